@@ -1,0 +1,382 @@
+// Golomb (Rice, M = 2^b) coding of the gaps between sent positions ("Sparse Binary
+// Compression", §II Optimal Position Encoding; Appendix A: the decoder needs no shapes).
+//
+// Codeword of gap d: q = d >> b one-bits, a zero-bit, then d mod 2^b in b bits, most significant
+// first; stream bit t is bit t % 32 of word t / 32.
+//
+// Encoder: codeword lengths -> device-wide exclusive scan (bit offsets) -> zero the stream ->
+// pack. A warp packs 32 codewords: it stages their offsets in shared memory and writes every
+// word that lies wholly inside its bit range with one plain store; only the two words it shares
+// with neighbouring warps are OR-ed atomically.
+// Decoder: with the side table, one thread per chunk of codewords decodes sequentially from its
+// recorded bit offset and checks that it ends where the next chunk starts.
+#include "common.cuh"
+
+namespace gs {
+namespace {
+
+constexpr int kScanThreads = 1024;
+
+struct GCtl {
+  int64_t begin, len;
+  int32_t abort;
+  int32_t pad;
+};
+
+__global__ void g_setup_kernel(const int64_t* d_begin, const int64_t* d_end, int64_t capacity,
+                               GCtl* ctl, int32_t* d_status) {
+  const int64_t b = d_begin ? *d_begin : 0;
+  const int64_t len = *d_end - b;
+  if (b < 0 || len < 0 || len > capacity) {
+    raise(d_status, GSPARSE_DERR_CAPACITY);
+    ctl->abort = 1;
+    ctl->len = 0;
+  } else {
+    ctl->abort = 0;
+    ctl->len = len;
+  }
+  ctl->begin = b;
+}
+
+// codeword length of entry j (validating the gap)
+__device__ __forceinline__ uint64_t code_len(const int32_t* idx, int64_t j, int64_t base, int b,
+                                             int32_t* d_status) {
+  const int64_t prev = j == 0 ? base - 1 : (int64_t)idx[j - 1];
+  int64_t d = (int64_t)idx[j] - prev - 1;
+  if (d < 0) {
+    raise(d_status, GSPARSE_DERR_INDEX_RANGE);
+    d = 0;
+  }
+  return (uint64_t)(d >> b) + 1u + (uint64_t)b;
+}
+
+// per-block totals of the codeword lengths
+__global__ void __launch_bounds__(kScanThreads) g_len_kernel(const int32_t* idx, const GCtl* ctl,
+                                                              int64_t base, int b, int64_t* block_tot,
+                                                              int32_t* d_status) {
+  __shared__ int64_t sh[33];
+  if (ctl->abort) return;
+  const int64_t len = ctl->len;
+  const int32_t* x = idx + ctl->begin;
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if ((int64_t)blockIdx.x * blockDim.x >= len) return;
+  const int64_t l = j < len ? (int64_t)code_len(x, j, base, b, d_status) : 0;
+  int64_t tot;
+  block_exclusive_scan(l, sh, &tot);
+  if (threadIdx.x == 0) block_tot[blockIdx.x] = tot;
+}
+
+// exclusive scan of the block totals (one CTA), total = stream length
+__global__ void __launch_bounds__(kScanThreads) g_scan_blocks_kernel(int64_t* block_tot,
+                                                                      const GCtl* ctl,
+                                                                      int64_t word_capacity,
+                                                                      uint64_t* d_nbits,
+                                                                      GCtl* wctl,
+                                                                      int32_t* d_status) {
+  __shared__ int64_t sh[33];
+  if (ctl->abort) {
+    if (threadIdx.x == 0) *d_nbits = 0;
+    return;
+  }
+  const int64_t nblk = cdiv(ctl->len, kScanThreads);
+  int64_t carry = 0;
+  for (int64_t base = 0; base < nblk; base += blockDim.x) {
+    const int64_t i = base + threadIdx.x;
+    const int64_t v = i < nblk ? block_tot[i] : 0;
+    int64_t tot;
+    const int64_t ex = block_exclusive_scan(v, sh, &tot);
+    if (i < nblk) block_tot[i] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) {
+    *d_nbits = (uint64_t)carry;
+    if (cdiv(carry, 32) > word_capacity) {
+      raise(d_status, GSPARSE_DERR_CAPACITY);
+      wctl->abort = 1;
+    }
+  }
+}
+
+// bit offset of every codeword, and the side table
+__global__ void __launch_bounds__(kScanThreads) g_offsets_kernel(const int32_t* idx, const GCtl* ctl,
+                                                                  int64_t base, int b,
+                                                                  const int64_t* block_pre,
+                                                                  uint64_t* offs, int64_t* table,
+                                                                  int32_t chunk) {
+  __shared__ int64_t sh[33];
+  if (ctl->abort) return;
+  const int64_t len = ctl->len;
+  const int32_t* x = idx + ctl->begin;
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if ((int64_t)blockIdx.x * blockDim.x >= len) return;
+  const int64_t l = j < len ? (int64_t)code_len(x, j, base, b, nullptr) : 0;
+  int64_t tot;
+  const int64_t ex = block_exclusive_scan(l, sh, &tot);
+  if (j < len) {
+    const int64_t o = block_pre[blockIdx.x] + ex;
+    offs[j] = (uint64_t)o;
+    if (table && j % chunk == 0) {
+      table[2 * (j / chunk)] = o;
+      table[2 * (j / chunk) + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
+    }
+  }
+}
+
+__global__ void g_zero_kernel(uint32_t* words, const uint64_t* d_nbits, int64_t bound,
+                              const GCtl* ctl, const GCtl* wctl) {
+  if (ctl->abort || wctl->abort) return;
+  const int64_t nw = cdiv((int64_t)*d_nbits, 32);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < nw && w < bound; w += stride)
+    words[w] = 0u;
+}
+
+struct Code {
+  uint64_t o;     // first bit
+  uint64_t q;     // unary length
+  uint32_t tail;  // (1 + b)-bit field after the unary run: terminator 0 then reversed remainder
+  uint32_t len_tail;
+};
+
+// bits of codeword c that fall in word w
+__device__ __forceinline__ uint32_t code_bits_in_word(const Code& c, uint64_t w) {
+  const uint64_t lo = w * 32, hi = lo + 32;
+  uint32_t bits = 0;
+  // unary ones [o, o + q)
+  const uint64_t a = c.o > lo ? c.o : lo;
+  const uint64_t e = (c.o + c.q) < hi ? (c.o + c.q) : hi;
+  if (a < e) {
+    const uint32_t n = (uint32_t)(e - a), s = (uint32_t)(a - lo);
+    bits |= (n == 32 ? 0xffffffffu : ((1u << n) - 1u)) << s;
+  }
+  // tail field at p = o + q
+  const uint64_t p = c.o + c.q;
+  if (p < hi && p + c.len_tail > lo) {
+    const uint64_t f = (uint64_t)c.tail;
+    if (p >= lo) bits |= (uint32_t)(f << (p - lo));
+    else bits |= (uint32_t)(f >> (lo - p));
+  }
+  return bits;
+}
+
+__global__ void __launch_bounds__(256) g_pack_kernel(const int32_t* idx, const GCtl* ctl,
+                                                      const GCtl* wctl, int64_t base, int b,
+                                                      const uint64_t* offs, uint32_t* words) {
+  __shared__ Code cs[8][32];
+  if (ctl->abort || wctl->abort) return;
+  const int64_t len = ctl->len;
+  const int32_t* x = idx + ctl->begin;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t j0 = ((int64_t)blockIdx.x * 8 + wid) * 32;
+  if (j0 >= len) return;
+  const int64_t j = j0 + lane;
+  const int nvalid = (int)((len - j0) < 32 ? (len - j0) : 32);
+  if (j < len) {
+    const int64_t prev = j == 0 ? base - 1 : (int64_t)x[j - 1];
+    int64_t d = (int64_t)x[j] - prev - 1;
+    if (d < 0) d = 0;  // reported by the length pass
+    Code c;
+    c.o = offs[j];
+    c.q = (uint64_t)(d >> b);
+    const uint32_t rem = (uint32_t)(d & ((int64_t(1) << b) - 1));
+    c.tail = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
+    c.len_tail = 1u + (uint32_t)b;
+    cs[wid][lane] = c;
+  }
+  __syncwarp();
+  const Code* C = cs[wid];
+  const uint64_t S = C[0].o;
+  const uint64_t E = C[nvalid - 1].o + C[nvalid - 1].q + C[nvalid - 1].len_tail;
+  const uint64_t wf = S >> 5, wl = (E - 1) >> 5;
+  for (uint64_t w = wf + lane; w <= wl; w += 32) {
+    // first codeword ending after the word starts
+    int lo = 0, hi = nvalid;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (C[mid].o + C[mid].q + C[mid].len_tail <= w * 32) lo = mid + 1; else hi = mid;
+    }
+    uint32_t bits = 0;
+    for (int k = lo; k < nvalid && C[k].o < w * 32 + 32; ++k) bits |= code_bits_in_word(C[k], w);
+    const bool shared_lo = (w == wf) && (S & 31);
+    const bool shared_hi = (w == wl) && (E & 31);
+    if (shared_lo || shared_hi) {
+      if (bits) atomicOr(&words[w], bits);
+    } else {
+      words[w] = bits;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// decoder
+
+__device__ __forceinline__ uint32_t word_at(const uint32_t* words, int64_t nw, int64_t w) {
+  return w < nw ? words[w] : 0u;
+}
+
+// Decodes `count` codewords from bit t; returns false (and raises) on a corrupt stream.
+__device__ bool decode_run(const uint32_t* words, uint64_t nbits, uint64_t& t, int64_t& prev,
+                           int64_t count, int b, int64_t n_limit, int32_t* out, int32_t* d_status) {
+  const int64_t nw = cdiv((int64_t)nbits, 32);
+  for (int64_t k = 0; k < count; ++k) {
+    uint64_t q = 0;
+    for (;;) {
+      if (t >= nbits) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+      const uint32_t sh = (uint32_t)(t & 31);
+      const uint32_t avail = 32 - sh;
+      const uint32_t v = word_at(words, nw, (int64_t)(t >> 5)) >> sh;
+      const uint32_t zeros = ~v & (avail == 32 ? 0xffffffffu : ((1u << avail) - 1u));
+      if (zeros) {
+        const uint32_t z = (uint32_t)__ffs(zeros) - 1u;
+        q += z;
+        t += z + 1;
+        break;
+      }
+      q += avail;
+      t += avail;
+    }
+    if (t > nbits) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+    uint32_t rem = 0;
+    if (b > 0) {
+      if (t + (uint64_t)b > nbits) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+      const uint64_t w = t >> 5;
+      const uint64_t win = (uint64_t)word_at(words, nw, (int64_t)w) |
+                           ((uint64_t)word_at(words, nw, (int64_t)w + 1) << 32);
+      const uint32_t raw = (uint32_t)(win >> (t & 31)) & ((1u << b) - 1u);
+      rem = __brev(raw) >> (32 - b);
+      t += (uint64_t)b;
+    }
+    if (q > (uint64_t)INT32_MAX) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); return false; }
+    const int64_t i = prev + 1 + (int64_t)((q << b) | rem);
+    if (i >= n_limit || i > INT32_MAX) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); return false; }
+    out[k] = (int32_t)i;
+    prev = i;
+  }
+  return true;
+}
+
+__global__ void g_decode_chunks_kernel(const uint32_t* words, int64_t word_capacity,
+                                       const uint64_t* d_nbits,
+                                       const int64_t* d_count, int64_t capacity, int b,
+                                       const int64_t* table, int32_t chunk, int64_t n_limit,
+                                       int32_t* out, int32_t* d_status) {
+  const int64_t K = *d_count;
+  if (K < 0 || K > capacity) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise(d_status, GSPARSE_DERR_CAPACITY);
+    return;
+  }
+  const int64_t nch = cdiv(K, chunk);
+  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= nch) return;
+  const uint64_t nbits = *d_nbits;
+  if (nbits > (uint64_t)word_capacity * 32u) {
+    if (c == 0) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+    return;
+  }
+  uint64_t t = (uint64_t)table[2 * c];
+  int64_t prev = table[2 * c + 1];
+  const int64_t first = c * chunk;
+  const int64_t count = (K - first) < chunk ? (K - first) : chunk;
+  if (t > nbits) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return; }
+  if (!decode_run(words, nbits, t, prev, count, b, n_limit, out + first, d_status)) return;
+  const bool last = c + 1 == nch;
+  const uint64_t end = last ? nbits : (uint64_t)table[2 * (c + 1)];
+  if (t != end || (!last && prev != table[2 * (c + 1) + 1])) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+}
+
+__global__ void g_decode_serial_kernel(const uint32_t* words, int64_t word_capacity,
+                                       const uint64_t* d_nbits,
+                                       const int64_t* d_count, int64_t capacity, int64_t base,
+                                       int b, int64_t n_limit, int32_t* out, int32_t* d_status) {
+  const int64_t K = *d_count;
+  if (K < 0 || K > capacity) { raise(d_status, GSPARSE_DERR_CAPACITY); return; }
+  const uint64_t nbits = *d_nbits;
+  if (nbits > (uint64_t)word_capacity * 32u) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return; }
+  uint64_t t = 0;
+  int64_t prev = base - 1;
+  if (!decode_run(words, nbits, t, prev, K, b, n_limit, out, d_status)) return;
+  if (t != nbits) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+}
+
+struct GLayout {
+  GCtl* ctl;
+  GCtl* wctl;
+  int64_t* block_tot;
+  uint64_t* offs;
+  size_t bytes;
+};
+
+GLayout g_carve(int64_t capacity, void* ws) {
+  GLayout L;
+  Carver cv(ws);
+  L.ctl = cv.take<GCtl>(1);
+  L.wctl = cv.take<GCtl>(1);
+  L.block_tot = cv.take<int64_t>(cdiv(capacity, kScanThreads) + 1);
+  L.offs = cv.take<uint64_t>(capacity);
+  L.bytes = cv.off + 256;
+  return L;
+}
+
+}  // namespace
+}  // namespace gs
+
+using namespace gs;
+
+extern "C" {
+
+size_t gsparse_golomb_encode_workspace_size(int64_t capacity) {
+  if (capacity < 0) return 0;
+  return g_carve(capacity, nullptr).bytes;
+}
+
+int gsparse_golomb_encode(const int32_t* idx, const int64_t* d_begin, const int64_t* d_end,
+                          int64_t capacity, int64_t base, int32_t b, uint32_t* words,
+                          int64_t word_capacity, uint64_t* d_nbits, int64_t* chunk_table,
+                          int32_t chunk, void* workspace, size_t workspace_bytes,
+                          int32_t* d_status, gsparse_stream stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  if (capacity < 0 || word_capacity < 0 || !d_end || !d_nbits || (capacity > 0 && (!idx || !words)) ||
+      (chunk_table && chunk <= 0))
+    return GSPARSE_ERR_INVALID_ARG;
+  if (b < 0 || b > 30 || capacity > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GSPARSE_ERR_WORKSPACE;
+  GLayout L = g_carve(capacity, workspace);
+  if (workspace_bytes < L.bytes) return GSPARSE_ERR_WORKSPACE;
+  g_setup_kernel<<<1, 1, 0, st>>>(d_begin, d_end, capacity, L.ctl, d_status);
+  if (cudaMemsetAsync(L.wctl, 0, sizeof(GCtl), st) != cudaSuccess) return GSPARSE_ERR_CUDA;
+  const unsigned nblk = (unsigned)cdiv(capacity > 0 ? capacity : 1, kScanThreads);
+  g_len_kernel<<<nblk, kScanThreads, 0, st>>>(idx, L.ctl, base, b, L.block_tot, d_status);
+  g_scan_blocks_kernel<<<1, kScanThreads, 0, st>>>(L.block_tot, L.ctl, word_capacity, d_nbits,
+                                                    L.wctl, d_status);
+  g_offsets_kernel<<<nblk, kScanThreads, 0, st>>>(idx, L.ctl, base, b, L.block_tot, L.offs,
+                                                   chunk_table, chunk);
+  const int64_t zb = cdiv(word_capacity > 0 ? word_capacity : 1, 256);
+  g_zero_kernel<<<(unsigned)(zb < 148 * 16 ? zb : 148 * 16), 256, 0, st>>>(words, d_nbits,
+                                                                            word_capacity, L.ctl, L.wctl);
+  const int64_t warps = cdiv(capacity > 0 ? capacity : 1, 32);
+  g_pack_kernel<<<(unsigned)cdiv(warps, 8), 256, 0, st>>>(idx, L.ctl, L.wctl, base, b, L.offs, words);
+  return launch_status();
+}
+
+int gsparse_golomb_decode(const uint32_t* words, int64_t word_capacity, const uint64_t* d_nbits,
+                          const int64_t* d_count, int64_t capacity, int64_t base, int32_t b,
+                          const int64_t* chunk_table, int32_t chunk, int64_t n_limit,
+                          int32_t* out_idx, int32_t* d_status, gsparse_stream stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  if (capacity < 0 || word_capacity < 0 || !d_nbits || !d_count || (capacity > 0 && (!words || !out_idx)) ||
+      (chunk_table && chunk <= 0))
+    return GSPARSE_ERR_INVALID_ARG;
+  if (b < 0 || b > 30 || capacity > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
+  if (chunk_table) {
+    const int64_t nch = cdiv(capacity > 0 ? capacity : 1, chunk);
+    g_decode_chunks_kernel<<<(unsigned)cdiv(nch, 128), 128, 0, st>>>(
+        words, word_capacity, d_nbits, d_count, capacity, b, chunk_table, chunk, n_limit, out_idx,
+        d_status);
+  } else {
+    g_decode_serial_kernel<<<1, 1, 0, st>>>(words, word_capacity, d_nbits, d_count, capacity, base,
+                                            b, n_limit, out_idx, d_status);
+  }
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,287 @@
+// Receive side: sum of W workers' sparse updates and its combination with the local gradient
+// ("Combining Global Sparse Gradients with Local Gradients in Distributed Neural Network
+// Training", Abstract; "Sparse Binary Compression", §I: the clients' updates are summed).
+//
+// Scatter-accumulate works on tiles of 8192 consecutive indices. One CTA owns a tile: it finds
+// each worker's entries in the tile by binary search (the lists are sorted), adds them worker by
+// worker into a shared-memory accumulator (fixed worker order, one fp32 add per entry, so the
+// result is bitwise reproducible), writes the dense tile with coalesced stores and counts the
+// touched indices. The merged sparse output is an ordered compaction of the touched indices
+// after a scan over the tile counts.
+#include "common.cuh"
+
+namespace gs {
+namespace {
+
+constexpr int kTile = 8192;
+constexpr int kTileThreads = 256;
+
+struct Lists {
+  const int32_t* idx[GSPARSE_MAX_WORKERS];
+  const float* val[GSPARSE_MAX_WORKERS];
+  const float* uni[GSPARSE_MAX_WORKERS];
+  const int64_t* cnt[GSPARSE_MAX_WORKERS];
+  int64_t cap[GSPARSE_MAX_WORKERS];
+};
+
+__device__ __forceinline__ int64_t list_count(const Lists& L, int w) {
+  int64_t c = *L.cnt[w];
+  if (c < 0) c = 0;
+  return c > L.cap[w] ? L.cap[w] : c;
+}
+
+// start[t][w] = first entry of worker w with index >= t * kTile, for t = 0..ntiles
+__global__ void sa_bounds_kernel(Lists L, int32_t W, int64_t n, int64_t ntiles, int64_t* start,
+                                 int32_t* d_status) {
+  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= (ntiles + 1) * W) return;
+  const int64_t t = k / W;
+  const int w = (int)(k % W);
+  const int64_t c = list_count(L, w);
+  if (t == 0 && c > 0) {
+    if (*L.cnt[w] > L.cap[w]) raise(d_status, GSPARSE_DERR_CAPACITY);
+    if (L.idx[w][0] < 0 || (int64_t)L.idx[w][c - 1] >= n) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
+  }
+  start[k] = t == ntiles ? c : lower_bound_i32(L.idx[w], c, t * kTile);
+}
+
+// Accumulates tile t into acc[] (zeroed) and sets touched bits.
+__device__ void accumulate_tile(const Lists& L, int32_t W, int64_t t, const int64_t* start,
+                                float* acc, uint32_t* touched, int32_t* d_status) {
+  const int64_t t0 = t * kTile;
+  for (int w = 0; w < W; ++w) {
+    const int64_t b = start[t * W + w], e = start[(t + 1) * W + w];
+    const int32_t* ix = L.idx[w];
+    const float* vv = L.val[w];
+    const float u = vv ? 0.0f : *L.uni[w];
+    for (int64_t j = b + threadIdx.x; j < e; j += blockDim.x) {
+      const int32_t i = ix[j];
+      if (j > 0 && ix[j - 1] >= i) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); continue; }
+      const int off = (int)(i - t0);
+      if (off < 0 || off >= kTile) continue;  // out of range, reported by the bounds pass
+      acc[off] = __fadd_rn(acc[off], vv ? vv[j] : u);
+      atomicOr(&touched[off >> 5], 1u << (off & 31));
+    }
+    __syncthreads();  // worker order: all of worker w before any of worker w + 1
+  }
+}
+
+__global__ void __launch_bounds__(kTileThreads) sa_tile_kernel(Lists L, int32_t W, int64_t n,
+                                                               const int64_t* start, float* dense,
+                                                               int64_t* tile_count,
+                                                               int32_t* d_status) {
+  __shared__ __align__(16) float acc[kTile];
+  __shared__ uint32_t touched[kTile / 32];
+  const int64_t t = blockIdx.x;
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) acc[i] = 0.0f;
+  for (int i = threadIdx.x; i < kTile / 32; i += blockDim.x) touched[i] = 0u;
+  __syncthreads();
+  accumulate_tile(L, W, t, start, acc, touched, d_status);
+  const int64_t t0 = t * kTile;
+  const int64_t m = (n - t0) < kTile ? (n - t0) : kTile;
+  if (dense) {
+    if (m == kTile) {
+      for (int v = threadIdx.x; v < kTile / 4; v += blockDim.x)
+        st_stream(dense + t0 + 4 * v, reinterpret_cast<const float4*>(acc)[v]);
+    } else {
+      for (int i = threadIdx.x; i < m; i += blockDim.x) dense[t0 + i] = acc[i];
+    }
+  }
+  if (tile_count) {
+    __shared__ int64_t sh[33];
+    int64_t c = 0;
+    for (int i = threadIdx.x; i < kTile / 32; i += blockDim.x) c += __popc(touched[i]);
+    int64_t tot;
+    block_exclusive_scan(c, sh, &tot);
+    if (threadIdx.x == 0) tile_count[t] = tot;
+  }
+}
+
+__global__ void __launch_bounds__(1024) sa_scan_kernel(int64_t* tile_count, int64_t ntiles,
+                                                       int64_t* d_merged_count, int64_t capacity,
+                                                       int32_t* ctl, int32_t* d_status) {
+  __shared__ int64_t sh[33];
+  int64_t carry = 0;
+  for (int64_t base = 0; base < ntiles; base += blockDim.x) {
+    const int64_t i = base + threadIdx.x;
+    const int64_t v = i < ntiles ? tile_count[i] : 0;
+    int64_t tot;
+    const int64_t ex = block_exclusive_scan(v, sh, &tot);
+    if (i < ntiles) tile_count[i] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) {
+    *d_merged_count = carry;
+    ctl[0] = carry > capacity;
+    if (carry > capacity) raise(d_status, GSPARSE_DERR_CAPACITY);
+  }
+}
+
+__global__ void __launch_bounds__(kTileThreads) sa_merge_kernel(Lists L, int32_t W, const int64_t* start,
+                                                                const int64_t* tile_off,
+                                                                int32_t* merged_idx, float* merged_val,
+                                                                const int32_t* ctl) {
+  __shared__ float acc[kTile];
+  __shared__ uint32_t touched[kTile / 32];
+  __shared__ int64_t sh[33];
+  if (ctl[0]) return;
+  const int64_t t = blockIdx.x;
+  // skip tiles no worker touches
+  bool any = false;
+  for (int w = 0; w < W; ++w) any |= start[t * W + w] != start[(t + 1) * W + w];
+  if (!any) return;
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) acc[i] = 0.0f;
+  for (int i = threadIdx.x; i < kTile / 32; i += blockDim.x) touched[i] = 0u;
+  __syncthreads();
+  accumulate_tile(L, W, t, start, acc, touched, nullptr);
+  // thread k owns bitmap word k (kTile / 32 == blockDim.x)
+  const uint32_t word = touched[threadIdx.x];
+  int64_t tot;
+  const int64_t pre = block_exclusive_scan(__popc(word), sh, &tot);
+  int64_t o = tile_off[t] + pre;
+  uint32_t wbits = word;
+  while (wbits) {
+    const int b = __ffs(wbits) - 1;
+    wbits &= wbits - 1;
+    const int off = threadIdx.x * 32 + b;
+    merged_idx[o] = (int32_t)(t * kTile + off);
+    merged_val[o] = acc[off];
+    ++o;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// combine
+
+__global__ void combine_kernel(const float* G, const float* Lg, float* out, int64_t n, float alpha,
+                               float beta) {
+  const int64_t nv = n >> 2;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nv; v += stride) {
+    const float4 g = ld_stream(G + 4 * v), l = ld_stream(Lg + 4 * v);
+    float4 o;
+    o.x = __fadd_rn(__fmul_rn(alpha, g.x), __fmul_rn(beta, l.x));
+    o.y = __fadd_rn(__fmul_rn(alpha, g.y), __fmul_rn(beta, l.y));
+    o.z = __fadd_rn(__fmul_rn(alpha, g.z), __fmul_rn(beta, l.z));
+    o.w = __fadd_rn(__fmul_rn(alpha, g.w), __fmul_rn(beta, l.w));
+    st_stream(out + 4 * v, o);
+  }
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < (n & 3)) {
+    const int64_t i = 4 * nv + t;
+    out[i] = __fadd_rn(__fmul_rn(alpha, G[i]), __fmul_rn(beta, Lg[i]));
+  }
+}
+
+__global__ void combine_partial_kernel(const float* G, const float* Lg, float* out, int64_t n,
+                                       float alpha, float beta, const int32_t* own_idx,
+                                       const float* own_val, const int64_t* d_count,
+                                       int64_t capacity, int32_t* d_status) {
+  int64_t K = *d_count;
+  if (K > capacity) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise(d_status, GSPARSE_DERR_CAPACITY);
+    K = capacity;
+  }
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= K) return;
+  const int32_t i = own_idx[j];
+  if (i < 0 || (int64_t)i >= n) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); return; }
+  const float gi = __fsub_rn(G[i], own_val[j]);
+  out[i] = __fadd_rn(__fmul_rn(alpha, gi), __fmul_rn(beta, Lg[i]));
+}
+
+struct SLayout {
+  int64_t* start;
+  int64_t* tile_count;
+  int32_t* ctl;
+  size_t bytes;
+};
+
+SLayout s_carve(int32_t W, int64_t n, void* ws) {
+  SLayout L;
+  Carver cv(ws);
+  const int64_t ntiles = cdiv(n, kTile);
+  L.start = cv.take<int64_t>((ntiles + 1) * W);
+  L.tile_count = cv.take<int64_t>(ntiles + 1);
+  L.ctl = cv.take<int32_t>(4);
+  L.bytes = cv.off + 256;
+  return L;
+}
+
+}  // namespace
+}  // namespace gs
+
+using namespace gs;
+
+extern "C" {
+
+size_t gsparse_scatter_accumulate_workspace_size(int32_t W, int64_t n) {
+  if (W < 1 || n < 0) return 0;
+  return s_carve(W, n, nullptr).bytes;
+}
+
+int gsparse_scatter_accumulate(const gsparse_list* lists, int32_t W, int64_t n, float* dense_out,
+                               int32_t* merged_idx, float* merged_val, int64_t* d_merged_count,
+                               int64_t merged_capacity, void* workspace, size_t workspace_bytes,
+                               int32_t* d_status, gsparse_stream stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!lists || W < 1 || n < 0 || merged_capacity < 0) return GSPARSE_ERR_INVALID_ARG;
+  if (W > GSPARSE_MAX_WORKERS || n > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
+  const bool merged = d_merged_count != nullptr;
+  if (merged && merged_capacity > 0 && (!merged_idx || !merged_val)) return GSPARSE_ERR_INVALID_ARG;
+  if (dense_out && !aligned16(dense_out)) return GSPARSE_ERR_INVALID_ARG;
+  Lists L{};
+  for (int w = 0; w < W; ++w) {
+    const gsparse_list& x = lists[w];
+    if (!x.d_count || x.capacity < 0 || (x.capacity > 0 && !x.idx) || (!x.val && !x.uniform_val))
+      return GSPARSE_ERR_INVALID_ARG;
+    L.idx[w] = x.idx;
+    L.val[w] = x.val;
+    L.uni[w] = x.uniform_val;
+    L.cnt[w] = x.d_count;
+    L.cap[w] = x.capacity;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GSPARSE_ERR_WORKSPACE;
+  SLayout S = s_carve(W, n, workspace);
+  if (workspace_bytes < S.bytes) return GSPARSE_ERR_WORKSPACE;
+  const int64_t ntiles = cdiv(n, kTile);
+  if (ntiles == 0) {
+    if (merged && cudaMemsetAsync(d_merged_count, 0, sizeof(int64_t), st) != cudaSuccess)
+      return GSPARSE_ERR_CUDA;
+    return launch_status();
+  }
+  const int64_t nb = (ntiles + 1) * W;
+  sa_bounds_kernel<<<(unsigned)cdiv(nb, 256), 256, 0, st>>>(L, W, n, ntiles, S.start, d_status);
+  sa_tile_kernel<<<(unsigned)ntiles, kTileThreads, 0, st>>>(L, W, n, S.start, dense_out,
+                                                            merged ? S.tile_count : nullptr, d_status);
+  if (merged) {
+    sa_scan_kernel<<<1, 1024, 0, st>>>(S.tile_count, ntiles, d_merged_count, merged_capacity, S.ctl,
+                                       d_status);
+    sa_merge_kernel<<<(unsigned)ntiles, kTileThreads, 0, st>>>(L, W, S.start, S.tile_count,
+                                                               merged_idx, merged_val, S.ctl);
+  }
+  return launch_status();
+}
+
+int gsparse_combine_local(const float* G, const float* L, float* out, int64_t n, float alpha,
+                          float beta, int32_t mode, const int32_t* own_idx, const float* own_val,
+                          const int64_t* d_own_count, int64_t own_capacity, int32_t* d_status,
+                          gsparse_stream stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  if (n < 0 || (mode != 0 && mode != 1)) return GSPARSE_ERR_INVALID_ARG;
+  if (n > 0 && (!G || !L || !out || !aligned16(G) || !aligned16(L) || !aligned16(out)))
+    return GSPARSE_ERR_INVALID_ARG;
+  if (mode == 1 && (!d_own_count || own_capacity < 0 || (own_capacity > 0 && (!own_idx || !own_val))))
+    return GSPARSE_ERR_INVALID_ARG;
+  if (mode == 1 && (out == G || out == L)) return GSPARSE_ERR_INVALID_ARG;
+  if (n > 0) {
+    const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
+    combine_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(G, L, out, n, alpha, beta);
+  }
+  if (mode == 1 && own_capacity > 0)
+    combine_partial_kernel<<<(unsigned)cdiv(own_capacity, 256), 256, 0, st>>>(
+        G, L, out, n, alpha, beta, own_idx, own_val, d_own_count, own_capacity, d_status);
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,1059 @@
+// Exact residual top-k and sparse binarisation on B200.
+//
+// Method: "Sparse Communication for Distributed Gradient Descent" (Aji & Heafield 2017),
+// Abstract — drop the 99% smallest updates by |value|; "Sparse Binary Compression" (Sattler et
+// al. 2018), §II Residual Accumulation, Sparse Binarization, Communication Delay.
+//
+// Design (one call = a fixed sequence of kernels on the caller's stream, no host sync):
+//  1. plan     per-segment sizes, k_s, output bases and the split of each segment into "pieces"
+//              (contiguous ranges of <= Lp entries, one warp each).
+//  2. sample   per segment, a 16384-entry sample of acc = g + r gives a candidate threshold
+//              T_lo that a little more than k_s entries reach (the exact k_s-th key when the
+//              whole segment fits in the sample).
+//  3. pass 1   the only full stream over the data: 128-bit loads of g and r, acc = fl(g + r),
+//              residual <- acc (or +0 for candidates in top-k mode, so sent entries never need
+//              a second write), candidates (key >= T_lo) appended per piece in index order by a
+//              warp-ballot compaction, and a shared-memory histogram of candidate keys.
+//  4. check    a segment whose sample threshold was too high (fewer than k_s candidates) is
+//              redone exhaustively; pieces whose candidate store overflowed are re-read from
+//              the residual. Both routes give the same result, only slower.
+//  5-7.        three radix-select levels (11 + 11 + 9 bits of the key) over the candidates give
+//              the exact k_s-th key T and how many entries equal to T are taken.
+//  8-9. count + scan per piece, then emit: selected candidates are written in index order;
+//              candidates not selected get their acc back into the residual.
+// Ties: keys equal to T are taken in ascending index order, so the lowest indices win.
+#include <math.h>
+
+#include "common.cuh"
+#include "osum.cuh"
+
+namespace gs {
+namespace {
+
+constexpr uint32_t kNone = 0x80000000u;  // a threshold no 31-bit key reaches
+constexpr int kBins1 = 2048, kBins2 = 2048, kBins3 = 512;
+constexpr int kHist = kBins1 + kBins2 + kBins3;  // per problem
+constexpr int64_t kGranule = 512;                // entries per warp iteration (32 lanes x 16)
+constexpr int64_t kTargetPieces = 148 * 32;      // warps streaming at once on a B200
+constexpr int kSample = 16384;                   // sampled entries per segment
+constexpr int kSampleChunks = kSample / 32;
+constexpr int kWarps = 8;                        // warps (pieces) per CTA
+constexpr int kThreads = kWarps * 32;
+
+struct Sel {
+  const float* g;
+  float* r;
+  int64_t n;
+  int32_t T, C;       // segments; classes: 1 = |x| (top-k), 2 = x > 0 and x < 0 (binarise)
+  int32_t zero_mode;  // top-k: write +0 for candidates in pass 1
+  int32_t pad;
+  int64_t Lp, Q, cap;
+  int64_t *seg_lo, *seg_n, *seg_k, *seg_kbase, *seg_pbase;
+  uint32_t *tlo, *redo, *pfx, *thr;
+  int64_t *keff, *krem, *need_eq;
+  uint32_t* hist;  // [P][kHist]
+  uint32_t *pcnt, *prsrc, *pgt, *peq, *ptake;
+  int64_t* poff;
+  int32_t* cidx;
+  float* cval;
+  int32_t* ctl;  // [0] abort, [1] any redo
+  int32_t* d_status;
+  // binarise
+  int32_t* lidx;
+  float* lval;
+  int32_t* bsel;
+};
+
+struct Piece {
+  int64_t lo, hi;
+  int32_t s;
+};
+
+__device__ __forceinline__ int64_t total_pieces(const Sel& a) { return a.seg_pbase[a.T]; }
+
+__device__ __forceinline__ Piece piece_of(const Sel& a, int64_t q) {
+  Piece p;
+  p.s = (int32_t)(upper_bound_i64(a.seg_pbase, a.T + 1, q) - 1);
+  p.lo = a.seg_lo[p.s] + (q - a.seg_pbase[p.s]) * a.Lp;
+  const int64_t end = a.seg_lo[p.s] + a.seg_n[p.s];
+  p.hi = p.lo + a.Lp < end ? p.lo + a.Lp : end;
+  return p;
+}
+
+// class of an accumulated value: top-k has one class; binarise splits by sign (zeros in none)
+template <int C>
+__device__ __forceinline__ int class_of(float x) {
+  if (C == 1) return 0;
+  return x > 0.0f ? 0 : (x < 0.0f ? 1 : -1);
+}
+
+__device__ __forceinline__ uint32_t* hist_of(const Sel& a, int64_t p, int level) {
+  return a.hist + p * kHist + (level == 1 ? 0 : (level == 2 ? kBins1 : kBins1 + kBins2));
+}
+
+// Histogram sink of a CTA: counts for the CTA's first segment go to shared memory and are
+// flushed once; counts for other segments (CTAs straddling a segment boundary) go straight to
+// global memory.
+template <int C, int BINS>
+struct CtaHist {
+  uint32_t sh[C * BINS];
+  int64_t primary;
+  __device__ void add(const Sel& a, int32_t s, int c, uint32_t bin, int level) {
+    if (s == primary) atomicAdd(&sh[c * BINS + bin], 1u);
+    else atomicAdd(hist_of(a, (int64_t)s * C + c, level) + bin, 1u);
+  }
+  __device__ void init(const Sel& a, int64_t q0) {
+    for (int i = threadIdx.x; i < C * BINS; i += blockDim.x) sh[i] = 0;
+    if (threadIdx.x == 0) primary = q0 < total_pieces(a) ? piece_of(a, q0).s : -1;
+  }
+  // adds the shared counts of bins [0, bins) to the primary segment's histograms
+  __device__ void flush(const Sel& a, int level, int bins) {
+    if (primary < 0) return;
+    for (int i = threadIdx.x; i < C * BINS; i += blockDim.x) {
+      const uint32_t h = sh[i];
+      if (h && (i % BINS) < bins) atomicAdd(hist_of(a, primary * C + i / BINS, level) + (i % BINS), h);
+    }
+  }
+};
+
+// ------------------------------------------------------------------------------------------
+// block helpers for the select steps (blockDim.x == 1024)
+
+// Given bin counts h[0..B) and a rank (1 = largest), find the bin b holding the rank-th largest
+// entry: sum(h[b+1..B)) < rank <= sum(h[b..B)). Returns b and the count above it.
+__device__ void block_find_bin(const uint32_t* h, int B, int64_t rank, uint32_t* bin_out,
+                               int64_t* above_out) {
+  __shared__ int64_t sh[33];
+  __shared__ uint32_t fb;
+  __shared__ int64_t fa;
+  const int per = (B + (int)blockDim.x - 1) / (int)blockDim.x;
+  // thread t owns bins [B - (t+1)*per, B - t*per) walked downwards
+  const int hi = B - (int)threadIdx.x * per;
+  int64_t mine = 0;
+  for (int j = 0; j < per; ++j) {
+    const int b = hi - 1 - j;
+    if (b >= 0) mine += h[b];
+  }
+  int64_t tot;
+  int64_t above = block_exclusive_scan(mine, sh, &tot);
+  if (threadIdx.x == 0) { fb = 0; fa = 0; }
+  __syncthreads();
+  for (int j = 0; j < per; ++j) {
+    const int b = hi - 1 - j;
+    if (b < 0) break;
+    const int64_t c = h[b];
+    if (above < rank && rank <= above + c) { fb = (uint32_t)b; fa = above; }
+    above += c;
+  }
+  __syncthreads();
+  *bin_out = fb;
+  *above_out = fa;
+  __syncthreads();
+}
+
+// rank-th largest of keys[0..cnt) in shared memory (1 <= rank <= cnt), by 11+11+9-bit radix steps.
+__device__ uint32_t block_select_key(const uint32_t* keys, int cnt, int64_t rank, uint32_t* hist) {
+  uint32_t prefix = 0;
+  const int shifts[3] = {20, 9, 0};
+  const int widths[3] = {11, 11, 9};
+  for (int L = 0; L < 3; ++L) {
+    const int sh = shifts[L], w = widths[L], B = 1 << w;
+    for (int i = threadIdx.x; i < B; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+      const uint32_t k = keys[i];
+      if ((k >> (sh + w)) == prefix) atomicAdd(&hist[(k >> sh) & (B - 1)], 1u);
+    }
+    __syncthreads();
+    uint32_t bin;
+    int64_t above;
+    block_find_bin(hist, B, rank, &bin, &above);
+    prefix = (prefix << w) | bin;
+    rank -= above;
+  }
+  return prefix;
+}
+
+// ------------------------------------------------------------------------------------------
+// 1. plan
+
+__global__ void __launch_bounds__(1024) plan_kernel(Sel a, const int64_t* seg, int64_t knum, int64_t kden,
+                            int64_t out_capacity, int64_t* out_offsets) {
+  __shared__ int64_t sh[33];
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  int64_t carry_k = 0, carry_p = 0;
+  for (int64_t base = 0; base < a.T; base += blockDim.x) {
+    const int64_t s = base + threadIdx.x;
+    int64_t k = 0, np = 0;
+    if (s < a.T) {
+      const int64_t lo = seg ? seg[s] : 0;
+      const int64_t hi = seg ? seg[s + 1] : a.n;
+      if (hi < lo || lo < 0 || hi > a.n || (s == 0 && lo != 0) || (s == a.T - 1 && hi != a.n)) bad = 1;
+      const int64_t ns = hi > lo ? hi - lo : 0;
+      k = kept_count(ns, knum, kden);
+      np = cdiv(ns, a.Lp);
+      a.seg_lo[s] = lo;
+      a.seg_n[s] = ns;
+      a.seg_k[s] = k;
+    }
+    int64_t tk, tp;
+    const int64_t ek = block_exclusive_scan(k, sh, &tk);
+    const int64_t ep = block_exclusive_scan(np, sh, &tp);
+    if (s < a.T) {
+      a.seg_kbase[s] = carry_k + ek;
+      a.seg_pbase[s] = carry_p + ep;
+    }
+    carry_k += tk;
+    carry_p += tp;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    a.seg_kbase[a.T] = carry_k;
+    a.seg_pbase[a.T] = carry_p;
+    if (bad || carry_p > a.Q) {
+      raise(a.d_status, GSPARSE_DERR_SEGMENTS);
+      a.ctl[0] = 1;
+      a.seg_pbase[a.T] = 0;
+    } else if (carry_k > out_capacity) {
+      raise(a.d_status, GSPARSE_DERR_CAPACITY);
+      a.ctl[0] = 1;
+      a.seg_pbase[a.T] = 0;
+    }
+  }
+  __syncthreads();
+  if (out_offsets && !a.ctl[0])
+    for (int64_t s = threadIdx.x; s <= a.T; s += blockDim.x) out_offsets[s] = a.seg_kbase[s];
+}
+
+// ------------------------------------------------------------------------------------------
+// 2. sample: candidate thresholds
+
+template <int C>
+__global__ void __launch_bounds__(1024) sample_kernel(Sel a, int exhaustive) {
+  extern __shared__ uint32_t skeys[];  // [C][kSample]
+  __shared__ uint32_t hist[kBins1];
+  __shared__ int cnt[2];
+  if (a.ctl[0]) return;
+  const int32_t s = blockIdx.x;
+  const int64_t lo = a.seg_lo[s], ns = a.seg_n[s], k = a.seg_k[s];
+  const int64_t P0 = (int64_t)s * C;
+  if (k == 0 || ns == 0) {
+    if (threadIdx.x < C) a.tlo[P0 + threadIdx.x] = kNone;
+    return;
+  }
+  if (exhaustive) {
+    if (threadIdx.x < C) a.tlo[P0 + threadIdx.x] = 0;
+    return;
+  }
+  if (threadIdx.x < 2) cnt[threadIdx.x] = 0;
+  __syncthreads();
+  const bool full = ns <= kSample;
+  const int S = full ? (int)ns : kSample;
+  for (int j = threadIdx.x; j < S; j += blockDim.x) {
+    int64_t i;
+    if (full) {
+      i = lo + j;
+    } else {  // 512 evenly spaced runs of 32 consecutive entries
+      const int64_t chunk = j >> 5;
+      i = lo + chunk * (ns - 32) / (kSampleChunks - 1) + (j & 31);
+    }
+    const float x = __fadd_rn(a.g[i], a.r[i]);
+    const int c = class_of<C>(x);
+    if (c < 0) continue;
+    const int pos = atomicAdd(&cnt[c], 1);
+    skeys[c * kSample + pos] = mag_key(x);
+  }
+  __syncthreads();
+  for (int c = 0; c < C; ++c) {
+    const int count = cnt[c];
+    uint32_t t;
+    if (full) {
+      const int64_t m = k < count ? k : count;
+      if (count == 0) t = kNone;                // class absent from the segment
+      else if (m == count) t = 0;               // every member is needed
+      else t = block_select_key(skeys + c * kSample, count, m, hist);
+    } else {
+      const double e = (double)k * (double)S / (double)ns;
+      const int64_t m = (int64_t)ceil(e + 4.0 * sqrt(e) + 8.0);
+      if (m >= count) t = 0;
+      else t = block_select_key(skeys + c * kSample, count, m, hist);
+    }
+    if (threadIdx.x == 0) a.tlo[P0 + c] = t;
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// 3. pass 1: the streaming pass
+
+template <int C>
+__global__ void __launch_bounds__(kThreads, 4) pass1_kernel(Sel a) {
+  __shared__ CtaHist<C, kBins1> H;
+  if (a.ctl[0]) return;
+  const int64_t q0 = (int64_t)blockIdx.x * kWarps;
+  H.init(a, q0);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t q = q0 + (threadIdx.x >> 5);
+  if (q < total_pieces(a)) {
+    const Piece P = piece_of(a, q);
+    uint32_t tl[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) tl[c] = a.tlo[(int64_t)P.s * C + c];
+    const int64_t cap = a.cap;
+    int32_t* cidx = a.cidx + q * cap;
+    float* cval = a.cval + q * cap;
+    uint32_t count = 0;
+    for (int64_t base = P.lo & ~(int64_t)3; base < P.hi; base += kGranule) {
+      float4 gv[4], rv[4];
+      bool full[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t v = base + u * 128 + lane * 4;
+        full[u] = v >= P.lo && v + 4 <= P.hi;
+        if (full[u]) {
+          gv[u] = ld_stream(a.g + v);
+          rv[u] = ld_stream(a.r + v);
+        } else {
+          float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int64_t i = v + e;
+            if (i >= P.lo && i < P.hi) { t0[e] = a.g[i]; t1[e] = a.r[i]; }
+          }
+          gv[u] = make_float4(t0[0], t0[1], t0[2], t0[3]);
+          rv[u] = make_float4(t1[0], t1[1], t1[2], t1[3]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t v = base + u * 128 + lane * 4;
+        float acc[4] = {__fadd_rn(gv[u].x, rv[u].x), __fadd_rn(gv[u].y, rv[u].y),
+                        __fadd_rn(gv[u].z, rv[u].z), __fadd_rn(gv[u].w, rv[u].w)};
+        uint32_t m4 = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int64_t i = v + e;
+          const int c = class_of<C>(acc[e]);
+          const bool cand = i >= P.lo && i < P.hi && c >= 0 && mag_key(acc[e]) >= tl[c < 0 ? 0 : c];
+          m4 |= (uint32_t)cand << e;
+        }
+        uint32_t tot;
+        const uint32_t pre = warp_prefix_small(__popc(m4), &tot);
+        uint32_t stored = 0;
+        if (tot) {
+          uint32_t pos = count + pre;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if ((m4 >> e) & 1u) {
+              if (pos < cap) {
+                cidx[pos] = (int32_t)(v + e);
+                cval[pos] = acc[e];
+                stored |= 1u << e;
+              }
+              H.add(a, P.s, class_of<C>(acc[e]) < 0 ? 0 : class_of<C>(acc[e]), mag_key(acc[e]) >> 20, 1);
+              ++pos;
+            }
+          }
+          count += tot;
+        }
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] = (a.zero_mode && ((stored >> e) & 1u)) ? 0.0f : acc[e];
+        if (full[u]) {
+          st_stream(a.r + v, make_float4(o[0], o[1], o[2], o[3]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int64_t i = v + e;
+            if (i >= P.lo && i < P.hi) a.r[i] = o[e];
+          }
+        }
+      }
+    }
+    if (lane == 0) a.pcnt[q] = count;
+  }
+  __syncthreads();
+  H.flush(a, 1, kBins1);
+}
+
+// ------------------------------------------------------------------------------------------
+// candidate iteration for the later steps (order not needed)
+
+// Calls f(i, x, c, key) for every candidate of piece q: from the piece's store, or, for pieces
+// marked to be re-read, from the residual (which then holds acc) filtered by class and T_lo.
+template <int C, class F>
+__device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, const Piece& P, F f) {
+  const int lane = threadIdx.x & 31;
+  if (!a.prsrc[q]) {
+    const uint32_t cnt = a.pcnt[q];
+    for (uint32_t j = lane; j < cnt; j += 32) {
+      const float x = a.cval[q * a.cap + j];
+      const int c = class_of<C>(x);
+      f((int64_t)a.cidx[q * a.cap + j], x, c < 0 ? 0 : c, mag_key(x));
+    }
+    return;
+  }
+  uint32_t tl[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) tl[c] = a.tlo[(int64_t)P.s * C + c];
+  for (int64_t base = P.lo & ~(int64_t)3; base < P.hi; base += 128) {
+    const int64_t v = base + lane * 4;
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (v >= P.lo && v + 4 <= P.hi) {
+      const float4 t = *reinterpret_cast<const float4*>(a.r + v);
+      x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (v + e >= P.lo && v + e < P.hi) x[e] = a.r[v + e];
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int64_t i = v + e;
+      if (i < P.lo || i >= P.hi) continue;
+      const int c = class_of<C>(x[e]);
+      if (c < 0) continue;
+      const uint32_t key = mag_key(x[e]);
+      if (key >= tl[c]) f(i, x[e], c, key);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// 4. check + restore
+
+__global__ void check_kernel(Sel a) {
+  __shared__ int64_t sh[33];
+  if (a.ctl[0]) return;
+  const int64_t p = blockIdx.x;
+  const int32_t s = (int32_t)(p / a.C);
+  uint32_t* h = hist_of(a, p, 1);
+  int64_t mine = 0;
+  for (int i = threadIdx.x; i < kBins1; i += blockDim.x) mine += h[i];
+  int64_t total;
+  block_exclusive_scan(mine, sh, &total);
+  const uint32_t t = a.tlo[p];
+  if (t != kNone && t != 0 && total < a.seg_k[s]) {
+    for (int i = threadIdx.x; i < kBins1; i += blockDim.x) h[i] = 0;
+    if (threadIdx.x == 0) {
+      a.redo[p] = 1;
+      a.tlo[p] = 0;
+      a.ctl[1] = 1;
+    }
+  }
+}
+
+template <int C>
+__global__ void __launch_bounds__(kThreads) restore_kernel(Sel a) {
+  __shared__ CtaHist<C, kBins1> H;
+  if (a.ctl[0]) return;
+  const int64_t q0 = (int64_t)blockIdx.x * kWarps;
+  H.init(a, q0);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t q = q0 + (threadIdx.x >> 5);
+  if (q < total_pieces(a)) {
+    const Piece P = piece_of(a, q);
+    bool redo = false;
+#pragma unroll
+    for (int c = 0; c < C; ++c) redo |= a.redo[(int64_t)P.s * C + c] != 0;
+    const uint32_t cnt = a.pcnt[q];
+    if (redo || cnt > a.cap) {
+      if (a.zero_mode) {
+        const uint32_t stored = cnt < a.cap ? cnt : (uint32_t)a.cap;
+        for (uint32_t j = lane; j < stored; j += 32) a.r[a.cidx[q * a.cap + j]] = a.cval[q * a.cap + j];
+      }
+      __syncwarp();
+      if (lane == 0) a.prsrc[q] = 1;
+      __syncwarp();
+      if (redo) {
+        // the redone classes count every member (their T_lo is now 0)
+        for_each_candidate<C>(a, q, P, [&](int64_t, float, int c, uint32_t key) {
+          if (a.redo[(int64_t)P.s * C + c]) H.add(a, P.s, c, key >> 20, 1);
+        });
+      }
+    }
+  }
+  __syncthreads();
+  // only redone problems received counts here
+  H.flush(a, 1, kBins1);
+}
+
+// ------------------------------------------------------------------------------------------
+// 5-7. radix-select levels
+
+__global__ void __launch_bounds__(1024) select_kernel(Sel a, int level) {
+  __shared__ uint32_t h[kBins1];
+  __shared__ int64_t sh[33];
+  if (a.ctl[0]) return;
+  const int64_t p = blockIdx.x;
+  const int32_t s = (int32_t)(p / a.C);
+  if (level > 1 && a.pfx[p] == kNone) return;
+  const int B = level == 3 ? kBins3 : kBins1;
+  const uint32_t* src = hist_of(a, p, level);
+  int64_t mine = 0;
+  for (int i = threadIdx.x; i < B; i += blockDim.x) {
+    h[i] = src[i];
+    mine += h[i];
+  }
+  int64_t total;
+  block_exclusive_scan(mine, sh, &total);
+  int64_t rank;
+  if (level == 1) {
+    const int64_t k = a.seg_k[s] < total ? a.seg_k[s] : total;
+    if (threadIdx.x == 0) a.keff[p] = k;
+    if (k == 0) {
+      if (threadIdx.x == 0) {
+        a.pfx[p] = kNone;
+        a.thr[p] = kNone;
+        a.need_eq[p] = 0;
+      }
+      return;
+    }
+    rank = k;
+  } else {
+    rank = a.krem[p];
+  }
+  uint32_t bin;
+  int64_t above;
+  block_find_bin(h, B, rank, &bin, &above);
+  if (threadIdx.x == 0) {
+    if (level == 1) {
+      a.pfx[p] = bin;
+      a.krem[p] = rank - above;
+    } else if (level == 2) {
+      a.pfx[p] = (a.pfx[p] << 11) | bin;
+      a.krem[p] = rank - above;
+    } else {
+      a.thr[p] = (a.pfx[p] << 9) | bin;
+      a.need_eq[p] = rank - above;
+    }
+  }
+}
+
+template <int C>
+__global__ void __launch_bounds__(kThreads) hist_kernel(Sel a, int level) {
+  constexpr int B = kBins1;  // level 3 uses the first 512 bins
+  __shared__ CtaHist<C, B> H;
+  if (a.ctl[0]) return;
+  const int64_t q0 = (int64_t)blockIdx.x * kWarps;
+  H.init(a, q0);
+  __syncthreads();
+  const int64_t q = q0 + (threadIdx.x >> 5);
+  if (q < total_pieces(a)) {
+    const Piece P = piece_of(a, q);
+    uint32_t pf[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) pf[c] = a.pfx[(int64_t)P.s * C + c];
+    for_each_candidate<C>(a, q, P, [&](int64_t, float, int c, uint32_t key) {
+      if (level == 2) {
+        if ((key >> 20) == pf[c]) H.add(a, P.s, c, (key >> 9) & 2047u, 2);
+      } else {
+        if ((key >> 9) == pf[c]) H.add(a, P.s, c, key & 511u, 3);
+      }
+    });
+  }
+  __syncthreads();
+  H.flush(a, level, level == 2 ? kBins2 : kBins3);
+}
+
+// ------------------------------------------------------------------------------------------
+// 8. count + scan
+
+template <int C>
+__global__ void __launch_bounds__(kThreads) count_kernel(Sel a) {
+  if (a.ctl[0]) return;
+  const int64_t q = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (q >= total_pieces(a)) return;
+  const Piece P = piece_of(a, q);
+  uint32_t th[C], gt[C], eq[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    th[c] = a.thr[(int64_t)P.s * C + c];
+    gt[c] = 0;
+    eq[c] = 0;
+  }
+  for_each_candidate<C>(a, q, P, [&](int64_t, float, int c, uint32_t key) {
+#pragma unroll
+    for (int cc = 0; cc < C; ++cc) {
+      if (cc == c) {
+        gt[cc] += key > th[cc] && th[cc] != kNone;
+        eq[cc] += key == th[cc];
+      }
+    }
+  });
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    const uint32_t G = warp_sum(gt[c]), E = warp_sum(eq[c]);
+    if ((threadIdx.x & 31) == 0) {
+      a.pgt[q * C + c] = G;
+      a.peq[q * C + c] = E;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(Sel a) {
+  __shared__ int64_t sh[33];
+  if (a.ctl[0]) return;
+  const int64_t p = blockIdx.x;
+  const int32_t s = (int32_t)(p / a.C);
+  const int c = (int)(p % a.C);
+  const int64_t first = a.seg_pbase[s], last = a.seg_pbase[s + 1];
+  const int64_t need = a.need_eq[p];
+  int64_t eq_carry = 0, sel_carry = 0;
+  for (int64_t base = first; base < last; base += blockDim.x) {
+    const int64_t q = base + threadIdx.x;
+    int64_t eq = 0, gt = 0;
+    if (q < last) {
+      eq = a.peq[q * a.C + c];
+      gt = a.pgt[q * a.C + c];
+    }
+    int64_t teq, tsel;
+    const int64_t eq_before = eq_carry + block_exclusive_scan(eq, sh, &teq);
+    int64_t take = need - eq_before;
+    take = take < 0 ? 0 : (take > eq ? eq : take);
+    const int64_t sel = gt + take;
+    const int64_t sel_before = sel_carry + block_exclusive_scan(sel, sh, &tsel);
+    if (q < last) {
+      a.poff[q * a.C + c] = sel_before;
+      a.ptake[q * a.C + c] = (uint32_t)take;
+    }
+    eq_carry += teq;
+    sel_carry += tsel;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// 9. emit, in index order
+
+template <int C>
+__global__ void __launch_bounds__(kThreads) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
+                                                        int64_t limit) {
+  if (a.ctl[0]) return;
+  const int64_t q = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (q >= total_pieces(a)) return;
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = lanemask_lt();
+  const Piece P = piece_of(a, q);
+  uint32_t th[C], take[C], eq_run[C], sel_run[C];
+  int64_t base_out[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    const int64_t p = (int64_t)P.s * C + c;
+    th[c] = a.thr[p];
+    take[c] = a.ptake[q * C + c];
+    eq_run[c] = 0;
+    sel_run[c] = 0;
+    // top-k: the segment's block of the output; binarise: the class list of the problem
+    base_out[c] = (C == 1 ? a.seg_kbase[P.s] : 2 * a.seg_kbase[P.s] + c * a.seg_k[P.s]) + a.poff[q * C + c];
+  }
+  auto is_sel = [&](int c, uint32_t key, bool eq_taken) {
+    return c >= 0 && th[c] != kNone && (key > th[c] || eq_taken);
+  };
+  if (!a.prsrc[q]) {
+    const uint32_t cnt = a.pcnt[q];
+    const int32_t* ci = a.cidx + q * a.cap;
+    const float* cv = a.cval + q * a.cap;
+    for (uint32_t j0 = 0; j0 < cnt; j0 += 32) {
+      const uint32_t j = j0 + lane;
+      const bool valid = j < cnt;
+      const int32_t i = valid ? ci[j] : 0;
+      const float x = valid ? cv[j] : 0.0f;
+      const int c = valid ? class_of<C>(x) : -1;
+      const uint32_t key = mag_key(x);
+      bool sel = false;
+      uint32_t pos = 0;
+#pragma unroll
+      for (int cc = 0; cc < C; ++cc) {
+        const bool eq = c == cc && key == th[cc];
+        const uint32_t be = __ballot_sync(kFull, eq);
+        const bool taken = eq && (eq_run[cc] + __popc(be & lt)) < take[cc];
+        const bool s_ = c == cc && is_sel(cc, key, taken);
+        const uint32_t bs = __ballot_sync(kFull, s_);
+        if (s_) { sel = true; pos = sel_run[cc] + __popc(bs & lt); }
+        eq_run[cc] += __popc(be);
+        sel_run[cc] += __popc(bs);
+      }
+      if (sel) {
+        const int64_t o = base_out[c] + pos;
+        if (o >= limit) raise(a.d_status, GSPARSE_DERR_CAPACITY);
+        else if (C == 1) { out_idx[o] = i; out_val[o] = x; }
+        else { a.lidx[o] = i; a.lval[o] = x; }
+      } else if (valid && a.zero_mode) {
+        a.r[i] = x;  // a candidate that is not sent keeps its acc in the residual
+      }
+    }
+    return;
+  }
+  // re-read piece: the residual holds acc; walk it in index order
+  for (int64_t vb = P.lo & ~(int64_t)3; vb < P.hi; vb += 128) {
+    const int64_t v = vb + lane * 4;
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (v >= P.lo && v + 4 <= P.hi) {
+      const float4 t = *reinterpret_cast<const float4*>(a.r + v);
+      x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (v + e >= P.lo && v + e < P.hi) x[e] = a.r[v + e];
+    }
+    int cls[4];
+    uint32_t key[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool in = v + e >= P.lo && v + e < P.hi;
+      cls[e] = in ? class_of<C>(x[e]) : -1;
+      key[e] = mag_key(x[e]);
+    }
+    uint32_t selm = 0;
+#pragma unroll
+    for (int cc = 0; cc < C; ++cc) {
+      uint32_t eqm = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) eqm |= (uint32_t)(cls[e] == cc && key[e] == th[cc]) << e;
+      uint32_t teq;
+      const uint32_t pre_eq = warp_prefix_small(__popc(eqm), &teq);
+      uint32_t sm = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool eq = (eqm >> e) & 1u;
+        const bool taken = eq && (eq_run[cc] + pre_eq + __popc(eqm & ((1u << e) - 1u))) < take[cc];
+        sm |= (uint32_t)(cls[e] == cc && is_sel(cc, key[e], taken)) << e;
+      }
+      uint32_t tsel;
+      const uint32_t pre_sel = warp_prefix_small(__popc(sm), &tsel);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if ((sm >> e) & 1u) {
+          const int64_t o = base_out[cc] + sel_run[cc] + pre_sel + __popc(sm & ((1u << e) - 1u));
+          if (o >= limit) raise(a.d_status, GSPARSE_DERR_CAPACITY);
+          else if (C == 1) { out_idx[o] = (int32_t)(v + e); out_val[o] = x[e]; }
+          else { a.lidx[o] = (int32_t)(v + e); a.lval[o] = x[e]; }
+        }
+      }
+      eq_run[cc] += teq;
+      sel_run[cc] += tsel;
+      selm |= sm;
+    }
+    if (a.zero_mode && selm) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((selm >> e) & 1u) a.r[v + e] = 0.0f;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// binarise: means, choice, output
+
+__global__ void __launch_bounds__(1024) bjobs_kernel(Sel a, SumJob* jobs) {
+  __shared__ int64_t sh[33];
+  if (a.ctl[0]) return;
+  const int64_t P = (int64_t)a.T * 2;
+  int64_t carry = 0;
+  for (int64_t base = 0; base < P; base += blockDim.x) {
+    const int64_t p = base + threadIdx.x;
+    int64_t leaves = 0;
+    if (p < P) leaves = cdiv(a.keff[p], kSumBlock);
+    int64_t tot;
+    const int64_t ex = block_exclusive_scan(leaves, sh, &tot);
+    if (p < P) {
+      const int32_t s = (int32_t)(p >> 1);
+      const int c = (int)(p & 1);
+      SumJob J;
+      J.vals = a.lval + 2 * a.seg_kbase[s] + c * a.seg_k[s];
+      J.len = a.keff[p];
+      J.mode = c == 0 ? kSumAll : kSumNegated;
+      J.pad = 0;
+      J.leaf_base = carry + ex;
+      J.count = 0;
+      J.sum = 0.0;
+      J.mean = 0.0f;
+      J.done_blocks = 0;
+      jobs[p] = J;
+    }
+    carry += tot;
+  }
+}
+
+__global__ void __launch_bounds__(1024) bchoose_kernel(Sel a, const SumJob* jobs, float* d_mean, int64_t* out_offsets) {
+  __shared__ int64_t sh[33];
+  if (a.ctl[0]) return;
+  int64_t carry = 0;
+  for (int64_t base = 0; base < a.T; base += blockDim.x) {
+    const int64_t s = base + threadIdx.x;
+    int64_t cnt = 0;
+    if (s < a.T) {
+      const int64_t kp = a.keff[2 * s], kn = a.keff[2 * s + 1];
+      const float mp = jobs[2 * s].mean, mn = jobs[2 * s + 1].mean;
+      const bool pos = kp > 0 && mp >= mn;
+      const bool neg = !pos && kn > 0;
+      a.bsel[s] = pos ? 0 : (neg ? 1 : -1);
+      d_mean[s] = pos ? mp : (neg ? -mn : 0.0f);
+      cnt = pos ? kp : (neg ? kn : 0);
+    }
+    int64_t tot;
+    const int64_t ex = block_exclusive_scan(cnt, sh, &tot);
+    if (s < a.T) out_offsets[s] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) out_offsets[a.T] = carry;
+}
+
+__global__ void bemit_kernel(Sel a, const float* d_mean, const int64_t* out_offsets,
+                             int64_t bound, int32_t* out_idx, float* out_val) {
+  if (a.ctl[0]) return;
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= bound || j >= out_offsets[a.T]) return;
+  const int32_t s = (int32_t)(upper_bound_i64(out_offsets, a.T + 1, j) - 1);
+  const int c = a.bsel[s];
+  const int64_t src = 2 * a.seg_kbase[s] + c * a.seg_k[s] + (j - out_offsets[s]);
+  const int32_t i = a.lidx[src];
+  const float m = d_mean[s];
+  out_idx[j] = i;
+  if (out_val) out_val[j] = m;
+  a.r[i] = __fsub_rn(a.lval[src], m);
+}
+
+// ------------------------------------------------------------------------------------------
+// accumulate only (keep 0): residual <- fl(g + residual)
+
+__global__ void accumulate_kernel(const float* g, float* r, int64_t n, const int32_t* ctl) {
+  if (ctl[0]) return;
+  const int64_t nv = n >> 2;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nv; v += stride) {
+    const float4 a = ld_stream(g + 4 * v), b = ld_stream(r + 4 * v);
+    st_stream(r + 4 * v, make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z),
+                                     __fadd_rn(a.w, b.w)));
+  }
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < (n & 3)) r[4 * nv + t] = __fadd_rn(g[4 * nv + t], r[4 * nv + t]);
+}
+
+// ------------------------------------------------------------------------------------------
+// host side
+
+struct Layout {
+  int64_t n, Lp, Q, cap, cap_rec;
+  int32_t T, C;
+  size_t fixed_bytes, total_bytes;
+  Sel a;
+  // binarise extras
+  SumJob* jobs;
+  double* leaves;
+  double* partials;
+  int64_t leaf_bound, per_job_leaf_bound, kbound;
+  char* zero_begin;
+  size_t zero_bytes;
+};
+
+int64_t pick_lp(int64_t n) {
+  int64_t lp = cdiv(n > 0 ? n : 1, kTargetPieces);
+  return round_up(lp < kGranule ? kGranule : lp, kGranule);
+}
+
+// k bound over all segmentations: sum_s ceil(n_s f) <= ceil(n f) + T
+int64_t k_bound(int64_t n, int32_t T, int64_t num, int64_t den) {
+  const int64_t kb = kept_count(n, num, den) + T;
+  return kb < n ? kb : n;
+}
+
+int64_t rec_cap(int64_t Lp, int32_t C, int64_t num, int64_t den) {
+  const double q = den > 0 ? (double)num / (double)den : 1.0;
+  const double f = q + 4.0 * sqrt(q / kSample) + 8.0 / kSample;
+  double cap = ceil((double)Lp * f * C * 1.25) + 64.0;
+  if (cap > (double)Lp) cap = (double)Lp;
+  return round_up((int64_t)cap, 32);
+}
+
+// Carves the workspace (ws may be null to measure). cap_req < 0: recommended capacity.
+Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws, size_t ws_bytes,
+             bool measure_rec) {
+  Layout L{};
+  L.n = n;
+  L.T = T;
+  L.C = C;
+  L.Lp = pick_lp(n);
+  L.Q = cdiv(n, L.Lp) + T;
+  const int64_t P = (int64_t)T * C;
+  Carver cv(ws);
+  Sel& a = L.a;
+  a.seg_lo = cv.take<int64_t>(T);
+  a.seg_n = cv.take<int64_t>(T);
+  a.seg_k = cv.take<int64_t>(T);
+  a.seg_kbase = cv.take<int64_t>(T + 1);
+  a.seg_pbase = cv.take<int64_t>(T + 1);
+  a.tlo = cv.take<uint32_t>(P);
+  a.pfx = cv.take<uint32_t>(P);
+  a.thr = cv.take<uint32_t>(P);
+  a.keff = cv.take<int64_t>(P);
+  a.krem = cv.take<int64_t>(P);
+  a.need_eq = cv.take<int64_t>(P);
+  a.pgt = cv.take<uint32_t>(L.Q * C);
+  a.peq = cv.take<uint32_t>(L.Q * C);
+  a.ptake = cv.take<uint32_t>(L.Q * C);
+  a.poff = cv.take<int64_t>(L.Q * C);
+  // zero-initialised block
+  const size_t zoff = (size_t)round_up((int64_t)cv.off, 256);
+  a.ctl = cv.take<int32_t>(64);
+  a.redo = cv.take<uint32_t>(P);
+  a.pcnt = cv.take<uint32_t>(L.Q);
+  a.prsrc = cv.take<uint32_t>(L.Q);
+  a.hist = cv.take<uint32_t>(P * kHist);
+  const size_t zend = cv.off;
+  L.zero_begin = ws ? (char*)ws + zoff : nullptr;
+  L.zero_bytes = zend - zoff;
+  if (C == 2) {
+    L.kbound = k_bound(n, T, num, den);
+    a.lidx = cv.take<int32_t>(2 * L.kbound);
+    a.lval = cv.take<float>(2 * L.kbound);
+    a.bsel = cv.take<int32_t>(T);
+    L.jobs = cv.take<SumJob>(P);
+    L.leaf_bound = cdiv(2 * L.kbound, kSumBlock) + P;
+    L.per_job_leaf_bound = cdiv(kept_count(n, num, den), kSumBlock);
+    L.leaves = cv.take<double>(L.leaf_bound);
+    L.partials = cv.take<double>(P * osum_partial_stride(L.per_job_leaf_bound));
+  }
+  L.fixed_bytes = cv.off + 512;
+  L.cap_rec = rec_cap(L.Lp, C, num, den);
+  int64_t cap;
+  if (measure_rec) {
+    cap = L.cap_rec;
+  } else {
+    const int64_t room = ws_bytes > L.fixed_bytes ? (int64_t)(ws_bytes - L.fixed_bytes) : 0;
+    cap = room / (L.Q * 8 > 0 ? L.Q * 8 : 1);
+    if (cap > L.Lp) cap = L.Lp;
+  }
+  L.cap = cap;
+  a.cidx = cv.take<int32_t>(L.Q * cap);
+  a.cval = cv.take<float>(L.Q * cap);
+  L.total_bytes = cv.off;
+  a.cap = cap;
+  a.Lp = L.Lp;
+  a.Q = L.Q;
+  a.n = n;
+  a.T = T;
+  a.C = C;
+  return L;
+}
+
+bool bad_keep(int64_t num, int64_t den) { return den <= 0 || num < 0 || num > den; }
+
+template <int C>
+int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t T, int64_t num,
+               int64_t den, int32_t* out_idx, float* out_val, float* d_mean, int64_t* out_offsets,
+               int64_t out_capacity, uint32_t flags, void* ws, size_t ws_bytes, int32_t* d_status,
+               cudaStream_t st) {
+  if (n < 0 || T < 1 || (seg == nullptr && T != 1) || bad_keep(num, den) || !out_offsets ||
+      out_capacity < 0)
+    return GSPARSE_ERR_INVALID_ARG;
+  if (n > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
+  if (n > 0 && (!g || !r || !aligned16(g) || !aligned16(r))) return GSPARSE_ERR_INVALID_ARG;
+  if (out_capacity > 0 && !out_idx) return GSPARSE_ERR_INVALID_ARG;
+  if (C == 1 && out_capacity > 0 && !out_val) return GSPARSE_ERR_INVALID_ARG;
+  if (C == 2 && !d_mean) return GSPARSE_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return GSPARSE_ERR_WORKSPACE;
+  Layout L = carve(n, T, C, num, den, ws, ws_bytes, false);
+  if (ws_bytes < L.total_bytes || ws_bytes < L.fixed_bytes) return GSPARSE_ERR_WORKSPACE;
+  Sel a = L.a;
+  a.g = g;
+  a.r = r;
+  a.zero_mode = C == 1;
+  a.d_status = d_status;
+  if (cudaMemsetAsync(L.zero_begin, 0, L.zero_bytes, st) != cudaSuccess) return GSPARSE_ERR_CUDA;
+  plan_kernel<<<1, 1024, 0, st>>>(a, seg, num, den, out_capacity, C == 1 ? out_offsets : nullptr);
+  if (num == 0 && C == 1) {  // communication delay step: accumulate only
+    if (n > 0) {
+      const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
+      accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, a.ctl);
+    }
+    return launch_status();
+  }
+  const unsigned piece_ctas = (unsigned)cdiv(L.Q, kWarps);
+  const size_t sample_smem = (size_t)C * kSample * sizeof(uint32_t);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GSPARSE_ERR_CUDA;
+  static bool attr_set[2][64] = {};
+  if (dev < 64 && !attr_set[C - 1][dev]) {
+    if (cudaFuncSetAttribute(sample_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sample_smem) != cudaSuccess)
+      return GSPARSE_ERR_CUDA;
+    attr_set[C - 1][dev] = true;
+  }
+  sample_kernel<C><<<T, 1024, sample_smem, st>>>(a, (flags & GSPARSE_SELECT_EXHAUSTIVE) ? 1 : 0);
+  if (piece_ctas) pass1_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
+  check_kernel<<<(unsigned)(T * C), 256, 0, st>>>(a);
+  if (piece_ctas) restore_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
+  select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 1);
+  if (piece_ctas) hist_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a, 2);
+  select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 2);
+  if (piece_ctas) hist_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a, 3);
+  select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 3);
+  if (piece_ctas) count_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
+  scan_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a);
+  if (piece_ctas)
+    emit_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a, out_idx, out_val,
+                                                    C == 1 ? out_capacity : 2 * L.kbound);
+  if (C == 2) {
+    bjobs_kernel<<<1, 1024, 0, st>>>(a, L.jobs);
+    osum_launch(L.jobs, T * 2, L.leaves, L.leaf_bound, L.per_job_leaf_bound, L.partials, a.ctl, st);
+    bchoose_kernel<<<1, 1024, 0, st>>>(a, L.jobs, d_mean, out_offsets);
+    if (L.kbound > 0)
+      bemit_kernel<<<(unsigned)cdiv(L.kbound, 256), 256, 0, st>>>(a, d_mean, out_offsets, L.kbound,
+                                                                  out_idx, out_val);
+  }
+  return launch_status();
+}
+
+}  // namespace
+}  // namespace gs
+
+using namespace gs;
+
+extern "C" {
+
+size_t gsparse_residual_topk_workspace_size(int64_t n, int32_t T, int64_t num, int64_t den) {
+  if (n < 0 || T < 1 || bad_keep(num, den)) return 0;
+  return carve(n, T, 1, num, den, nullptr, 0, true).total_bytes + 256;
+}
+
+size_t gsparse_residual_topk_workspace_min(int64_t n, int32_t T) {
+  if (n < 0 || T < 1) return 0;
+  return carve(n, T, 1, 1, 1, nullptr, 0, false).fixed_bytes;
+}
+
+int gsparse_residual_topk(const float* g, float* residual, int64_t n, const int64_t* seg_offsets,
+                          int32_t num_segments, int64_t keep_num, int64_t keep_den, int32_t* out_idx,
+                          float* out_val, int64_t* out_offsets, int64_t out_capacity, uint32_t flags,
+                          void* workspace, size_t workspace_bytes, int32_t* d_status,
+                          gsparse_stream stream) {
+  return run_select<1>(g, residual, n, seg_offsets, num_segments, keep_num, keep_den, out_idx,
+                       out_val, nullptr, out_offsets, out_capacity, flags, workspace,
+                       workspace_bytes, d_status, (cudaStream_t)stream);
+}
+
+size_t gsparse_binarize_workspace_size(int64_t n, int32_t T, int64_t num, int64_t den) {
+  if (n < 0 || T < 1 || bad_keep(num, den)) return 0;
+  return carve(n, T, 2, num, den, nullptr, 0, true).total_bytes + 256;
+}
+
+size_t gsparse_binarize_workspace_min(int64_t n, int32_t T, int64_t num, int64_t den) {
+  if (n < 0 || T < 1 || bad_keep(num, den)) return 0;
+  return carve(n, T, 2, num, den, nullptr, 0, false).fixed_bytes;
+}
+
+int gsparse_binarize(const float* g, float* residual, int64_t n, const int64_t* seg_offsets,
+                     int32_t num_segments, int64_t keep_num, int64_t keep_den, int32_t* out_idx,
+                     float* out_val, float* d_mean, int64_t* out_offsets, int64_t out_capacity,
+                     uint32_t flags, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                     gsparse_stream stream) {
+  return run_select<2>(g, residual, n, seg_offsets, num_segments, keep_num, keep_den, out_idx,
+                       out_val, d_mean, out_offsets, out_capacity, flags, workspace,
+                       workspace_bytes, d_status, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,352 @@
+"""CUDA path vs the CPU oracle, element by element, on seeded inputs (bit-exact on indices,
+counts, residuals, bitstreams; fp32 means and sums are compared bitwise too, which is stricter
+than the 1e-6 relative bound)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.gpu_util import bits, dev, gpu_binarize, gpu_topk, host
+
+import compressed_sgd_b200 as gs
+
+pytestmark = pytest.mark.gpu
+
+
+def assert_topk_equal(got, want):
+    gi, gv, go, gr, st = got
+    wi, wv, wo, wr = want
+    assert st == 0
+    assert np.array_equal(go, wo), (go, wo)
+    assert np.array_equal(gi, wi)
+    assert np.array_equal(bits(gv), bits(wv))
+    assert np.array_equal(bits(gr), bits(wr))
+
+
+# ------------------------------------------------------------------------------------ top-k
+
+SIZES = [0, 1, 2, 5, 31, 32, 33, 127, 1000, 4097, 65537, 300001, (1 << 20) + 3]
+KEEPS = [(1, 100), (1, 10), (1, 2), (1, 1), (0, 1), (1, 1000), (7, 9)]
+
+
+@pytest.mark.parametrize("n", SIZES)
+def test_topk_global_sizes(n):
+    g = synth.gaussian(n, n)
+    r = synth.gaussian(n, n + 1, sigma=3e-4)
+    for keep in KEEPS:
+        assert_topk_equal(gpu_topk(g, r, keep), oracle.residual_topk(g, r, keep))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_topk_ties_and_zeros(seed):
+    n = 20000 + 977 * seed
+    g = synth.tied_values(n, seed, levels=3, zero_frac=0.3)
+    r = synth.tied_values(n, seed + 50, levels=2, zero_frac=0.6)
+    for keep in [(1, 100), (1, 4), (1, 2), (9, 10), (1, 1)]:
+        assert_topk_equal(gpu_topk(g, r, keep), oracle.residual_topk(g, r, keep))
+
+
+def test_topk_all_zero_and_constant():
+    n = 50001
+    z = np.zeros(n, np.float32)
+    for keep in [(1, 100), (1, 2)]:
+        assert_topk_equal(gpu_topk(z, z, keep), oracle.residual_topk(z, z, keep))
+    c = np.full(n, -0.5, np.float32)
+    assert_topk_equal(gpu_topk(c, z, (1, 7)), oracle.residual_topk(c, z, (1, 7)))
+
+
+@pytest.mark.parametrize("layout", [
+    [37, 1, 500, 64, 0, 1023],
+    [0, 0, 5],
+    [100000, 3, 250000, 1],
+    [16384, 16385, 16383, 70000],
+    [1] * 200,
+])
+def test_topk_per_segment(layout):
+    seg = np.concatenate([[0], np.cumsum(layout)]).astype(np.int64)
+    n = int(seg[-1])
+    g = synth.gaussian(n, 7)
+    r = synth.tied_values(n, 8, levels=3) * np.float32(1e-3)
+    for keep in [(1, 100), (1, 10), (1, 1), (0, 1)]:
+        assert_topk_equal(gpu_topk(g, r, keep, seg=seg), oracle.residual_topk(g, r, keep, seg=seg))
+
+
+@pytest.mark.parametrize("route", ["exhaustive", "min_workspace", "tiny_workspace"])
+def test_topk_fallback_routes_identical(route):
+    n = 400003
+    g = synth.flat_mixture(n, seed=3)
+    r = synth.gaussian(n, 4, sigma=1e-4)
+    seg = np.array([0, 1000, 200000, n], np.int64)
+    for keep, s in [((1, 100), None), ((1, 10), seg), ((1, 2), None)]:
+        T = 1 if s is None else len(s) - 1
+        kw = {}
+        if route == "exhaustive":
+            kw["flags"] = gs.GSPARSE_SELECT_EXHAUSTIVE
+        elif route == "min_workspace":
+            kw["workspace_bytes"] = int(gs.lib().gsparse_residual_topk_workspace_min(n, T))
+        else:
+            kw["workspace_bytes"] = int(gs.lib().gsparse_residual_topk_workspace_min(n, T)) + 64 * 1024
+        assert_topk_equal(gpu_topk(g, r, keep, seg=s, **kw), oracle.residual_topk(g, r, keep, seg=s))
+
+
+def test_topk_sample_threshold_too_high_is_redone():
+    # a segment whose sampled runs miss a dense block of large values: the sampled threshold
+    # leaves fewer than k candidates and the segment is redone exhaustively
+    n = 1 << 20
+    g = synth.gaussian(n, 11, sigma=1e-6)
+    g[777000:777000 + 20000] = synth.gaussian(20000, 12, sigma=1.0)
+    r = np.zeros(n, np.float32)
+    assert_topk_equal(gpu_topk(g, r, (1, 60)), oracle.residual_topk(g, r, (1, 60)))
+
+
+def test_topk_multi_step_residual_carried():
+    lay = synth.mlp_layout()
+    seg = synth.offsets(lay)
+    n = int(seg[-1])
+    r_o = np.zeros(n, np.float32)
+    rd = dev(r_o)
+    for step in range(4):
+        g = synth.mlp_gradient(0, step)
+        wi, wv, wo, r_o = oracle.residual_topk(g, r_o, (1, 100), seg=seg)
+        idx, val, off = gs.residual_topk(dev(g), rd, (1, 100), seg_offsets=dev(seg))
+        K = int(host(off)[-1])
+        assert np.array_equal(host(off), wo)
+        assert np.array_equal(host(idx)[:K], wi)
+        assert np.array_equal(bits(host(val)[:K]), bits(wv))
+        assert np.array_equal(bits(host(rd)), bits(r_o))
+
+
+def test_topk_bad_segments_and_capacity_flagged():
+    n = 1000
+    g = synth.gaussian(n, 1)
+    r = np.zeros(n, np.float32)
+    _, _, _, rr, st = gpu_topk(g, r, (1, 10), seg=np.array([0, 600, 500, n], np.int64))
+    assert st & gs.DERR_SEGMENTS and np.array_equal(rr, r)     # nothing touched
+    _, _, _, rr, st = gpu_topk(g, r, (1, 10), seg=np.array([0, 600, n - 1], np.int64))
+    assert st & gs.DERR_SEGMENTS
+    _, _, _, rr, st = gpu_topk(g, r, (1, 10), capacity=50)
+    assert st & gs.DERR_CAPACITY and np.array_equal(rr, r)
+
+
+def test_topk_host_argument_errors():
+    x = torch.zeros(16, device="cuda")
+    with pytest.raises(gs.GsparseError):
+        gs.residual_topk(x, x, (2, 1))                      # keep fraction above 1
+    with pytest.raises(gs.GsparseError):
+        gs.residual_topk(x[1:], x[1:], (1, 2))              # misaligned
+    with pytest.raises(gs.GsparseError):
+        ws = torch.empty(64, dtype=torch.uint8, device="cuda")
+        gs.residual_topk(x, x.clone(), (1, 2), workspace=ws)
+
+
+# ------------------------------------------------------------------------------------ quantise
+
+@pytest.mark.parametrize("K", [0, 1, 31, 33, 255, 256, 257, 5000, 70001, 600000])
+def test_quantize_parity(K):
+    n = max(4 * K, 1)
+    gen = np.random.default_rng(K)
+    idx = np.sort(gen.choice(n, K, replace=False)).astype(np.int32)
+    val = synth.gaussian(K, K, sigma=1e-2)
+    if K > 10:
+        val[::11] = 0.0
+        val[5::13] = -0.0
+    res = synth.gaussian(n, 3, sigma=1e-4)
+    wb, wm, wval, wres = oracle.quantize(idx, val, residual=res, write_dequantized=True)
+    vd, rd = dev(val), dev(res)
+    end = torch.tensor([K], dtype=torch.int64, device="cuda")
+    st = gs.status_tensor()
+    sb, means = gs.quantize(dev(idx), vd, end, residual=rd, write_dequantized=True, d_status=st, capacity=K)
+    assert int(host(st)[0]) == 0
+    assert np.array_equal(bits(host(means)), bits(wm))
+    assert np.array_equal(host(sb)[:(K + 31) // 32].view(np.uint32), wb)
+    assert np.array_equal(bits(host(vd)), bits(wval))
+    assert np.array_equal(bits(host(rd)), bits(wres))
+
+
+def test_quantize_sublist_with_begin_end():
+    K = 3000
+    idx = np.arange(0, 3 * K, 3, dtype=np.int32)
+    val = synth.gaussian(K, 5, sigma=1e-2)
+    b, e = 700, 2333
+    wb, wm, _, _ = oracle.quantize(idx[b:e], val[b:e])
+    sb, means = gs.quantize(dev(idx), dev(val), torch.tensor([e], device="cuda"),
+                            d_begin=torch.tensor([b], device="cuda"), capacity=K)
+    assert np.array_equal(bits(host(means)), bits(wm))
+    assert np.array_equal(host(sb)[:(e - b + 31) // 32].view(np.uint32), wb)
+
+
+# ------------------------------------------------------------------------------------ binarise
+
+def assert_binarize_equal(got, want):
+    gi, gv, gm, go, gr, st = got
+    wi, wv, wm, wo, wr = want
+    assert st == 0
+    assert np.array_equal(go, wo)
+    assert np.array_equal(gi, wi)
+    assert np.array_equal(bits(gm), bits(wm))
+    assert np.array_equal(bits(gv), bits(wv))
+    assert np.array_equal(bits(gr), bits(wr))
+
+
+@pytest.mark.parametrize("n", [1, 2, 33, 1000, 65537, 300001, (1 << 20) + 5])
+def test_binarize_global(n):
+    g = synth.gaussian(n, n, sigma=1e-2)
+    r = synth.gaussian(n, n + 2, sigma=1e-3)
+    for keep in [(1, 1000), (1, 100), (1, 3), (1, 1)]:
+        assert_binarize_equal(gpu_binarize(g, r, keep), oracle.binarize(g, r, keep))
+
+
+def test_binarize_skewed_ties_segments_and_routes():
+    n = 200000
+    g = synth.tied_values(n, 4, levels=3, zero_frac=0.2)
+    g[: n // 2] = np.abs(g[: n // 2])
+    r = np.zeros(n, np.float32)
+    seg = np.array([0, 10, 10, 150000, n], np.int64)
+    for keep in [(1, 1000), (1, 50), (1, 2)]:
+        want = oracle.binarize(g, r, keep, seg=seg)
+        assert_binarize_equal(gpu_binarize(g, r, keep, seg=seg), want)
+        assert_binarize_equal(gpu_binarize(g, r, keep, seg=seg, flags=gs.GSPARSE_SELECT_EXHAUSTIVE), want)
+        mn = int(gs.lib().gsparse_binarize_workspace_min(n, 4, *keep))
+        assert_binarize_equal(gpu_binarize(g, r, keep, seg=seg, workspace_bytes=mn), want)
+
+
+def test_binarize_one_sign_only():
+    n = 5000
+    g = np.abs(synth.gaussian(n, 1))
+    r = np.zeros(n, np.float32)
+    assert_binarize_equal(gpu_binarize(g, r, (1, 100)), oracle.binarize(g, r, (1, 100)))
+    assert_binarize_equal(gpu_binarize(-g, r, (1, 100)), oracle.binarize(-g, r, (1, 100)))
+    z = np.zeros(n, np.float32)
+    assert_binarize_equal(gpu_binarize(z, z, (1, 100)), oracle.binarize(z, z, (1, 100)))
+
+
+# ------------------------------------------------------------------------------------ Golomb
+
+@pytest.mark.parametrize("b", [0, 1, 3, 6, 9, 15, 30])
+@pytest.mark.parametrize("K", [0, 1, 31, 32, 33, 1000, 65537])
+def test_golomb_parity(b, K):
+    n = 1 << 22 if b else 1 << 14
+    gen = np.random.default_rng(b * 1000 + K)
+    idx = np.sort(gen.choice(n, min(K, n), replace=False)).astype(np.int32)
+    K = idx.size
+    base = 0
+    wwords, wbits, wtable = oracle.golomb_encode(idx, b, base, chunk=64)
+    end = torch.tensor([K], dtype=torch.int64, device="cuda")
+    st = gs.status_tensor()
+    words, nbits, table = gs.golomb_encode(dev(idx), end, b, n, base=base, chunk=64, d_status=st, capacity=K)
+    nb = int(host(nbits)[0])
+    assert int(host(st)[0]) == 0 and nb == wbits
+    assert np.array_equal(host(words)[:(nb + 31) // 32].view(np.uint32), wwords)
+    if K:
+        assert np.array_equal(host(table)[: wtable.shape[0]], wtable)
+    out = gs.golomb_decode(words, nbits, end, K, b, base=base, table=table, chunk=64, n_limit=n, d_status=st)
+    assert int(host(st)[0]) == 0
+    assert np.array_equal(host(out)[:K], idx)
+    out2 = gs.golomb_decode(words, nbits, end, K, b, base=base, table=None, n_limit=n, d_status=st)
+    assert np.array_equal(host(out2)[:K], idx)
+
+
+def test_golomb_huge_gaps_and_base():
+    idx = np.array([5, 6, 100000, 100001, 2_000_000_000], np.int32)
+    for b in [0, 2, 20]:
+        ww, wb, wt = oracle.golomb_encode(idx, b, base=5, chunk=2)
+        end = torch.tensor([idx.size], device="cuda")
+        words, nbits, table = gs.golomb_encode(dev(idx), end, b, 2**31 - 1, base=5, chunk=2)
+        nb = int(host(nbits)[0])
+        assert nb == wb and np.array_equal(host(words)[:(nb + 31) // 32].view(np.uint32), ww)
+        out = gs.golomb_decode(words, nbits, end, idx.size, b, base=5, table=table, chunk=2)
+        assert np.array_equal(host(out)[: idx.size], idx)
+
+
+def test_golomb_corrupt_streams_flagged():
+    idx = np.sort(np.random.default_rng(0).choice(100000, 3000, replace=False)).astype(np.int32)
+    end = torch.tensor([idx.size], device="cuda")
+    words, nbits, table = gs.golomb_encode(dev(idx), end, 6, 100000, chunk=32)
+    # truncated stream
+    st = gs.status_tensor()
+    short = nbits - 5
+    gs.golomb_decode(words, short, end, idx.size, 6, table=table, chunk=32, d_status=st)
+    assert int(host(st)[0]) & gs.DERR_CORRUPT_STREAM
+    # flipped bits (host-made corruption), both decoders: flagged or, if still a valid code,
+    # the decoded indices differ; never a fault
+    for flip in [3, 1000, 7777]:
+        w = words.clone()
+        w.view(torch.int32)[flip // 32] ^= (1 << (flip % 32))
+        for tb in [table, None]:
+            st = gs.status_tensor()
+            out = gs.golomb_decode(w, nbits, end, idx.size, 6, table=tb, chunk=32, n_limit=100000, d_status=st)
+            s = int(host(st)[0])
+            assert s != 0 or not np.array_equal(host(out)[: idx.size], idx)
+    # not ascending
+    bad = idx.copy()
+    bad[10] = bad[9]
+    st = gs.status_tensor()
+    gs.golomb_encode(dev(bad), end, 6, 100000, d_status=st)
+    assert int(host(st)[0]) & gs.DERR_INDEX_RANGE
+
+
+# ------------------------------------------------------------------------------------ scatter
+
+@pytest.mark.parametrize("W", [1, 2, 4, 8])
+@pytest.mark.parametrize("n", [1, 8191, 8192, 100003])
+def test_scatter_parity(W, n):
+    gen = np.random.default_rng(W * n)
+    host_lists, lists, keep = [], [], []
+    for w in range(W):
+        k = int(min(n, gen.integers(0, max(n // 10, 2))))
+        idx = np.sort(gen.choice(n, k, replace=False)).astype(np.int32)
+        val = synth.gaussian(k, w, sigma=1e-2)
+        cnt = torch.tensor([k], dtype=torch.int64, device="cuda")
+        if w == 1:   # a binarised worker: one value for every entry
+            u = torch.tensor([0.125], device="cuda")
+            host_lists.append((idx, None, np.float32(0.125)))
+            t = (dev(idx), cnt, u)
+            lists.append(gs.make_list(t[0], cnt, uniform_val=u, capacity=k))
+        else:
+            host_lists.append((idx, val))
+            t = (dev(idx), cnt, dev(val))
+            lists.append(gs.make_list(t[0], cnt, val=t[2], capacity=k))
+        keep.append(t)
+    wd, wi, wv = oracle.scatter_accumulate(host_lists, n)
+    st = gs.status_tensor()
+    dense, mi, mv, mc = gs.scatter_accumulate(lists, n, merged=True, d_status=st)
+    assert int(host(st)[0]) == 0
+    assert np.array_equal(bits(host(dense)[:n]), bits(wd))
+    U = int(host(mc)[0])
+    assert U == wi.size
+    assert np.array_equal(host(mi)[:U], wi)
+    assert np.array_equal(bits(host(mv)[:U]), bits(wv))
+
+
+def test_scatter_bad_indices_flagged():
+    n = 1000
+    idx = torch.tensor([5, 3, 7], dtype=torch.int32, device="cuda")
+    val = torch.ones(3, device="cuda")
+    cnt = torch.tensor([3], device="cuda")
+    st = gs.status_tensor()
+    gs.scatter_accumulate([gs.make_list(idx, cnt, val=val)], n, d_status=st)
+    assert int(host(st)[0]) & gs.DERR_INDEX_RANGE
+    idx = torch.tensor([5, 3000], dtype=torch.int32, device="cuda")
+    st = gs.status_tensor()
+    gs.scatter_accumulate([gs.make_list(idx, torch.tensor([2], device="cuda"), val=val[:2])], n, d_status=st)
+    assert int(host(st)[0]) & gs.DERR_INDEX_RANGE
+
+
+# ------------------------------------------------------------------------------------ combine
+
+@pytest.mark.parametrize("n", [1, 3, 4, 1000, 100001])
+def test_combine_parity(n):
+    G = synth.gaussian(n, 1, sigma=1e-2)
+    L = synth.gaussian(n, 2, sigma=1e-2)
+    for alpha, beta in [(1.0, 1.0), (0.25, 0.25), (0.0, 0.5), (1.0 / 3, 0.7)]:
+        want = oracle.combine_local(G, L, alpha, beta)
+        got = gs.combine_local(dev(G), dev(L), alpha=alpha, beta=beta)
+        assert np.array_equal(bits(host(got)), bits(want))
+    k = max(n // 7, 1)
+    own_idx = np.sort(np.random.default_rng(n).choice(n, k, replace=False)).astype(np.int32)
+    own_val = synth.gaussian(k, 9, sigma=1e-2)
+    want = oracle.combine_local(G, L, 1.0, 1.0, mode=1, own_idx=own_idx, own_val=own_val)
+    got = gs.combine_local(dev(G), dev(L), mode=1, own_idx=dev(own_idx), own_val=dev(own_val),
+                           own_count=torch.tensor([k], device="cuda"), own_capacity=k)
+    assert np.array_equal(bits(host(got)), bits(want))
