@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Benchmark of the gradient-compression hot path on B200.
+
+Workload: a flat fp32 gradient of 2^30 entries (4 GiB) per worker, Laplace(0, 1e-3) with 0.1%
+Laplace(0, 1e-1) outliers, W = 2 workers resident on one GPU, residual carried from step to step.
+One step:
+  per worker: residual top-k at a 99% drop (keep 1/100) -> 2-bit quantisation with the error fed
+              back into the residual -> Golomb encode (b* = 6) -> Golomb decode
+  then:       scatter-accumulate of the W decoded updates into the dense global sum G
+              -> combination with each worker's own gradient (out_w = G + g_w)
+Metric: gradient GB/s compressed = W * 4 * n bytes per step / step time (whole job over all
+ranks), with the residual-top-k call's share of HBM bandwidth reported beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--drop 0.99]
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent replica of the step:
+the path has no exchange on one node's simulated workers, so there is no collective in the data
+path; the barrier and the max-over-ranks reduction use NCCL. Rank 0 prints one JSON line.
+The reference arm is the CPU oracle (single thread) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "gradient GB/s compressed (top-1% residual select+compact)"
+UNIT = "GB/s"
+PROFILE = os.path.join(ROOT, "profiles", "pass1_kernel_flat_fp32.md")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def workload_config(n, workers, drop, b, extra=None):
+    cfg = {"workload": f"flat fp32 gradient of {n} entries per worker, Laplace(0,1e-3) with 0.1% "
+                       f"Laplace(0,1e-1) outliers, {workers} workers on one GPU, residual carried",
+           "n": n, "workers": workers, "drop": drop, "keep": f"1/{round(1 / (1 - drop))}",
+           "golomb_b": b, "step": "topk+quantise+golomb enc/dec per worker, scatter-accumulate, combine",
+           "l2": "inputs larger than L2 (8 GiB of gradients + 8 GiB of residuals per step)"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def keep_of(drop):
+    den = round(1.0 / (1.0 - drop))
+    return (1, den)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(n):
+    """Per-launch DRAM bytes of the pass-1 kernel from the committed ncu summary, scaled to n
+    entries; None if the summary is missing or the kernel source changed since the capture."""
+    try:
+        text = open(PROFILE).read()
+        src = open(os.path.join(ROOT, "compressed_sgd_b200", "csrc", "select.cu"), "rb").read()
+        sha = hashlib.sha256(src).hexdigest()[:16]
+        m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+        m_b = re.search(r"dram_bytes_per_entry:\s*([0-9.]+)", text)
+        if not m_sha or not m_b or m_sha.group(1) != sha:
+            return None
+        return float(m_b.group(1)) * n
+    except Exception:
+        return None
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = f"/tmp/gsparse_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.index)], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = max(smax, float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.remove(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+
+def run_ours(args, rank, world, dist):
+    import torch
+    import compressed_sgd_b200 as gs
+    import synth
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    n, W = args.n, args.workers
+    keep = keep_of(args.drop)
+    b = gs.golomb_b_star(1.0 - args.drop)
+    cap = gs.k_for(n, keep)
+    chunk = 64
+
+    # inputs: generated on the host (pinned, for the end-to-end leg), copied once to the device
+    g_host = []
+    for w in range(W):
+        t = torch.empty(n, dtype=torch.float32, pin_memory=True)
+        t.numpy()[:] = synth.laplace_outliers(w + 2 * rank, n)
+        g_host.append(t)
+    g = [t.to(dev) for t in g_host]
+    r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)]
+    idx = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(W)]
+    val = [torch.empty(cap, dtype=torch.float32, device=dev) for _ in range(W)]
+    off = [torch.empty(2, dtype=torch.int64, device=dev) for _ in range(W)]
+    end = [o[1:2] for o in off]
+    sb = [torch.empty((cap + 31) // 32, dtype=torch.int32, device=dev) for _ in range(W)]
+    means = [torch.empty(2, dtype=torch.float32, device=dev) for _ in range(W)]
+    nwords = gs.golomb_word_capacity(cap, b, n)
+    words = [torch.empty(nwords, dtype=torch.int32, device=dev) for _ in range(W)]
+    nbits = [torch.zeros(1, dtype=torch.int64, device=dev) for _ in range(W)]
+    table = [torch.empty(((cap + chunk - 1) // chunk, 2), dtype=torch.int64, device=dev) for _ in range(W)]
+    dec = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(W)]
+    G = torch.empty(n, dtype=torch.float32, device=dev)
+    out = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
+    ws_t = [torch.empty(gs.residual_topk_workspace_size(n, 1, keep), dtype=torch.uint8, device=dev) for _ in range(W)]
+    ws_q = [torch.empty(gs.lib().gsparse_quantize_workspace_size(cap), dtype=torch.uint8, device=dev) for _ in range(W)]
+    ws_g = [torch.empty(gs.lib().gsparse_golomb_encode_workspace_size(cap), dtype=torch.uint8, device=dev)
+            for _ in range(W)]
+    ws_s = torch.empty(gs.lib().gsparse_scatter_accumulate_workspace_size(W, n), dtype=torch.uint8, device=dev)
+    st = gs.status_tensor(dev)
+    lists = [gs.make_list(dec[w], end[w], val=val[w], capacity=cap) for w in range(W)]
+    # payload read back in the end-to-end leg: Golomb words, sign bits, means, bit count
+    payload = [(words[w], sb[w], means[w], nbits[w], off[w]) for w in range(W)]
+    payload_host = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in p] for p in payload]
+    d2h_bytes = sum(t.numel() * t.element_size() for p in payload for t in p)
+    h2d_bytes = W * n * 4
+
+    stage_names = ["residual_topk", "quantize", "golomb_encode", "golomb_decode"]
+    stage_ms = {k: [] for k in stage_names + ["scatter_accumulate", "combine_local"]}
+    pass1_ms = []
+
+    def step(events=None, p1=None):
+        e = iter(events) if events is not None else None
+        rec = (lambda: next(e).record()) if e is not None else (lambda: None)
+        for w in range(W):
+            rec()
+            if p1 is not None:
+                gs.set_pass1_events(p1[w][0], p1[w][1])
+            gs.residual_topk(g[w], r[w], keep, out_idx=idx[w], out_val=val[w], out_offsets=off[w],
+                             workspace=ws_t[w], d_status=st, capacity=cap)
+            if p1 is not None:
+                gs.set_pass1_events(None, None)
+            rec()
+            gs.quantize(idx[w], val[w], end[w], residual=r[w], write_dequantized=True, sign_bits=sb[w],
+                        means=means[w], workspace=ws_q[w], d_status=st, capacity=cap)
+            rec()
+            gs.golomb_encode(idx[w], end[w], b, n, chunk=chunk, words=words[w], nbits=nbits[w], table=table[w],
+                             workspace=ws_g[w], d_status=st, capacity=cap)
+            rec()
+            gs.golomb_decode(words[w], nbits[w], end[w], cap, b, table=table[w], chunk=chunk, n_limit=n,
+                             out_idx=dec[w], d_status=st)
+        rec()
+        gs.scatter_accumulate(lists, n, dense_out=G, workspace=ws_s, d_status=st, device=dev)
+        rec()
+        for w in range(W):
+            gs.combine_local(G, g[w], out=out[w])
+        rec()
+
+    n_ev = 4 * W + 3
+
+    def new_events(k):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(k)]
+        for ev in evs:
+            ev.record()       # materialise the CUDA event before handing it to the library
+        return evs
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} after warm-up")
+
+    K = args.steps
+    ev = [new_events(n_ev) for _ in range(K)]
+    p1 = [[new_events(2) for _ in range(W)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(dev.index if dev.index is not None else 0)
+    barrier()
+    clocks.start()
+    t0.record()
+    for k in range(K):
+        step(ev[k], p1[k])
+    t1.record()
+    barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / K
+    for k in range(K):
+        e = ev[k]
+        for w in range(W):
+            for s, name in enumerate(stage_names):
+                stage_ms[name].append(e[4 * w + s].elapsed_time(e[4 * w + s + 1]))
+            pass1_ms.append(p1[k][w][0].elapsed_time(p1[k][w][1]))
+        stage_ms["scatter_accumulate"].append(e[4 * W].elapsed_time(e[4 * W + 1]))
+        stage_ms["combine_local"].append(e[4 * W + 1].elapsed_time(e[4 * W + 2]))
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the timed region")
+
+    # kernels of this library launched per step, counted by the CUDA profiler on one extra step
+    launches_per_step = None
+    if not args.no_launch_count:
+      try:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step()
+            torch.cuda.synchronize(dev)
+        names = [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+        launches_per_step = len([x for x in names if "gs::" in x])
+      except Exception:
+        launches_per_step = None
+
+    # end-to-end through the public API: pinned host gradients in, compressed payload out
+    e2e_ms = None
+    if args.e2e_steps > 0:
+        def e2e_step():
+            for w in range(W):
+                g[w].copy_(g_host[w], non_blocking=True)
+            step()
+            for w in range(W):
+                for src, dst in zip(payload[w], payload_host[w]):
+                    dst.copy_(src, non_blocking=True)
+        e2e_step()
+        barrier()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        z.record()
+        barrier()
+        e2e_ms = a.elapsed_time(z) / args.e2e_steps
+
+    # max over ranks
+    if world > 1:
+        tt = torch.tensor([ms, e2e_ms or 0.0], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(tt[0]), (float(tt[1]) if e2e_ms is not None else None)
+
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peaks()
+    grad_bytes = world * W * 4 * n
+    value = grad_bytes / (ms * 1e-3) / 1e9
+    p1 = statistics.mean(pass1_ms)
+    p1_bytes = 12 * n
+    achieved = p1_bytes / (p1 * 1e-3) / 1e9
+    topk_ms = statistics.mean(stage_ms["residual_topk"])
+    topk_bytes = 12 * n + 8 * cap
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(n, W, args.drop, b, {"parallelism": f"replicas x{world}"}),
+        "roofline": {"bound": "hbm", "kernel": "pass1_kernel (streaming pass of residual top-k)",
+                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(n),
+                     "algorithmic_bytes_per_launch": p1_bytes, "launch_ms": round(p1, 4)},
+        "residual_topk_call": {"ms": round(topk_ms, 4), "algorithmic_bytes": topk_bytes,
+                               "gbs": round(topk_bytes / (topk_ms * 1e-3) / 1e9, 1),
+                               "frac_of_peak": round(topk_bytes / (topk_ms * 1e-3) / 1e9 / peak, 4),
+                               "frac_of_8000": round(topk_bytes / (topk_ms * 1e-3) / 1e9 / 8000.0, 4),
+                               "gradient_gbs": round(4 * n / (topk_ms * 1e-3) / 1e9, 1)},
+        "stages_ms": {k: round(statistics.median(v), 4) for k, v in stage_ms.items()},
+        "gpu_launches": (launches_per_step * K) if launches_per_step is not None else None,
+        "gpu_launches_per_step": launches_per_step,
+        "clocks": clk,
+    }
+    if e2e_ms is not None:
+        line["e2e"] = {"value": round(grad_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+                       "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
+                       "ms_per_step": round(e2e_ms, 3)}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args, args.cpu_n)
+    return line
+
+
+# ---------------------------------------------------------------------------------------------
+# the CPU oracle (reference arm and cpu_baseline)
+
+def oracle_step(gs_list, rs, keep, b, n):
+    import oracle
+    lists = []
+    for g, r in zip(gs_list, rs):
+        idx, val, off, r2 = oracle.residual_topk(g, r, keep)
+        bits, means, val, r2 = oracle.quantize(idx, val, residual=r2, write_dequantized=True)
+        words, nb, table = oracle.golomb_encode(idx, b, chunk=64)
+        dec = oracle.golomb_decode(words, nb, idx.size, b, n_limit=n)
+        lists.append((dec, val))
+        r[:] = r2
+    dense, _, _ = oracle.scatter_accumulate(lists, n, merged=False)
+    for g in gs_list:
+        oracle.combine_local(dense, g)
+
+
+def cpu_baseline(args, n_s):
+    import oracle
+    import synth
+    oracle.build()
+    keep = keep_of(args.drop)
+    b = oracle.golomb_b_star(1.0 - args.drop)
+    gsl = [synth.laplace_outliers(w, n_s) for w in range(args.workers)]
+    rs = [np.zeros(n_s, np.float32) for _ in range(args.workers)]
+    oracle_step(gsl, rs, keep, b, n_s)          # warm
+    t = time.perf_counter()
+    reps = 0
+    while True:
+        oracle_step(gsl, rs, keep, b, n_s)
+        reps += 1
+        if time.perf_counter() - t > 8.0 or reps >= 5:
+            break
+    dt = (time.perf_counter() - t) / reps
+    return {"value": round(args.workers * 4 * n_s / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"the same step on {n_s} entries per worker ({args.workers} workers), {reps} timed steps, "
+                      f"single-threaded C++ oracle", "host_cpus": os.cpu_count()}
+
+
+def run_reference(args):
+    import oracle
+    import synth
+    oracle.build()
+    keep = keep_of(args.drop)
+    b = oracle.golomb_b_star(1.0 - args.drop)
+    n_s = args.ref_n
+    gsl = [synth.laplace_outliers(w, n_s) for w in range(args.workers)]
+    rs = [np.zeros(n_s, np.float32) for _ in range(args.workers)]
+    for _ in range(args.warmup):
+        oracle_step(gsl, rs, keep, b, n_s)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(gsl, rs, keep, b, n_s)
+    dt = (time.perf_counter() - t) / args.steps
+    value = round(args.workers * 4 * n_s / dt / 1e9, 4)
+    sample = (f"each step the full hot path on {n_s} entries per worker ({args.workers} workers) instead of "
+              f"{args.n}; single-threaded C++ oracle")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": workload_config(args.n, args.workers, args.drop, b, {"sample_n": n_s}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--drop", type=float, default=0.99)
+    ap.add_argument("--n", type=int, default=1 << 30)
+    ap.add_argument("--workers", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-launch-count", action="store_true", help="skip the profiler-based kernel count")
+    ap.add_argument("--cpu-n", type=int, default=1 << 24)
+    ap.add_argument("--ref-n", type=int, default=1 << 20)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        line = run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

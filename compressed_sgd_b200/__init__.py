@@ -39,6 +39,7 @@ class GsparseList(ctypes.Structure):
 _SIGNATURES = {
     "gsparse_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gsparse_version": (ctypes.c_char_p, []),
+    "gsparse_set_pass1_events": (None, [_vp, _vp]),
     "gsparse_k_for": (_i64, [_i64, _i64, _i64]),
     "gsparse_golomb_b_star": (_i32, [_f64]),
     "gsparse_residual_topk_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
@@ -114,6 +115,15 @@ def k_for(n_s: int, keep: Tuple[int, int]) -> int:
 
 def golomb_b_star(p: float) -> int:
     return int(lib().gsparse_golomb_b_star(p))
+
+
+def set_pass1_events(before: Optional[torch.cuda.Event], after: Optional[torch.cuda.Event]):
+    """Measurement hook: record these events around the streaming pass of every following
+    residual_topk / binarize call (None, None turns it off)."""
+    if before is None or after is None:
+        lib().gsparse_set_pass1_events(None, None)
+    else:
+        lib().gsparse_set_pass1_events(before.cuda_event, after.cuda_event)
 
 
 def status_tensor(device="cuda") -> torch.Tensor:

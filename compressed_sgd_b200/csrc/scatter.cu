@@ -53,7 +53,7 @@ __device__ void accumulate_tile(const Lists& L, int32_t W, int64_t t, const int6
     const int64_t b = start[t * W + w], e = start[(t + 1) * W + w];
     const int32_t* ix = L.idx[w];
     const float* vv = L.val[w];
-    const float u = vv ? 0.0f : *L.uni[w];
+    const float u = (vv || !L.uni[w]) ? 0.0f : *L.uni[w];
     for (int64_t j = b + threadIdx.x; j < e; j += blockDim.x) {
       const int32_t i = ix[j];
       if (j > 0 && ix[j - 1] >= i) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); continue; }
@@ -233,7 +233,7 @@ int gsparse_scatter_accumulate(const gsparse_list* lists, int32_t W, int64_t n, 
   Lists L{};
   for (int w = 0; w < W; ++w) {
     const gsparse_list& x = lists[w];
-    if (!x.d_count || x.capacity < 0 || (x.capacity > 0 && !x.idx) || (!x.val && !x.uniform_val))
+    if (!x.d_count || x.capacity < 0 || (x.capacity > 0 && (!x.idx || (!x.val && !x.uniform_val))))
       return GSPARSE_ERR_INVALID_ARG;
     L.idx[w] = x.idx;
     L.val[w] = x.val;

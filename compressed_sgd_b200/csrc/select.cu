@@ -943,6 +943,8 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
 
 bool bad_keep(int64_t num, int64_t den) { return den <= 0 || num < 0 || num > den; }
 
+cudaEvent_t g_pass1_before = nullptr, g_pass1_after = nullptr;
+
 template <int C>
 int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t T, int64_t num,
                int64_t den, int32_t* out_idx, float* out_val, float* d_mean, int64_t* out_offsets,
@@ -985,7 +987,10 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
     attr_set[C - 1][dev] = true;
   }
   sample_kernel<C><<<T, 1024, sample_smem, st>>>(a, (flags & GSPARSE_SELECT_EXHAUSTIVE) ? 1 : 0);
+  const bool timed = g_pass1_before && g_pass1_after;
+  if (timed) cudaEventRecord(g_pass1_before, st);
   if (piece_ctas) pass1_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
+  if (timed) cudaEventRecord(g_pass1_after, st);
   check_kernel<<<(unsigned)(T * C), 256, 0, st>>>(a);
   if (piece_ctas) restore_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
   select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 1);
@@ -1015,6 +1020,11 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
 using namespace gs;
 
 extern "C" {
+
+void gsparse_set_pass1_events(gsparse_event before, gsparse_event after) {
+  g_pass1_before = (cudaEvent_t)before;
+  g_pass1_after = (cudaEvent_t)after;
+}
 
 size_t gsparse_residual_topk_workspace_size(int64_t n, int32_t T, int64_t num, int64_t den) {
   if (n < 0 || T < 1 || bad_keep(num, den)) return 0;

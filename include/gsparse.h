@@ -41,8 +41,9 @@
 extern "C" {
 #endif
 
-/* Same type as cudaStream_t. */
+/* Same types as cudaStream_t and cudaEvent_t. */
 typedef struct CUstream_st* gsparse_stream;
+typedef struct CUevent_st* gsparse_event;
 
 /* Host-side status. */
 enum gsparse_status {
@@ -71,6 +72,12 @@ enum gsparse_select_flags {
 
 const char* gsparse_status_string(int status);
 const char* gsparse_version(void);
+
+/* Measurement hook, off by default and not thread-safe: while both events are non-NULL, every
+ * gsparse_residual_topk and gsparse_binarize call records `before` on its stream right before
+ * its streaming pass over g and the residual, and `after` right after it, so that pass can be
+ * timed alone with cudaEventElapsedTime. Passing NULLs turns it off. */
+void gsparse_set_pass1_events(gsparse_event before, gsparse_event after);
 
 /* ---------------------------------------------------------------------------------------------
  * Host helpers.
