@@ -46,6 +46,7 @@ _SIGNATURES = {
     "gsparse_residual_topk_workspace_min": (_sz, [_i64, _i32]),
     "gsparse_residual_topk": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _i64, _u32,
                                              _vp, _sz, _vp, _vp]),
+    "gsparse_residual_topk_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp]),
     "gsparse_quantize_workspace_size": (_sz, [_i64]),
     "gsparse_quantize": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp, _sz, _vp, _vp]),
     "gsparse_binarize_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
@@ -170,6 +171,35 @@ def residual_topk(g: torch.Tensor, residual: torch.Tensor, keep=(1, 100), seg_of
                                      _ptr(out_idx), _ptr(out_val), _ptr(out_offsets), capacity, flags,
                                      _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev))
     _check(st, "gsparse_residual_topk")
+    return out_idx, out_val, out_offsets
+
+
+NOALLOC_MAX_N = 1 << 24
+
+
+def residual_topk_noalloc(g: torch.Tensor, residual: torch.Tensor, keep=(1, 100),
+                          out_idx: Optional[torch.Tensor] = None, out_val: Optional[torch.Tensor] = None,
+                          out_offsets: Optional[torch.Tensor] = None, d_status: Optional[torch.Tensor] = None,
+                          capacity: Optional[int] = None):
+    """Global residual top-k whose scratch is the library's own fixed device array (for callers that
+    must not allocate; n <= NOALLOC_MAX_N). Outputs as for residual_topk; pass them in to allocate
+    nothing here either."""
+    _dev(g, torch.float32, "g")
+    _dev(residual, torch.float32, "residual")
+    n = g.numel()
+    dev = g.device
+    if capacity is None:
+        capacity = k_for(n, keep)
+    if out_idx is None:
+        out_idx = torch.empty(max(capacity, 1), dtype=torch.int32, device=dev)
+    if out_val is None:
+        out_val = torch.empty(max(capacity, 1), dtype=torch.float32, device=dev)
+    if out_offsets is None:
+        out_offsets = torch.empty(2, dtype=torch.int64, device=dev)
+    st = lib().gsparse_residual_topk_noalloc(_ptr(g), _ptr(residual), n, keep[0], keep[1], _ptr(out_idx),
+                                             _ptr(out_val), _ptr(out_offsets), capacity, _ptr(d_status),
+                                             _stream(dev))
+    _check(st, "gsparse_residual_topk_noalloc")
     return out_idx, out_val, out_offsets
 
 

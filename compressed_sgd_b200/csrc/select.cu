@@ -1014,6 +1014,25 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   return launch_status();
 }
 
+// Scratch of gsparse_residual_topk_noalloc: one array per device, in the library's own memory.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GSPARSE_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the array on the current device, looked up once per device. In host code
+// the symbol itself is only a host-side stand-in, never a device address.
+int noalloc_scratch(void** out) {
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GSPARSE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return GSPARSE_ERR_UNSUPPORTED;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GSPARSE_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return GSPARSE_OK;
+}
+
 }  // namespace
 }  // namespace gs
 
@@ -1054,6 +1073,19 @@ size_t gsparse_binarize_workspace_size(int64_t n, int32_t T, int64_t num, int64_
 size_t gsparse_binarize_workspace_min(int64_t n, int32_t T, int64_t num, int64_t den) {
   if (n < 0 || T < 1 || bad_keep(num, den)) return 0;
   return carve(n, T, 2, num, den, nullptr, 0, false).fixed_bytes;
+}
+
+int gsparse_residual_topk_noalloc(const float* g, float* residual, int64_t n, int64_t keep_num,
+                                  int64_t keep_den, int32_t* out_idx, float* out_val,
+                                  int64_t* out_offsets, int64_t out_capacity, int32_t* d_status,
+                                  gsparse_stream stream) {
+  if (n > GSPARSE_NOALLOC_MAX_N) return GSPARSE_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  const int st = noalloc_scratch(&scratch);
+  if (st != GSPARSE_OK) return st;
+  return run_select<1>(g, residual, n, nullptr, 1, keep_num, keep_den, out_idx, out_val, nullptr,
+                       out_offsets, out_capacity, 0, scratch, GSPARSE_NOALLOC_SCRATCH_BYTES, d_status,
+                       (cudaStream_t)stream);
 }
 
 int gsparse_binarize(const float* g, float* residual, int64_t n, const int64_t* seg_offsets,

@@ -128,6 +128,33 @@ int gsparse_residual_topk(const float* g, float* residual, int64_t n, const int6
                           gsparse_stream stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Residual top-k without caller-provided scratch  (no counterpart in the pages: this entry point
+ * exists for callers, not for the method)
+ *
+ * Some callers cannot call cudaMalloc or hand over a workspace: code that runs inside a host
+ * framework whose caching allocator owns the whole device and budgets every byte (an allocation
+ * of our own would fail or fight that allocator), or code invoked from that allocator's own hooks
+ * (allocating there would re-enter it). This call needs neither: its scratch is a fixed array of
+ * GSPARSE_NOALLOC_SCRATCH_BYTES in the library's own device memory, created when the library is
+ * loaded and held by every GPU that loads it until the process exits. It allocates nothing.
+ *
+ * Same result as gsparse_residual_topk with seg_offsets = NULL and num_segments = 1 (one global
+ * selection) and flags = 0, bit for bit. The caller still owns g, residual and the outputs.
+ * - n above GSPARSE_NOALLOC_MAX_N returns GSPARSE_ERR_UNSUPPORTED before any launch.
+ * - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current; make that first call before any stream capture on the device.
+ * - All calls on a device share the one array and it keeps the last call's contents; each call
+ *   clears the parts that must start at zero. Calls whose kernels overlap on the GPU (concurrent
+ *   streams, or several host threads) race on the array: serialise them.
+ */
+#define GSPARSE_NOALLOC_MAX_N (1 << 24)
+#define GSPARSE_NOALLOC_SCRATCH_BYTES (16u << 20)
+int gsparse_residual_topk_noalloc(const float* g, float* residual, int64_t n, int64_t keep_num,
+                                  int64_t keep_den, int32_t* out_idx, float* out_val,
+                                  int64_t* out_offsets, int64_t out_capacity, int32_t* d_status,
+                                  gsparse_stream stream);
+
+/* ---------------------------------------------------------------------------------------------
  * 2-bit quantisation of a sent list  (Aji & Heafield 2017, Abstract: sparsification combined
  * with quantisation)
  *
