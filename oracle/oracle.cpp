@@ -53,20 +53,20 @@ int64_t kept_count(int64_t n_s, int64_t num, int64_t den) {
 }
 
 // The k largest of `cand` under the total order (key descending, index ascending), returned in
-// ascending index order. The order is a plain definition of "largest by magnitude, ties to the
-// lower index"; std::nth_element places exactly the k smallest-under-`before` first.
+// ascending index order. Each entry is packed as (~key << 32 | index) so that ascending order of
+// the packed integer is exactly that total order ("largest by magnitude, ties to the lower
+// index"); std::nth_element then places the k smallest packed values first.
 template <class KeyFn>
-std::vector<int64_t> top_k(std::vector<int64_t> cand, int64_t k, KeyFn key) {
-  auto before = [&](int64_t a, int64_t b) {
-    uint32_t ka = key(a), kb = key(b);
-    if (ka != kb) return ka > kb;
-    return a < b;
-  };
-  if (k > (int64_t)cand.size()) k = (int64_t)cand.size();
-  if (k < (int64_t)cand.size()) std::nth_element(cand.begin(), cand.begin() + k, cand.end(), before);
-  cand.resize(k);
-  std::sort(cand.begin(), cand.end());
-  return cand;
+std::vector<int64_t> top_k(const std::vector<int64_t>& cand, int64_t k, KeyFn key) {
+  std::vector<uint64_t> packed(cand.size());
+  for (size_t j = 0; j < cand.size(); ++j)
+    packed[j] = ((uint64_t)(~key(cand[j])) << 32) | (uint64_t)(uint32_t)cand[j];
+  if (k > (int64_t)packed.size()) k = (int64_t)packed.size();
+  if (k < (int64_t)packed.size()) std::nth_element(packed.begin(), packed.begin() + k, packed.end());
+  std::vector<int64_t> out(k);
+  for (int64_t j = 0; j < k; ++j) out[j] = (int64_t)(uint32_t)(packed[j] & 0xffffffffu);
+  std::sort(out.begin(), out.end());
+  return out;
 }
 
 // Fixed-order fp64 sum of the member entries of a list. READING: the pages give no summation
@@ -265,7 +265,7 @@ int orc_golomb_encode(const int32_t* idx, int64_t K, int64_t base, int32_t b, ui
   std::vector<uint8_t> bits;
   int64_t prev = base - 1;
   for (int64_t j = 0; j < K; ++j) {
-    const int64_t d = (int64_t)idx[j] - prev - 1;
+    const int64_t d = (int64_t)idx[j] - prev;
     if (d < 0) return kRange;
     if (chunk_table && j % chunk == 0) {
       chunk_table[2 * (j / chunk)] = (int64_t)bits.size();
