@@ -56,17 +56,22 @@ int64_t kept_count(int64_t n_s, int64_t num, int64_t den) {
 // ascending index order. Each entry is packed as (~key << 32 | index) so that ascending order of
 // the packed integer is exactly that total order ("largest by magnitude, ties to the lower
 // index"); std::nth_element then places the k smallest packed values first.
-template <class KeyFn>
-std::vector<int64_t> top_k(const std::vector<int64_t>& cand, int64_t k, KeyFn key) {
-  std::vector<uint64_t> packed(cand.size());
-  for (size_t j = 0; j < cand.size(); ++j)
-    packed[j] = ((uint64_t)(~key(cand[j])) << 32) | (uint64_t)(uint32_t)cand[j];
+std::vector<int64_t> top_k_packed(std::vector<uint64_t>& packed, int64_t k) {
   if (k > (int64_t)packed.size()) k = (int64_t)packed.size();
   if (k < (int64_t)packed.size()) std::nth_element(packed.begin(), packed.begin() + k, packed.end());
   std::vector<int64_t> out(k);
   for (int64_t j = 0; j < k; ++j) out[j] = (int64_t)(uint32_t)(packed[j] & 0xffffffffu);
   std::sort(out.begin(), out.end());
   return out;
+}
+
+uint64_t pack(uint32_t key, int64_t index) { return ((uint64_t)(~key) << 32) | (uint64_t)(uint32_t)index; }
+
+template <class KeyFn>
+std::vector<int64_t> top_k(const std::vector<int64_t>& cand, int64_t k, KeyFn key) {
+  std::vector<uint64_t> packed(cand.size());
+  for (size_t j = 0; j < cand.size(); ++j) packed[j] = pack(key(cand[j]), cand[j]);
+  return top_k_packed(packed, k);
 }
 
 // Fixed-order fp64 sum of the member entries of a list. READING: the pages give no summation
@@ -150,9 +155,9 @@ int orc_residual_topk(const float* g, float* r, int64_t n, const int64_t* seg, i
   out_off[0] = 0;
   for (int64_t i = 0; i < n; ++i) r[i] = acc[i];
   for (int32_t s = 0; s < T; ++s) {
-    std::vector<int64_t> cand(seg[s + 1] - seg[s]);
-    std::iota(cand.begin(), cand.end(), seg[s]);
-    std::vector<int64_t> sent = top_k(cand, kept_count(seg[s + 1] - seg[s], num, den), key);
+    std::vector<uint64_t> packed(seg[s + 1] - seg[s]);
+    for (int64_t i = seg[s]; i < seg[s + 1]; ++i) packed[i - seg[s]] = pack(key(i), i);
+    std::vector<int64_t> sent = top_k_packed(packed, kept_count(seg[s + 1] - seg[s], num, den));
     for (int64_t i : sent) {
       out_idx[o] = (int32_t)i;
       out_val[o] = acc[i];
@@ -265,7 +270,7 @@ int orc_golomb_encode(const int32_t* idx, int64_t K, int64_t base, int32_t b, ui
   std::vector<uint8_t> bits;
   int64_t prev = base - 1;
   for (int64_t j = 0; j < K; ++j) {
-    const int64_t d = (int64_t)idx[j] - prev;
+    const int64_t d = (int64_t)idx[j] - prev - 1;
     if (d < 0) return kRange;
     if (chunk_table && j % chunk == 0) {
       chunk_table[2 * (j / chunk)] = (int64_t)bits.size();
