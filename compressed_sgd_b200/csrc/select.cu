@@ -35,8 +35,9 @@ constexpr int kBins1 = 2048, kBins2 = 2048, kBins3 = 512;
 constexpr int kHist = kBins1 + kBins2 + kBins3;  // per problem
 constexpr int64_t kGranule = 512;                // entries per warp iteration (32 lanes x 16)
 constexpr int64_t kTargetPieces = 148 * 32;      // warps streaming at once on a B200
-constexpr int kSample = 16384;                   // sampled entries per segment
-constexpr int kSampleChunks = kSample / 32;
+constexpr int kSample = 1 << 18;                 // sampled entries per segment
+constexpr int kSampleRuns = kSample / 32;        // ... as evenly spaced runs of 32 entries
+constexpr int kSampleCtas = 256;                 // CTAs sharing one segment's sample
 constexpr int kWarps = 8;                        // warps (pieces) per CTA
 constexpr int kThreads = kWarps * 32;
 
@@ -57,6 +58,9 @@ struct Sel {
   int32_t* cidx;
   float* cval;
   int32_t* ctl;  // [0] abort, [1] any redo
+  // sample: two-level histogram of the sampled keys per problem
+  uint32_t *shist, *scount, *sdone, *sb1;
+  int64_t* srank;
   int32_t* d_status;
   // binarise
   int32_t* lidx;
@@ -151,29 +155,6 @@ __device__ void block_find_bin(const uint32_t* h, int B, int64_t rank, uint32_t*
   __syncthreads();
 }
 
-// rank-th largest of keys[0..cnt) in shared memory (1 <= rank <= cnt), by 11+11+9-bit radix steps.
-__device__ uint32_t block_select_key(const uint32_t* keys, int cnt, int64_t rank, uint32_t* hist) {
-  uint32_t prefix = 0;
-  const int shifts[3] = {20, 9, 0};
-  const int widths[3] = {11, 11, 9};
-  for (int L = 0; L < 3; ++L) {
-    const int sh = shifts[L], w = widths[L], B = 1 << w;
-    for (int i = threadIdx.x; i < B; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-      const uint32_t k = keys[i];
-      if ((k >> (sh + w)) == prefix) atomicAdd(&hist[(k >> sh) & (B - 1)], 1u);
-    }
-    __syncthreads();
-    uint32_t bin;
-    int64_t above;
-    block_find_bin(hist, B, rank, &bin, &above);
-    prefix = (prefix << w) | bin;
-    rank -= above;
-  }
-  return prefix;
-}
-
 // ------------------------------------------------------------------------------------------
 // 1. plan
 
@@ -229,58 +210,112 @@ __global__ void __launch_bounds__(1024) plan_kernel(Sel a, const int64_t* seg, i
 
 // ------------------------------------------------------------------------------------------
 // 2. sample: candidate thresholds
+//
+// Each segment's sample (the whole segment when it has at most kSample entries, else kSample
+// entries in evenly spaced runs of 32) is split over kSampleCtas CTAs. Level 1 histograms the
+// top 11 key bits; the last CTA to finish picks the bin holding the m-th largest sampled key.
+// Level 2 re-reads the sample, histograms the next 11 bits inside that bin, and its last CTA sets
+// T_lo to the lower edge of the 22-bit bucket holding the m-th key. With the whole segment in the
+// sample m = k, so at least k entries reach T_lo; otherwise m sits three standard deviations (plus
+// 16) above the expected sample count, and a shortfall is caught and redone by the check step.
+
+__device__ __forceinline__ int64_t sample_pos(int64_t lo, int64_t ns, int64_t j) {
+  if (ns <= kSample) return lo + j;
+  return lo + (j >> 5) * (ns - 32) / (kSampleRuns - 1) + (j & 31);
+}
+
+__device__ __forceinline__ uint32_t* shist_of(const Sel& a, int64_t p, int level) {
+  return a.shist + p * (2 * kBins1) + (level == 1 ? 0 : kBins1);
+}
 
 template <int C>
-__global__ void __launch_bounds__(1024) sample_kernel(Sel a, int exhaustive) {
-  extern __shared__ uint32_t skeys[];  // [C][kSample]
-  __shared__ uint32_t hist[kBins1];
-  __shared__ int cnt[2];
+__global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhaustive) {
+  __shared__ uint32_t h[C * kBins1];
+  __shared__ uint32_t cnt[C];
+  __shared__ int last;
   if (a.ctl[0]) return;
-  const int32_t s = blockIdx.x;
+  const int32_t s = blockIdx.y;
   const int64_t lo = a.seg_lo[s], ns = a.seg_n[s], k = a.seg_k[s];
   const int64_t P0 = (int64_t)s * C;
-  if (k == 0 || ns == 0) {
-    if (threadIdx.x < C) a.tlo[P0 + threadIdx.x] = kNone;
-    return;
-  }
-  if (exhaustive) {
-    if (threadIdx.x < C) a.tlo[P0 + threadIdx.x] = 0;
-    return;
-  }
-  if (threadIdx.x < 2) cnt[threadIdx.x] = 0;
-  __syncthreads();
-  const bool full = ns <= kSample;
-  const int S = full ? (int)ns : kSample;
-  for (int j = threadIdx.x; j < S; j += blockDim.x) {
-    int64_t i;
-    if (full) {
-      i = lo + j;
-    } else {  // 512 evenly spaced runs of 32 consecutive entries
-      const int64_t chunk = j >> 5;
-      i = lo + chunk * (ns - 32) / (kSampleChunks - 1) + (j & 31);
+  if (k == 0 || ns == 0 || exhaustive) {
+    if (level == 1 && blockIdx.x == 0 && threadIdx.x < C) {
+      a.tlo[P0 + threadIdx.x] = (k == 0 || ns == 0) ? kNone : 0u;
+      a.sb1[P0 + threadIdx.x] = kNone;
     }
+    return;
+  }
+  uint32_t b1[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) b1[c] = level == 2 ? a.sb1[P0 + c] : 0u;
+  if (level == 2) {
+    bool any = false;
+#pragma unroll
+    for (int c = 0; c < C; ++c) any |= b1[c] != kNone;
+    if (!any) return;
+  }
+  for (int i = threadIdx.x; i < C * kBins1; i += blockDim.x) h[i] = 0;
+  if (threadIdx.x < C) cnt[threadIdx.x] = 0;
+  __syncthreads();
+  const int64_t S = ns < kSample ? ns : kSample;
+  const int64_t j0 = S * blockIdx.x / gridDim.x, j1 = S * (blockIdx.x + 1) / gridDim.x;
+  for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+    const int64_t i = sample_pos(lo, ns, j);
     const float x = __fadd_rn(a.g[i], a.r[i]);
     const int c = class_of<C>(x);
     if (c < 0) continue;
-    const int pos = atomicAdd(&cnt[c], 1);
-    skeys[c * kSample + pos] = mag_key(x);
+    const uint32_t key = mag_key(x);
+    if (level == 1) {
+      atomicAdd(&h[c * kBins1 + (key >> 20)], 1u);
+      atomicAdd(&cnt[c], 1u);
+    } else if ((key >> 20) == b1[c]) {
+      atomicAdd(&h[c * kBins1 + ((key >> 9) & 2047u)], 1u);
+    }
   }
   __syncthreads();
+  for (int i = threadIdx.x; i < C * kBins1; i += blockDim.x)
+    if (h[i]) atomicAdd(shist_of(a, P0 + i / kBins1, level) + (i % kBins1), h[i]);
+  if (level == 1 && threadIdx.x < C && cnt[threadIdx.x]) atomicAdd(&a.scount[P0 + threadIdx.x], cnt[threadIdx.x]);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&a.sdone[2 * s + level - 1], 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
   for (int c = 0; c < C; ++c) {
-    const int count = cnt[c];
-    uint32_t t;
-    if (full) {
-      const int64_t m = k < count ? k : count;
-      if (count == 0) t = kNone;                // class absent from the segment
-      else if (m == count) t = 0;               // every member is needed
-      else t = block_select_key(skeys + c * kSample, count, m, hist);
+    const int64_t p = P0 + c;
+    if (level == 2 && b1[c] == kNone) continue;
+    for (int i = threadIdx.x; i < kBins1; i += blockDim.x) h[i] = ((volatile uint32_t*)shist_of(a, p, level))[i];
+    __syncthreads();
+    if (level == 1) {
+      const int64_t count = ((volatile uint32_t*)a.scount)[p];
+      int64_t m;
+      if (ns <= kSample) {
+        m = k < count ? k : count;                 // the whole segment is in the sample
+      } else {
+        const double e = (double)k * (double)S / (double)ns;
+        m = (int64_t)ceil(e + 3.0 * sqrt(e) + 16.0);
+      }
+      if (count == 0 || m >= count) {
+        // every member is needed (or the class is absent from a fully sampled segment)
+        if (threadIdx.x == 0) {
+          a.tlo[p] = (count == 0 && ns <= kSample) ? kNone : 0u;
+          a.sb1[p] = kNone;
+        }
+      } else {
+        uint32_t bin;
+        int64_t above;
+        block_find_bin(h, kBins1, m, &bin, &above);
+        if (threadIdx.x == 0) {
+          a.sb1[p] = bin;
+          a.srank[p] = m - above;
+        }
+      }
     } else {
-      const double e = (double)k * (double)S / (double)ns;
-      const int64_t m = (int64_t)ceil(e + 4.0 * sqrt(e) + 8.0);
-      if (m >= count) t = 0;
-      else t = block_select_key(skeys + c * kSample, count, m, hist);
+      uint32_t bin;
+      int64_t above;
+      block_find_bin(h, kBins1, a.srank[p], &bin, &above);
+      if (threadIdx.x == 0) a.tlo[p] = ((b1[c] << 11) | bin) << 9;
     }
-    if (threadIdx.x == 0) a.tlo[P0 + c] = t;
     __syncthreads();
   }
 }
@@ -288,88 +323,146 @@ __global__ void __launch_bounds__(1024) sample_kernel(Sel a, int exhaustive) {
 // ------------------------------------------------------------------------------------------
 // 3. pass 1: the streaming pass
 
+// Candidate test of one accumulated value: its key reaches T_lo of its class. Binarise: the sign
+// picks the class, and zeros and NaN belong to neither (same classes as class_of<2>).
+template <int C>
+__device__ __forceinline__ uint32_t cand_bit(float x, const uint32_t* tl) {
+  const uint32_t u = __float_as_uint(x);
+  const uint32_t key = u & 0x7fffffffu;
+  if (C == 1) return key >= tl[0];
+  const uint32_t t = (u >> 31) ? tl[1] : tl[0];
+  return key >= t && key != 0u && key <= 0x7f800000u;
+}
+
+template <int C>
+__device__ __forceinline__ int cand_class(float x) {
+  return C == 1 ? 0 : (int)(__float_as_uint(x) >> 31);
+}
+
 template <int C>
 __global__ void __launch_bounds__(kThreads, 4) pass1_kernel(Sel a) {
   __shared__ CtaHist<C, kBins1> H;
+  __shared__ __align__(16) float stage[kWarps * 4 * 32 * 4];  // [warp][u][lane][e]
   if (a.ctl[0]) return;
   const int64_t q0 = (int64_t)blockIdx.x * kWarps;
   H.init(a, q0);
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int64_t q = q0 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t q = q0 + wid;
   if (q < total_pieces(a)) {
     const Piece P = piece_of(a, q);
     uint32_t tl[C];
 #pragma unroll
     for (int c = 0; c < C; ++c) tl[c] = a.tlo[(int64_t)P.s * C + c];
-    const int64_t cap = a.cap;
-    int32_t* cidx = a.cidx + q * cap;
-    float* cval = a.cval + q * cap;
+    const uint32_t cap = (uint32_t)a.cap;
+    int32_t* cidx = a.cidx + q * a.cap;
+    float* cval = a.cval + q * a.cap;
+    // histogram sink: this CTA's shared counts, or global counts for a second segment
+    const bool sh_sink = P.s == H.primary;
+    uint32_t* hsink = sh_sink ? H.sh : hist_of(a, (int64_t)P.s * C, 1);
+    const int hstride = sh_sink ? kBins1 : kHist;
+    const uint32_t lo = (uint32_t)P.lo, hi = (uint32_t)P.hi;  // indices are below 2^31
+    const float* g = a.g;
+    float* r = a.r;
+    float* st = stage + wid * 512;
     uint32_t count = 0;
-    for (int64_t base = P.lo & ~(int64_t)3; base < P.hi; base += kGranule) {
-      float4 gv[4], rv[4];
-      bool full[4];
+    for (uint32_t base = lo & ~3u; base < hi; base += (uint32_t)kGranule) {
+      if (base >= lo && base + (uint32_t)kGranule <= hi) {
+        // ---- fast path: the whole 512-entry chunk lies in the piece ----
+        float4 gv[4], rv[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t v = base + u * 128 + lane * 4;
-        full[u] = v >= P.lo && v + 4 <= P.hi;
-        if (full[u]) {
-          gv[u] = ld_stream(a.g + v);
-          rv[u] = ld_stream(a.r + v);
+        for (int u = 0; u < 4; ++u) {
+          gv[u] = ld_stream(g + base + u * 128 + lane * 4);
+          rv[u] = ld_stream(r + base + u * 128 + lane * 4);
+        }
+        float4 av[4];
+        uint32_t m16 = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          av[u] = make_float4(__fadd_rn(gv[u].x, rv[u].x), __fadd_rn(gv[u].y, rv[u].y),
+                              __fadd_rn(gv[u].z, rv[u].z), __fadd_rn(gv[u].w, rv[u].w));
+          m16 |= (cand_bit<C>(av[u].x, tl) | (cand_bit<C>(av[u].y, tl) << 1) |
+                  (cand_bit<C>(av[u].z, tl) << 2) | (cand_bit<C>(av[u].w, tl) << 3)) << (4 * u);
+        }
+        // per-quarter counts packed in bytes; one warp scan serves all four quarters
+        const uint32_t packed = __popc(m16 & 0xFu) | (__popc(m16 & 0xF0u) << 8) |
+                                (__popc(m16 & 0xF00u) << 16) | (__popc(m16 & 0xF000u) << 24);
+        const uint32_t incl = warp_inclusive_scan(packed);
+        const uint32_t tot = __shfl_sync(kFull, incl, 31);
+        if (tot == 0) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) st_stream(r + base + u * 128 + lane * 4, av[u]);
+          continue;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) reinterpret_cast<float4*>(st)[u * 32 + lane] = av[u];
+        __syncwarp();
+        const uint32_t excl = incl - packed;
+        const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu;
+        uint32_t stored = 0;
+        for (uint32_t m = m16; m; m &= m - 1) {
+          const int b = __ffs(m) - 1;
+          const int u = b >> 2, e = b & 3;
+          const uint32_t before = (u >= 1 ? t0 : 0u) + (u >= 2 ? t1 : 0u) + (u >= 3 ? t2 : 0u);
+          const uint32_t pos = count + before + ((excl >> (8 * u)) & 0xFFu) +
+                               __popc(m16 & ((1u << b) - 1u) & (0xFu << (4 * u)));
+          const float x = st[(u * 32 + lane) * 4 + e];
+          if (pos < cap) {
+            cidx[pos] = (int32_t)(base + u * 128 + lane * 4 + e);
+            cval[pos] = x;
+            stored |= 1u << b;
+          }
+          atomicAdd(hsink + cand_class<C>(x) * hstride + (mag_key(x) >> 20), 1u);
+        }
+        count += t0 + t1 + t2 + (tot >> 24);
+        if (a.zero_mode) {
+          for (uint32_t m = stored; m; m &= m - 1) {
+            const int b = __ffs(m) - 1;
+            st[((b >> 2) * 32 + lane) * 4 + (b & 3)] = 0.0f;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            st_stream(r + base + u * 128 + lane * 4, reinterpret_cast<const float4*>(st)[u * 32 + lane]);
         } else {
-          float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) st_stream(r + base + u * 128 + lane * 4, av[u]);
+        }
+        __syncwarp();
+      } else {
+        // ---- edge path: first or last chunk of the piece, element-wise bounds ----
+#pragma unroll 1
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t v = base + u * 128 + lane * 4;
+          float x[4];
+          uint32_t m4 = 0;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int64_t i = v + e;
-            if (i >= P.lo && i < P.hi) { t0[e] = a.g[i]; t1[e] = a.r[i]; }
+            const uint32_t i = v + e;
+            const bool in = i >= lo && i < hi;
+            x[e] = in ? __fadd_rn(g[i], r[i]) : 0.0f;
+            m4 |= (in ? cand_bit<C>(x[e], tl) : 0u) << e;
           }
-          gv[u] = make_float4(t0[0], t0[1], t0[2], t0[3]);
-          rv[u] = make_float4(t1[0], t1[1], t1[2], t1[3]);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t v = base + u * 128 + lane * 4;
-        float acc[4] = {__fadd_rn(gv[u].x, rv[u].x), __fadd_rn(gv[u].y, rv[u].y),
-                        __fadd_rn(gv[u].z, rv[u].z), __fadd_rn(gv[u].w, rv[u].w)};
-        uint32_t m4 = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int64_t i = v + e;
-          const int c = class_of<C>(acc[e]);
-          const bool cand = i >= P.lo && i < P.hi && c >= 0 && mag_key(acc[e]) >= tl[c < 0 ? 0 : c];
-          m4 |= (uint32_t)cand << e;
-        }
-        uint32_t tot;
-        const uint32_t pre = warp_prefix_small(__popc(m4), &tot);
-        uint32_t stored = 0;
-        if (tot) {
+          uint32_t tot;
+          const uint32_t pre = warp_prefix_small(__popc(m4), &tot);
           uint32_t pos = count + pre;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
+            const uint32_t i = v + e;
+            if (i < lo || i >= hi) continue;
+            float o = x[e];
             if ((m4 >> e) & 1u) {
               if (pos < cap) {
-                cidx[pos] = (int32_t)(v + e);
-                cval[pos] = acc[e];
-                stored |= 1u << e;
+                cidx[pos] = (int32_t)i;
+                cval[pos] = x[e];
+                if (a.zero_mode) o = 0.0f;
               }
-              H.add(a, P.s, class_of<C>(acc[e]) < 0 ? 0 : class_of<C>(acc[e]), mag_key(acc[e]) >> 20, 1);
+              atomicAdd(hsink + cand_class<C>(x[e]) * hstride + (mag_key(x[e]) >> 20), 1u);
               ++pos;
             }
+            r[i] = o;
           }
           count += tot;
-        }
-        float o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[e] = (a.zero_mode && ((stored >> e) & 1u)) ? 0.0f : acc[e];
-        if (full[u]) {
-          st_stream(a.r + v, make_float4(o[0], o[1], o[2], o[3]));
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int64_t i = v + e;
-            if (i >= P.lo && i < P.hi) a.r[i] = o[e];
-          }
         }
       }
     }
@@ -382,17 +475,29 @@ __global__ void __launch_bounds__(kThreads, 4) pass1_kernel(Sel a) {
 // ------------------------------------------------------------------------------------------
 // candidate iteration for the later steps (order not needed)
 
-// Calls f(i, x, c, key) for every candidate of piece q: from the piece's store, or, for pieces
-// marked to be re-read, from the residual (which then holds acc) filtered by class and T_lo.
+// Calls f(x, c, key) for every candidate value of piece q: from the piece's store (values only;
+// two float4 loads per lane in flight), or, for pieces marked to be re-read, from the residual
+// (which then holds acc) filtered by class and T_lo.
 template <int C, class F>
 __device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, const Piece& P, F f) {
   const int lane = threadIdx.x & 31;
   if (!a.prsrc[q]) {
+    // the store of a piece starts 16-byte aligned (cap is a multiple of 4): four per lane
     const uint32_t cnt = a.pcnt[q];
-    for (uint32_t j = lane; j < cnt; j += 32) {
-      const float x = a.cval[q * a.cap + j];
-      const int c = class_of<C>(x);
-      f((int64_t)a.cidx[q * a.cap + j], x, c < 0 ? 0 : c, mag_key(x));
+    const float4* cv = reinterpret_cast<const float4*>(a.cval + q * a.cap);
+    const uint32_t n4 = (cnt + 3) / 4;
+    for (uint32_t j4 = lane; j4 < n4; j4 += 64) {
+      const float4 X0 = cv[j4];
+      const float4 X1 = j4 + 32 < n4 ? cv[j4 + 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float xv[8] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t j = 4 * (j4 + (e >> 2) * 32) + (e & 3);
+        if (j < cnt) {
+          const int c = class_of<C>(xv[e]);
+          f(xv[e], c < 0 ? 0 : c, mag_key(xv[e]));
+        }
+      }
     }
     return;
   }
@@ -417,7 +522,7 @@ __device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, cons
       const int c = class_of<C>(x[e]);
       if (c < 0) continue;
       const uint32_t key = mag_key(x[e]);
-      if (key >= tl[c]) f(i, x[e], c, key);
+      if (key >= tl[c]) f(x[e], c, key);
     }
   }
 }
@@ -471,7 +576,7 @@ __global__ void __launch_bounds__(kThreads) restore_kernel(Sel a) {
       __syncwarp();
       if (redo) {
         // the redone classes count every member (their T_lo is now 0)
-        for_each_candidate<C>(a, q, P, [&](int64_t, float, int c, uint32_t key) {
+        for_each_candidate<C>(a, q, P, [&](float, int c, uint32_t key) {
           if (a.redo[(int64_t)P.s * C + c]) H.add(a, P.s, c, key >> 20, 1);
         });
       }
@@ -548,7 +653,7 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(Sel a, int level) {
     uint32_t pf[C];
 #pragma unroll
     for (int c = 0; c < C; ++c) pf[c] = a.pfx[(int64_t)P.s * C + c];
-    for_each_candidate<C>(a, q, P, [&](int64_t, float, int c, uint32_t key) {
+    for_each_candidate<C>(a, q, P, [&](float, int c, uint32_t key) {
       if (level == 2) {
         if ((key >> 20) == pf[c]) H.add(a, P.s, c, (key >> 9) & 2047u, 2);
       } else {
@@ -576,7 +681,7 @@ __global__ void __launch_bounds__(kThreads) count_kernel(Sel a) {
     gt[c] = 0;
     eq[c] = 0;
   }
-  for_each_candidate<C>(a, q, P, [&](int64_t, float, int c, uint32_t key) {
+  for_each_candidate<C>(a, q, P, [&](float, int c, uint32_t key) {
 #pragma unroll
     for (int cc = 0; cc < C; ++cc) {
       if (cc == c) {
@@ -654,36 +759,67 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(Sel a, int32_t* out_idx,
     return c >= 0 && th[c] != kNone && (key > th[c] || eq_taken);
   };
   if (!a.prsrc[q]) {
+    // the store in index order, four consecutive candidates per lane
     const uint32_t cnt = a.pcnt[q];
-    const int32_t* ci = a.cidx + q * a.cap;
-    const float* cv = a.cval + q * a.cap;
-    for (uint32_t j0 = 0; j0 < cnt; j0 += 32) {
-      const uint32_t j = j0 + lane;
-      const bool valid = j < cnt;
-      const int32_t i = valid ? ci[j] : 0;
-      const float x = valid ? cv[j] : 0.0f;
-      const int c = valid ? class_of<C>(x) : -1;
-      const uint32_t key = mag_key(x);
-      bool sel = false;
-      uint32_t pos = 0;
+    const int4* ci = reinterpret_cast<const int4*>(a.cidx + q * a.cap);
+    const float4* cv = reinterpret_cast<const float4*>(a.cval + q * a.cap);
+    // software pipelined: the next 128 candidates are in flight while these are placed
+    int4 In = make_int4(0, 0, 0, 0);
+    float4 Xn = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (4 * lane < cnt) { In = ci[lane]; Xn = cv[lane]; }
+    for (uint32_t j0 = 0; j0 < cnt; j0 += 128) {
+      const uint32_t j = j0 + 4 * lane;
+      const int4 I = In;
+      const float4 X = Xn;
+      if (j + 128 < cnt) { In = ci[(j >> 2) + 32]; Xn = cv[(j >> 2) + 32]; }
+      int32_t iv[4] = {0, 0, 0, 0};
+      float xv[4] = {0.f, 0.f, 0.f, 0.f};
+      if (j < cnt) {
+        iv[0] = I.x; iv[1] = I.y; iv[2] = I.z; iv[3] = I.w;
+        xv[0] = X.x; xv[1] = X.y; xv[2] = X.z; xv[3] = X.w;
+      }
+      int cls[4];
+      uint32_t key[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        cls[e] = j + e < cnt ? class_of<C>(xv[e]) : -1;
+        key[e] = mag_key(xv[e]);
+      }
+      uint32_t selm = 0;
 #pragma unroll
       for (int cc = 0; cc < C; ++cc) {
-        const bool eq = c == cc && key == th[cc];
-        const uint32_t be = __ballot_sync(kFull, eq);
-        const bool taken = eq && (eq_run[cc] + __popc(be & lt)) < take[cc];
-        const bool s_ = c == cc && is_sel(cc, key, taken);
-        const uint32_t bs = __ballot_sync(kFull, s_);
-        if (s_) { sel = true; pos = sel_run[cc] + __popc(bs & lt); }
-        eq_run[cc] += __popc(be);
-        sel_run[cc] += __popc(bs);
+        uint32_t eqm = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) eqm |= (uint32_t)(cls[e] == cc && key[e] == th[cc]) << e;
+        uint32_t teq;
+        const uint32_t pre_eq = warp_prefix_small(__popc(eqm), &teq);
+        uint32_t sm = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool eq = (eqm >> e) & 1u;
+          const bool taken = eq && (eq_run[cc] + pre_eq + __popc(eqm & ((1u << e) - 1u))) < take[cc];
+          sm |= (uint32_t)(cls[e] == cc && is_sel(cc, key[e], taken)) << e;
+        }
+        uint32_t tsel;
+        const uint32_t pre_sel = warp_prefix_small(__popc(sm), &tsel);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if ((sm >> e) & 1u) {
+            const int64_t o = base_out[cc] + sel_run[cc] + pre_sel + __popc(sm & ((1u << e) - 1u));
+            if (o >= limit) raise(a.d_status, GSPARSE_DERR_CAPACITY);
+            else if (C == 1) { out_idx[o] = iv[e]; out_val[o] = xv[e]; }
+            else { a.lidx[o] = iv[e]; a.lval[o] = xv[e]; }
+          }
+        }
+        eq_run[cc] += teq;
+        sel_run[cc] += tsel;
+        selm |= sm;
       }
-      if (sel) {
-        const int64_t o = base_out[c] + pos;
-        if (o >= limit) raise(a.d_status, GSPARSE_DERR_CAPACITY);
-        else if (C == 1) { out_idx[o] = i; out_val[o] = x; }
-        else { a.lidx[o] = i; a.lval[o] = x; }
-      } else if (valid && a.zero_mode) {
-        a.r[i] = x;  // a candidate that is not sent keeps its acc in the residual
+      if (a.zero_mode) {
+        // a candidate that is not sent keeps its acc in the residual
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (j + e < cnt && !((selm >> e) & 1u)) a.r[iv[e]] = xv[e];
       }
     }
     return;
@@ -864,7 +1000,7 @@ int64_t k_bound(int64_t n, int32_t T, int64_t num, int64_t den) {
 
 int64_t rec_cap(int64_t Lp, int32_t C, int64_t num, int64_t den) {
   const double q = den > 0 ? (double)num / (double)den : 1.0;
-  const double f = q + 4.0 * sqrt(q / kSample) + 8.0 / kSample;
+  const double f = q + 3.0 * sqrt(q / kSample) + 16.0 / kSample;
   double cap = ceil((double)Lp * f * C * 1.25) + 64.0;
   if (cap > (double)Lp) cap = (double)Lp;
   return round_up((int64_t)cap, 32);
@@ -904,7 +1040,12 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
   a.pcnt = cv.take<uint32_t>(L.Q);
   a.prsrc = cv.take<uint32_t>(L.Q);
   a.hist = cv.take<uint32_t>(P * kHist);
+  a.shist = cv.take<uint32_t>(P * 2 * kBins1);
+  a.scount = cv.take<uint32_t>(P);
+  a.sdone = cv.take<uint32_t>(2 * (int64_t)T);
   const size_t zend = cv.off;
+  a.sb1 = cv.take<uint32_t>(P);
+  a.srank = cv.take<int64_t>(P);
   L.zero_begin = ws ? (char*)ws + zoff : nullptr;
   L.zero_bytes = zend - zoff;
   if (C == 2) {
@@ -925,7 +1066,7 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
     cap = L.cap_rec;
   } else {
     const int64_t room = ws_bytes > L.fixed_bytes ? (int64_t)(ws_bytes - L.fixed_bytes) : 0;
-    cap = room / (L.Q * 8 > 0 ? L.Q * 8 : 1);
+    cap = (room / (L.Q * 8 > 0 ? L.Q * 8 : 1)) & ~(int64_t)3;  // int4-aligned per-piece stores
     if (cap > L.Lp) cap = L.Lp;
   }
   L.cap = cap;
@@ -976,17 +1117,10 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
     return launch_status();
   }
   const unsigned piece_ctas = (unsigned)cdiv(L.Q, kWarps);
-  const size_t sample_smem = (size_t)C * kSample * sizeof(uint32_t);
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GSPARSE_ERR_CUDA;
-  static bool attr_set[2][64] = {};
-  if (dev < 64 && !attr_set[C - 1][dev]) {
-    if (cudaFuncSetAttribute(sample_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sample_smem) != cudaSuccess)
-      return GSPARSE_ERR_CUDA;
-    attr_set[C - 1][dev] = true;
-  }
-  sample_kernel<C><<<T, 1024, sample_smem, st>>>(a, (flags & GSPARSE_SELECT_EXHAUSTIVE) ? 1 : 0);
+  const int exhaustive = (flags & GSPARSE_SELECT_EXHAUSTIVE) ? 1 : 0;
+  const dim3 sgrid(kSampleCtas, (unsigned)T);
+  sample_kernel<C><<<sgrid, 256, 0, st>>>(a, 1, exhaustive);
+  sample_kernel<C><<<sgrid, 256, 0, st>>>(a, 2, exhaustive);
   const bool timed = g_pass1_before && g_pass1_after;
   if (timed) cudaEventRecord(g_pass1_before, st);
   if (piece_ctas) pass1_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
