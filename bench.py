@@ -6,8 +6,8 @@ Laplace(0, 1e-1) outliers, W = 2 workers resident on one GPU, residual carried f
 One step:
   per worker: residual top-k at a 99% drop (keep 1/100) -> 2-bit quantisation with the error fed
               back into the residual -> Golomb encode (b* = 6) -> Golomb decode
-  then:       scatter-accumulate of the W decoded updates into the dense global sum G
-              -> combination with each worker's own gradient (out_w = G + g_w)
+  then, per worker (the receive side): the worker-ordered sum G of the W decoded updates combined
+              with the worker's own gradient, out_w = G + g_w, in one fused pass that never writes G
 Metric: gradient GB/s compressed = W * 4 * n bytes per step / step time (whole job over all
 ranks), with the residual-top-k call's share of HBM bandwidth reported beside it.
 
@@ -45,7 +45,7 @@ def workload_config(n, workers, drop, b, extra=None):
     cfg = {"workload": f"flat fp32 gradient of {n} entries per worker, Laplace(0,1e-3) with 0.1% "
                        f"Laplace(0,1e-1) outliers, {workers} workers on one GPU, residual carried",
            "n": n, "workers": workers, "drop": drop, "keep": f"1/{round(1 / (1 - drop))}",
-           "golomb_b": b, "step": "topk+quantise+golomb enc/dec per worker, scatter-accumulate, combine",
+           "golomb_b": b, "step": "per worker: topk+quantise+golomb enc/dec; per worker: fused accumulate+combine",
            "l2": "inputs larger than L2 (8 GiB of gradients + 8 GiB of residuals per step)"}
     if extra:
         cfg.update(extra)
@@ -169,13 +169,12 @@ def run_ours(args, rank, world, dist):
     nbits = [torch.zeros(1, dtype=torch.int64, device=dev) for _ in range(W)]
     table = [torch.empty(((cap + chunk - 1) // chunk, 2), dtype=torch.int64, device=dev) for _ in range(W)]
     dec = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(W)]
-    G = torch.empty(n, dtype=torch.float32, device=dev)
     out = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(W)]
     ws_t = [torch.empty(gs.residual_topk_workspace_size(n, 1, keep), dtype=torch.uint8, device=dev) for _ in range(W)]
     ws_q = [torch.empty(gs.lib().gsparse_quantize_workspace_size(cap), dtype=torch.uint8, device=dev) for _ in range(W)]
     ws_g = [torch.empty(gs.lib().gsparse_golomb_encode_workspace_size(cap), dtype=torch.uint8, device=dev)
             for _ in range(W)]
-    ws_s = torch.empty(gs.lib().gsparse_scatter_accumulate_workspace_size(W, n), dtype=torch.uint8, device=dev)
+    ws_s = torch.empty(gs.lib().gsparse_accumulate_combine_workspace_size(W, n), dtype=torch.uint8, device=dev)
     st = gs.status_tensor(dev)
     lists = [gs.make_list(dec[w], end[w], val=val[w], capacity=cap) for w in range(W)]
     # payload read back in the end-to-end leg: Golomb words, sign bits, means, bit count
@@ -185,7 +184,7 @@ def run_ours(args, rank, world, dist):
     h2d_bytes = W * n * 4
 
     stage_names = ["residual_topk", "quantize", "golomb_encode", "golomb_decode"]
-    stage_ms = {k: [] for k in stage_names + ["scatter_accumulate", "combine_local"]}
+    stage_ms = {k: [] for k in stage_names + ["receive"]}
     pass1_ms = []
 
     def step(events=None, p1=None):
@@ -209,13 +208,11 @@ def run_ours(args, rank, world, dist):
             gs.golomb_decode(words[w], nbits[w], end[w], cap, b, table=table[w], chunk=chunk, n_limit=n,
                              out_idx=dec[w], d_status=st)
         rec()
-        gs.scatter_accumulate(lists, n, dense_out=G, workspace=ws_s, d_status=st, device=dev)
-        rec()
         for w in range(W):
-            gs.combine_local(G, g[w], out=out[w])
+            gs.accumulate_combine(lists, n, g[w], out=out[w], workspace=ws_s, d_status=st)
         rec()
 
-    n_ev = 4 * W + 3
+    n_ev = 4 * W + 2
 
     def new_events(k):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(k)]
@@ -254,8 +251,7 @@ def run_ours(args, rank, world, dist):
             for s, name in enumerate(stage_names):
                 stage_ms[name].append(e[4 * w + s].elapsed_time(e[4 * w + s + 1]))
             pass1_ms.append(p1[k][w][0].elapsed_time(p1[k][w][1]))
-        stage_ms["scatter_accumulate"].append(e[4 * W].elapsed_time(e[4 * W + 1]))
-        stage_ms["combine_local"].append(e[4 * W + 1].elapsed_time(e[4 * W + 2]))
+        stage_ms["receive"].append(e[4 * W].elapsed_time(e[4 * W + 1]))
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} in the timed region")
 

@@ -61,6 +61,9 @@ _SIGNATURES = {
     "gsparse_scatter_accumulate_workspace_size": (_sz, [_i32, _i64]),
     "gsparse_scatter_accumulate": (ctypes.c_int, [ctypes.POINTER(GsparseList), _i32, _i64, _vp, _vp, _vp, _vp,
                                                   _i64, _vp, _sz, _vp, _vp]),
+    "gsparse_accumulate_combine_workspace_size": (_sz, [_i32, _i64]),
+    "gsparse_accumulate_combine": (ctypes.c_int, [ctypes.POINTER(GsparseList), _i32, _i64, _vp, _vp, _f32, _f32,
+                                                  _i32, _i32, _vp, _vp, _sz, _vp, _vp]),
     "gsparse_combine_local": (ctypes.c_int, [_vp, _vp, _vp, _i64, _f32, _f32, _i32, _vp, _vp, _vp, _i64, _vp,
                                              _vp]),
 }
@@ -339,6 +342,23 @@ def scatter_accumulate(lists: Sequence[GsparseList], n: int, dense_out: Optional
                                           _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev))
     _check(st, "gsparse_scatter_accumulate")
     return dense_out, mi, mv, mc
+
+
+def accumulate_combine(lists: Sequence[GsparseList], n: int, L: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       alpha: float = 1.0, beta: float = 1.0, mode: int = 0, own: int = -1,
+                       dense_out: Optional[torch.Tensor] = None, workspace=None, d_status=None):
+    """Fused receive side: out = combine(scatter_accumulate(lists), L) without materialising G."""
+    W = len(lists)
+    arr = (GsparseList * W)(*lists)
+    dev = L.device
+    if out is None:
+        out = torch.empty_like(L)
+    if workspace is None:
+        workspace = _workspace(lib().gsparse_accumulate_combine_workspace_size(W, n), dev)
+    st = lib().gsparse_accumulate_combine(arr, W, n, _ptr(L), _ptr(out), alpha, beta, mode, own, _ptr(dense_out),
+                                          _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev))
+    _check(st, "gsparse_accumulate_combine")
+    return out
 
 
 def combine_local(G: torch.Tensor, L: torch.Tensor, out: Optional[torch.Tensor] = None, alpha: float = 1.0,

@@ -150,6 +150,60 @@ __global__ void __launch_bounds__(kTileThreads) sa_merge_kernel(Lists L, int32_t
   }
 }
 
+// Fused receive side: per tile, the worker-ordered sum G lives only in shared memory and the
+// combined gradient is streamed out directly (G itself is written only when asked for).
+__global__ void __launch_bounds__(kTileThreads) sa_combine_kernel(Lists L, int32_t W, int64_t n,
+                                                                  const int64_t* start, const float* Lg,
+                                                                  float* out, float alpha, float beta,
+                                                                  int32_t own, float* dense,
+                                                                  int32_t* d_status) {
+  __shared__ __align__(16) float acc[kTile];
+  __shared__ uint32_t touched[kTile / 32];
+  const int64_t t = blockIdx.x;
+  for (int i = threadIdx.x; i < kTile; i += blockDim.x) acc[i] = 0.0f;
+  for (int i = threadIdx.x; i < kTile / 32; i += blockDim.x) touched[i] = 0u;
+  __syncthreads();
+  accumulate_tile(L, W, t, start, acc, touched, d_status);
+  const int64_t t0 = t * kTile;
+  const int64_t m = (n - t0) < kTile ? (n - t0) : kTile;
+  if (dense) {
+    if (m == kTile) {
+      for (int v = threadIdx.x; v < kTile / 4; v += blockDim.x)
+        st_stream(dense + t0 + 4 * v, reinterpret_cast<const float4*>(acc)[v]);
+    } else {
+      for (int i = threadIdx.x; i < m; i += blockDim.x) dense[t0 + i] = acc[i];
+    }
+  }
+  if (own >= 0) {
+    // partial mode: the worker's own sent values leave G before the combination
+    __syncthreads();
+    const int64_t b = start[t * W + own], e = start[(t + 1) * W + own];
+    const int32_t* ix = L.idx[own];
+    const float* vv = L.val[own];
+    const float u = (vv || !L.uni[own]) ? 0.0f : *L.uni[own];
+    for (int64_t j = b + threadIdx.x; j < e; j += blockDim.x) {
+      const int off = (int)(ix[j] - t0);
+      if (off >= 0 && off < kTile) acc[off] = __fsub_rn(acc[off], vv ? vv[j] : u);
+    }
+    __syncthreads();
+  }
+  if (m == kTile) {
+    for (int v = threadIdx.x; v < kTile / 4; v += blockDim.x) {
+      const float4 g = reinterpret_cast<const float4*>(acc)[v];
+      const float4 l = ld_stream(Lg + t0 + 4 * v);
+      float4 o;
+      o.x = __fadd_rn(__fmul_rn(alpha, g.x), __fmul_rn(beta, l.x));
+      o.y = __fadd_rn(__fmul_rn(alpha, g.y), __fmul_rn(beta, l.y));
+      o.z = __fadd_rn(__fmul_rn(alpha, g.z), __fmul_rn(beta, l.z));
+      o.w = __fadd_rn(__fmul_rn(alpha, g.w), __fmul_rn(beta, l.w));
+      st_stream(out + t0 + 4 * v, o);
+    }
+  } else {
+    for (int i = threadIdx.x; i < m; i += blockDim.x)
+      out[t0 + i] = __fadd_rn(__fmul_rn(alpha, acc[i]), __fmul_rn(beta, Lg[t0 + i]));
+  }
+}
+
 // ---------------------------------------------------------------------------------------------
 // combine
 
@@ -260,6 +314,43 @@ int gsparse_scatter_accumulate(const gsparse_list* lists, int32_t W, int64_t n, 
     sa_merge_kernel<<<(unsigned)ntiles, kTileThreads, 0, st>>>(L, W, S.start, S.tile_count,
                                                                merged_idx, merged_val, S.ctl);
   }
+  return launch_status();
+}
+
+size_t gsparse_accumulate_combine_workspace_size(int32_t W, int64_t n) {
+  return gsparse_scatter_accumulate_workspace_size(W, n);
+}
+
+int gsparse_accumulate_combine(const gsparse_list* lists, int32_t W, int64_t n, const float* L,
+                               float* out, float alpha, float beta, int32_t mode, int32_t own,
+                               float* dense_out, void* workspace, size_t workspace_bytes,
+                               int32_t* d_status, gsparse_stream stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!lists || W < 1 || n < 0 || (mode != 0 && mode != 1)) return GSPARSE_ERR_INVALID_ARG;
+  if (W > GSPARSE_MAX_WORKERS || n > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
+  if (mode == 1 && (own < 0 || own >= W)) return GSPARSE_ERR_INVALID_ARG;
+  if (n > 0 && (!L || !out || !aligned16(L) || !aligned16(out))) return GSPARSE_ERR_INVALID_ARG;
+  if (dense_out && !aligned16(dense_out)) return GSPARSE_ERR_INVALID_ARG;
+  Lists Ls{};
+  for (int w = 0; w < W; ++w) {
+    const gsparse_list& x = lists[w];
+    if (!x.d_count || x.capacity < 0 || (x.capacity > 0 && (!x.idx || (!x.val && !x.uniform_val))))
+      return GSPARSE_ERR_INVALID_ARG;
+    Ls.idx[w] = x.idx;
+    Ls.val[w] = x.val;
+    Ls.uni[w] = x.uniform_val;
+    Ls.cnt[w] = x.d_count;
+    Ls.cap[w] = x.capacity;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GSPARSE_ERR_WORKSPACE;
+  SLayout S = s_carve(W, n, workspace);
+  if (workspace_bytes < S.bytes) return GSPARSE_ERR_WORKSPACE;
+  const int64_t ntiles = cdiv(n, kTile);
+  if (ntiles == 0) return launch_status();
+  const int64_t nb = (ntiles + 1) * W;
+  sa_bounds_kernel<<<(unsigned)cdiv(nb, 256), 256, 0, st>>>(Ls, W, n, ntiles, S.start, d_status);
+  sa_combine_kernel<<<(unsigned)ntiles, kTileThreads, 0, st>>>(Ls, W, n, S.start, L, out, alpha, beta,
+                                                               mode == 1 ? own : -1, dense_out, d_status);
   return launch_status();
 }
 

@@ -265,6 +265,25 @@ int gsparse_scatter_accumulate(const gsparse_list* lists, int32_t W, int64_t n, 
                                int32_t* d_status, gsparse_stream stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Receive side in one pass: scatter-accumulate fused with the combination  (Aji, Heafield &
+ * Bogoychev 2019, Abstract)
+ *
+ * out = the result of gsparse_combine_local(G, L, out, n, alpha, beta, mode, own list) with G the
+ * result of gsparse_scatter_accumulate(lists, W, n), bit for bit, without writing G to memory:
+ * per tile of 8192 indices the worker-ordered sum is formed in shared memory and the combined
+ * gradient streamed out, so the call moves 8n bytes plus the lists instead of 20n.
+ * mode 0: out_i = fl(fl(alpha * G_i) + fl(beta * L_i)); mode 1: G_i becomes fl(G_i - s_i) on the
+ * entries of lists[own] (the worker's own sent update) first.
+ * L, out fp32[n], 16-byte aligned, not aliased with each other. dense_out fp32[n] or NULL: also
+ * receives G. Device errors as for gsparse_scatter_accumulate.
+ */
+size_t gsparse_accumulate_combine_workspace_size(int32_t W, int64_t n);
+int gsparse_accumulate_combine(const gsparse_list* lists, int32_t W, int64_t n, const float* L,
+                               float* out, float alpha, float beta, int32_t mode, int32_t own,
+                               float* dense_out, void* workspace, size_t workspace_bytes,
+                               int32_t* d_status, gsparse_stream stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Combination with the local gradient  (Aji, Heafield & Bogoychev 2019, Abstract)
  *
  * mode 0 (sum):     out_i = fl(fl(alpha * G_i) + fl(beta * L_i))

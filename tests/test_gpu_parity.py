@@ -350,3 +350,38 @@ def test_combine_parity(n):
     got = gs.combine_local(dev(G), dev(L), mode=1, own_idx=dev(own_idx), own_val=dev(own_val),
                            own_count=torch.tensor([k], device="cuda"), own_capacity=k)
     assert np.array_equal(bits(host(got)), bits(want))
+
+
+# ------------------------------------------------------------------------------------ fused receive
+
+@pytest.mark.parametrize("W", [1, 2, 4, 8])
+@pytest.mark.parametrize("n", [3, 8192, 8193, 200003])
+def test_accumulate_combine_parity(W, n):
+    gen = np.random.default_rng(77 * W + n)
+    host_lists, lists, keep = [], [], []
+    for w in range(W):
+        k = int(min(n, gen.integers(1, max(n // 10, 2) + 1)))
+        idx = np.sort(gen.choice(n, k, replace=False)).astype(np.int32)
+        val = synth.gaussian(k, 40 + w, sigma=1e-2)
+        cnt = torch.tensor([k], dtype=torch.int64, device="cuda")
+        t = (dev(idx), cnt, dev(val))
+        keep.append(t)
+        host_lists.append((idx, val))
+        lists.append(gs.make_list(t[0], cnt, val=t[2], capacity=k))
+    Lh = synth.gaussian(n, 5, sigma=1e-2)
+    L = dev(Lh)
+    wd, _, _ = oracle.scatter_accumulate(host_lists, n, merged=False)
+    for alpha, beta in [(1.0, 1.0), (0.25, 0.75)]:
+        for mode in (0, 1):
+            own = W - 1 if mode == 1 else -1
+            kw = {} if mode == 0 else {"own_idx": host_lists[own][0], "own_val": host_lists[own][1]}
+            want = oracle.combine_local(wd, Lh, alpha, beta, mode=mode, **kw)
+            dense = torch.empty(n, device="cuda")
+            st = gs.status_tensor()
+            out = gs.accumulate_combine(lists, n, L, alpha=alpha, beta=beta, mode=mode, own=own, dense_out=dense,
+                                        d_status=st)
+            assert int(host(st)[0]) == 0
+            assert np.array_equal(bits(host(out)), bits(want))
+            assert np.array_equal(bits(host(dense)), bits(wd))
+            out2 = gs.accumulate_combine(lists, n, L, alpha=alpha, beta=beta, mode=mode, own=own)
+            assert np.array_equal(bits(host(out2)), bits(want))
