@@ -4,8 +4,9 @@
 Workload: a flat fp32 gradient of 2^30 entries (4 GiB) per worker, Laplace(0, 1e-3) with 0.1%
 Laplace(0, 1e-1) outliers, W = 2 workers resident on one GPU, residual carried from step to step.
 One step:
-  per worker: residual top-k at a 99% drop (keep 1/100) -> 2-bit quantisation with the error fed
-              back into the residual -> Golomb encode (b* = 6) -> Golomb decode
+  per worker: residual top-k at a 99% drop (keep 1/100), which first applies the previous step's
+              quantisation error to the residual -> 2-bit quantisation (its error kept as a list for
+              the next step) -> Golomb encode (b* = 6) -> Golomb decode
   then, per worker (the receive side): the worker-ordered sum G of the W decoded updates combined
               with the worker's own gradient, out_w = G + g_w, in one fused pass that never writes G
 Metric: gradient GB/s compressed = W * 4 * n bytes per step / step time (whole job over all
@@ -158,10 +159,14 @@ def run_ours(args, rank, world, dist):
         g_host.append(t)
     g = [t.to(dev) for t in g_host]
     r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)]
-    idx = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(W)]
-    val = [torch.empty(cap, dtype=torch.float32, device=dev) for _ in range(W)]
-    off = [torch.empty(2, dtype=torch.int64, device=dev) for _ in range(W)]
-    end = [o[1:2] for o in off]
+    # sent lists alternate between two buffers: step t applies step t-1's quantisation error
+    idx2 = [[torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(W)] for _ in range(2)]
+    val2 = [[torch.empty(cap, dtype=torch.float32, device=dev) for _ in range(W)] for _ in range(2)]
+    fb2 = [[torch.empty(cap, dtype=torch.float32, device=dev) for _ in range(W)] for _ in range(2)]
+    off2 = [[torch.zeros(2, dtype=torch.int64, device=dev) for _ in range(W)] for _ in range(2)]
+    pend2 = [[gs.make_pending(idx2[p][w], fb2[p][w], off2[p][w][1:2], capacity=cap) for w in range(W)]
+             for p in range(2)]
+    parity = [0]
     sb = [torch.empty((cap + 31) // 32, dtype=torch.int32, device=dev) for _ in range(W)]
     means = [torch.empty(2, dtype=torch.float32, device=dev) for _ in range(W)]
     nwords = gs.golomb_word_capacity(cap, b, n)
@@ -176,9 +181,10 @@ def run_ours(args, rank, world, dist):
             for _ in range(W)]
     ws_s = torch.empty(gs.lib().gsparse_accumulate_combine_workspace_size(W, n), dtype=torch.uint8, device=dev)
     st = gs.status_tensor(dev)
-    lists = [gs.make_list(dec[w], end[w], val=val[w], capacity=cap) for w in range(W)]
+    lists2 = [[gs.make_list(dec[w], off2[p][w][1:2], val=val2[p][w], capacity=cap) for w in range(W)]
+              for p in range(2)]
     # payload read back in the end-to-end leg: Golomb words, sign bits, means, bit count
-    payload = [(words[w], sb[w], means[w], nbits[w], off[w]) for w in range(W)]
+    payload = [(words[w], sb[w], means[w], nbits[w], off2[0][w], off2[1][w]) for w in range(W)]
     payload_host = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in p] for p in payload]
     d2h_bytes = sum(t.numel() * t.element_size() for p in payload for t in p)
     h2d_bytes = W * n * 4
@@ -190,26 +196,30 @@ def run_ours(args, rank, world, dist):
     def step(events=None, p1=None):
         e = iter(events) if events is not None else None
         rec = (lambda: next(e).record()) if e is not None else (lambda: None)
+        cur, prev = parity[0], 1 - parity[0]
+        parity[0] = prev
         for w in range(W):
+            idx, val, off, fb = idx2[cur][w], val2[cur][w], off2[cur][w], fb2[cur][w]
+            end = off[1:2]
             rec()
             if p1 is not None:
                 gs.set_pass1_events(p1[w][0], p1[w][1])
-            gs.residual_topk(g[w], r[w], keep, out_idx=idx[w], out_val=val[w], out_offsets=off[w],
-                             workspace=ws_t[w], d_status=st, capacity=cap)
+            gs.residual_topk(g[w], r[w], keep, out_idx=idx, out_val=val, out_offsets=off, workspace=ws_t[w],
+                             d_status=st, capacity=cap, pending=pend2[prev][w])
             if p1 is not None:
                 gs.set_pass1_events(None, None)
             rec()
-            gs.quantize(idx[w], val[w], end[w], residual=r[w], write_dequantized=True, sign_bits=sb[w],
-                        means=means[w], workspace=ws_q[w], d_status=st, capacity=cap)
+            gs.quantize(idx, val, end, write_dequantized=True, feedback_out=fb, sign_bits=sb[w], means=means[w],
+                        workspace=ws_q[w], d_status=st, capacity=cap)
             rec()
-            gs.golomb_encode(idx[w], end[w], b, n, chunk=chunk, words=words[w], nbits=nbits[w], table=table[w],
+            gs.golomb_encode(idx, end, b, n, chunk=chunk, words=words[w], nbits=nbits[w], table=table[w],
                              workspace=ws_g[w], d_status=st, capacity=cap)
             rec()
-            gs.golomb_decode(words[w], nbits[w], end[w], cap, b, table=table[w], chunk=chunk, n_limit=n,
+            gs.golomb_decode(words[w], nbits[w], end, cap, b, table=table[w], chunk=chunk, n_limit=n,
                              out_idx=dec[w], d_status=st)
         rec()
         for w in range(W):
-            gs.accumulate_combine(lists, n, g[w], out=out[w], workspace=ws_s, d_status=st)
+            gs.accumulate_combine(lists2[cur], n, g[w], out=out[w], workspace=ws_s, d_status=st)
         rec()
 
     n_ev = 4 * W + 2
@@ -254,6 +264,8 @@ def run_ours(args, rank, world, dist):
         stage_ms["receive"].append(e[4 * W].elapsed_time(e[4 * W + 1]))
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} in the timed region")
+    if getattr(args, "step_hook", None) is not None:
+        args.step_hook(step, dev)
 
     # kernels of this library launched per step, counted by the CUDA profiler on one extra step
     launches_per_step = None

@@ -31,6 +31,10 @@ class GsparseError(RuntimeError):
     pass
 
 
+class GsparsePending(ctypes.Structure):
+    _fields_ = [("idx", _vp), ("val", _vp), ("d_count", _vp), ("capacity", _i64)]
+
+
 class GsparseList(ctypes.Structure):
     _fields_ = [("idx", _vp), ("val", _vp), ("uniform_val", _vp), ("d_count", _vp), ("capacity", _i64)]
 
@@ -44,11 +48,12 @@ _SIGNATURES = {
     "gsparse_golomb_b_star": (_i32, [_f64]),
     "gsparse_residual_topk_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_residual_topk_workspace_min": (_sz, [_i64, _i32]),
-    "gsparse_residual_topk": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _i64, _u32,
-                                             _vp, _sz, _vp, _vp]),
+    "gsparse_residual_topk": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _i64,
+                                             ctypes.POINTER(GsparsePending), _u32, _vp, _sz, _vp, _vp]),
     "gsparse_residual_topk_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp]),
     "gsparse_quantize_workspace_size": (_sz, [_i64]),
-    "gsparse_quantize": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp, _sz, _vp, _vp]),
+    "gsparse_quantize": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _sz, _vp,
+                                        _vp]),
     "gsparse_binarize_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_binarize_workspace_min": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_binarize": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _u32,
@@ -150,9 +155,11 @@ def residual_topk_capacity(n: int, seg_sizes: Optional[Sequence[int]], keep) -> 
 def residual_topk(g: torch.Tensor, residual: torch.Tensor, keep=(1, 100), seg_offsets: Optional[torch.Tensor] = None,
                   out_idx: Optional[torch.Tensor] = None, out_val: Optional[torch.Tensor] = None,
                   out_offsets: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                  flags: int = 0, d_status: Optional[torch.Tensor] = None, capacity: Optional[int] = None):
+                  flags: int = 0, d_status: Optional[torch.Tensor] = None, capacity: Optional[int] = None,
+                  pending: Optional[GsparsePending] = None):
     """residual <- acc with the sent entries zeroed. Returns (idx, val, offsets) device tensors;
-    idx/val hold `capacity` slots of which offsets[-1] are used."""
+    idx/val hold `capacity` slots of which offsets[-1] are used. `pending` (make_pending) are
+    residual writes applied first."""
     _dev(g, torch.float32, "g")
     _dev(residual, torch.float32, "residual")
     n = g.numel()
@@ -170,8 +177,9 @@ def residual_topk(g: torch.Tensor, residual: torch.Tensor, keep=(1, 100), seg_of
         out_offsets = torch.empty(T + 1, dtype=torch.int64, device=dev)
     if workspace is None:
         workspace = _workspace(residual_topk_workspace_size(n, T, keep), dev)
+    pend = ctypes.byref(pending) if pending is not None else None
     st = lib().gsparse_residual_topk(_ptr(g), _ptr(residual), n, _ptr(seg_offsets), T, keep[0], keep[1],
-                                     _ptr(out_idx), _ptr(out_val), _ptr(out_offsets), capacity, flags,
+                                     _ptr(out_idx), _ptr(out_val), _ptr(out_offsets), capacity, pend, flags,
                                      _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev))
     _check(st, "gsparse_residual_topk")
     return out_idx, out_val, out_offsets
@@ -209,8 +217,16 @@ def residual_topk_noalloc(g: torch.Tensor, residual: torch.Tensor, keep=(1, 100)
 # ---------------------------------------------------------------------------------------------
 # quantise
 
+def make_pending(idx: torch.Tensor, val: torch.Tensor, d_count: torch.Tensor,
+                 capacity: Optional[int] = None) -> GsparsePending:
+    """Residual writes residual[idx_j] <- val_j for the next residual_topk (e.g. quantize's feedback)."""
+    cap = idx.numel() if capacity is None else capacity
+    return GsparsePending(_ptr(idx), _ptr(val), _ptr(d_count), cap)
+
+
 def quantize(idx: torch.Tensor, val: torch.Tensor, d_end: torch.Tensor, d_begin: Optional[torch.Tensor] = None,
              residual: Optional[torch.Tensor] = None, write_dequantized: bool = False,
+             feedback_out: Optional[torch.Tensor] = None,
              sign_bits: Optional[torch.Tensor] = None, means: Optional[torch.Tensor] = None,
              workspace: Optional[torch.Tensor] = None, d_status: Optional[torch.Tensor] = None,
              capacity: Optional[int] = None):
@@ -225,8 +241,8 @@ def quantize(idx: torch.Tensor, val: torch.Tensor, d_end: torch.Tensor, d_begin:
         workspace = _workspace(lib().gsparse_quantize_workspace_size(capacity), dev)
     n = 0 if residual is None else residual.numel()
     st = lib().gsparse_quantize(_ptr(idx), _ptr(val), _ptr(d_begin), _ptr(d_end), capacity, _ptr(residual), n,
-                                _ptr(sign_bits), _ptr(means), int(write_dequantized), _ptr(workspace),
-                                workspace.numel(), _ptr(d_status), _stream(dev))
+                                _ptr(feedback_out), _ptr(sign_bits), _ptr(means), int(write_dequantized),
+                                _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev))
     _check(st, "gsparse_quantize")
     return sign_bits, means
 

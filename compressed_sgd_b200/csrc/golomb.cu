@@ -16,6 +16,9 @@ namespace gs {
 namespace {
 
 constexpr int kScanThreads = 1024;
+constexpr int kPer = 4;                      // codewords per thread
+constexpr int kCodeThreads = 256;
+constexpr int kBlockCodes = kPer * kCodeThreads;  // codewords per block of the length and pack passes
 
 struct GCtl {
   int64_t begin, len;
@@ -24,7 +27,7 @@ struct GCtl {
 };
 
 __global__ void g_setup_kernel(const int64_t* d_begin, const int64_t* d_end, int64_t capacity,
-                               GCtl* ctl, int32_t* d_status) {
+                               GCtl* ctl, GCtl* wctl, int32_t* d_status) {
   const int64_t b = d_begin ? *d_begin : 0;
   const int64_t len = *d_end - b;
   if (b < 0 || len < 0 || len > capacity) {
@@ -36,31 +39,45 @@ __global__ void g_setup_kernel(const int64_t* d_begin, const int64_t* d_end, int
     ctl->len = len;
   }
   ctl->begin = b;
+  wctl->abort = 0;
 }
 
-// codeword length of entry j (validating the gap)
-__device__ __forceinline__ uint64_t code_len(const int32_t* idx, int64_t j, int64_t base, int b,
-                                             int32_t* d_status) {
-  const int64_t prev = j == 0 ? base - 1 : (int64_t)idx[j - 1];
-  int64_t d = (int64_t)idx[j] - prev - 1;
-  if (d < 0) {
-    raise(d_status, GSPARSE_DERR_INDEX_RANGE);
-    d = 0;
+// Gaps of this thread's kPer consecutive codewords (entries j0 .. j0+kPer-1 of the list); an
+// invalid (negative) gap is reported and coded as 0.
+__device__ __forceinline__ void thread_gaps(const int32_t* x, int64_t len, int64_t base, int64_t j0,
+                                            int64_t (&d)[kPer], int32_t* d_status) {
+  int64_t prev = j0 == 0 ? base - 1 : (j0 - 1 < len ? (int64_t)x[j0 - 1] : 0);
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int64_t j = j0 + e;
+    d[e] = 0;
+    if (j < len) {
+      const int64_t cur = x[j];
+      d[e] = cur - prev - 1;
+      if (d[e] < 0) {
+        if (d_status) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
+        d[e] = 0;
+      }
+      prev = cur;
+    }
   }
-  return (uint64_t)(d >> b) + 1u + (uint64_t)b;
 }
 
 // per-block totals of the codeword lengths
-__global__ void __launch_bounds__(kScanThreads) g_len_kernel(const int32_t* idx, const GCtl* ctl,
+__global__ void __launch_bounds__(kCodeThreads) g_len_kernel(const int32_t* idx, const GCtl* ctl,
                                                               int64_t base, int b, int64_t* block_tot,
                                                               int32_t* d_status) {
   __shared__ int64_t sh[33];
   if (ctl->abort) return;
   const int64_t len = ctl->len;
-  const int32_t* x = idx + ctl->begin;
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if ((int64_t)blockIdx.x * blockDim.x >= len) return;
-  const int64_t l = j < len ? (int64_t)code_len(x, j, base, b, d_status) : 0;
+  if ((int64_t)blockIdx.x * kBlockCodes >= len) return;
+  const int64_t j0 = (int64_t)blockIdx.x * kBlockCodes + (int64_t)threadIdx.x * kPer;
+  int64_t d[kPer];
+  thread_gaps(idx + ctl->begin, len, base, j0, d, d_status);
+  int64_t l = 0;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e)
+    if (j0 + e < len) l += (d[e] >> b) + 1 + b;
   int64_t tot;
   block_exclusive_scan(l, sh, &tot);
   if (threadIdx.x == 0) block_tot[blockIdx.x] = tot;
@@ -78,7 +95,7 @@ __global__ void __launch_bounds__(kScanThreads) g_scan_blocks_kernel(int64_t* bl
     if (threadIdx.x == 0) *d_nbits = 0;
     return;
   }
-  const int64_t nblk = cdiv(ctl->len, kScanThreads);
+  const int64_t nblk = cdiv(ctl->len, kBlockCodes);
   int64_t carry = 0;
   for (int64_t base = 0; base < nblk; base += blockDim.x) {
     const int64_t i = base + threadIdx.x;
@@ -93,31 +110,6 @@ __global__ void __launch_bounds__(kScanThreads) g_scan_blocks_kernel(int64_t* bl
     if (cdiv(carry, 32) > word_capacity) {
       raise(d_status, GSPARSE_DERR_CAPACITY);
       wctl->abort = 1;
-    }
-  }
-}
-
-// bit offset of every codeword, and the side table
-__global__ void __launch_bounds__(kScanThreads) g_offsets_kernel(const int32_t* idx, const GCtl* ctl,
-                                                                  int64_t base, int b,
-                                                                  const int64_t* block_pre,
-                                                                  uint64_t* offs, int64_t* table,
-                                                                  int32_t chunk) {
-  __shared__ int64_t sh[33];
-  if (ctl->abort) return;
-  const int64_t len = ctl->len;
-  const int32_t* x = idx + ctl->begin;
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if ((int64_t)blockIdx.x * blockDim.x >= len) return;
-  const int64_t l = j < len ? (int64_t)code_len(x, j, base, b, nullptr) : 0;
-  int64_t tot;
-  const int64_t ex = block_exclusive_scan(l, sh, &tot);
-  if (j < len) {
-    const int64_t o = block_pre[blockIdx.x] + ex;
-    offs[j] = (uint64_t)o;
-    if (table && j % chunk == 0) {
-      table[2 * (j / chunk)] = o;
-      table[2 * (j / chunk) + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
     }
   }
 }
@@ -159,44 +151,61 @@ __device__ __forceinline__ uint32_t code_bits_in_word(const Code& c, uint64_t w)
   return bits;
 }
 
-__global__ void __launch_bounds__(256) g_pack_kernel(const int32_t* idx, const GCtl* ctl,
-                                                      const GCtl* wctl, int64_t base, int b,
-                                                      const uint64_t* offs, uint32_t* words) {
-  __shared__ Code cs[8][32];
+// Offsets of this block's codewords (block prefix + in-block scan), the side table, and the
+// packing: the block stages its codewords in shared memory and writes every word of its bit range
+// once; only the first and last word, which it may share with neighbouring blocks, are OR-ed.
+__global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx, const GCtl* ctl,
+                                                               const GCtl* wctl, int64_t base, int b,
+                                                               const int64_t* block_pre,
+                                                               int64_t* table, int32_t chunk,
+                                                               uint32_t* words) {
+  __shared__ Code cs[kBlockCodes];
+  __shared__ int64_t sh[33];
   if (ctl->abort || wctl->abort) return;
   const int64_t len = ctl->len;
+  if ((int64_t)blockIdx.x * kBlockCodes >= len) return;
   const int32_t* x = idx + ctl->begin;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int64_t j0 = ((int64_t)blockIdx.x * 8 + wid) * 32;
-  if (j0 >= len) return;
-  const int64_t j = j0 + lane;
-  const int nvalid = (int)((len - j0) < 32 ? (len - j0) : 32);
-  if (j < len) {
-    const int64_t prev = j == 0 ? base - 1 : (int64_t)x[j - 1];
-    int64_t d = (int64_t)x[j] - prev - 1;
-    if (d < 0) d = 0;  // reported by the length pass
+  const int64_t jb = (int64_t)blockIdx.x * kBlockCodes;
+  const int64_t j0 = jb + (int64_t)threadIdx.x * kPer;
+  int64_t d[kPer];
+  thread_gaps(x, len, base, j0, d, nullptr);
+  int64_t l = 0;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e)
+    if (j0 + e < len) l += (d[e] >> b) + 1 + b;
+  int64_t tot;
+  int64_t o = block_pre[blockIdx.x] + block_exclusive_scan(l, sh, &tot);
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int64_t j = j0 + e;
+    if (j >= len) break;
     Code c;
-    c.o = offs[j];
-    c.q = (uint64_t)(d >> b);
-    const uint32_t rem = (uint32_t)(d & ((int64_t(1) << b) - 1));
+    c.o = (uint64_t)o;
+    c.q = (uint64_t)(d[e] >> b);
+    const uint32_t rem = (uint32_t)(d[e] & ((int64_t(1) << b) - 1));
     c.tail = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
     c.len_tail = 1u + (uint32_t)b;
-    cs[wid][lane] = c;
+    cs[threadIdx.x * kPer + e] = c;
+    if (table && j % chunk == 0) {
+      table[2 * (j / chunk)] = o;
+      table[2 * (j / chunk) + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
+    }
+    o += (int64_t)c.q + c.len_tail;
   }
-  __syncwarp();
-  const Code* C = cs[wid];
-  const uint64_t S = C[0].o;
-  const uint64_t E = C[nvalid - 1].o + C[nvalid - 1].q + C[nvalid - 1].len_tail;
+  __syncthreads();
+  const int nvalid = (int)((len - jb) < kBlockCodes ? (len - jb) : kBlockCodes);
+  const uint64_t S = cs[0].o;
+  const uint64_t E = cs[nvalid - 1].o + cs[nvalid - 1].q + cs[nvalid - 1].len_tail;
   const uint64_t wf = S >> 5, wl = (E - 1) >> 5;
-  for (uint64_t w = wf + lane; w <= wl; w += 32) {
+  for (uint64_t w = wf + threadIdx.x; w <= wl; w += blockDim.x) {
     // first codeword ending after the word starts
     int lo = 0, hi = nvalid;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (C[mid].o + C[mid].q + C[mid].len_tail <= w * 32) lo = mid + 1; else hi = mid;
+      if (cs[mid].o + cs[mid].q + cs[mid].len_tail <= w * 32) lo = mid + 1; else hi = mid;
     }
     uint32_t bits = 0;
-    for (int k = lo; k < nvalid && C[k].o < w * 32 + 32; ++k) bits |= code_bits_in_word(C[k], w);
+    for (int k = lo; k < nvalid && cs[k].o < w * 32 + 32; ++k) bits |= code_bits_in_word(cs[k], w);
     const bool shared_lo = (w == wf) && (S & 31);
     const bool shared_hi = (w == wl) && (E & 31);
     if (shared_lo || shared_hi) {
@@ -302,7 +311,6 @@ struct GLayout {
   GCtl* ctl;
   GCtl* wctl;
   int64_t* block_tot;
-  uint64_t* offs;
   size_t bytes;
 };
 
@@ -311,8 +319,7 @@ GLayout g_carve(int64_t capacity, void* ws) {
   Carver cv(ws);
   L.ctl = cv.take<GCtl>(1);
   L.wctl = cv.take<GCtl>(1);
-  L.block_tot = cv.take<int64_t>(cdiv(capacity, kScanThreads) + 1);
-  L.offs = cv.take<uint64_t>(capacity);
+  L.block_tot = cv.take<int64_t>(cdiv(capacity, kBlockCodes) + 1);
   L.bytes = cv.off + 256;
   return L;
 }
@@ -342,19 +349,16 @@ int gsparse_golomb_encode(const int32_t* idx, const int64_t* d_begin, const int6
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GSPARSE_ERR_WORKSPACE;
   GLayout L = g_carve(capacity, workspace);
   if (workspace_bytes < L.bytes) return GSPARSE_ERR_WORKSPACE;
-  g_setup_kernel<<<1, 1, 0, st>>>(d_begin, d_end, capacity, L.ctl, d_status);
-  if (cudaMemsetAsync(L.wctl, 0, sizeof(GCtl), st) != cudaSuccess) return GSPARSE_ERR_CUDA;
-  const unsigned nblk = (unsigned)cdiv(capacity > 0 ? capacity : 1, kScanThreads);
-  g_len_kernel<<<nblk, kScanThreads, 0, st>>>(idx, L.ctl, base, b, L.block_tot, d_status);
+  g_setup_kernel<<<1, 1, 0, st>>>(d_begin, d_end, capacity, L.ctl, L.wctl, d_status);
+  const unsigned nblk = (unsigned)cdiv(capacity > 0 ? capacity : 1, kBlockCodes);
+  g_len_kernel<<<nblk, kCodeThreads, 0, st>>>(idx, L.ctl, base, b, L.block_tot, d_status);
   g_scan_blocks_kernel<<<1, kScanThreads, 0, st>>>(L.block_tot, L.ctl, word_capacity, d_nbits,
                                                     L.wctl, d_status);
-  g_offsets_kernel<<<nblk, kScanThreads, 0, st>>>(idx, L.ctl, base, b, L.block_tot, L.offs,
-                                                   chunk_table, chunk);
   const int64_t zb = cdiv(word_capacity > 0 ? word_capacity : 1, 256);
   g_zero_kernel<<<(unsigned)(zb < 148 * 16 ? zb : 148 * 16), 256, 0, st>>>(words, d_nbits,
                                                                             word_capacity, L.ctl, L.wctl);
-  const int64_t warps = cdiv(capacity > 0 ? capacity : 1, 32);
-  g_pack_kernel<<<(unsigned)cdiv(warps, 8), 256, 0, st>>>(idx, L.ctl, L.wctl, base, b, L.offs, words);
+  g_pack_kernel<<<nblk, kCodeThreads, 0, st>>>(idx, L.ctl, L.wctl, base, b, L.block_tot, chunk_table,
+                                               chunk, words);
   return launch_status();
 }
 

@@ -3,50 +3,79 @@
 
 namespace gs {
 
-__global__ void osum_leaves_kernel(SumJob* jobs, int32_t njobs, double* leaves, int64_t leaf_bound,
-                                   const int32_t* abort_flag) {
+// One warp sums 32 consecutive leaves (one per lane). The values are read coalesced, 32 leaves x
+// 64 positions at a time, into a padded shared tile; each lane then adds its own leaf's positions
+// strictly left to right, so every leaf sum is the plain sequential fp64 sum of its block.
+constexpr int kLeafWarps = 4;
+constexpr int kLeafRound = 64;
+
+__global__ void __launch_bounds__(kLeafWarps * 32) osum_leaves_kernel(SumJob* jobs, int32_t njobs,
+                                                                      double* leaves, int64_t leaf_bound,
+                                                                      const int32_t* abort_flag) {
+  __shared__ float tile[kLeafWarps][32][kLeafRound + 1];
+  __shared__ const float* lptr[kLeafWarps][32];
+  __shared__ int lcnt[kLeafWarps][32];
   if (abort_flag && *abort_flag) return;
-  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  unsigned long long members = 0;
-  int32_t job = -1;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t t = ((int64_t)blockIdx.x * kLeafWarps + wid) * 32 + lane;
+  int32_t job = -1, mode = kSumAll, cnt = 0;
+  const float* ptr = nullptr;
   if (t < leaf_bound) {
     // the job owning leaf t: the last job whose first leaf is <= t
     int32_t lo = 0, hi = njobs;
     while (lo < hi) {
-      int32_t mid = (lo + hi) >> 1;
+      const int32_t mid = (lo + hi) >> 1;
       if (jobs[mid].leaf_base <= t) lo = mid + 1; else hi = mid;
     }
     job = lo - 1;
     if (job >= 0) {
       const SumJob& J = jobs[job];
       const int64_t leaf = t - J.leaf_base;
-      const int64_t nleaves = cdiv(J.len, kSumBlock);
-      if (leaf < nleaves) {
+      if (leaf < cdiv(J.len, kSumBlock)) {
         const int64_t b = leaf * kSumBlock;
-        const int64_t e = b + kSumBlock < J.len ? b + kSumBlock : J.len;
-        double s = 0.0;
-        const float* v = J.vals;
-        switch (J.mode) {
-          case kSumPositive:
-            for (int64_t j = b; j < e; ++j) { float x = v[j]; if (x > 0.0f) { s = __dadd_rn(s, (double)x); ++members; } }
-            break;
-          case kSumNegative:
-            for (int64_t j = b; j < e; ++j) { float x = v[j]; if (x < 0.0f) { s = __dadd_rn(s, (double)x); ++members; } }
-            break;
-          case kSumNegated:
-            for (int64_t j = b; j < e; ++j) s = __dadd_rn(s, -(double)v[j]);
-            members = (unsigned long long)(e - b);
-            break;
-          default:
-            for (int64_t j = b; j < e; ++j) s = __dadd_rn(s, (double)v[j]);
-            members = (unsigned long long)(e - b);
-        }
-        leaves[t] = s;
+        cnt = (int)((J.len - b) < kSumBlock ? (J.len - b) : kSumBlock);
+        ptr = J.vals + b;
+        mode = J.mode;
       } else {
         job = -1;
       }
     }
   }
+  lptr[wid][lane] = ptr;
+  lcnt[wid][lane] = cnt;
+  __syncwarp();
+  double s = 0.0;
+  unsigned long long members = 0;
+  for (int base = 0; base < kSumBlock; base += kLeafRound) {
+    // 32 leaves x 64 positions: lane l fetches position (base + l) and (base + 32 + l) of every
+    // leaf, all 64 loads independent, then the values go to the shared tile
+    float v0[32], v1[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const float* pc = lptr[wid][c];
+      const int nc = lcnt[wid][c];
+      v0[c] = base + lane < nc ? pc[base + lane] : 0.0f;
+      v1[c] = base + 32 + lane < nc ? pc[base + 32 + lane] : 0.0f;
+    }
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      tile[wid][c][lane] = v0[c];
+      tile[wid][c][32 + lane] = v1[c];
+    }
+    __syncwarp();
+    const int m = cnt - base < kLeafRound ? cnt - base : kLeafRound;
+    for (int j = 0; j < m; ++j) {
+      const float x = tile[wid][lane][j];
+      switch (mode) {
+        case kSumPositive: if (x > 0.0f) { s = __dadd_rn(s, (double)x); ++members; } break;
+        case kSumNegative: if (x < 0.0f) { s = __dadd_rn(s, (double)x); ++members; } break;
+        case kSumNegated: s = __dadd_rn(s, -(double)x); ++members; break;
+        default: s = __dadd_rn(s, (double)x); ++members;
+      }
+    }
+    __syncwarp();
+  }
+  if (job >= 0) leaves[t] = s;
   // member counts are integers, so the order of the atomics does not matter: the lowest lane of
   // each group of lanes working on the same job adds the group's total
   const uint32_t same = __match_any_sync(kFull, job);
@@ -132,7 +161,7 @@ void osum_launch(SumJob* jobs, int32_t njobs, double* leaves, int64_t leaf_bound
                  cudaStream_t s) {
   if (njobs <= 0) return;
   if (leaf_bound > 0) {
-    const int threads = 256;
+    const int threads = kLeafWarps * 32;
     osum_leaves_kernel<<<(unsigned)cdiv(leaf_bound, threads), threads, 0, s>>>(jobs, njobs, leaves,
                                                                                leaf_bound, abort_flag);
   }

@@ -32,7 +32,7 @@ struct SumJob {
   uint32_t done_blocks;  // completion counter of the tree kernel (must start at 0)
 };
 
-// Leaf sums: one thread per 256-position block of one job.
+// Leaf sums: one sequential fp64 sum per 256-position block of one job (one lane per block).
 __global__ void osum_leaves_kernel(SumJob* jobs, int32_t njobs, double* leaves, int64_t leaf_bound,
                                    const int32_t* abort_flag);
 

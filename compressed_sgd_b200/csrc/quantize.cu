@@ -42,8 +42,8 @@ __global__ void q_setup_kernel(const float* val, const int64_t* d_begin, const i
 
 __global__ void q_apply_kernel(const int32_t* idx, float* val, const int64_t* d_begin,
                                const int64_t* d_end, const SumJob* jobs, float* residual, int64_t n,
-                               uint32_t* sign_bits, float* d_means, int32_t write_deq,
-                               const int32_t* ctl, int32_t* d_status) {
+                               float* feedback, uint32_t* sign_bits, float* d_means,
+                               int32_t write_deq, const int32_t* ctl, int32_t* d_status) {
   if (ctl[0]) return;
   const int64_t b = d_begin ? *d_begin : 0;
   const int64_t len = *d_end - b;
@@ -68,6 +68,7 @@ __global__ void q_apply_kernel(const int32_t* idx, float* val, const int64_t* d_
     if (i < 0 || (int64_t)i >= n) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
     else residual[i] = __fsub_rn(x, q);
   }
+  if (feedback) feedback[j] = __fsub_rn(x, q);
   if (write_deq) val[b + j] = q;
 }
 
@@ -106,9 +107,10 @@ size_t gsparse_quantize_workspace_size(int64_t capacity) {
 }
 
 int gsparse_quantize(const int32_t* idx, float* val, const int64_t* d_begin, const int64_t* d_end,
-                     int64_t capacity, float* residual, int64_t n, uint32_t* sign_bits,
-                     float* d_means, int32_t write_dequantized, void* workspace,
-                     size_t workspace_bytes, int32_t* d_status, gsparse_stream stream) {
+                     int64_t capacity, float* residual, int64_t n, float* feedback_out,
+                     uint32_t* sign_bits, float* d_means, int32_t write_dequantized,
+                     void* workspace, size_t workspace_bytes, int32_t* d_status,
+                     gsparse_stream stream) {
   cudaStream_t st = (cudaStream_t)stream;
   if (capacity < 0 || n < 0 || !d_end || !d_means || (capacity > 0 && (!val || !sign_bits)) ||
       (residual && capacity > 0 && !idx))
@@ -122,8 +124,8 @@ int gsparse_quantize(const int32_t* idx, float* val, const int64_t* d_begin, con
   const int64_t threads = 256;
   const int64_t blocks = cdiv(capacity > 0 ? capacity : 1, threads);
   q_apply_kernel<<<(unsigned)blocks, (unsigned)threads, 0, st>>>(
-      idx, val, d_begin, d_end, L.jobs, residual, n, sign_bits, d_means, write_dequantized, L.ctl,
-      d_status);
+      idx, val, d_begin, d_end, L.jobs, residual, n, feedback_out, sign_bits, d_means,
+      write_dequantized, L.ctl, d_status);
   return launch_status();
 }
 

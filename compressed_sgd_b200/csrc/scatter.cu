@@ -157,15 +157,22 @@ __global__ void __launch_bounds__(kTileThreads) sa_combine_kernel(Lists L, int32
                                                                   float* out, float alpha, float beta,
                                                                   int32_t own, float* dense,
                                                                   int32_t* d_status) {
+  constexpr int kVec = kTile / 4 / kTileThreads;  // float4s of the tile per thread
   __shared__ __align__(16) float acc[kTile];
   __shared__ uint32_t touched[kTile / 32];
   const int64_t t = blockIdx.x;
+  const int64_t t0 = t * kTile;
+  const int64_t m = (n - t0) < kTile ? (n - t0) : kTile;
+  // the local-gradient tile is requested first, so its latency overlaps the accumulation
+  float4 lv[kVec];
+  if (m == kTile) {
+#pragma unroll
+    for (int k = 0; k < kVec; ++k) lv[k] = ld_stream(Lg + t0 + 4 * (threadIdx.x + k * kTileThreads));
+  }
   for (int i = threadIdx.x; i < kTile; i += blockDim.x) acc[i] = 0.0f;
   for (int i = threadIdx.x; i < kTile / 32; i += blockDim.x) touched[i] = 0u;
   __syncthreads();
   accumulate_tile(L, W, t, start, acc, touched, d_status);
-  const int64_t t0 = t * kTile;
-  const int64_t m = (n - t0) < kTile ? (n - t0) : kTile;
   if (dense) {
     if (m == kTile) {
       for (int v = threadIdx.x; v < kTile / 4; v += blockDim.x)
@@ -188,14 +195,15 @@ __global__ void __launch_bounds__(kTileThreads) sa_combine_kernel(Lists L, int32
     __syncthreads();
   }
   if (m == kTile) {
-    for (int v = threadIdx.x; v < kTile / 4; v += blockDim.x) {
+#pragma unroll
+    for (int k = 0; k < kVec; ++k) {
+      const int v = threadIdx.x + k * kTileThreads;
       const float4 g = reinterpret_cast<const float4*>(acc)[v];
-      const float4 l = ld_stream(Lg + t0 + 4 * v);
       float4 o;
-      o.x = __fadd_rn(__fmul_rn(alpha, g.x), __fmul_rn(beta, l.x));
-      o.y = __fadd_rn(__fmul_rn(alpha, g.y), __fmul_rn(beta, l.y));
-      o.z = __fadd_rn(__fmul_rn(alpha, g.z), __fmul_rn(beta, l.z));
-      o.w = __fadd_rn(__fmul_rn(alpha, g.w), __fmul_rn(beta, l.w));
+      o.x = __fadd_rn(__fmul_rn(alpha, g.x), __fmul_rn(beta, lv[k].x));
+      o.y = __fadd_rn(__fmul_rn(alpha, g.y), __fmul_rn(beta, lv[k].y));
+      o.z = __fadd_rn(__fmul_rn(alpha, g.z), __fmul_rn(beta, lv[k].z));
+      o.w = __fadd_rn(__fmul_rn(alpha, g.w), __fmul_rn(beta, lv[k].w));
       st_stream(out + t0 + 4 * v, o);
     }
   } else {

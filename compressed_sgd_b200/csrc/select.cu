@@ -38,6 +38,8 @@ constexpr int64_t kTargetPieces = 148 * 32;      // warps streaming at once on a
 constexpr int kSample = 1 << 18;                 // sampled entries per segment
 constexpr int kSampleRuns = kSample / 32;        // ... as evenly spaced runs of 32 entries
 constexpr int kSampleCtas = 256;                 // CTAs sharing one segment's sample
+static_assert(kSample % (32 * kSampleCtas) == 0 && kSample / kSampleCtas <= 1024,
+              "each sample CTA takes whole runs, at most 32 of them");
 constexpr int kWarps = 8;                        // warps (pieces) per CTA
 constexpr int kThreads = kWarps * 32;
 
@@ -61,6 +63,11 @@ struct Sel {
   // sample: two-level histogram of the sampled keys per problem
   uint32_t *shist, *scount, *sdone, *sb1;
   int64_t* srank;
+  // pending residual writes applied in the sample and pass 1 (null: none)
+  const int32_t* pw_idx;
+  const float* pw_val;
+  const int64_t* pw_count;
+  int64_t pw_cap;
   int32_t* d_status;
   // binarise
   int32_t* lidx;
@@ -219,6 +226,23 @@ __global__ void __launch_bounds__(1024) plan_kernel(Sel a, const int64_t* seg, i
 // sample m = k, so at least k entries reach T_lo; otherwise m sits three standard deviations (plus
 // 16) above the expected sample count, and a shortfall is caught and redone by the check step.
 
+__device__ __forceinline__ uint32_t pending_count(const Sel& a) {
+  if (!a.pw_idx) return 0;
+  int64_t c = *a.pw_count;
+  c = c < 0 ? 0 : (c > a.pw_cap ? a.pw_cap : c);
+  return (uint32_t)c;
+}
+
+// The residual value of entry i with the pending writes applied (the writes in [b, e) of the
+// list, which must hold every write of the caller's range).
+__device__ __forceinline__ float residual_at(const Sel& a, int64_t i, uint32_t b, uint32_t e) {
+  if (b < e) {
+    const int64_t pos = lower_bound_i32(a.pw_idx + b, e - b, i);
+    if (pos < (int64_t)(e - b) && a.pw_idx[b + pos] == i) return a.pw_val[b + pos];
+  }
+  return a.r[i];
+}
+
 __device__ __forceinline__ int64_t sample_pos(int64_t lo, int64_t ns, int64_t j) {
   if (ns <= kSample) return lo + j;
   return lo + (j >> 5) * (ns - 32) / (kSampleRuns - 1) + (j & 31);
@@ -258,9 +282,38 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
   __syncthreads();
   const int64_t S = ns < kSample ? ns : kSample;
   const int64_t j0 = S * blockIdx.x / gridDim.x, j1 = S * (blockIdx.x + 1) / gridDim.x;
+  // The sample sees the pending residual writes. A fully sampled segment: the writes of this
+  // CTA's contiguous slice. A sparsely sampled one: per run of 32 entries, the writes falling in
+  // the run (one binary search per run, by the lanes of the first warp).
+  __shared__ uint32_t pwb, pwe;
+  __shared__ uint32_t run_b[32], run_e[32];
+  const uint32_t pc = pending_count(a);
+  const bool runs = pc && ns > kSample;
+  if (threadIdx.x == 0) {
+    pwb = pwe = 0;
+    if (pc && ns <= kSample) {
+      pwb = (uint32_t)lower_bound_i32(a.pw_idx, pc, lo + j0);
+      pwe = (uint32_t)lower_bound_i32(a.pw_idx, pc, lo + j1);
+    }
+  }
+  if (runs && threadIdx.x < 32) {
+    const int64_t jr = j0 + 32 * threadIdx.x;       // j0 is a multiple of 32 here
+    uint32_t b = 0, e = 0;
+    if (jr < j1) {
+      const int64_t start = sample_pos(lo, ns, jr);
+      b = (uint32_t)lower_bound_i32(a.pw_idx, pc, start);
+      const uint32_t span = pc - b < 33u ? pc - b : 33u;
+      e = b + (uint32_t)lower_bound_i32(a.pw_idx + b, span, start + 32);
+    }
+    run_b[threadIdx.x] = b;
+    run_e[threadIdx.x] = e;
+  }
+  __syncthreads();
   for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
     const int64_t i = sample_pos(lo, ns, j);
-    const float x = __fadd_rn(a.g[i], a.r[i]);
+    const uint32_t cb = runs ? run_b[(j - j0) >> 5] : pwb;
+    const uint32_t ce = runs ? run_e[(j - j0) >> 5] : pwe;
+    const float x = __fadd_rn(a.g[i], residual_at(a, i, cb, ce));
     const int c = class_of<C>(x);
     if (c < 0) continue;
     const uint32_t key = mag_key(x);
@@ -342,7 +395,7 @@ __device__ __forceinline__ int cand_class(float x) {
 template <int C>
 __global__ void __launch_bounds__(kThreads, 4) pass1_kernel(Sel a) {
   __shared__ CtaHist<C, kBins1> H;
-  __shared__ __align__(16) float stage[kWarps * 4 * 32 * 4];  // [warp][u][lane][e]
+  __shared__ __align__(16) float stage[kWarps * kGranule];  // per warp: one chunk, entry order
   if (a.ctl[0]) return;
   const int64_t q0 = (int64_t)blockIdx.x * kWarps;
   H.init(a, q0);
@@ -364,38 +417,87 @@ __global__ void __launch_bounds__(kThreads, 4) pass1_kernel(Sel a) {
     const uint32_t lo = (uint32_t)P.lo, hi = (uint32_t)P.hi;  // indices are below 2^31
     const float* g = a.g;
     float* r = a.r;
-    float* st = stage + wid * 512;
+    float* st = stage + wid * kGranule;
+    float4* st4 = reinterpret_cast<float4*>(st);
+    // pending residual writes of this piece: [cp, cend) of the sorted list
+    const uint32_t cend = pending_count(a);
+    uint32_t cp = 0;
+    if (cend) cp = __shfl_sync(kFull, lane == 0 ? (uint32_t)lower_bound_i32(a.pw_idx, cend, lo) : 0u, 0);
     uint32_t count = 0;
     for (uint32_t base = lo & ~3u; base < hi; base += (uint32_t)kGranule) {
-      if (base >= lo && base + (uint32_t)kGranule <= hi) {
-        // ---- fast path: the whole 512-entry chunk lies in the piece ----
-        float4 gv[4], rv[4];
+      const bool full = base >= lo && base + (uint32_t)kGranule <= hi;  // warp-uniform
+      float4 gv[4], rv[4];
+      uint32_t valid = 0xFFFFu;
+      if (full) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           gv[u] = ld_stream(g + base + u * 128 + lane * 4);
           rv[u] = ld_stream(r + base + u * 128 + lane * 4);
         }
-        float4 av[4];
-        uint32_t m16 = 0;
+      } else {
+        // first or last chunk of the piece: entry-wise bounds
+        valid = 0;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          av[u] = make_float4(__fadd_rn(gv[u].x, rv[u].x), __fadd_rn(gv[u].y, rv[u].y),
-                              __fadd_rn(gv[u].z, rv[u].z), __fadd_rn(gv[u].w, rv[u].w));
-          m16 |= (cand_bit<C>(av[u].x, tl) | (cand_bit<C>(av[u].y, tl) << 1) |
-                  (cand_bit<C>(av[u].z, tl) << 2) | (cand_bit<C>(av[u].w, tl) << 3)) << (4 * u);
-        }
-        // per-quarter counts packed in bytes; one warp scan serves all four quarters
-        const uint32_t packed = __popc(m16 & 0xFu) | (__popc(m16 & 0xF0u) << 8) |
-                                (__popc(m16 & 0xF00u) << 16) | (__popc(m16 & 0xF000u) << 24);
-        const uint32_t incl = warp_inclusive_scan(packed);
-        const uint32_t tot = __shfl_sync(kFull, incl, 31);
-        if (tot == 0) {
+          float t0[4], t1[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) st_stream(r + base + u * 128 + lane * 4, av[u]);
-          continue;
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t i = base + u * 128 + lane * 4 + e;
+            const bool in = i >= lo && i < hi;
+            t0[e] = in ? g[i] : 0.0f;
+            t1[e] = in ? r[i] : 0.0f;
+            valid |= (uint32_t)in << (4 * u + e);
+          }
+          gv[u] = make_float4(t0[0], t0[1], t0[2], t0[3]);
+          rv[u] = make_float4(t1[0], t1[1], t1[2], t1[3]);
         }
+      }
+      if (cp < cend) {
+        // pending residual writes that fall in this chunk replace those residual entries
+        const uint32_t lim = base + (uint32_t)kGranule < hi ? base + (uint32_t)kGranule : hi;
+        bool staged = false;
+        for (;;) {
+          const uint32_t j = cp + lane;
+          const int32_t ci = j < cend ? a.pw_idx[j] : INT32_MAX;
+          const bool in = ci >= (int32_t)base && ci < (int32_t)lim;
+          const uint32_t mask = __ballot_sync(kFull, in);
+          if (!mask) break;
+          if (!staged) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) reinterpret_cast<float4*>(st)[u * 32 + lane] = av[u];
+            for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = rv[u];
+            __syncwarp();
+            staged = true;
+          }
+          if (in) st[ci - (int32_t)base] = a.pw_val[j];
+          cp += __popc(mask);
+          __syncwarp();
+          if (mask != kFull) break;
+        }
+        if (staged) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) rv[u] = st4[u * 32 + lane];
+          __syncwarp();
+        }
+      }
+      float4 av[4];
+      uint32_t m16 = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        av[u] = make_float4(__fadd_rn(gv[u].x, rv[u].x), __fadd_rn(gv[u].y, rv[u].y),
+                            __fadd_rn(gv[u].z, rv[u].z), __fadd_rn(gv[u].w, rv[u].w));
+        m16 |= (cand_bit<C>(av[u].x, tl) | (cand_bit<C>(av[u].y, tl) << 1) |
+                (cand_bit<C>(av[u].z, tl) << 2) | (cand_bit<C>(av[u].w, tl) << 3)) << (4 * u);
+      }
+      m16 &= valid;
+      // per-quarter counts packed in bytes; one warp scan serves all four quarters
+      const uint32_t packed = __popc(m16 & 0xFu) | (__popc(m16 & 0xF0u) << 8) |
+                              (__popc(m16 & 0xF00u) << 16) | (__popc(m16 & 0xF000u) << 24);
+      const uint32_t incl = warp_inclusive_scan(packed);
+      const uint32_t tot = __shfl_sync(kFull, incl, 31);
+      bool from_stage = false;
+      if (tot) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = av[u];
         __syncwarp();
         const uint32_t excl = incl - packed;
         const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu;
@@ -416,60 +518,52 @@ __global__ void __launch_bounds__(kThreads, 4) pass1_kernel(Sel a) {
         }
         count += t0 + t1 + t2 + (tot >> 24);
         if (a.zero_mode) {
+          // stored candidates leave the residual as +0 (the not-sent ones get acc back later)
           for (uint32_t m = stored; m; m &= m - 1) {
             const int b = __ffs(m) - 1;
             st[((b >> 2) * 32 + lane) * 4 + (b & 3)] = 0.0f;
           }
           __syncwarp();
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            st_stream(r + base + u * 128 + lane * 4, reinterpret_cast<const float4*>(st)[u * 32 + lane]);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) st_stream(r + base + u * 128 + lane * 4, av[u]);
-        }
-        __syncwarp();
-      } else {
-        // ---- edge path: first or last chunk of the piece, element-wise bounds ----
-#pragma unroll 1
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t v = base + u * 128 + lane * 4;
-          float x[4];
-          uint32_t m4 = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t i = v + e;
-            const bool in = i >= lo && i < hi;
-            x[e] = in ? __fadd_rn(g[i], r[i]) : 0.0f;
-            m4 |= (in ? cand_bit<C>(x[e], tl) : 0u) << e;
-          }
-          uint32_t tot;
-          const uint32_t pre = warp_prefix_small(__popc(m4), &tot);
-          uint32_t pos = count + pre;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t i = v + e;
-            if (i < lo || i >= hi) continue;
-            float o = x[e];
-            if ((m4 >> e) & 1u) {
-              if (pos < cap) {
-                cidx[pos] = (int32_t)i;
-                cval[pos] = x[e];
-                if (a.zero_mode) o = 0.0f;
-              }
-              atomicAdd(hsink + cand_class<C>(x[e]) * hstride + (mag_key(x[e]) >> 20), 1u);
-              ++pos;
-            }
-            r[i] = o;
-          }
-          count += tot;
+          from_stage = true;
         }
       }
+      if (full) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          st_stream(r + base + u * 128 + lane * 4, from_stage ? st4[u * 32 + lane] : av[u]);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 o = from_stage ? st4[u * 32 + lane] : av[u];
+          const float ov[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if ((valid >> (4 * u + e)) & 1u) r[base + u * 128 + lane * 4 + e] = ov[e];
+        }
+      }
+      __syncwarp();
     }
     if (lane == 0) a.pcnt[q] = count;
   }
   __syncthreads();
   H.flush(a, 1, kBins1);
+}
+
+// The pending residual writes must be strictly ascending indices in [0, n): anything else stops
+// the call before it touches the residual.
+__global__ void pending_check_kernel(Sel a) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j == 0 && *a.pw_count > a.pw_cap) {
+    raise(a.d_status, GSPARSE_DERR_CAPACITY);
+    a.ctl[0] = 1;
+  }
+  const uint32_t c = pending_count(a);
+  if (j >= c) return;
+  const int32_t i = a.pw_idx[j];
+  if (i < 0 || (int64_t)i >= a.n || (j > 0 && a.pw_idx[j - 1] >= i)) {
+    raise(a.d_status, GSPARSE_DERR_INDEX_RANGE);
+    a.ctl[0] = 1;
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1089,8 +1183,11 @@ cudaEvent_t g_pass1_before = nullptr, g_pass1_after = nullptr;
 template <int C>
 int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t T, int64_t num,
                int64_t den, int32_t* out_idx, float* out_val, float* d_mean, int64_t* out_offsets,
-               int64_t out_capacity, uint32_t flags, void* ws, size_t ws_bytes, int32_t* d_status,
-               cudaStream_t st) {
+               int64_t out_capacity, const gsparse_pending* pending, uint32_t flags, void* ws,
+               size_t ws_bytes, int32_t* d_status, cudaStream_t st) {
+  if (pending && (!pending->d_count || pending->capacity < 0 ||
+                  (pending->capacity > 0 && (!pending->idx || !pending->val))))
+    return GSPARSE_ERR_INVALID_ARG;
   if (n < 0 || T < 1 || (seg == nullptr && T != 1) || bad_keep(num, den) || !out_offsets ||
       out_capacity < 0)
     return GSPARSE_ERR_INVALID_ARG;
@@ -1107,9 +1204,16 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   a.r = r;
   a.zero_mode = C == 1;
   a.d_status = d_status;
+  const bool has_pending = pending && pending->capacity > 0;
+  a.pw_idx = has_pending ? pending->idx : nullptr;
+  a.pw_val = has_pending ? pending->val : nullptr;
+  a.pw_count = has_pending ? pending->d_count : nullptr;
+  a.pw_cap = has_pending ? pending->capacity : 0;
   if (cudaMemsetAsync(L.zero_begin, 0, L.zero_bytes, st) != cudaSuccess) return GSPARSE_ERR_CUDA;
   plan_kernel<<<1, 1024, 0, st>>>(a, seg, num, den, out_capacity, C == 1 ? out_offsets : nullptr);
-  if (num == 0 && C == 1) {  // communication delay step: accumulate only
+  if (has_pending)
+    pending_check_kernel<<<(unsigned)cdiv(a.pw_cap, 256), 256, 0, st>>>(a);
+  if (num == 0 && C == 1 && !has_pending) {  // communication delay step: accumulate only
     if (n > 0) {
       const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
       accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, a.ctl);
@@ -1191,11 +1295,11 @@ size_t gsparse_residual_topk_workspace_min(int64_t n, int32_t T) {
 
 int gsparse_residual_topk(const float* g, float* residual, int64_t n, const int64_t* seg_offsets,
                           int32_t num_segments, int64_t keep_num, int64_t keep_den, int32_t* out_idx,
-                          float* out_val, int64_t* out_offsets, int64_t out_capacity, uint32_t flags,
-                          void* workspace, size_t workspace_bytes, int32_t* d_status,
-                          gsparse_stream stream) {
+                          float* out_val, int64_t* out_offsets, int64_t out_capacity,
+                          const gsparse_pending* pending, uint32_t flags, void* workspace,
+                          size_t workspace_bytes, int32_t* d_status, gsparse_stream stream) {
   return run_select<1>(g, residual, n, seg_offsets, num_segments, keep_num, keep_den, out_idx,
-                       out_val, nullptr, out_offsets, out_capacity, flags, workspace,
+                       out_val, nullptr, out_offsets, out_capacity, pending, flags, workspace,
                        workspace_bytes, d_status, (cudaStream_t)stream);
 }
 
@@ -1218,8 +1322,8 @@ int gsparse_residual_topk_noalloc(const float* g, float* residual, int64_t n, in
   const int st = noalloc_scratch(&scratch);
   if (st != GSPARSE_OK) return st;
   return run_select<1>(g, residual, n, nullptr, 1, keep_num, keep_den, out_idx, out_val, nullptr,
-                       out_offsets, out_capacity, 0, scratch, GSPARSE_NOALLOC_SCRATCH_BYTES, d_status,
-                       (cudaStream_t)stream);
+                       out_offsets, out_capacity, nullptr, 0, scratch, GSPARSE_NOALLOC_SCRATCH_BYTES,
+                       d_status, (cudaStream_t)stream);
 }
 
 int gsparse_binarize(const float* g, float* residual, int64_t n, const int64_t* seg_offsets,
@@ -1228,7 +1332,7 @@ int gsparse_binarize(const float* g, float* residual, int64_t n, const int64_t* 
                      uint32_t flags, void* workspace, size_t workspace_bytes, int32_t* d_status,
                      gsparse_stream stream) {
   return run_select<2>(g, residual, n, seg_offsets, num_segments, keep_num, keep_den, out_idx,
-                       out_val, d_mean, out_offsets, out_capacity, flags, workspace,
+                       out_val, d_mean, out_offsets, out_capacity, nullptr, flags, workspace,
                        workspace_bytes, d_status, (cudaStream_t)stream);
 }
 

@@ -114,18 +114,32 @@ int32_t gsparse_golomb_b_star(double p);
  * out_offsets      int64[num_segments+1] device: exclusive offsets of each segment's entries.
  * out_capacity     host bound; if sum_s k_s exceeds it, GSPARSE_DERR_CAPACITY is raised and
  *                  neither outputs nor residual are touched.
- * workspace        at least gsparse_residual_topk_workspace_min(); the recommended size is
- *                  gsparse_residual_topk_workspace_size(). Less room only costs speed.
- * Data errors: GSPARSE_DERR_SEGMENTS, GSPARSE_DERR_CAPACITY.
+ * pending          HOST pointer to a list of residual writes applied before the step, or NULL:
+ *                  residual[idx_j] <- val_j for every entry j (idx strictly ascending in [0, n)).
+ *                  It carries the quantisation error of the previous step (gsparse_quantize's
+ *                  feedback_out) into this call, which applies it inside its streaming pass rather
+ *                  than as a separate scattered write; the result equals writing it first.
+ * workspace        256-byte aligned, at least gsparse_residual_topk_workspace_min(); the
+ *                  recommended size is gsparse_residual_topk_workspace_size(). Less room only
+ *                  costs speed.
+ * Data errors: GSPARSE_DERR_SEGMENTS, GSPARSE_DERR_CAPACITY, GSPARSE_DERR_INDEX_RANGE (a pending
+ * list that is not strictly ascending in [0, n)); on any of them nothing is written.
  */
+typedef struct {
+  const int32_t* idx;      /* device, strictly ascending */
+  const float* val;        /* device */
+  const int64_t* d_count;  /* device int64: number of entries */
+  int64_t capacity;        /* host bound on *d_count */
+} gsparse_pending;
+
 size_t gsparse_residual_topk_workspace_size(int64_t n, int32_t num_segments, int64_t keep_num,
                                             int64_t keep_den);
 size_t gsparse_residual_topk_workspace_min(int64_t n, int32_t num_segments);
 int gsparse_residual_topk(const float* g, float* residual, int64_t n, const int64_t* seg_offsets,
                           int32_t num_segments, int64_t keep_num, int64_t keep_den, int32_t* out_idx,
-                          float* out_val, int64_t* out_offsets, int64_t out_capacity, uint32_t flags,
-                          void* workspace, size_t workspace_bytes, int32_t* d_status,
-                          gsparse_stream stream);
+                          float* out_val, int64_t* out_offsets, int64_t out_capacity,
+                          const gsparse_pending* pending, uint32_t flags, void* workspace,
+                          size_t workspace_bytes, int32_t* d_status, gsparse_stream stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Residual top-k without caller-provided scratch  (no counterpart in the pages: this entry point
@@ -171,13 +185,18 @@ int gsparse_residual_topk_noalloc(const float* g, float* residual, int64_t n, in
  * residual    fp32[n] or NULL: residual[idx_j] <- fl(val_j - q_j), the quantisation error fed back
  *             (Sattler et al. §II Residual Accumulation). Indices outside [0, n) raise
  *             GSPARSE_DERR_INDEX_RANGE and are skipped.
+ * feedback_out fp32[capacity] or NULL: feedback_out[j] <- fl(val_j - q_j) (position j counted
+ *             from begin), the same error as a contiguous list; handed to the next
+ *             gsparse_residual_topk as its pending writes (with idx) it has the effect of the
+ *             residual argument without the scattered write.
  * write_dequantized  nonzero: val_j <- q_j in place.
  */
 size_t gsparse_quantize_workspace_size(int64_t capacity);
 int gsparse_quantize(const int32_t* idx, float* val, const int64_t* d_begin, const int64_t* d_end,
-                     int64_t capacity, float* residual, int64_t n, uint32_t* sign_bits,
-                     float* d_means, int32_t write_dequantized, void* workspace,
-                     size_t workspace_bytes, int32_t* d_status, gsparse_stream stream);
+                     int64_t capacity, float* residual, int64_t n, float* feedback_out,
+                     uint32_t* sign_bits, float* d_means, int32_t write_dequantized,
+                     void* workspace, size_t workspace_bytes, int32_t* d_status,
+                     gsparse_stream stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Sparse binarisation  (Sattler et al. §II Sparse Binarization)

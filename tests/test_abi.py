@@ -59,7 +59,7 @@ def test_workspace_queries(gs):
     assert lib.gsparse_residual_topk_workspace_size(-1, 1, 1, 100) == 0
     assert lib.gsparse_binarize_workspace_size(1000, 3, 1, 1000) > lib.gsparse_binarize_workspace_min(1000, 3, 1, 1000) - 1
     assert lib.gsparse_quantize_workspace_size(10 ** 6) > 0
-    assert lib.gsparse_golomb_encode_workspace_size(10 ** 6) >= 8 * 10 ** 6
+    assert 0 < lib.gsparse_golomb_encode_workspace_size(10 ** 6) < 10 ** 5     # block totals only
     assert lib.gsparse_scatter_accumulate_workspace_size(4, 1 << 20) > 0
     for s in range(6):
         assert lib.gsparse_status_string(s)

@@ -385,3 +385,56 @@ def test_accumulate_combine_parity(W, n):
             assert np.array_equal(bits(host(dense)), bits(wd))
             out2 = gs.accumulate_combine(lists, n, L, alpha=alpha, beta=beta, mode=mode, own=own)
             assert np.array_equal(bits(host(out2)), bits(want))
+
+
+# ------------------------------------------------------------------------------------ pending writes
+
+@pytest.mark.parametrize("mode", ["global", "per_tensor", "delay"])
+def test_quantisation_feedback_as_pending_writes_matches_immediate(mode):
+    """Quantise with feedback_out, hand (idx, feedback) to the next residual_topk as pending writes:
+    after every top-k the residual and the outputs equal the oracle chain that writes the
+    quantisation error into the residual at once."""
+    lay = [70000, 3, 130001, 64] if mode == "per_tensor" else [200071]
+    seg = np.concatenate([[0], np.cumsum(lay)]).astype(np.int64)
+    n, T = int(seg[-1]), len(lay)
+    seg_arg = seg if mode == "per_tensor" else None
+    r_o = np.zeros(n, np.float32)
+    r_d = torch.zeros(n, device="cuda")
+    pend = None
+    keepalive = []
+    st = gs.status_tensor()
+    for step in range(6):
+        keep = (0, 1) if (mode == "delay" and step % 2 == 1) else (1, 50)
+        g = synth.flat_mixture(n, seed=300 + step)
+        wi, wv, wo, r_o = oracle.residual_topk(g, r_o, keep, seg=seg_arg)
+        idx, val, off = gs.residual_topk(dev(g), r_d, keep, seg_offsets=None if seg_arg is None else dev(seg),
+                                         d_status=st, pending=pend)
+        K = int(wo[-1])
+        assert np.array_equal(host(off), wo), step
+        assert np.array_equal(host(idx)[:K], wi), step
+        assert np.array_equal(bits(host(val)[:K]), bits(wv)), step
+        assert np.array_equal(bits(host(r_d)), bits(r_o)), step
+        pend = None
+        if K:
+            fb = torch.empty(idx.numel(), device="cuda")
+            for s in range(T):
+                b, e = int(wo[s]), int(wo[s + 1])
+                _, _, wv_s, r_o = oracle.quantize(wi[b:e], wv[b:e], residual=r_o, write_dequantized=True)
+                gs.quantize(idx, val, off[s + 1:s + 2], d_begin=off[s:s + 1], write_dequantized=True,
+                            feedback_out=fb[b:], d_status=st, capacity=idx.numel())
+            pend = gs.make_pending(idx, fb, off[T:T + 1])
+            keepalive.append((idx, val, off, fb))
+    assert int(host(st)[0]) == 0
+
+
+def test_pending_writes_must_be_ascending():
+    n = 5000
+    g = synth.gaussian(n, 1)
+    r = torch.zeros(n, device="cuda")
+    pidx = torch.tensor([10, 20, 15], dtype=torch.int32, device="cuda")
+    pval = torch.ones(3, device="cuda")
+    st = gs.status_tensor()
+    gs.residual_topk(dev(g), r, (1, 10), d_status=st,
+                     pending=gs.make_pending(pidx, pval, torch.tensor([3], device="cuda")))
+    assert int(host(st)[0]) & gs.DERR_INDEX_RANGE
+    assert bool((r == 0).all())                       # nothing written
