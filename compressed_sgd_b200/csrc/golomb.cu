@@ -16,9 +16,10 @@ namespace gs {
 namespace {
 
 constexpr int kScanThreads = 1024;
-constexpr int kPer = 4;                      // codewords per thread
+constexpr int kPer = 8;                      // codewords per thread
 constexpr int kCodeThreads = 256;
 constexpr int kBlockCodes = kPer * kCodeThreads;  // codewords per block of the length and pack passes
+constexpr int kPackWords = 4096;             // shared word buffer of the pack pass (128 Kbit)
 
 struct GCtl {
   int64_t begin, len;
@@ -152,15 +153,18 @@ __device__ __forceinline__ uint32_t code_bits_in_word(const Code& c, uint64_t w)
 }
 
 // Offsets of this block's codewords (block prefix + in-block scan), the side table, and the
-// packing: the block stages its codewords in shared memory and writes every word of its bit range
-// once; only the first and last word, which it may share with neighbouring blocks, are OR-ed.
+// packing: when the block's bits fit the shared word buffer, each thread ORs its codewords in
+// with shared atomics and the words go out in one coalesced sweep (the first and last word, which
+// the block may share with its neighbours, are OR-ed into the zeroed stream). Otherwise (long
+// unary runs) every codeword is OR-ed straight into the zeroed stream.
 __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx, const GCtl* ctl,
                                                                const GCtl* wctl, int64_t base, int b,
                                                                const int64_t* block_pre,
                                                                int64_t* table, int32_t chunk,
                                                                uint32_t* words) {
-  __shared__ Code cs[kBlockCodes];
+  __shared__ uint32_t wbuf[kPackWords];
   __shared__ int64_t sh[33];
+  __shared__ uint64_t span_lo, span_hi;
   if (ctl->abort || wctl->abort) return;
   const int64_t len = ctl->len;
   if ((int64_t)blockIdx.x * kBlockCodes >= len) return;
@@ -174,42 +178,53 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
   for (int e = 0; e < kPer; ++e)
     if (j0 + e < len) l += (d[e] >> b) + 1 + b;
   int64_t tot;
-  int64_t o = block_pre[blockIdx.x] + block_exclusive_scan(l, sh, &tot);
+  const int64_t o0 = block_pre[blockIdx.x] + block_exclusive_scan(l, sh, &tot);
+  if (threadIdx.x == 0) span_lo = (uint64_t)o0;
+  if (threadIdx.x == blockDim.x - 1) span_hi = (uint64_t)(o0 + l);   // the block's last bit + 1
+  Code cs[kPer];
+  int64_t o = o0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     const int64_t j = j0 + e;
-    if (j >= len) break;
-    Code c;
-    c.o = (uint64_t)o;
-    c.q = (uint64_t)(d[e] >> b);
+    cs[e].o = (uint64_t)o;
+    cs[e].q = (uint64_t)(d[e] >> b);
     const uint32_t rem = (uint32_t)(d[e] & ((int64_t(1) << b) - 1));
-    c.tail = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
-    c.len_tail = 1u + (uint32_t)b;
-    cs[threadIdx.x * kPer + e] = c;
-    if (table && j % chunk == 0) {
-      table[2 * (j / chunk)] = o;
-      table[2 * (j / chunk) + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
+    cs[e].tail = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
+    cs[e].len_tail = 1u + (uint32_t)b;
+    if (j < len) {
+      if (table && j % chunk == 0) {
+        table[2 * (j / chunk)] = o;
+        table[2 * (j / chunk) + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
+      }
+      o += (int64_t)cs[e].q + cs[e].len_tail;
     }
-    o += (int64_t)c.q + c.len_tail;
   }
   __syncthreads();
-  const int nvalid = (int)((len - jb) < kBlockCodes ? (len - jb) : kBlockCodes);
-  const uint64_t S = cs[0].o;
-  const uint64_t E = cs[nvalid - 1].o + cs[nvalid - 1].q + cs[nvalid - 1].len_tail;
+  const uint64_t S = span_lo, E = span_hi;
   const uint64_t wf = S >> 5, wl = (E - 1) >> 5;
-  for (uint64_t w = wf + threadIdx.x; w <= wl; w += blockDim.x) {
-    // first codeword ending after the word starts
-    int lo = 0, hi = nvalid;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (cs[mid].o + cs[mid].q + cs[mid].len_tail <= w * 32) lo = mid + 1; else hi = mid;
+  const bool fits = wl - wf + 1 <= (uint64_t)kPackWords;
+  if (fits) {
+    for (int i = threadIdx.x; i < kPackWords; i += blockDim.x) wbuf[i] = 0u;
+    __syncthreads();
+  }
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    if (j0 + e >= len) break;
+    const Code& c = cs[e];
+    const uint64_t w0 = c.o >> 5, w1 = (c.o + c.q + c.len_tail - 1) >> 5;
+    for (uint64_t w = w0; w <= w1; ++w) {
+      const uint32_t bits = code_bits_in_word(c, w);
+      if (!bits) continue;
+      if (fits) atomicOr(&wbuf[w - wf], bits);
+      else atomicOr(&words[w], bits);
     }
-    uint32_t bits = 0;
-    for (int k = lo; k < nvalid && cs[k].o < w * 32 + 32; ++k) bits |= code_bits_in_word(cs[k], w);
-    const bool shared_lo = (w == wf) && (S & 31);
-    const bool shared_hi = (w == wl) && (E & 31);
-    if (shared_lo || shared_hi) {
-      if (bits) atomicOr(&words[w], bits);
+  }
+  if (!fits) return;
+  __syncthreads();
+  for (uint64_t w = wf + threadIdx.x; w <= wl; w += blockDim.x) {
+    const uint32_t bits = wbuf[w - wf];
+    if ((w == wf && (S & 31)) || (w == wl && (E & 31))) {
+      if (bits) atomicOr(&words[w], bits);   // shared with a neighbouring block
     } else {
       words[w] = bits;
     }
@@ -219,21 +234,23 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
 // ---------------------------------------------------------------------------------------------
 // decoder
 
-__device__ __forceinline__ uint32_t word_at(const uint32_t* words, int64_t nw, int64_t w) {
-  return w < nw ? words[w] : 0u;
+// Word w of the stream, read from a window holding words [base_w, lim_w) (zero outside).
+__device__ __forceinline__ uint32_t word_at(const uint32_t* src, int64_t base_w, int64_t lim_w,
+                                            int64_t w) {
+  return (w >= base_w && w < lim_w) ? src[w - base_w] : 0u;
 }
 
 // Decodes `count` codewords from bit t; returns false (and raises) on a corrupt stream.
-__device__ bool decode_run(const uint32_t* words, uint64_t nbits, uint64_t& t, int64_t& prev,
-                           int64_t count, int b, int64_t n_limit, int32_t* out, int32_t* d_status) {
-  const int64_t nw = cdiv((int64_t)nbits, 32);
+__device__ bool decode_run(const uint32_t* src, int64_t base_w, int64_t lim_w, uint64_t nbits,
+                           uint64_t& t, int64_t& prev, int64_t count, int b, int64_t n_limit,
+                           int32_t* out, int32_t* d_status) {
   for (int64_t k = 0; k < count; ++k) {
     uint64_t q = 0;
     for (;;) {
       if (t >= nbits) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
       const uint32_t sh = (uint32_t)(t & 31);
       const uint32_t avail = 32 - sh;
-      const uint32_t v = word_at(words, nw, (int64_t)(t >> 5)) >> sh;
+      const uint32_t v = word_at(src, base_w, lim_w, (int64_t)(t >> 5)) >> sh;
       const uint32_t zeros = ~v & (avail == 32 ? 0xffffffffu : ((1u << avail) - 1u));
       if (zeros) {
         const uint32_t z = (uint32_t)__ffs(zeros) - 1u;
@@ -248,9 +265,9 @@ __device__ bool decode_run(const uint32_t* words, uint64_t nbits, uint64_t& t, i
     uint32_t rem = 0;
     if (b > 0) {
       if (t + (uint64_t)b > nbits) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
-      const uint64_t w = t >> 5;
-      const uint64_t win = (uint64_t)word_at(words, nw, (int64_t)w) |
-                           ((uint64_t)word_at(words, nw, (int64_t)w + 1) << 32);
+      const int64_t w = (int64_t)(t >> 5);
+      const uint64_t win = (uint64_t)word_at(src, base_w, lim_w, w) |
+                           ((uint64_t)word_at(src, base_w, lim_w, w + 1) << 32);
       const uint32_t raw = (uint32_t)(win >> (t & 31)) & ((1u << b) - 1u);
       rem = __brev(raw) >> (32 - b);
       t += (uint64_t)b;
@@ -264,33 +281,86 @@ __device__ bool decode_run(const uint32_t* words, uint64_t nbits, uint64_t& t, i
   return true;
 }
 
-__global__ void g_decode_chunks_kernel(const uint32_t* words, int64_t word_capacity,
-                                       const uint64_t* d_nbits,
-                                       const int64_t* d_count, int64_t capacity, int b,
-                                       const int64_t* table, int32_t chunk, int64_t n_limit,
-                                       int32_t* out, int32_t* d_status) {
+// One thread per chunk of codewords, kDecThreads chunks per CTA. The CTA's stream words (a
+// contiguous bit range given by the side table) are staged in shared memory when they fit, and
+// the decoded indices leave through shared memory in one coalesced sweep.
+constexpr int kDecThreads = 64;
+constexpr int kDecMaxChunk = 64;
+constexpr int kDecWords = 4096;   // 128 Kbit of staged stream per CTA
+
+__global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
+    const uint32_t* words, int64_t word_capacity, const uint64_t* d_nbits, const int64_t* d_count,
+    int64_t capacity, int b, const int64_t* table, int32_t chunk, int64_t n_limit, int32_t* out,
+    int32_t* d_status) {
+  __shared__ uint32_t sw[kDecWords];
+  __shared__ int32_t so[kDecThreads * (kDecMaxChunk + 1)];
   const int64_t K = *d_count;
   if (K < 0 || K > capacity) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise(d_status, GSPARSE_DERR_CAPACITY);
     return;
   }
-  const int64_t nch = cdiv(K, chunk);
-  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= nch) return;
   const uint64_t nbits = *d_nbits;
   if (nbits > (uint64_t)word_capacity * 32u) {
-    if (c == 0) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
     return;
   }
-  uint64_t t = (uint64_t)table[2 * c];
-  int64_t prev = table[2 * c + 1];
-  const int64_t first = c * chunk;
-  const int64_t count = (K - first) < chunk ? (K - first) : chunk;
-  if (t > nbits) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return; }
-  if (!decode_run(words, nbits, t, prev, count, b, n_limit, out + first, d_status)) return;
-  const bool last = c + 1 == nch;
-  const uint64_t end = last ? nbits : (uint64_t)table[2 * (c + 1)];
-  if (t != end || (!last && prev != table[2 * (c + 1) + 1])) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+  const int64_t nch = cdiv(K, chunk);
+  const int64_t c0 = (int64_t)blockIdx.x * kDecThreads;
+  if (c0 >= nch) return;
+  const int64_t c = c0 + threadIdx.x;
+  const int64_t c1 = c0 + kDecThreads < nch ? c0 + kDecThreads : nch;  // chunks of this CTA
+  // the CTA's bit range, clamped to the stream
+  uint64_t ba = (uint64_t)table[2 * c0];
+  uint64_t bz = c1 < nch ? (uint64_t)table[2 * c1] : nbits;
+  ba = ba < nbits ? ba : nbits;
+  bz = bz < nbits ? (bz > ba ? bz : ba) : nbits;
+  const int64_t nw = cdiv((int64_t)nbits, 32);
+  const int64_t wa = (int64_t)(ba >> 5), wz = cdiv((int64_t)bz, 32) + 1;   // one spare word
+  const bool staged = wz - wa <= kDecWords && chunk <= kDecMaxChunk;
+  if (staged) {
+    const int span = (int)(wz - wa);
+#pragma unroll 8
+    for (int k = threadIdx.x; k < span; k += kDecThreads) sw[k] = wa + k < nw ? words[wa + k] : 0u;
+    __syncthreads();
+  }
+  bool ok = true;
+  if (c < nch) {
+    uint64_t t = (uint64_t)table[2 * c];
+    int64_t prev = table[2 * c + 1];
+    const int64_t first = c * chunk;
+    const int64_t count = (K - first) < chunk ? (K - first) : chunk;
+    int32_t* dst = staged ? so + threadIdx.x * (kDecMaxChunk + 1) : out + first;
+    if (t > nbits) {
+      raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+      ok = false;
+    } else if (staged && (t < ba || t > bz)) {
+      raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);  // the side table is not ascending
+      ok = false;
+    } else {
+      const uint32_t* src = staged ? sw : words;
+      const int64_t base_w = staged ? wa : 0;
+      const int64_t lim_w = staged ? wz : nw;
+      ok = decode_run(src, base_w, lim_w, nbits, t, prev, count, b, n_limit, dst, d_status);
+      if (ok) {
+        const bool last = c + 1 == nch;
+        const uint64_t end = last ? nbits : (uint64_t)table[2 * (c + 1)];
+        if (t != end || (!last && prev != table[2 * (c + 1) + 1])) {
+          raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+          ok = false;
+        }
+      }
+    }
+  }
+  if (staged) {
+    __syncthreads();
+    // chunk by chunk: the CTA's indices are contiguous in the output
+    for (int cc = 0; cc < (int)(c1 - c0); ++cc) {
+      const int64_t first = (c0 + cc) * chunk;
+      const int cnt = (int)((K - first) < chunk ? (K - first) : chunk);
+      for (int kk = threadIdx.x; kk < cnt; kk += kDecThreads) out[first + kk] = so[cc * (kDecMaxChunk + 1) + kk];
+    }
+  }
+  (void)ok;
 }
 
 __global__ void g_decode_serial_kernel(const uint32_t* words, int64_t word_capacity,
@@ -303,7 +373,8 @@ __global__ void g_decode_serial_kernel(const uint32_t* words, int64_t word_capac
   if (nbits > (uint64_t)word_capacity * 32u) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return; }
   uint64_t t = 0;
   int64_t prev = base - 1;
-  if (!decode_run(words, nbits, t, prev, K, b, n_limit, out, d_status)) return;
+  if (!decode_run(words, 0, cdiv((int64_t)nbits, 32), nbits, t, prev, K, b, n_limit, out, d_status))
+    return;
   if (t != nbits) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
 }
 
@@ -373,7 +444,7 @@ int gsparse_golomb_decode(const uint32_t* words, int64_t word_capacity, const ui
   if (b < 0 || b > 30 || capacity > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
   if (chunk_table) {
     const int64_t nch = cdiv(capacity > 0 ? capacity : 1, chunk);
-    g_decode_chunks_kernel<<<(unsigned)cdiv(nch, 128), 128, 0, st>>>(
+    g_decode_chunks_kernel<<<(unsigned)cdiv(nch, kDecThreads), kDecThreads, 0, st>>>(
         words, word_capacity, d_nbits, d_count, capacity, b, chunk_table, chunk, n_limit, out_idx,
         d_status);
   } else {

@@ -150,66 +150,129 @@ __global__ void __launch_bounds__(kTileThreads) sa_merge_kernel(Lists L, int32_t
   }
 }
 
-// Fused receive side: per tile, the worker-ordered sum G lives only in shared memory and the
-// combined gradient is streamed out directly (G itself is written only when asked for).
-__global__ void __launch_bounds__(kTileThreads) sa_combine_kernel(Lists L, int32_t W, int64_t n,
-                                                                  const int64_t* start, const float* Lg,
-                                                                  float* out, float alpha, float beta,
+// Fused receive side. A persistent CTA owns a contiguous run of tiles; for each tile it
+// requests the local-gradient tile first, adds the workers' entries falling in the tile into a
+// shared accumulator (worker by worker, so the sums keep the fixed order), streams out
+// fl(fl(alpha * G) + fl(beta * L)) and finally clears only the entries it touched, so the
+// accumulator is zeroed once per CTA rather than once per tile. The sorted lists are walked
+// forward from one binary search per worker at the CTA's first tile: no bounds pass.
+constexpr int kCombThreads = 256;
+
+__global__ void __launch_bounds__(kCombThreads) sa_combine_kernel(Lists L, int32_t W, int64_t n,
+                                                                  int64_t tiles_per_cta,
+                                                                  const float* Lg, float* out,
+                                                                  float alpha, float beta,
                                                                   int32_t own, float* dense,
                                                                   int32_t* d_status) {
-  constexpr int kVec = kTile / 4 / kTileThreads;  // float4s of the tile per thread
+  constexpr int kVec = kTile / 4 / kCombThreads;  // float4s of a tile per thread
   __shared__ __align__(16) float acc[kTile];
   __shared__ uint32_t touched[kTile / 32];
-  const int64_t t = blockIdx.x;
-  const int64_t t0 = t * kTile;
-  const int64_t m = (n - t0) < kTile ? (n - t0) : kTile;
-  // the local-gradient tile is requested first, so its latency overlaps the accumulation
-  float4 lv[kVec];
-  if (m == kTile) {
-#pragma unroll
-    for (int k = 0; k < kVec; ++k) lv[k] = ld_stream(Lg + t0 + 4 * (threadIdx.x + k * kTileThreads));
-  }
+  __shared__ int64_t cur[GSPARSE_MAX_WORKERS], cnt[GSPARSE_MAX_WORKERS];
+  __shared__ int64_t own_b, own_e;
+  const int64_t ntiles = cdiv(n, kTile);
+  const int64_t T0 = (int64_t)blockIdx.x * tiles_per_cta;
+  const int64_t T1 = T0 + tiles_per_cta < ntiles ? T0 + tiles_per_cta : ntiles;
+  if (T0 >= T1) return;
   for (int i = threadIdx.x; i < kTile; i += blockDim.x) acc[i] = 0.0f;
   for (int i = threadIdx.x; i < kTile / 32; i += blockDim.x) touched[i] = 0u;
+  for (int w = threadIdx.x; w < W; w += blockDim.x) {
+    const int64_t c = list_count(L, w);
+    cnt[w] = c;
+    cur[w] = lower_bound_i32(L.idx[w], c, T0 * kTile);
+    if (T0 == 0 && c > 0 && L.idx[w][0] < 0) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
+    if (*L.cnt[w] > L.cap[w] && blockIdx.x == 0) raise(d_status, GSPARSE_DERR_CAPACITY);
+  }
   __syncthreads();
-  accumulate_tile(L, W, t, start, acc, touched, d_status);
-  if (dense) {
+  for (int64_t t = T0; t < T1; ++t) {
+    const int64_t t0 = t * kTile;
+    const int64_t m = (n - t0) < kTile ? (n - t0) : kTile;
+    const int64_t tend = t0 + m;
+    float4 lv[kVec];
     if (m == kTile) {
-      for (int v = threadIdx.x; v < kTile / 4; v += blockDim.x)
-        st_stream(dense + t0 + 4 * v, reinterpret_cast<const float4*>(acc)[v]);
-    } else {
-      for (int i = threadIdx.x; i < m; i += blockDim.x) dense[t0 + i] = acc[i];
-    }
-  }
-  if (own >= 0) {
-    // partial mode: the worker's own sent values leave G before the combination
-    __syncthreads();
-    const int64_t b = start[t * W + own], e = start[(t + 1) * W + own];
-    const int32_t* ix = L.idx[own];
-    const float* vv = L.val[own];
-    const float u = (vv || !L.uni[own]) ? 0.0f : *L.uni[own];
-    for (int64_t j = b + threadIdx.x; j < e; j += blockDim.x) {
-      const int off = (int)(ix[j] - t0);
-      if (off >= 0 && off < kTile) acc[off] = __fsub_rn(acc[off], vv ? vv[j] : u);
-    }
-    __syncthreads();
-  }
-  if (m == kTile) {
 #pragma unroll
-    for (int k = 0; k < kVec; ++k) {
-      const int v = threadIdx.x + k * kTileThreads;
-      const float4 g = reinterpret_cast<const float4*>(acc)[v];
-      float4 o;
-      o.x = __fadd_rn(__fmul_rn(alpha, g.x), __fmul_rn(beta, lv[k].x));
-      o.y = __fadd_rn(__fmul_rn(alpha, g.y), __fmul_rn(beta, lv[k].y));
-      o.z = __fadd_rn(__fmul_rn(alpha, g.z), __fmul_rn(beta, lv[k].z));
-      o.w = __fadd_rn(__fmul_rn(alpha, g.w), __fmul_rn(beta, lv[k].w));
-      st_stream(out + t0 + 4 * v, o);
+      for (int k = 0; k < kVec; ++k) lv[k] = ld_stream(Lg + t0 + 4 * (threadIdx.x + k * kCombThreads));
     }
-  } else {
-    for (int i = threadIdx.x; i < m; i += blockDim.x)
-      out[t0 + i] = __fadd_rn(__fmul_rn(alpha, acc[i]), __fmul_rn(beta, Lg[t0 + i]));
+    for (int w = 0; w < W; ++w) {
+      const int32_t* ix = L.idx[w];
+      const float* vv = L.val[w];
+      const float u = (vv || !L.uni[w]) ? 0.0f : *L.uni[w];
+      const int64_t c = cnt[w];
+      int64_t b = cur[w];
+      if (w == own && threadIdx.x == 0) own_b = b;
+      for (;;) {
+        const int64_t j = b + threadIdx.x;
+        const int32_t i = j < c ? ix[j] : INT32_MAX;
+        const bool in = i < tend;             // a prefix: the list is ascending
+        if (in) {
+          if (j > 0 && ix[j - 1] >= i) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
+          const int off = (int)(i - t0);
+          if (off >= 0 && off < kTile) {
+            acc[off] = __fadd_rn(acc[off], vv ? vv[j] : u);
+            atomicOr(&touched[off >> 5], 1u << (off & 31));
+          }
+        }
+        const int nin = __syncthreads_count(in);
+        b += nin;
+        if (nin < kCombThreads) break;
+      }
+      if (threadIdx.x == 0) {
+        cur[w] = b;
+        if (w == own) own_e = b;
+      }
+      __syncthreads();  // worker order: all of worker w before any of worker w + 1
+    }
+    if (dense) {
+      if (m == kTile) {
+        for (int v = threadIdx.x; v < kTile / 4; v += blockDim.x)
+          st_stream(dense + t0 + 4 * v, reinterpret_cast<const float4*>(acc)[v]);
+      } else {
+        for (int i = threadIdx.x; i < m; i += blockDim.x) dense[t0 + i] = acc[i];
+      }
+    }
+    if (own >= 0) {
+      // partial mode: the worker's own sent values leave G before the combination
+      const int32_t* ix = L.idx[own];
+      const float* vv = L.val[own];
+      const float u = (vv || !L.uni[own]) ? 0.0f : *L.uni[own];
+      for (int64_t j = own_b + threadIdx.x; j < own_e; j += blockDim.x) {
+        const int off = (int)(ix[j] - t0);
+        if (off >= 0 && off < kTile) acc[off] = __fsub_rn(acc[off], vv ? vv[j] : u);
+      }
+      __syncthreads();
+    }
+    if (m == kTile) {
+#pragma unroll
+      for (int k = 0; k < kVec; ++k) {
+        const int v = threadIdx.x + k * kCombThreads;
+        const float4 g = reinterpret_cast<const float4*>(acc)[v];
+        float4 o;
+        o.x = __fadd_rn(__fmul_rn(alpha, g.x), __fmul_rn(beta, lv[k].x));
+        o.y = __fadd_rn(__fmul_rn(alpha, g.y), __fmul_rn(beta, lv[k].y));
+        o.z = __fadd_rn(__fmul_rn(alpha, g.z), __fmul_rn(beta, lv[k].z));
+        o.w = __fadd_rn(__fmul_rn(alpha, g.w), __fmul_rn(beta, lv[k].w));
+        st_stream(out + t0 + 4 * v, o);
+      }
+    } else {
+      for (int i = threadIdx.x; i < m; i += blockDim.x)
+        out[t0 + i] = __fadd_rn(__fmul_rn(alpha, acc[i]), __fmul_rn(beta, Lg[t0 + i]));
+    }
+    __syncthreads();
+    // clear what this tile touched (thread k owns bitmap word k)
+    for (int k = threadIdx.x; k < kTile / 32; k += blockDim.x) {
+      uint32_t word = touched[k];
+      touched[k] = 0u;
+      while (word) {
+        const int bit = __ffs(word) - 1;
+        word &= word - 1;
+        acc[k * 32 + bit] = 0.0f;
+      }
+    }
+    __syncthreads();
   }
+  // entries at or beyond n belong to no tile: the CTA with the last tile reports them
+  if (T1 == ntiles)
+    for (int w = threadIdx.x; w < W; w += blockDim.x)
+      if (cur[w] < cnt[w]) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -355,10 +418,11 @@ int gsparse_accumulate_combine(const gsparse_list* lists, int32_t W, int64_t n, 
   if (workspace_bytes < S.bytes) return GSPARSE_ERR_WORKSPACE;
   const int64_t ntiles = cdiv(n, kTile);
   if (ntiles == 0) return launch_status();
-  const int64_t nb = (ntiles + 1) * W;
-  sa_bounds_kernel<<<(unsigned)cdiv(nb, 256), 256, 0, st>>>(Ls, W, n, ntiles, S.start, d_status);
-  sa_combine_kernel<<<(unsigned)ntiles, kTileThreads, 0, st>>>(Ls, W, n, S.start, L, out, alpha, beta,
-                                                               mode == 1 ? own : -1, dense_out, d_status);
+  (void)S;
+  const int64_t ctas_target = (int64_t)sm_count() * 4;
+  const int64_t per = cdiv(ntiles, ctas_target < ntiles ? ctas_target : ntiles);
+  sa_combine_kernel<<<(unsigned)cdiv(ntiles, per), kCombThreads, 0, st>>>(
+      Ls, W, n, per, L, out, alpha, beta, mode == 1 ? own : -1, dense_out, d_status);
   return launch_status();
 }
 

@@ -552,15 +552,18 @@ __global__ void __launch_bounds__(kThreads, 4) pass1_kernel(Sel a) {
 // The pending residual writes must be strictly ascending indices in [0, n): anything else stops
 // the call before it touches the residual.
 __global__ void pending_check_kernel(Sel a) {
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (j == 0 && *a.pw_count > a.pw_cap) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t == 0 && *a.pw_count > a.pw_cap) {
     raise(a.d_status, GSPARSE_DERR_CAPACITY);
     a.ctl[0] = 1;
   }
   const uint32_t c = pending_count(a);
-  if (j >= c) return;
-  const int32_t i = a.pw_idx[j];
-  if (i < 0 || (int64_t)i >= a.n || (j > 0 && a.pw_idx[j - 1] >= i)) {
+  bool bad = false;
+  for (int64_t j = t; j < c; j += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t i = a.pw_idx[j];
+    bad |= i < 0 || (int64_t)i >= a.n || (j > 0 && a.pw_idx[j - 1] >= i);
+  }
+  if (__any_sync(kFull, bad) && (threadIdx.x & 31) == 0) {
     raise(a.d_status, GSPARSE_DERR_INDEX_RANGE);
     a.ctl[0] = 1;
   }
@@ -1212,7 +1215,8 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   if (cudaMemsetAsync(L.zero_begin, 0, L.zero_bytes, st) != cudaSuccess) return GSPARSE_ERR_CUDA;
   plan_kernel<<<1, 1024, 0, st>>>(a, seg, num, den, out_capacity, C == 1 ? out_offsets : nullptr);
   if (has_pending)
-    pending_check_kernel<<<(unsigned)cdiv(a.pw_cap, 256), 256, 0, st>>>(a);
+    pending_check_kernel<<<(unsigned)(cdiv(a.pw_cap, 256) < 148 * 8 ? cdiv(a.pw_cap, 256) : 148 * 8), 256, 0,
+                           st>>>(a);
   if (num == 0 && C == 1 && !has_pending) {  // communication delay step: accumulate only
     if (n > 0) {
       const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
