@@ -392,8 +392,159 @@ __device__ __forceinline__ int cand_class(float x) {
   return C == 1 ? 0 : (int)(__float_as_uint(x) >> 31);
 }
 
+// Per-warp state of pass 1 over one piece.
+struct P1State {
+  uint32_t count;   // candidates found so far
+  uint32_t cp;      // next pending write of this piece
+  int32_t win_idx;  // pending window (entry cp + lane), loaded one chunk ahead
+  float win_val;
+};
+
+__device__ __forceinline__ void load_window(const Sel& a, uint32_t cp, uint32_t cend, int lane,
+                                            P1State& S) {
+  const uint32_t j = cp + lane;
+  S.win_idx = j < cend ? a.pw_idx[j] : INT32_MAX;
+  S.win_val = j < cend ? a.pw_val[j] : 0.0f;
+}
+
+// One chunk of 512 entries [base, base + 512) of the piece [lo, hi): pending writes, acc, the
+// candidate test and ordered store, the histogram, and the residual write-back. gv/rv hold the
+// chunk (entries outside the piece, as marked by `valid`, are ignored).
 template <int C>
-__global__ void __launch_bounds__(kThreads, 4) pass1_kernel(Sel a) {
+__device__ __forceinline__ void pass1_chunk(const Sel& a, uint32_t base, uint32_t lo, uint32_t hi,
+                                            bool full, uint32_t valid, float4 (&gv)[4],
+                                            float4 (&rv)[4], P1State& S, uint32_t cend,
+                                            const uint32_t (&tl)[C], float* st, uint32_t cap,
+                                            int32_t* cidx, float* cval, uint32_t* hsink,
+                                            int hstride, int lane) {
+  float4* st4 = reinterpret_cast<float4*>(st);
+  float* r = a.r;
+  if (S.cp < cend) {
+    // pending residual writes that fall in this chunk replace those residual entries
+    const uint32_t lim = base + (uint32_t)kGranule < hi ? base + (uint32_t)kGranule : hi;
+    bool staged = false;
+    for (;;) {
+      const bool in = S.win_idx >= (int32_t)base && S.win_idx < (int32_t)lim;
+      const uint32_t mask = __ballot_sync(kFull, in);
+      if (!mask) break;
+      if (!staged) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = rv[u];
+        __syncwarp();
+        staged = true;
+      }
+      if (in) st[S.win_idx - (int32_t)base] = S.win_val;
+      S.cp += __popc(mask);
+      __syncwarp();
+      load_window(a, S.cp, cend, lane, S);   // the next window (for this chunk if it was full)
+      if (mask != kFull) break;
+    }
+    if (staged) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) rv[u] = st4[u * 32 + lane];
+      __syncwarp();
+    }
+  }
+  float4 av[4];
+  uint32_t m16 = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    av[u] = make_float4(__fadd_rn(gv[u].x, rv[u].x), __fadd_rn(gv[u].y, rv[u].y),
+                        __fadd_rn(gv[u].z, rv[u].z), __fadd_rn(gv[u].w, rv[u].w));
+    m16 |= (cand_bit<C>(av[u].x, tl) | (cand_bit<C>(av[u].y, tl) << 1) |
+            (cand_bit<C>(av[u].z, tl) << 2) | (cand_bit<C>(av[u].w, tl) << 3)) << (4 * u);
+  }
+  m16 &= valid;
+  // per-quarter counts packed in bytes; one warp scan serves all four quarters
+  const uint32_t packed = __popc(m16 & 0xFu) | (__popc(m16 & 0xF0u) << 8) |
+                          (__popc(m16 & 0xF00u) << 16) | (__popc(m16 & 0xF000u) << 24);
+  const uint32_t incl = warp_inclusive_scan(packed);
+  const uint32_t tot = __shfl_sync(kFull, incl, 31);
+  bool from_stage = false;
+  if (tot) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = av[u];
+    __syncwarp();
+    const uint32_t excl = incl - packed;
+    const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu;
+    uint32_t stored = 0;
+    for (uint32_t m = m16; m; m &= m - 1) {
+      const int b = __ffs(m) - 1;
+      const int u = b >> 2, e = b & 3;
+      const uint32_t before = (u >= 1 ? t0 : 0u) + (u >= 2 ? t1 : 0u) + (u >= 3 ? t2 : 0u);
+      const uint32_t pos = S.count + before + ((excl >> (8 * u)) & 0xFFu) +
+                           __popc(m16 & ((1u << b) - 1u) & (0xFu << (4 * u)));
+      const float x = st[(u * 32 + lane) * 4 + e];
+      if (pos < cap) {
+        cidx[pos] = (int32_t)(base + u * 128 + lane * 4 + e);
+        cval[pos] = x;
+        stored |= 1u << b;
+      }
+      atomicAdd(hsink + cand_class<C>(x) * hstride + (mag_key(x) >> 20), 1u);
+    }
+    S.count += t0 + t1 + t2 + (tot >> 24);
+    if (a.zero_mode) {
+      // stored candidates leave the residual as +0 (the not-sent ones get acc back later)
+      for (uint32_t m = stored; m; m &= m - 1) {
+        const int b = __ffs(m) - 1;
+        st[((b >> 2) * 32 + lane) * 4 + (b & 3)] = 0.0f;
+      }
+      __syncwarp();
+      from_stage = true;
+    }
+  }
+  if (full) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      st_stream(r + base + u * 128 + lane * 4, from_stage ? st4[u * 32 + lane] : av[u]);
+  } else {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 o = from_stage ? st4[u * 32 + lane] : av[u];
+      const float ov[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((valid >> (4 * u + e)) & 1u) r[base + u * 128 + lane * 4 + e] = ov[e];
+    }
+  }
+  __syncwarp();
+}
+
+// First or last chunk of a piece: entry-wise bounds.
+__device__ __forceinline__ uint32_t load_edge(const Sel& a, uint32_t base, uint32_t lo, uint32_t hi,
+                                              int lane, float4 (&gv)[4], float4 (&rv)[4]) {
+  uint32_t valid = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    float t0[4], t1[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t i = base + u * 128 + lane * 4 + e;
+      const bool in = i >= lo && i < hi;
+      t0[e] = in ? a.g[i] : 0.0f;
+      t1[e] = in ? a.r[i] : 0.0f;
+      valid |= (uint32_t)in << (4 * u + e);
+    }
+    gv[u] = make_float4(t0[0], t0[1], t0[2], t0[3]);
+    rv[u] = make_float4(t1[0], t1[1], t1[2], t1[3]);
+  }
+  return valid;
+}
+
+__device__ __forceinline__ void load_full(const Sel& a, uint32_t base, int lane, float4 (&gv)[4],
+                                          float4 (&rv)[4]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    gv[u] = ld_stream(a.g + base + u * 128 + lane * 4);
+    rv[u] = ld_stream(a.r + base + u * 128 + lane * 4);
+  }
+}
+
+// The streaming pass: one warp per piece. Interior chunks are software pipelined: the next
+// chunk's g and r (and the next window of pending writes) are in flight while this one is
+// processed.
+template <int C>
+__global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
   __shared__ CtaHist<C, kBins1> H;
   __shared__ __align__(16) float stage[kWarps * kGranule];  // per warp: one chunk, entry order
   if (a.ctl[0]) return;
@@ -415,135 +566,43 @@ __global__ void __launch_bounds__(kThreads, 4) pass1_kernel(Sel a) {
     uint32_t* hsink = sh_sink ? H.sh : hist_of(a, (int64_t)P.s * C, 1);
     const int hstride = sh_sink ? kBins1 : kHist;
     const uint32_t lo = (uint32_t)P.lo, hi = (uint32_t)P.hi;  // indices are below 2^31
-    const float* g = a.g;
-    float* r = a.r;
     float* st = stage + wid * kGranule;
-    float4* st4 = reinterpret_cast<float4*>(st);
-    // pending residual writes of this piece: [cp, cend) of the sorted list
+    // pending residual writes of this piece start at the first index >= lo
     const uint32_t cend = pending_count(a);
-    uint32_t cp = 0;
-    if (cend) cp = __shfl_sync(kFull, lane == 0 ? (uint32_t)lower_bound_i32(a.pw_idx, cend, lo) : 0u, 0);
-    uint32_t count = 0;
-    for (uint32_t base = lo & ~3u; base < hi; base += (uint32_t)kGranule) {
-      const bool full = base >= lo && base + (uint32_t)kGranule <= hi;  // warp-uniform
-      float4 gv[4], rv[4];
-      uint32_t valid = 0xFFFFu;
-      if (full) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          gv[u] = ld_stream(g + base + u * 128 + lane * 4);
-          rv[u] = ld_stream(r + base + u * 128 + lane * 4);
-        }
-      } else {
-        // first or last chunk of the piece: entry-wise bounds
-        valid = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float t0[4], t1[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t i = base + u * 128 + lane * 4 + e;
-            const bool in = i >= lo && i < hi;
-            t0[e] = in ? g[i] : 0.0f;
-            t1[e] = in ? r[i] : 0.0f;
-            valid |= (uint32_t)in << (4 * u + e);
-          }
-          gv[u] = make_float4(t0[0], t0[1], t0[2], t0[3]);
-          rv[u] = make_float4(t1[0], t1[1], t1[2], t1[3]);
-        }
-      }
-      if (cp < cend) {
-        // pending residual writes that fall in this chunk replace those residual entries
-        const uint32_t lim = base + (uint32_t)kGranule < hi ? base + (uint32_t)kGranule : hi;
-        bool staged = false;
-        for (;;) {
-          const uint32_t j = cp + lane;
-          const int32_t ci = j < cend ? a.pw_idx[j] : INT32_MAX;
-          const bool in = ci >= (int32_t)base && ci < (int32_t)lim;
-          const uint32_t mask = __ballot_sync(kFull, in);
-          if (!mask) break;
-          if (!staged) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = rv[u];
-            __syncwarp();
-            staged = true;
-          }
-          if (in) st[ci - (int32_t)base] = a.pw_val[j];
-          cp += __popc(mask);
-          __syncwarp();
-          if (mask != kFull) break;
-        }
-        if (staged) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) rv[u] = st4[u * 32 + lane];
-          __syncwarp();
-        }
-      }
-      float4 av[4];
-      uint32_t m16 = 0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        av[u] = make_float4(__fadd_rn(gv[u].x, rv[u].x), __fadd_rn(gv[u].y, rv[u].y),
-                            __fadd_rn(gv[u].z, rv[u].z), __fadd_rn(gv[u].w, rv[u].w));
-        m16 |= (cand_bit<C>(av[u].x, tl) | (cand_bit<C>(av[u].y, tl) << 1) |
-                (cand_bit<C>(av[u].z, tl) << 2) | (cand_bit<C>(av[u].w, tl) << 3)) << (4 * u);
-      }
-      m16 &= valid;
-      // per-quarter counts packed in bytes; one warp scan serves all four quarters
-      const uint32_t packed = __popc(m16 & 0xFu) | (__popc(m16 & 0xF0u) << 8) |
-                              (__popc(m16 & 0xF00u) << 16) | (__popc(m16 & 0xF000u) << 24);
-      const uint32_t incl = warp_inclusive_scan(packed);
-      const uint32_t tot = __shfl_sync(kFull, incl, 31);
-      bool from_stage = false;
-      if (tot) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = av[u];
-        __syncwarp();
-        const uint32_t excl = incl - packed;
-        const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu;
-        uint32_t stored = 0;
-        for (uint32_t m = m16; m; m &= m - 1) {
-          const int b = __ffs(m) - 1;
-          const int u = b >> 2, e = b & 3;
-          const uint32_t before = (u >= 1 ? t0 : 0u) + (u >= 2 ? t1 : 0u) + (u >= 3 ? t2 : 0u);
-          const uint32_t pos = count + before + ((excl >> (8 * u)) & 0xFFu) +
-                               __popc(m16 & ((1u << b) - 1u) & (0xFu << (4 * u)));
-          const float x = st[(u * 32 + lane) * 4 + e];
-          if (pos < cap) {
-            cidx[pos] = (int32_t)(base + u * 128 + lane * 4 + e);
-            cval[pos] = x;
-            stored |= 1u << b;
-          }
-          atomicAdd(hsink + cand_class<C>(x) * hstride + (mag_key(x) >> 20), 1u);
-        }
-        count += t0 + t1 + t2 + (tot >> 24);
-        if (a.zero_mode) {
-          // stored candidates leave the residual as +0 (the not-sent ones get acc back later)
-          for (uint32_t m = stored; m; m &= m - 1) {
-            const int b = __ffs(m) - 1;
-            st[((b >> 2) * 32 + lane) * 4 + (b & 3)] = 0.0f;
-          }
-          __syncwarp();
-          from_stage = true;
-        }
-      }
-      if (full) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          st_stream(r + base + u * 128 + lane * 4, from_stage ? st4[u * 32 + lane] : av[u]);
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 o = from_stage ? st4[u * 32 + lane] : av[u];
-          const float ov[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if ((valid >> (4 * u + e)) & 1u) r[base + u * 128 + lane * 4 + e] = ov[e];
-        }
-      }
-      __syncwarp();
+    P1State S;
+    S.count = 0;
+    S.cp = 0;
+    if (cend) S.cp = __shfl_sync(kFull, lane == 0 ? (uint32_t)lower_bound_i32(a.pw_idx, cend, lo) : 0u, 0);
+    load_window(a, S.cp, cend, lane, S);
+    uint32_t base = lo & ~3u;
+    float4 gv[4], rv[4];
+    if (base < lo || base + (uint32_t)kGranule > hi) {
+      const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
+      pass1_chunk<C>(a, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, cap, cidx, cval, hsink,
+                     hstride, lane);
+      base += (uint32_t)kGranule;
     }
-    if (lane == 0) a.pcnt[q] = count;
+    if (base < hi && base + (uint32_t)kGranule <= hi) {
+      float4 gn[4], rn[4];
+      load_full(a, base, lane, gn, rn);
+      for (;;) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) { gv[u] = gn[u]; rv[u] = rn[u]; }
+        const uint32_t nb = base + (uint32_t)kGranule;
+        const bool more = nb + (uint32_t)kGranule <= hi;
+        if (more) load_full(a, nb, lane, gn, rn);
+        pass1_chunk<C>(a, base, lo, hi, true, 0xFFFFu, gv, rv, S, cend, tl, st, cap, cidx, cval,
+                       hsink, hstride, lane);
+        base = nb;
+        if (!more) break;
+      }
+    }
+    if (base < hi) {
+      const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
+      pass1_chunk<C>(a, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, cap, cidx, cval, hsink,
+                     hstride, lane);
+    }
+    if (lane == 0) a.pcnt[q] = S.count;
   }
   __syncthreads();
   H.flush(a, 1, kBins1);
