@@ -135,6 +135,17 @@ class Clocks:
                 "samples": len(sm)}
 
 
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of a list of floats over all ranks (every rank gets the result); a
+    None entry (a leg that did not run) stays None. With dist None: the values themselves."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor([-1.0 if v is None else float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [None if v is None else float(x) for v, x in zip(values, t.tolist())]
+
+
 # ---------------------------------------------------------------------------------------------
 # our arm
 
@@ -301,10 +312,7 @@ def run_ours(args, rank, world, dist):
         e2e_ms = a.elapsed_time(z) / args.e2e_steps
 
     # max over ranks
-    if world > 1:
-        tt = torch.tensor([ms, e2e_ms or 0.0], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(tt[0]), (float(tt[1]) if e2e_ms is not None else None)
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dist if world > 1 else None, dev)
 
     if rank != 0:
         return None
