@@ -183,6 +183,8 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
   if (threadIdx.x == blockDim.x - 1) span_hi = (uint64_t)(o0 + l);   // the block's last bit + 1
   Code cs[kPer];
   int64_t o = o0;
+  // position of j0 inside its side-table chunk (one 32-bit division per thread; indices < 2^31)
+  uint32_t in_chunk = table ? (uint32_t)j0 % (uint32_t)chunk : 1u;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     const int64_t j = j0 + e;
@@ -192,12 +194,14 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
     cs[e].tail = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
     cs[e].len_tail = 1u + (uint32_t)b;
     if (j < len) {
-      if (table && j % chunk == 0) {
-        table[2 * (j / chunk)] = o;
-        table[2 * (j / chunk) + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
+      if (table && in_chunk == 0) {
+        const int64_t c = (int64_t)((uint32_t)j / (uint32_t)chunk);
+        table[2 * c] = o;
+        table[2 * c + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
       }
       o += (int64_t)cs[e].q + cs[e].len_tail;
     }
+    if (table && ++in_chunk == (uint32_t)chunk) in_chunk = 0;
   }
   __syncthreads();
   const uint64_t S = span_lo, E = span_hi;
@@ -211,12 +215,25 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
   for (int e = 0; e < kPer; ++e) {
     if (j0 + e >= len) break;
     const Code& c = cs[e];
-    const uint64_t w0 = c.o >> 5, w1 = (c.o + c.q + c.len_tail - 1) >> 5;
-    for (uint64_t w = w0; w <= w1; ++w) {
-      const uint32_t bits = code_bits_in_word(c, w);
-      if (!bits) continue;
-      if (fits) atomicOr(&wbuf[w - wf], bits);
-      else atomicOr(&words[w], bits);
+    if (fits) {
+      // positions relative to the block's first word: the block spans < 2^17 bits here
+      uint32_t p = (uint32_t)(c.o - 32u * wf);
+      uint32_t q = (uint32_t)c.q;
+      while (q) {  // the unary run of ones
+        const uint32_t sh = p & 31u, nrun = q < 32u - sh ? q : 32u - sh;
+        atomicOr(&wbuf[p >> 5], (nrun == 32u ? 0xffffffffu : ((1u << nrun) - 1u)) << sh);
+        p += nrun;
+        q -= nrun;
+      }
+      const uint64_t v = (uint64_t)c.tail << (p & 31u);  // terminator + remainder, <= 31 bits
+      if ((uint32_t)v) atomicOr(&wbuf[p >> 5], (uint32_t)v);
+      if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(p >> 5) + 1], (uint32_t)(v >> 32));
+    } else {
+      const uint64_t w0 = c.o >> 5, w1 = (c.o + c.q + c.len_tail - 1) >> 5;
+      for (uint64_t w = w0; w <= w1; ++w) {
+        const uint32_t bits = code_bits_in_word(c, w);
+        if (bits) atomicOr(&words[w], bits);
+      }
     }
   }
   if (!fits) return;
@@ -281,19 +298,59 @@ __device__ bool decode_run(const uint32_t* src, int64_t base_w, int64_t lim_w, u
   return true;
 }
 
+// Decodes `count` codewords from a staged window: sw holds stream words [wa, wa + nwin) (the last
+// one a zero spare), t is the bit position relative to bit 32 * wa, and nb_rel the stream end
+// relative to the same origin (at most 32 * (nwin - 1)). 32-bit positions throughout.
+__device__ bool decode_run_local(const uint32_t* sw, uint32_t nb_rel, uint32_t& t, int64_t& prev,
+                                 int count, int b, int64_t n_limit, int32_t* out, int stride,
+                                 int32_t* d_status) {
+  for (int k = 0; k < count; ++k) {
+    uint32_t q = 0;
+    for (;;) {
+      if (t >= nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+      const uint32_t sh = t & 31u;
+      const uint32_t zeros = ~(sw[t >> 5] >> sh) & (0xffffffffu >> sh);
+      if (zeros) {
+        const uint32_t z = (uint32_t)__ffs(zeros) - 1u;
+        q += z;
+        t += z + 1u;
+        break;
+      }
+      q += 32u - sh;
+      t += 32u - sh;
+    }
+    uint32_t rem = 0;
+    if (b > 0) {
+      if (t > nb_rel || nb_rel - t < (uint32_t)b) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+      const uint32_t w = t >> 5;
+      const uint64_t win = (uint64_t)sw[w] | ((uint64_t)sw[w + 1] << 32);
+      rem = __brev((uint32_t)(win >> (t & 31u)) & ((1u << b) - 1u)) >> (32 - b);
+      t += (uint32_t)b;
+    } else if (t > nb_rel) {
+      raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+      return false;
+    }
+    const int64_t i = prev + 1 + (int64_t)(((uint64_t)q << b) | rem);
+    if (i >= n_limit || i > INT32_MAX) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); return false; }
+    out[k * stride] = (int32_t)i;
+    prev = i;
+  }
+  return true;
+}
+
 // One thread per chunk of codewords, kDecThreads chunks per CTA. The CTA's stream words (a
 // contiguous bit range given by the side table) are staged in shared memory when they fit, and
-// the decoded indices leave through shared memory in one coalesced sweep.
+// decoded there with 32-bit positions; otherwise the thread reads global memory.
 constexpr int kDecThreads = 64;
-constexpr int kDecMaxChunk = 64;
-constexpr int kDecWords = 4096;   // 128 Kbit of staged stream per CTA
+constexpr int kDecWords = 2048;   // 64 Kbit of staged stream per CTA
+constexpr int kDecMaxChunk = 64;  // outputs staged when the chunk is at most this long
 
 __global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
     const uint32_t* words, int64_t word_capacity, const uint64_t* d_nbits, const int64_t* d_count,
     int64_t capacity, int b, const int64_t* table, int32_t chunk, int64_t n_limit, int32_t* out,
     int32_t* d_status) {
   __shared__ uint32_t sw[kDecWords];
-  __shared__ int32_t so[kDecThreads * (kDecMaxChunk + 1)];
+  __shared__ int32_t so[kDecMaxChunk * (kDecThreads + 1)];  // [codeword][chunk], padded
   const int64_t K = *d_count;
   if (K < 0 || K > capacity) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise(d_status, GSPARSE_DERR_CAPACITY);
@@ -315,52 +372,53 @@ __global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
   ba = ba < nbits ? ba : nbits;
   bz = bz < nbits ? (bz > ba ? bz : ba) : nbits;
   const int64_t nw = cdiv((int64_t)nbits, 32);
-  const int64_t wa = (int64_t)(ba >> 5), wz = cdiv((int64_t)bz, 32) + 1;   // one spare word
-  const bool staged = wz - wa <= kDecWords && chunk <= kDecMaxChunk;
+  const int64_t wa = (int64_t)(ba >> 5), wz = cdiv((int64_t)bz, 32) + 1;   // one zero spare word
+  const bool staged = wz - wa <= kDecWords;
   if (staged) {
     const int span = (int)(wz - wa);
-#pragma unroll 8
+#pragma unroll 4
     for (int k = threadIdx.x; k < span; k += kDecThreads) sw[k] = wa + k < nw ? words[wa + k] : 0u;
     __syncthreads();
   }
-  bool ok = true;
+  // outputs go through shared memory when staged, so they leave as whole rows (coalesced)
+  const bool stage_out = staged && chunk <= kDecMaxChunk;
   if (c < nch) {
     uint64_t t = (uint64_t)table[2 * c];
     int64_t prev = table[2 * c + 1];
     const int64_t first = c * chunk;
-    const int64_t count = (K - first) < chunk ? (K - first) : chunk;
-    int32_t* dst = staged ? so + threadIdx.x * (kDecMaxChunk + 1) : out + first;
-    if (t > nbits) {
-      raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
-      ok = false;
-    } else if (staged && (t < ba || t > bz)) {
-      raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);  // the side table is not ascending
-      ok = false;
+    const int count = (int)((K - first) < chunk ? (K - first) : chunk);
+    if (t > nbits || (staged && (t < ba || t > bz))) {
+      raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);   // the side table does not fit the stream
     } else {
-      const uint32_t* src = staged ? sw : words;
-      const int64_t base_w = staged ? wa : 0;
-      const int64_t lim_w = staged ? wz : nw;
-      ok = decode_run(src, base_w, lim_w, nbits, t, prev, count, b, n_limit, dst, d_status);
+      bool ok;
+      if (staged) {
+        // the window's end: this CTA's range, so a chunk cannot run into the next CTA's bits
+        uint32_t tl = (uint32_t)(t - 32u * (uint64_t)wa);
+        const uint32_t nb_rel = (uint32_t)(bz - 32u * (uint64_t)wa);
+        if (stage_out)
+          ok = decode_run_local(sw, nb_rel, tl, prev, count, b, n_limit, so + threadIdx.x,
+                               kDecThreads + 1, d_status);
+        else
+          ok = decode_run_local(sw, nb_rel, tl, prev, count, b, n_limit, out + first, 1, d_status);
+        t = 32u * (uint64_t)wa + tl;
+      } else {
+        ok = decode_run(words, 0, nw, nbits, t, prev, count, b, n_limit, out + first, d_status);
+      }
       if (ok) {
         const bool last = c + 1 == nch;
         const uint64_t end = last ? nbits : (uint64_t)table[2 * (c + 1)];
-        if (t != end || (!last && prev != table[2 * (c + 1) + 1])) {
-          raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
-          ok = false;
-        }
+        if (t != end || (!last && prev != table[2 * (c + 1) + 1])) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
       }
     }
   }
-  if (staged) {
+  if (stage_out) {
     __syncthreads();
-    // chunk by chunk: the CTA's indices are contiguous in the output
     for (int cc = 0; cc < (int)(c1 - c0); ++cc) {
       const int64_t first = (c0 + cc) * chunk;
       const int cnt = (int)((K - first) < chunk ? (K - first) : chunk);
-      for (int kk = threadIdx.x; kk < cnt; kk += kDecThreads) out[first + kk] = so[cc * (kDecMaxChunk + 1) + kk];
+      if ((int)threadIdx.x < cnt) out[first + threadIdx.x] = so[threadIdx.x * (kDecThreads + 1) + cc];
     }
   }
-  (void)ok;
 }
 
 __global__ void g_decode_serial_kernel(const uint32_t* words, int64_t word_capacity,

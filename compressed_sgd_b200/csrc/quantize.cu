@@ -40,36 +40,49 @@ __global__ void q_setup_kernel(const float* val, const int64_t* d_begin, const i
   }
 }
 
-__global__ void q_apply_kernel(const int32_t* idx, float* val, const int64_t* d_begin,
-                               const int64_t* d_end, const SumJob* jobs, float* residual, int64_t n,
-                               float* feedback, uint32_t* sign_bits, float* d_means,
-                               int32_t write_deq, const int32_t* ctl, int32_t* d_status) {
+// Four list positions per thread, j = blockIdx.x * 1024 + k * 256 + threadIdx.x (k = 0..3), so
+// the 32 lanes of a warp always hold 32 consecutive positions and one ballot is one sign word.
+constexpr int kApplyThreads = 256, kApplyPer = 4;
+
+__global__ void __launch_bounds__(kApplyThreads) q_apply_kernel(
+    const int32_t* idx, float* val, const int64_t* d_begin, const int64_t* d_end, const SumJob* jobs,
+    float* residual, int64_t n, float* feedback, uint32_t* sign_bits, float* d_means,
+    int32_t write_deq, const int32_t* ctl, int32_t* d_status) {
   if (ctl[0]) return;
   const int64_t b = d_begin ? *d_begin : 0;
   const int64_t len = *d_end - b;
   const float mp = jobs[0].mean, mn = jobs[1].mean;
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (j == 0) {
+  const int64_t j0 = (int64_t)blockIdx.x * (kApplyThreads * kApplyPer);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
     d_means[0] = mp;
     d_means[1] = mn;
   }
-  // whole warps cover 32 consecutive list positions, so one ballot is one sign word
-  const int64_t w0 = j & ~(int64_t)31;
-  if (w0 >= len) return;
-  const bool in = j < len;
-  const float x = in ? val[b + j] : 0.0f;
-  const bool neg = in && x < 0.0f;
-  const uint32_t word = __ballot_sync(kFull, neg);
-  if ((threadIdx.x & 31) == 0) sign_bits[j >> 5] = word;
-  if (!in) return;
-  const float q = x > 0.0f ? mp : (neg ? mn : 0.0f);
-  if (residual) {
-    const int32_t i = idx[b + j];
-    if (i < 0 || (int64_t)i >= n) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
-    else residual[i] = __fsub_rn(x, q);
+  float xv[kApplyPer];
+#pragma unroll
+  for (int k = 0; k < kApplyPer; ++k) {
+    const int64_t j = j0 + k * kApplyThreads + threadIdx.x;
+    xv[k] = j < len ? val[b + j] : 0.0f;
   }
-  if (feedback) feedback[j] = __fsub_rn(x, q);
-  if (write_deq) val[b + j] = q;
+#pragma unroll
+  for (int k = 0; k < kApplyPer; ++k) {
+    const int64_t j = j0 + k * kApplyThreads + threadIdx.x;
+    if ((j & ~(int64_t)31) >= len) break;  // warp-uniform: the warp's 32 positions all lie beyond
+    const bool in = j < len;
+    const float x = xv[k];
+    const bool neg = in && x < 0.0f;
+    const uint32_t word = __ballot_sync(kFull, neg);
+    if ((threadIdx.x & 31) == 0) sign_bits[j >> 5] = word;
+    if (!in) continue;
+    const float q = x > 0.0f ? mp : (neg ? mn : 0.0f);
+    const float err = __fsub_rn(x, q);
+    if (residual) {
+      const int32_t i = idx[b + j];
+      if (i < 0 || (int64_t)i >= n) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
+      else residual[i] = err;
+    }
+    if (feedback) feedback[j] = err;
+    if (write_deq) val[b + j] = q;
+  }
 }
 
 struct QLayout {
@@ -121,9 +134,8 @@ int gsparse_quantize(const int32_t* idx, float* val, const int64_t* d_begin, con
   if (workspace_bytes < L.bytes) return GSPARSE_ERR_WORKSPACE;
   q_setup_kernel<<<1, 1, 0, st>>>(val, d_begin, d_end, capacity, L.jobs, L.ctl, d_status);
   osum_launch(L.jobs, 2, L.leaves, L.leaf_bound, L.per_job, L.partials, L.ctl, st);
-  const int64_t threads = 256;
-  const int64_t blocks = cdiv(capacity > 0 ? capacity : 1, threads);
-  q_apply_kernel<<<(unsigned)blocks, (unsigned)threads, 0, st>>>(
+  const int64_t blocks = cdiv(capacity > 0 ? capacity : 1, kApplyThreads * kApplyPer);
+  q_apply_kernel<<<(unsigned)blocks, kApplyThreads, 0, st>>>(
       idx, val, d_begin, d_end, L.jobs, residual, n, feedback_out, sign_bits, d_means,
       write_dequantized, L.ctl, d_status);
   return launch_status();

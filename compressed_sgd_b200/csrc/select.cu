@@ -632,7 +632,7 @@ __global__ void pending_check_kernel(Sel a) {
 // candidate iteration for the later steps (order not needed)
 
 // Calls f(x, c, key) for every candidate value of piece q: from the piece's store (values only;
-// two float4 loads per lane in flight), or, for pieces marked to be re-read, from the residual
+// four float4 loads per lane in flight), or, for pieces marked to be re-read, from the residual
 // (which then holds acc) filtered by class and T_lo.
 template <int C, class F>
 __device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, const Piece& P, F f) {
@@ -642,16 +642,21 @@ __device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, cons
     const uint32_t cnt = a.pcnt[q];
     const float4* cv = reinterpret_cast<const float4*>(a.cval + q * a.cap);
     const uint32_t n4 = (cnt + 3) / 4;
-    for (uint32_t j4 = lane; j4 < n4; j4 += 64) {
-      const float4 X0 = cv[j4];
-      const float4 X1 = j4 + 32 < n4 ? cv[j4 + 32] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float xv[8] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w};
+    for (uint32_t j4 = lane; j4 < n4; j4 += 128) {
+      float4 X[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t j = 4 * (j4 + (e >> 2) * 32) + (e & 3);
-        if (j < cnt) {
-          const int c = class_of<C>(xv[e]);
-          f(xv[e], c < 0 ? 0 : c, mag_key(xv[e]));
+      for (int h = 0; h < 4; ++h)
+        X[h] = j4 + 32 * h < n4 ? cv[j4 + 32 * h] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float xv[4] = {X[h].x, X[h].y, X[h].z, X[h].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t j = 4 * (j4 + 32 * h) + e;
+          if (j < cnt) {
+            const int c = class_of<C>(xv[e]);
+            f(xv[e], c < 0 ? 0 : c, mag_key(xv[e]));
+          }
         }
       }
     }
@@ -891,7 +896,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(Sel a) {
 // 9. emit, in index order
 
 template <int C>
-__global__ void __launch_bounds__(kThreads) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
+__global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
                                                         int64_t limit) {
   if (a.ctl[0]) return;
   const int64_t q = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -919,15 +924,27 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(Sel a, int32_t* out_idx,
     const uint32_t cnt = a.pcnt[q];
     const int4* ci = reinterpret_cast<const int4*>(a.cidx + q * a.cap);
     const float4* cv = reinterpret_cast<const float4*>(a.cval + q * a.cap);
-    // software pipelined: the next 128 candidates are in flight while these are placed
-    int4 In = make_int4(0, 0, 0, 0);
-    float4 Xn = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (4 * lane < cnt) { In = ci[lane]; Xn = cv[lane]; }
+    // software pipelined: three batches of 128 candidates are in flight while one is placed
+    constexpr int kAhead = 3;
+    int4 Iq[kAhead];
+    float4 Xq[kAhead];
+#pragma unroll
+    for (int h = 0; h < kAhead; ++h) {
+      const uint32_t jj = 128 * h + 4 * lane;
+      Iq[h] = jj < cnt ? ci[jj >> 2] : make_int4(0, 0, 0, 0);
+      Xq[h] = jj < cnt ? cv[jj >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     for (uint32_t j0 = 0; j0 < cnt; j0 += 128) {
       const uint32_t j = j0 + 4 * lane;
-      const int4 I = In;
-      const float4 X = Xn;
-      if (j + 128 < cnt) { In = ci[(j >> 2) + 32]; Xn = cv[(j >> 2) + 32]; }
+      const int4 I = Iq[0];
+      const float4 X = Xq[0];
+#pragma unroll
+      for (int h = 0; h + 1 < kAhead; ++h) { Iq[h] = Iq[h + 1]; Xq[h] = Xq[h + 1]; }
+      {
+        const uint32_t jj = j + 128 * kAhead;
+        Iq[kAhead - 1] = jj < cnt ? ci[jj >> 2] : make_int4(0, 0, 0, 0);
+        Xq[kAhead - 1] = jj < cnt ? cv[jj >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
       int32_t iv[4] = {0, 0, 0, 0};
       float xv[4] = {0.f, 0.f, 0.f, 0.f};
       if (j < cnt) {
@@ -944,30 +961,37 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(Sel a, int32_t* out_idx,
       uint32_t selm = 0;
 #pragma unroll
       for (int cc = 0; cc < C; ++cc) {
-        uint32_t eqm = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) eqm |= (uint32_t)(cls[e] == cc && key[e] == th[cc]) << e;
-        uint32_t teq;
-        const uint32_t pre_eq = warp_prefix_small(__popc(eqm), &teq);
-        uint32_t sm = 0;
+        uint32_t eqm = 0, gtm = 0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const bool eq = (eqm >> e) & 1u;
-          const bool taken = eq && (eq_run[cc] + pre_eq + __popc(eqm & ((1u << e) - 1u))) < take[cc];
-          sm |= (uint32_t)(cls[e] == cc && is_sel(cc, key[e], taken)) << e;
+          eqm |= (uint32_t)(cls[e] == cc && key[e] == th[cc]) << e;
+          gtm |= (uint32_t)(cls[e] == cc && th[cc] != kNone && key[e] > th[cc]) << e;
+        }
+        uint32_t sm = gtm;
+        if (__any_sync(kFull, eqm)) {
+          // keys equal to the threshold: the first `take` of them in index order are sent
+          uint32_t teq;
+          const uint32_t pre_eq = warp_prefix_small(__popc(eqm), &teq);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (((eqm >> e) & 1u) && (eq_run[cc] + pre_eq + __popc(eqm & ((1u << e) - 1u))) < take[cc])
+              sm |= 1u << e;
+          eq_run[cc] += teq;
         }
         uint32_t tsel;
         const uint32_t pre_sel = warp_prefix_small(__popc(sm), &tsel);
+        if (sm) {
+          const int64_t o0 = base_out[cc] + sel_run[cc] + pre_sel;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if ((sm >> e) & 1u) {
-            const int64_t o = base_out[cc] + sel_run[cc] + pre_sel + __popc(sm & ((1u << e) - 1u));
-            if (o >= limit) raise(a.d_status, GSPARSE_DERR_CAPACITY);
-            else if (C == 1) { out_idx[o] = iv[e]; out_val[o] = xv[e]; }
-            else { a.lidx[o] = iv[e]; a.lval[o] = xv[e]; }
+          for (int e = 0; e < 4; ++e) {
+            if ((sm >> e) & 1u) {
+              const int64_t o = o0 + __popc(sm & ((1u << e) - 1u));
+              if (o >= limit) raise(a.d_status, GSPARSE_DERR_CAPACITY);
+              else if (C == 1) { out_idx[o] = iv[e]; out_val[o] = xv[e]; }
+              else { a.lidx[o] = iv[e]; a.lval[o] = xv[e]; }
+            }
           }
         }
-        eq_run[cc] += teq;
         sel_run[cc] += tsel;
         selm |= sm;
       }
