@@ -353,6 +353,182 @@ def run_ours(args, rank, world, dist):
 
 
 # ---------------------------------------------------------------------------------------------
+# the other workloads (one JSON line each; not the default line)
+
+WORKLOADS = {
+    "flat2e20": "flat fp32 gradient of 2^20 entries (95% N(0,1e-4^2), 5% N(0,1e-2^2)), 1 worker, global 99% "
+                "drop; step: residual top-k, Golomb encode/decode (b*=6), scatter-accumulate",
+    "mlp": "3-layer MNIST MLP gradient (1,863,690 entries, 6 tensors), 4 workers, per-tensor 99% drop; step per "
+           "worker: residual top-k, 2-bit quantisation per tensor with error feedback; then scatter-accumulate",
+    "nmt": "NMT-shaped gradient (147,337,216 entries), 4 workers, global 99% drop; step per worker: residual "
+           "top-k; then per worker the fused receive (sum of the 4 updates + own gradient)",
+    "resnet50": "ResNet-50-shaped gradient (25,557,032 entries, 161 tensors), 8 workers; round per worker: 9 "
+                "accumulate-only steps, sparse binarisation p=0.001, Golomb encode/decode (b*=9); then "
+                "scatter-accumulate of the 8 binarised updates",
+}
+
+
+def workload_oracle(name, g_host, n, seg, keep, b):
+    """One step of a smaller workload through the CPU oracle (zero starting residual)."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    W = len(g_host)
+    T = 1 if seg is None else len(seg) - 1
+    lists_h = []
+    for w in range(W):
+        rr = np.zeros(n, np.float32)
+        if name == "resnet50":
+            for _ in range(9):
+                _, _, _, rr = oracle.residual_topk(g_host[w], rr, (0, 1))
+            oi, ov, _, oo, rr = oracle.binarize(g_host[w], rr, keep)
+        else:
+            oi, ov, oo, rr = oracle.residual_topk(g_host[w], rr, keep, seg=seg)
+        if name == "mlp":
+            for s_ in range(T):
+                bb, ee = int(oo[s_]), int(oo[s_ + 1])
+                _, _, ov[bb:ee], rr = oracle.quantize(oi[bb:ee], ov[bb:ee], residual=rr, write_dequantized=True)
+        if name in ("flat2e20", "resnet50"):
+            ww, nb_, _ = oracle.golomb_encode(oi, b, chunk=64)
+            oi = oracle.golomb_decode(ww, nb_, oi.size, b, n_limit=n)
+        lists_h.append((oi, ov))
+    dense_h, _, _ = oracle.scatter_accumulate(lists_h, n, merged=False)
+    outs = [oracle.combine_local(dense_h, g_host[w]) for w in range(W)] if name == "nmt" else None
+    return dense_h, outs
+
+
+def run_workload(args):
+    """Times one of the smaller workloads on cuda:0 and the oracle on the same step."""
+    import numpy as np
+    import torch
+    import compressed_sgd_b200 as gs
+    import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    name = args.workload
+    keep = (1, 100)
+    seg = None
+    if name == "flat2e20":
+        n, W = 1 << 20, 1
+        gen = lambda w: synth.flat_mixture(n, seed=w)
+    elif name == "mlp":
+        seg = synth.offsets(synth.mlp_layout())
+        n, W = int(seg[-1]), 4
+        gen = lambda w: synth.mlp_gradient(w, 0)
+    elif name == "nmt":
+        n, W = int(synth.offsets(synth.nmt_layout())[-1]), 4
+        gen = lambda w: synth.nmt_gradient(w, 0)
+    else:
+        n, W = int(synth.offsets(synth.resnet50_layout())[-1]), 8
+        keep = (1, 1000)
+        gen = lambda w: synth.resnet50_gradient(w, 0)
+    T = 1 if seg is None else len(seg) - 1
+    seg_d = None if seg is None else torch.from_numpy(seg).to(dev)
+    b = gs.golomb_b_star(keep[0] / keep[1])
+    cap = gs.k_for(n, keep) + (T if T > 1 else 0)
+    g_host = [gen(w) for w in range(W)]
+    g = [torch.from_numpy(x).to(dev) for x in g_host]
+    r = [torch.zeros(n, device=dev) for _ in range(W)]
+    st = gs.status_tensor(dev)
+    idx = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(W)]
+    val = [torch.empty(cap, device=dev) for _ in range(W)]
+    off = [torch.zeros(T + 1, dtype=torch.int64, device=dev) for _ in range(W)]
+    mean = [torch.zeros(T, device=dev) for _ in range(W)]
+    words = [torch.empty(gs.golomb_word_capacity(cap, b, n), dtype=torch.int32, device=dev) for _ in range(W)]
+    nbits = [torch.zeros(1, dtype=torch.int64, device=dev) for _ in range(W)]
+    table = [torch.empty(((cap + 63) // 64, 2), dtype=torch.int64, device=dev) for _ in range(W)]
+    dec = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(W)]
+    out = [torch.empty(n, device=dev) for _ in range(W)]
+    dense = torch.empty(n, device=dev)
+    ws_t = torch.empty(max(gs.residual_topk_workspace_size(n, T, keep), gs.residual_topk_workspace_size(n, T, (0, 1)),
+                           gs.binarize_workspace_size(n, 1, keep)), dtype=torch.uint8, device=dev)
+    none_i = torch.empty(1, dtype=torch.int32, device=dev)
+    none_v = torch.empty(1, device=dev)
+    none_o = torch.zeros(2, dtype=torch.int64, device=dev)
+    ws_q = torch.empty(gs.lib().gsparse_quantize_workspace_size(cap), dtype=torch.uint8, device=dev)
+    ws_g = torch.empty(gs.lib().gsparse_golomb_encode_workspace_size(cap), dtype=torch.uint8, device=dev)
+    ws_s = torch.empty(max(gs.lib().gsparse_scatter_accumulate_workspace_size(W, n),
+                           gs.lib().gsparse_accumulate_combine_workspace_size(W, n)), dtype=torch.uint8, device=dev)
+    sb = [torch.empty((cap + 31) // 32, dtype=torch.int32, device=dev) for _ in range(W)]
+    means = [torch.empty(2, device=dev) for _ in range(W)]
+
+    def step(ev=None):
+        rec = (lambda k: ev[k].record()) if ev is not None else (lambda k: None)
+        rec(0)
+        for w in range(W):
+            if name == "resnet50":
+                for _ in range(9):
+                    gs.residual_topk(g[w], r[w], (0, 1), out_idx=none_i, out_val=none_v, out_offsets=none_o,
+                                     workspace=ws_t, d_status=st, capacity=0)
+                gs.binarize(g[w], r[w], keep, out_idx=idx[w], out_val=val[w], mean=mean[w], out_offsets=off[w],
+                            workspace=ws_t, d_status=st, capacity=cap)
+            else:
+                gs.residual_topk(g[w], r[w], keep, seg_offsets=seg_d, out_idx=idx[w], out_val=val[w],
+                                 out_offsets=off[w], workspace=ws_t, d_status=st, capacity=cap)
+            if name == "mlp":
+                for s_ in range(T):
+                    gs.quantize(idx[w], val[w], off[w][s_ + 1:s_ + 2], d_begin=off[w][s_:s_ + 1], residual=r[w],
+                                write_dequantized=True, sign_bits=sb[w], means=means[w], workspace=ws_q,
+                                d_status=st, capacity=cap)
+            if name in ("flat2e20", "resnet50"):
+                end = off[w][T:T + 1]
+                gs.golomb_encode(idx[w], end, b, n, chunk=64, words=words[w], nbits=nbits[w], table=table[w],
+                                 workspace=ws_g, d_status=st, capacity=cap)
+                gs.golomb_decode(words[w], nbits[w], end, cap, b, table=table[w], chunk=64, n_limit=n,
+                                 out_idx=dec[w], d_status=st)
+        rec(1)
+        src = dec if name in ("flat2e20", "resnet50") else idx
+        lists = [gs.make_list(src[w], off[w][T:T + 1], val=val[w], capacity=cap) for w in range(W)]
+        if name == "nmt":
+            for w in range(W):
+                gs.accumulate_combine(lists, n, g[w], out=out[w], workspace=ws_s, d_status=st)
+        else:
+            gs.scatter_accumulate(lists, n, dense_out=dense, workspace=ws_s, d_status=st, device=dev)
+        rec(2)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for k in range(K):
+        step(evs[k])
+    t1.record()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())}")
+    ms = t0.elapsed_time(t1) / K
+    compress = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    receive = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+
+    # the oracle on the same step (first step, zero residual), single thread
+    t = time.perf_counter()
+    if not args.no_oracle:
+        workload_oracle(name, g_host, n, seg, keep, b)
+    oms = (time.perf_counter() - t) * 1e3
+    grad = W * 4 * n
+    # algorithmic HBM bytes of the step: every residual pass reads g and r and writes r (12 B per
+    # entry); the receive writes the dense sum (scatter) or reads L and writes out per worker
+    # (combine); the lists themselves are < 1% of that and left out
+    passes = 10 if name == "resnet50" else 1
+    algo = W * passes * 12 * n + (W * 8 * n if name == "nmt" else 4 * n)
+    peak, peak_kind = measured_peaks()
+    ach = algo / (ms * 1e-3) / 1e9
+    return {"metric": METRIC, "workload": name, "description": WORKLOADS[name], "n": n, "workers": W,
+            "value": round(grad / (ms * 1e-3) / 1e9, 2), "unit": UNIT, "ms_per_step": round(ms, 4),
+            "roofline": {"bound": "hbm", "scope": "whole step", "achieved": round(ach, 1), "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
+                         "algorithmic_bytes_per_step": algo},
+            "stages_ms": {"compress": round(compress, 4), "receive": round(receive, 4)}, "steps": K,
+            "oracle": None if args.no_oracle else {
+                "ms_per_step": round(oms, 1), "value": round(grad / (oms * 1e-3) / 1e9, 4), "cores": 1,
+                "sample": "the same step on the full workload, zero residual, single-threaded C++ oracle"}}
+
+
+# ---------------------------------------------------------------------------------------------
 # the CPU oracle (reference arm and cpu_baseline)
 
 def oracle_step(gs_list, rs, keep, b, n):
@@ -432,11 +608,18 @@ def main():
     ap.add_argument("--no-launch-count", action="store_true", help="skip the profiler-based kernel count")
     ap.add_argument("--cpu-n", type=int, default=1 << 24)
     ap.add_argument("--ref-n", type=int, default=1 << 20)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
+                    help="time one of the smaller workloads instead of the default flat 2^30 line")
+    ap.add_argument("--no-oracle", action="store_true", help="with --workload: skip the oracle timing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.workload is not None:
+        if rank == 0:
+            print(json.dumps(run_workload(args)), flush=True)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)

@@ -2,12 +2,12 @@
 // ("Combining Global Sparse Gradients with Local Gradients in Distributed Neural Network
 // Training", Abstract; "Sparse Binary Compression", §I: the clients' updates are summed).
 //
-// Scatter-accumulate works on tiles of 8192 consecutive indices. One CTA owns a tile: it finds
-// each worker's entries in the tile by binary search (the lists are sorted), adds them worker by
-// worker into a shared-memory accumulator (fixed worker order, one fp32 add per entry, so the
-// result is bitwise reproducible), writes the dense tile with coalesced stores and counts the
-// touched indices. The merged sparse output is an ordered compaction of the touched indices
-// after a scan over the tile counts.
+// Scatter-accumulate works on tiles of 8192 consecutive indices. A streaming pass over the sorted
+// lists first records where each worker's entries of every tile start. One CTA owns a tile: it
+// adds the workers' entries of the tile worker by worker into a shared-memory accumulator (fixed
+// worker order, one fp32 add per entry, so the result is bitwise reproducible), writes the dense
+// tile with coalesced stores and counts the touched indices. The merged sparse output is an
+// ordered compaction of the touched indices after a scan over the tile counts.
 #include "common.cuh"
 
 namespace gs {
@@ -30,19 +30,71 @@ __device__ __forceinline__ int64_t list_count(const Lists& L, int w) {
   return c > L.cap[w] ? L.cap[w] : c;
 }
 
-// start[t][w] = first entry of worker w with index >= t * kTile, for t = 0..ntiles
-__global__ void sa_bounds_kernel(Lists L, int32_t W, int64_t n, int64_t ntiles, int64_t* start,
-                                 int32_t* d_status) {
-  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= (ntiles + 1) * W) return;
-  const int64_t t = k / W;
-  const int w = (int)(k % W);
+// start[t * W + w] = first entry of worker w with index >= t * kTile, for t = 0..ntiles, in one
+// streaming pass over each list: entry j starts every tile after its predecessor's tile up to its
+// own (index clamped to [0, n] by tile), and the end of the list closes the remaining tiles. For
+// an ascending list every table entry is written exactly once; a descent between tiles is flagged
+// (and the readers clamp the table to the list). Grid: (x, W).
+__device__ __forceinline__ int64_t tile_of_index(int32_t i, int64_t ntiles) {
+  if (i < 0) return 0;
+  const int64_t t = (int64_t)i / kTile;
+  return t < ntiles ? t : ntiles;
+}
+
+__device__ __forceinline__ void starts_at(const int32_t* ix, int64_t j, int64_t c, int32_t cur,
+                                          int32_t prev, int64_t ntiles, int32_t W, int w,
+                                          int64_t* start, int32_t* d_status) {
+  const int64_t tj = j < c ? tile_of_index(cur, ntiles) : ntiles;
+  const int64_t tp = j > 0 ? tile_of_index(prev, ntiles) : -1;
+  if (tj < tp) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
+  for (int64_t t = tp + 1; t <= tj; ++t) start[t * W + w] = j;
+}
+
+// Sixteen consecutive entries per thread (four 16-byte loads in flight when the list is 16-byte
+// aligned).
+constexpr int kStartsPer = 16;
+
+__global__ void __launch_bounds__(256) sa_starts_kernel(Lists L, int32_t W, int64_t n, int64_t ntiles,
+                                                        int64_t* start, uint32_t* next_tile,
+                                                        int32_t* d_status) {
+  const int w = blockIdx.y;
   const int64_t c = list_count(L, w);
-  if (t == 0 && c > 0) {
+  const int32_t* ix = L.idx[w];
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (w == 0 && next_tile) *next_tile = 0u;  // the combine kernel's tile counter
     if (*L.cnt[w] > L.cap[w]) raise(d_status, GSPARSE_DERR_CAPACITY);
-    if (L.idx[w][0] < 0 || (int64_t)L.idx[w][c - 1] >= n) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
+    if (c > 0 && (ix[0] < 0 || (int64_t)ix[c - 1] >= n)) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
   }
-  start[k] = t == ntiles ? c : lower_bound_i32(L.idx[w], c, t * kTile);
+  const int64_t j0 = kStartsPer * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  if (j0 > c) return;
+  int32_t v[kStartsPer];
+  if (j0 + kStartsPer <= c && (reinterpret_cast<uintptr_t>(ix) & 15u) == 0) {
+#pragma unroll
+    for (int h = 0; h < kStartsPer / 4; ++h) {
+      const int4 q = *reinterpret_cast<const int4*>(ix + j0 + 4 * h);
+      v[4 * h] = q.x; v[4 * h + 1] = q.y; v[4 * h + 2] = q.z; v[4 * h + 3] = q.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kStartsPer; ++e) v[e] = j0 + e < c ? ix[j0 + e] : 0;
+  }
+  int32_t prev = j0 > 0 ? ix[j0 - 1] : 0;
+#pragma unroll
+  for (int e = 0; e < kStartsPer; ++e) {
+    if (j0 + e > c) break;
+    starts_at(ix, j0 + e, c, v[e], prev, ntiles, W, w, start, d_status);
+    prev = v[e];
+  }
+}
+
+// The entries [b, e) of worker w in tile t, clamped to the list.
+__device__ __forceinline__ void tile_range(const int64_t* start, int64_t t, int32_t W, int w,
+                                           int64_t c, int64_t* b, int64_t* e) {
+  int64_t lo = start[t * W + w], hi = start[(t + 1) * W + w];
+  lo = lo < 0 ? 0 : (lo > c ? c : lo);
+  hi = hi < lo ? lo : (hi > c ? c : hi);
+  *b = lo;
+  *e = hi;
 }
 
 // Accumulates tile t into acc[] (zeroed) and sets touched bits.
@@ -50,7 +102,8 @@ __device__ void accumulate_tile(const Lists& L, int32_t W, int64_t t, const int6
                                 float* acc, uint32_t* touched, int32_t* d_status) {
   const int64_t t0 = t * kTile;
   for (int w = 0; w < W; ++w) {
-    const int64_t b = start[t * W + w], e = start[(t + 1) * W + w];
+    int64_t b, e;
+    tile_range(start, t, W, w, list_count(L, w), &b, &e);
     const int32_t* ix = L.idx[w];
     const float* vv = L.val[w];
     const float u = (vv || !L.uni[w]) ? 0.0f : *L.uni[w];
@@ -128,7 +181,11 @@ __global__ void __launch_bounds__(kTileThreads) sa_merge_kernel(Lists L, int32_t
   const int64_t t = blockIdx.x;
   // skip tiles no worker touches
   bool any = false;
-  for (int w = 0; w < W; ++w) any |= start[t * W + w] != start[(t + 1) * W + w];
+  for (int w = 0; w < W; ++w) {
+    int64_t b, e;
+    tile_range(start, t, W, w, list_count(L, w), &b, &e);
+    any |= b != e;
+  }
   if (!any) return;
   for (int i = threadIdx.x; i < kTile; i += blockDim.x) acc[i] = 0.0f;
   for (int i = threadIdx.x; i < kTile / 32; i += blockDim.x) touched[i] = 0u;
@@ -150,16 +207,21 @@ __global__ void __launch_bounds__(kTileThreads) sa_merge_kernel(Lists L, int32_t
   }
 }
 
-// Fused receive side. A persistent CTA owns a contiguous run of tiles; for each tile it
-// requests the local-gradient tile first, adds the workers' entries falling in the tile into a
-// shared accumulator (worker by worker, so the sums keep the fixed order), streams out
-// fl(fl(alpha * G) + fl(beta * L)) and finally clears only the entries it touched, so the
-// accumulator is zeroed once per CTA rather than once per tile. The sorted lists are walked
-// forward from one binary search per worker at the CTA's first tile: no bounds pass.
+// Fused receive side. The tile-start table (the bounds kernel above) gives each worker's entries
+// of every tile. Persistent CTAs take tiles from a shared counter, so tiles crowded with entries
+// (dense embedding rows) do not hold up the others. For each tile a CTA requests the
+// local-gradient tile first, adds the workers' entries of the tile into a shared accumulator
+// (worker by worker, so the sums keep the fixed order; four independent list loads per thread in
+// flight), streams out fl(fl(alpha * G) + fl(beta * L)) and finally clears only the entries it
+// touched, so the accumulator is zeroed once per CTA rather than once per tile.
 constexpr int kCombThreads = 256;
+constexpr int kCombPer = 4;
 
-__global__ void __launch_bounds__(kCombThreads) sa_combine_kernel(Lists L, int32_t W, int64_t n,
-                                                                  int64_t tiles_per_cta,
+constexpr int kCombPre = 2;  // workers whose first batch of entries is requested together
+
+__global__ void __launch_bounds__(kCombThreads, 4) sa_combine_kernel(Lists L, int32_t W, int64_t n,
+                                                                  const int64_t* start,
+                                                                  uint32_t* next_tile,
                                                                   const float* Lg, float* out,
                                                                   float alpha, float beta,
                                                                   int32_t own, float* dense,
@@ -167,60 +229,82 @@ __global__ void __launch_bounds__(kCombThreads) sa_combine_kernel(Lists L, int32
   constexpr int kVec = kTile / 4 / kCombThreads;  // float4s of a tile per thread
   __shared__ __align__(16) float acc[kTile];
   __shared__ uint32_t touched[kTile / 32];
-  __shared__ int64_t cur[GSPARSE_MAX_WORKERS], cnt[GSPARSE_MAX_WORKERS];
-  __shared__ int64_t own_b, own_e;
+  __shared__ uint32_t tnext;
+  __shared__ int64_t cnt[GSPARSE_MAX_WORKERS], rb[GSPARSE_MAX_WORKERS], re[GSPARSE_MAX_WORKERS];
   const int64_t ntiles = cdiv(n, kTile);
-  const int64_t T0 = (int64_t)blockIdx.x * tiles_per_cta;
-  const int64_t T1 = T0 + tiles_per_cta < ntiles ? T0 + tiles_per_cta : ntiles;
-  if (T0 >= T1) return;
   for (int i = threadIdx.x; i < kTile; i += blockDim.x) acc[i] = 0.0f;
   for (int i = threadIdx.x; i < kTile / 32; i += blockDim.x) touched[i] = 0u;
-  for (int w = threadIdx.x; w < W; w += blockDim.x) {
-    const int64_t c = list_count(L, w);
-    cnt[w] = c;
-    cur[w] = lower_bound_i32(L.idx[w], c, T0 * kTile);
-    if (T0 == 0 && c > 0 && L.idx[w][0] < 0) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
-    if (*L.cnt[w] > L.cap[w] && blockIdx.x == 0) raise(d_status, GSPARSE_DERR_CAPACITY);
-  }
+  if (threadIdx.x == 0) tnext = atomicAdd(next_tile, 1u);
   __syncthreads();
-  for (int64_t t = T0; t < T1; ++t) {
+  int64_t t = tnext;
+  // the entry ranges of the tile being worked on sit in rb/re; those of the next tile are loaded
+  // (by thread w for worker w) while the current tile is finished
+  for (int w = threadIdx.x; w < W; w += blockDim.x) {
+    cnt[w] = list_count(L, w);
+    if (t < ntiles) tile_range(start, t, W, w, cnt[w], &rb[w], &re[w]);
+  }
+  while (t < ntiles) {
+    __syncthreads();  // every thread has read tnext; rb/re hold tile t
+    if (threadIdx.x == 0) tnext = atomicAdd(next_tile, 1u);  // claimed now, read after the tile
     const int64_t t0 = t * kTile;
     const int64_t m = (n - t0) < kTile ? (n - t0) : kTile;
-    const int64_t tend = t0 + m;
     float4 lv[kVec];
     if (m == kTile) {
 #pragma unroll
       for (int k = 0; k < kVec; ++k) lv[k] = ld_stream(Lg + t0 + 4 * (threadIdx.x + k * kCombThreads));
     }
+    // first batch of the first kCombPre workers, requested together
+    int32_t pi[kCombPre];
+    float px[kCombPre];
+#pragma unroll
+    for (int w = 0; w < kCombPre; ++w) {
+      pi[w] = 0;
+      px[w] = 0.0f;
+      if (w < W) {
+        const int64_t j = rb[w] + threadIdx.x;
+        if (j < re[w]) {
+          pi[w] = L.idx[w][j];
+          px[w] = L.val[w] ? L.val[w][j] : (L.uni[w] ? *L.uni[w] : 0.0f);
+        }
+      }
+    }
     for (int w = 0; w < W; ++w) {
       const int32_t* ix = L.idx[w];
       const float* vv = L.val[w];
       const float u = (vv || !L.uni[w]) ? 0.0f : *L.uni[w];
-      const int64_t c = cnt[w];
-      int64_t b = cur[w];
-      if (w == own && threadIdx.x == 0) own_b = b;
-      for (;;) {
-        const int64_t j = b + threadIdx.x;
-        const int32_t i = j < c ? ix[j] : INT32_MAX;
-        const bool in = i < tend;             // a prefix: the list is ascending
-        if (in) {
-          if (j > 0 && ix[j - 1] >= i) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
-          const int off = (int)(i - t0);
-          if (off >= 0 && off < kTile) {
-            acc[off] = __fadd_rn(acc[off], vv ? vv[j] : u);
-            atomicOr(&touched[off >> 5], 1u << (off & 31));
+      const int64_t b = rb[w], e = re[w];
+      for (int64_t jb = b; jb < e; jb += kCombThreads * kCombPer) {
+        int32_t iv[kCombPer];
+        float xv[kCombPer];
+#pragma unroll
+        for (int k = 0; k < kCombPer; ++k) {
+          const int64_t j = jb + k * kCombThreads + threadIdx.x;
+          if (k == 0 && jb == b && w < kCombPre) {
+#pragma unroll
+            for (int ww = 0; ww < kCombPre; ++ww)
+              if (ww == w) { iv[0] = pi[ww]; xv[0] = px[ww]; }
+          } else {
+            iv[k] = j < e ? ix[j] : 0;
+            xv[k] = j < e ? (vv ? vv[j] : u) : 0.0f;
           }
         }
-        const int nin = __syncthreads_count(in);
-        b += nin;
-        if (nin < kCombThreads) break;
-      }
-      if (threadIdx.x == 0) {
-        cur[w] = b;
-        if (w == own) own_e = b;
+#pragma unroll
+        for (int k = 0; k < kCombPer; ++k) {
+          const int64_t j = jb + k * kCombThreads + threadIdx.x;
+          if (j >= e) continue;
+          if (j > 0 && ix[j - 1] >= iv[k]) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); continue; }
+          const int off = (int)(iv[k] - t0);
+          if (off < 0 || off >= kTile) continue;  // out of range, reported by the bounds pass
+          acc[off] = __fadd_rn(acc[off], xv[k]);
+          atomicOr(&touched[off >> 5], 1u << (off & 31));
+        }
       }
       __syncthreads();  // worker order: all of worker w before any of worker w + 1
     }
+    // the next tile's ranges (tnext is visible after the syncs above)
+    const int64_t tn = tnext;
+    int64_t nb_ = 0, ne_ = 0;
+    if (threadIdx.x < W && tn < ntiles) tile_range(start, tn, W, threadIdx.x, cnt[threadIdx.x], &nb_, &ne_);
     if (dense) {
       if (m == kTile) {
         for (int v = threadIdx.x; v < kTile / 4; v += blockDim.x)
@@ -234,7 +318,7 @@ __global__ void __launch_bounds__(kCombThreads) sa_combine_kernel(Lists L, int32
       const int32_t* ix = L.idx[own];
       const float* vv = L.val[own];
       const float u = (vv || !L.uni[own]) ? 0.0f : *L.uni[own];
-      for (int64_t j = own_b + threadIdx.x; j < own_e; j += blockDim.x) {
+      for (int64_t j = rb[own] + threadIdx.x; j < re[own]; j += blockDim.x) {
         const int off = (int)(ix[j] - t0);
         if (off >= 0 && off < kTile) acc[off] = __fsub_rn(acc[off], vv ? vv[j] : u);
       }
@@ -267,12 +351,12 @@ __global__ void __launch_bounds__(kCombThreads) sa_combine_kernel(Lists L, int32
         acc[k * 32 + bit] = 0.0f;
       }
     }
-    __syncthreads();
+    if (threadIdx.x < W) {
+      rb[threadIdx.x] = nb_;
+      re[threadIdx.x] = ne_;
+    }
+    t = tn;
   }
-  // entries at or beyond n belong to no tile: the CTA with the last tile reports them
-  if (T1 == ntiles)
-    for (int w = threadIdx.x; w < W; w += blockDim.x)
-      if (cur[w] < cnt[w]) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -321,6 +405,15 @@ struct SLayout {
   int32_t* ctl;
   size_t bytes;
 };
+
+void launch_starts(const Lists& L, int32_t W, int64_t n, int64_t ntiles, int64_t* start,
+                   uint32_t* next_tile, int32_t* d_status, cudaStream_t st) {
+  int64_t most = 0;
+  for (int w = 0; w < W; ++w) most = L.cap[w] > most ? L.cap[w] : most;
+  const int64_t bx = cdiv(most + 1, kStartsPer * 256);  // entries 0..count of every list
+  sa_starts_kernel<<<dim3((unsigned)bx, (unsigned)W), 256, 0, st>>>(L, W, n, ntiles, start, next_tile,
+                                                                      d_status);
+}
 
 SLayout s_carve(int32_t W, int64_t n, void* ws) {
   SLayout L;
@@ -375,8 +468,7 @@ int gsparse_scatter_accumulate(const gsparse_list* lists, int32_t W, int64_t n, 
       return GSPARSE_ERR_CUDA;
     return launch_status();
   }
-  const int64_t nb = (ntiles + 1) * W;
-  sa_bounds_kernel<<<(unsigned)cdiv(nb, 256), 256, 0, st>>>(L, W, n, ntiles, S.start, d_status);
+  launch_starts(L, W, n, ntiles, S.start, nullptr, d_status, st);
   sa_tile_kernel<<<(unsigned)ntiles, kTileThreads, 0, st>>>(L, W, n, S.start, dense_out,
                                                             merged ? S.tile_count : nullptr, d_status);
   if (merged) {
@@ -418,11 +510,11 @@ int gsparse_accumulate_combine(const gsparse_list* lists, int32_t W, int64_t n, 
   if (workspace_bytes < S.bytes) return GSPARSE_ERR_WORKSPACE;
   const int64_t ntiles = cdiv(n, kTile);
   if (ntiles == 0) return launch_status();
-  (void)S;
-  const int64_t ctas_target = (int64_t)sm_count() * 4;
-  const int64_t per = cdiv(ntiles, ctas_target < ntiles ? ctas_target : ntiles);
-  sa_combine_kernel<<<(unsigned)cdiv(ntiles, per), kCombThreads, 0, st>>>(
-      Ls, W, n, per, L, out, alpha, beta, mode == 1 ? own : -1, dense_out, d_status);
+  uint32_t* next_tile = reinterpret_cast<uint32_t*>(S.ctl + 1);
+  launch_starts(Ls, W, n, ntiles, S.start, next_tile, d_status, st);
+  const int64_t ctas = (int64_t)sm_count() * 4 < ntiles ? (int64_t)sm_count() * 4 : ntiles;
+  sa_combine_kernel<<<(unsigned)ctas, kCombThreads, 0, st>>>(
+      Ls, W, n, S.start, next_tile, L, out, alpha, beta, mode == 1 ? own : -1, dense_out, d_status);
   return launch_status();
 }
 

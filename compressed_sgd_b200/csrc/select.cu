@@ -41,6 +41,7 @@ constexpr int kSampleCtas = 256;                 // CTAs sharing one segment's s
 static_assert(kSample % (32 * kSampleCtas) == 0 && kSample / kSampleCtas <= 1024,
               "each sample CTA takes whole runs, at most 32 of them");
 constexpr int kWarps = 8;                        // warps (pieces) per CTA
+constexpr int kMaxChunks = 64;                   // pool chunks one piece may claim
 constexpr int kThreads = kWarps * 32;
 
 struct Sel {
@@ -57,12 +58,19 @@ struct Sel {
   uint32_t* hist;  // [P][kHist]
   uint32_t *pcnt, *prsrc, *pgt, *peq, *ptake;
   int64_t* poff;
+  // candidate stores: Q primary stores of cap slots, then a pool of chunks of 2^chunk_shift slots
+  // that a piece claims (at most max_chunks) once its primary store is full
   int32_t* cidx;
   float* cval;
-  int32_t* ctl;  // [0] abort, [1] any redo
+  int32_t* pchunk;    // [Q][max_chunks] pool chunk ids claimed by each piece, in order
+  uint32_t* pnch;     // [Q] chunks claimed
+  int64_t pool_chunks;
+  int32_t chunk_shift, max_chunks;
+  int32_t* ctl;  // [0] abort, [1] any redo, [2] next free pool chunk
   // sample: two-level histogram of the sampled keys per problem
-  uint32_t *shist, *scount, *sdone, *sb1;
-  int64_t* srank;
+  uint32_t *shist, *scount, *sdone, *sb1, *sblo, *ssub;
+  int64_t *srank, *sabove, *smcap;
+  unsigned long long* svar;  // per problem: sum and sum of squares of the per-run counts
   // pending residual writes applied in the sample and pass 1 (null: none)
   const int32_t* pw_idx;
   const float* pw_val;
@@ -89,6 +97,19 @@ __device__ __forceinline__ Piece piece_of(const Sel& a, int64_t q) {
   const int64_t end = a.seg_lo[p.s] + a.seg_n[p.s];
   p.hi = p.lo + a.Lp < end ? p.lo + a.Lp : end;
   return p;
+}
+
+// Slots of a piece's candidate store: positions [0, cap) in its primary store, later positions in
+// its pool chunks (chunk c holds positions cap + c * 2^chunk_shift onwards).
+__device__ __forceinline__ uint32_t room_of(const Sel& a, int64_t q) {
+  return (uint32_t)a.cap + (a.pnch[q] << a.chunk_shift);
+}
+
+__device__ __forceinline__ int64_t slot_of(const Sel& a, int64_t q, uint32_t pos) {
+  if (pos < (uint32_t)a.cap) return q * a.cap + pos;
+  const uint32_t o = pos - (uint32_t)a.cap;
+  const int64_t c = a.pchunk[q * a.max_chunks + (o >> a.chunk_shift)];
+  return a.Q * a.cap + (c << a.chunk_shift) + (o & ((1u << a.chunk_shift) - 1u));
 }
 
 // class of an accumulated value: top-k has one class; binarise splits by sign (zeros in none)
@@ -220,11 +241,17 @@ __global__ void __launch_bounds__(1024) plan_kernel(Sel a, const int64_t* seg, i
 //
 // Each segment's sample (the whole segment when it has at most kSample entries, else kSample
 // entries in evenly spaced runs of 32) is split over kSampleCtas CTAs. Level 1 histograms the
-// top 11 key bits; the last CTA to finish picks the bin holding the m-th largest sampled key.
-// Level 2 re-reads the sample, histograms the next 11 bits inside that bin, and its last CTA sets
-// T_lo to the lower edge of the 22-bit bucket holding the m-th key. With the whole segment in the
-// sample m = k, so at least k entries reach T_lo; otherwise m sits three standard deviations (plus
-// 16) above the expected sample count, and a shortfall is caught and redone by the check step.
+// top 11 key bits. Level 2 re-reads the sample and histograms the keys of a range of level-1
+// bins at a finer resolution; its last CTA sets T_lo to the lower edge of the fine bucket holding
+// the m-th largest sampled key. With the whole segment in the sample m = k, so at least k
+// entries reach T_lo. Otherwise m sits three standard deviations (plus 16) above the expected
+// sample count e = k * S / n_s. Entries of one run can be strongly correlated (a run inside an
+// all-zero embedding row, or inside a tensor of larger scale), so the deviation is estimated
+// from the spread of the per-run counts measured at level 2, never below the independent-entry
+// figure sqrt(e) and never above sqrt(32 e), which bounds the variance of a sum of run counts in
+// [0, 32]. Level 1 therefore picks the bins of both ends, m0 = e + 3 sqrt(e) + 16 and
+// m_max = e + 3 sqrt(32 e) + 16, and level 2 covers the bins between them. A shortfall (fewer than
+// k entries reaching T_lo) is still caught and redone by the check step.
 
 __device__ __forceinline__ uint32_t pending_count(const Sel& a) {
   if (!a.pw_idx) return 0;
@@ -252,10 +279,14 @@ __device__ __forceinline__ uint32_t* shist_of(const Sel& a, int64_t p, int level
   return a.shist + p * (2 * kBins1) + (level == 1 ? 0 : kBins1);
 }
 
+// smallest s with 2^s >= v (v >= 1)
+__device__ __forceinline__ uint32_t ceil_log2(uint32_t v) { return v <= 1 ? 0u : 32u - __clz(v - 1u); }
+
 template <int C>
 __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhaustive) {
   __shared__ uint32_t h[C * kBins1];
   __shared__ uint32_t cnt[C];
+  __shared__ unsigned long long vsum[C], vsq[C];
   __shared__ int last;
   if (a.ctl[0]) return;
   const int32_t s = blockIdx.y;
@@ -268,9 +299,14 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
     }
     return;
   }
-  uint32_t b1[C];
+  // level 2: per class the level-1 bins [blo, b1] at 2^sub fine bins each
+  uint32_t b1[C], blo[C], sub[C];
 #pragma unroll
-  for (int c = 0; c < C; ++c) b1[c] = level == 2 ? a.sb1[P0 + c] : 0u;
+  for (int c = 0; c < C; ++c) {
+    b1[c] = level == 2 ? a.sb1[P0 + c] : kNone;
+    blo[c] = level == 2 && b1[c] != kNone ? a.sblo[P0 + c] : 0u;
+    sub[c] = level == 2 && b1[c] != kNone ? a.ssub[P0 + c] : 0u;
+  }
   if (level == 2) {
     bool any = false;
 #pragma unroll
@@ -278,7 +314,11 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
     if (!any) return;
   }
   for (int i = threadIdx.x; i < C * kBins1; i += blockDim.x) h[i] = 0;
-  if (threadIdx.x < C) cnt[threadIdx.x] = 0;
+  if (threadIdx.x < C) {
+    cnt[threadIdx.x] = 0;
+    vsum[threadIdx.x] = 0;
+    vsq[threadIdx.x] = 0;
+  }
   __syncthreads();
   const int64_t S = ns < kSample ? ns : kSample;
   const int64_t j0 = S * blockIdx.x / gridDim.x, j1 = S * (blockIdx.x + 1) / gridDim.x;
@@ -288,7 +328,9 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
   __shared__ uint32_t pwb, pwe;
   __shared__ uint32_t run_b[32], run_e[32];
   const uint32_t pc = pending_count(a);
-  const bool runs = pc && ns > kSample;
+  const bool sparse = ns > kSample;  // then j1 - j0 is a multiple of blockDim.x and one warp
+                                     // iteration is one run
+  const bool runs = pc && sparse;
   if (threadIdx.x == 0) {
     pwb = pwe = 0;
     if (pc && ns <= kSample) {
@@ -315,25 +357,42 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
     const uint32_t ce = runs ? run_e[(j - j0) >> 5] : pwe;
     const float x = __fadd_rn(a.g[i], residual_at(a, i, cb, ce));
     const int c = class_of<C>(x);
-    if (c < 0) continue;
     const uint32_t key = mag_key(x);
+    if (level == 2 && sparse) {
+      // this run's count of class members in bin b1 or above
+#pragma unroll
+      for (int cc = 0; cc < C; ++cc) {
+        const bool hit = c == cc && b1[cc] != kNone && (key >> 20) >= b1[cc];
+        const uint32_t nr = __popc(__ballot_sync(kFull, hit));
+        if ((threadIdx.x & 31) == 0 && nr) {
+          atomicAdd(&vsum[cc], (unsigned long long)nr);
+          atomicAdd(&vsq[cc], (unsigned long long)(nr * nr));
+        }
+      }
+    }
+    if (c < 0) continue;
     if (level == 1) {
       atomicAdd(&h[c * kBins1 + (key >> 20)], 1u);
       atomicAdd(&cnt[c], 1u);
-    } else if ((key >> 20) == b1[c]) {
-      atomicAdd(&h[c * kBins1 + ((key >> 9) & 2047u)], 1u);
+    } else if (b1[c] != kNone && (key >> 20) >= blo[c] && (key >> 20) <= b1[c]) {
+      atomicAdd(&h[c * kBins1 + ((key >> (20 - sub[c])) - (blo[c] << sub[c]))], 1u);
     }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < C * kBins1; i += blockDim.x)
     if (h[i]) atomicAdd(shist_of(a, P0 + i / kBins1, level) + (i % kBins1), h[i]);
   if (level == 1 && threadIdx.x < C && cnt[threadIdx.x]) atomicAdd(&a.scount[P0 + threadIdx.x], cnt[threadIdx.x]);
+  if (level == 2 && threadIdx.x < C && vsum[threadIdx.x]) {
+    atomicAdd(&a.svar[2 * (P0 + threadIdx.x)], vsum[threadIdx.x]);
+    atomicAdd(&a.svar[2 * (P0 + threadIdx.x) + 1], vsq[threadIdx.x]);
+  }
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) last = atomicAdd(&a.sdone[2 * s + level - 1], 1u) == gridDim.x - 1;
   __syncthreads();
   if (!last) return;
   __threadfence();
+  const double e = (double)k * (double)S / (double)ns;
   for (int c = 0; c < C; ++c) {
     const int64_t p = P0 + c;
     if (level == 2 && b1[c] == kNone) continue;
@@ -341,33 +400,51 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
     __syncthreads();
     if (level == 1) {
       const int64_t count = ((volatile uint32_t*)a.scount)[p];
-      int64_t m;
-      if (ns <= kSample) {
-        m = k < count ? k : count;                 // the whole segment is in the sample
+      int64_t m0, mmax;
+      if (!sparse) {
+        m0 = mmax = k < count ? k : count;          // the whole segment is in the sample
       } else {
-        const double e = (double)k * (double)S / (double)ns;
-        m = (int64_t)ceil(e + 3.0 * sqrt(e) + 16.0);
+        m0 = (int64_t)ceil(e + 3.0 * sqrt(e) + 16.0);
+        mmax = (int64_t)ceil(e + 3.0 * sqrt(32.0 * e) + 16.0);
       }
-      if (count == 0 || m >= count) {
+      if (count == 0 || m0 >= count) {
         // every member is needed (or the class is absent from a fully sampled segment)
         if (threadIdx.x == 0) {
-          a.tlo[p] = (count == 0 && ns <= kSample) ? kNone : 0u;
+          a.tlo[p] = (count == 0 && !sparse) ? kNone : 0u;
           a.sb1[p] = kNone;
         }
       } else {
-        uint32_t bin;
-        int64_t above;
-        block_find_bin(h, kBins1, m, &bin, &above);
+        if (mmax > count) mmax = count;
+        uint32_t bin, binlo;
+        int64_t above, above_lo;
+        block_find_bin(h, kBins1, m0, &bin, &above);
+        block_find_bin(h, kBins1, mmax, &binlo, &above_lo);
         if (threadIdx.x == 0) {
           a.sb1[p] = bin;
-          a.srank[p] = m - above;
+          a.sblo[p] = binlo;
+          a.ssub[p] = 11u - ceil_log2(bin - binlo + 1u);
+          a.srank[p] = m0;
+          a.sabove[p] = above;
+          a.smcap[p] = mmax;
         }
       }
     } else {
+      int64_t m = a.srank[p];
+      if (sparse) {
+        // the deviation of the sampled count, from the spread of the per-run counts
+        const double R = (double)kSampleRuns;
+        const double mean = (double)((volatile unsigned long long*)a.svar)[2 * p] / R;
+        const double sq = (double)((volatile unsigned long long*)a.svar)[2 * p + 1] / R;
+        const double var = sq - mean * mean > 0.0 ? sq - mean * mean : 0.0;
+        const double sd = sqrt(R * var) > sqrt(e) ? sqrt(R * var) : sqrt(e);
+        const int64_t ma = (int64_t)ceil(e + 3.0 * sd + 16.0);
+        const int64_t mcap = a.smcap[p];
+        m = ma < m ? m : (ma > mcap ? mcap : ma);
+      }
       uint32_t bin;
       int64_t above;
-      block_find_bin(h, kBins1, a.srank[p], &bin, &above);
-      if (threadIdx.x == 0) a.tlo[p] = ((b1[c] << 11) | bin) << 9;
+      block_find_bin(h, kBins1, m - a.sabove[p], &bin, &above);
+      if (threadIdx.x == 0) a.tlo[p] = ((blo[c] << sub[c]) + bin) << (20 - sub[c]);
     }
     __syncthreads();
   }
@@ -398,7 +475,32 @@ struct P1State {
   uint32_t cp;      // next pending write of this piece
   int32_t win_idx;  // pending window (entry cp + lane), loaded one chunk ahead
   float win_val;
+  // the store: positions below `room` have slots; the newest region (primary store or pool
+  // chunk) starts at position ch_lo, slot ch_base; the one before it at pv_lo, pv_base
+  uint32_t room, nch, ch_lo, pv_lo;
+  int64_t ch_base, pv_base;
 };
+
+// Makes room for `need` more candidates (need <= 512 <= a chunk) by claiming one pool chunk.
+// Warp-uniform; once a candidate has been dropped nothing more is claimed (the piece is re-read).
+__device__ __forceinline__ void p1_reserve(const Sel& a, int64_t q, uint32_t need, P1State& S,
+                                           int lane) {
+  if (S.count + need <= S.room || S.count > S.room) return;
+  uint32_t c = 0xFFFFFFFFu;
+  if (lane == 0 && S.nch < (uint32_t)a.max_chunks) {
+    c = atomicAdd(reinterpret_cast<uint32_t*>(a.ctl + 2), 1u);
+    if (c >= (uint64_t)a.pool_chunks) c = 0xFFFFFFFFu;
+    else a.pchunk[q * a.max_chunks + S.nch] = (int32_t)c;
+  }
+  c = __shfl_sync(kFull, c, 0);
+  if (c == 0xFFFFFFFFu) return;
+  S.pv_lo = S.ch_lo;
+  S.pv_base = S.ch_base;
+  S.ch_lo = S.room;
+  S.ch_base = a.Q * a.cap + ((int64_t)c << a.chunk_shift);
+  S.room += 1u << a.chunk_shift;
+  S.nch += 1;
+}
 
 __device__ __forceinline__ void load_window(const Sel& a, uint32_t cp, uint32_t cend, int lane,
                                             P1State& S) {
@@ -411,12 +513,11 @@ __device__ __forceinline__ void load_window(const Sel& a, uint32_t cp, uint32_t 
 // candidate test and ordered store, the histogram, and the residual write-back. gv/rv hold the
 // chunk (entries outside the piece, as marked by `valid`, are ignored).
 template <int C>
-__device__ __forceinline__ void pass1_chunk(const Sel& a, uint32_t base, uint32_t lo, uint32_t hi,
-                                            bool full, uint32_t valid, float4 (&gv)[4],
-                                            float4 (&rv)[4], P1State& S, uint32_t cend,
-                                            const uint32_t (&tl)[C], float* st, uint32_t cap,
-                                            int32_t* cidx, float* cval, uint32_t* hsink,
-                                            int hstride, int lane) {
+__device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t base, uint32_t lo,
+                                            uint32_t hi, bool full, uint32_t valid,
+                                            float4 (&gv)[4], float4 (&rv)[4], P1State& S,
+                                            uint32_t cend, const uint32_t (&tl)[C], float* st,
+                                            uint32_t* hsink, int hstride, int lane) {
   float4* st4 = reinterpret_cast<float4*>(st);
   float* r = a.r;
   if (S.cp < cend) {
@@ -467,6 +568,7 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, uint32_t base, uint32_
     __syncwarp();
     const uint32_t excl = incl - packed;
     const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu;
+    p1_reserve(a, q, t0 + t1 + t2 + (tot >> 24), S, lane);
     uint32_t stored = 0;
     for (uint32_t m = m16; m; m &= m - 1) {
       const int b = __ffs(m) - 1;
@@ -475,9 +577,10 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, uint32_t base, uint32_
       const uint32_t pos = S.count + before + ((excl >> (8 * u)) & 0xFFu) +
                            __popc(m16 & ((1u << b) - 1u) & (0xFu << (4 * u)));
       const float x = st[(u * 32 + lane) * 4 + e];
-      if (pos < cap) {
-        cidx[pos] = (int32_t)(base + u * 128 + lane * 4 + e);
-        cval[pos] = x;
+      if (pos < S.room) {
+        const int64_t slot = pos >= S.ch_lo ? S.ch_base + (pos - S.ch_lo) : S.pv_base + (pos - S.pv_lo);
+        a.cidx[slot] = (int32_t)(base + u * 128 + lane * 4 + e);
+        a.cval[slot] = x;
         stored |= 1u << b;
       }
       atomicAdd(hsink + cand_class<C>(x) * hstride + (mag_key(x) >> 20), 1u);
@@ -558,9 +661,6 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     uint32_t tl[C];
 #pragma unroll
     for (int c = 0; c < C; ++c) tl[c] = a.tlo[(int64_t)P.s * C + c];
-    const uint32_t cap = (uint32_t)a.cap;
-    int32_t* cidx = a.cidx + q * a.cap;
-    float* cval = a.cval + q * a.cap;
     // histogram sink: this CTA's shared counts, or global counts for a second segment
     const bool sh_sink = P.s == H.primary;
     uint32_t* hsink = sh_sink ? H.sh : hist_of(a, (int64_t)P.s * C, 1);
@@ -572,14 +672,17 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     P1State S;
     S.count = 0;
     S.cp = 0;
+    S.room = (uint32_t)a.cap;
+    S.nch = 0;
+    S.ch_lo = S.pv_lo = 0;
+    S.ch_base = S.pv_base = q * a.cap;
     if (cend) S.cp = __shfl_sync(kFull, lane == 0 ? (uint32_t)lower_bound_i32(a.pw_idx, cend, lo) : 0u, 0);
     load_window(a, S.cp, cend, lane, S);
     uint32_t base = lo & ~3u;
     float4 gv[4], rv[4];
     if (base < lo || base + (uint32_t)kGranule > hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
-      pass1_chunk<C>(a, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, cap, cidx, cval, hsink,
-                     hstride, lane);
+      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, hsink, hstride, lane);
       base += (uint32_t)kGranule;
     }
     if (base < hi && base + (uint32_t)kGranule <= hi) {
@@ -591,18 +694,20 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
         const uint32_t nb = base + (uint32_t)kGranule;
         const bool more = nb + (uint32_t)kGranule <= hi;
         if (more) load_full(a, nb, lane, gn, rn);
-        pass1_chunk<C>(a, base, lo, hi, true, 0xFFFFu, gv, rv, S, cend, tl, st, cap, cidx, cval,
-                       hsink, hstride, lane);
+        pass1_chunk<C>(a, q, base, lo, hi, true, 0xFFFFu, gv, rv, S, cend, tl, st, hsink, hstride,
+                       lane);
         base = nb;
         if (!more) break;
       }
     }
     if (base < hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
-      pass1_chunk<C>(a, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, cap, cidx, cval, hsink,
-                     hstride, lane);
+      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, hsink, hstride, lane);
     }
-    if (lane == 0) a.pcnt[q] = S.count;
+    if (lane == 0) {
+      a.pcnt[q] = S.count;
+      a.pnch[q] = S.nch;
+    }
   }
   __syncthreads();
   H.flush(a, 1, kBins1);
@@ -638,15 +743,16 @@ template <int C, class F>
 __device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, const Piece& P, F f) {
   const int lane = threadIdx.x & 31;
   if (!a.prsrc[q]) {
-    // the store of a piece starts 16-byte aligned (cap is a multiple of 4): four per lane
+    // every store region starts 16-byte aligned (cap and the chunk size are multiples of 4):
+    // four per lane
     const uint32_t cnt = a.pcnt[q];
-    const float4* cv = reinterpret_cast<const float4*>(a.cval + q * a.cap);
     const uint32_t n4 = (cnt + 3) / 4;
     for (uint32_t j4 = lane; j4 < n4; j4 += 128) {
       float4 X[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h)
-        X[h] = j4 + 32 * h < n4 ? cv[j4 + 32 * h] : make_float4(0.f, 0.f, 0.f, 0.f);
+        X[h] = j4 + 32 * h < n4 ? *reinterpret_cast<const float4*>(a.cval + slot_of(a, q, 4 * (j4 + 32 * h)))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         const float xv[4] = {X[h].x, X[h].y, X[h].z, X[h].w};
@@ -727,10 +833,14 @@ __global__ void __launch_bounds__(kThreads) restore_kernel(Sel a) {
 #pragma unroll
     for (int c = 0; c < C; ++c) redo |= a.redo[(int64_t)P.s * C + c] != 0;
     const uint32_t cnt = a.pcnt[q];
-    if (redo || cnt > a.cap) {
+    const uint32_t room = room_of(a, q);
+    if (redo || cnt > room) {
       if (a.zero_mode) {
-        const uint32_t stored = cnt < a.cap ? cnt : (uint32_t)a.cap;
-        for (uint32_t j = lane; j < stored; j += 32) a.r[a.cidx[q * a.cap + j]] = a.cval[q * a.cap + j];
+        const uint32_t stored = cnt < room ? cnt : room;
+        for (uint32_t j = lane; j < stored; j += 32) {
+          const int64_t sl = slot_of(a, q, j);
+          a.r[a.cidx[sl]] = a.cval[sl];
+        }
       }
       __syncwarp();
       if (lane == 0) a.prsrc[q] = 1;
@@ -922,8 +1032,8 @@ __global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_i
   if (!a.prsrc[q]) {
     // the store in index order, four consecutive candidates per lane
     const uint32_t cnt = a.pcnt[q];
-    const int4* ci = reinterpret_cast<const int4*>(a.cidx + q * a.cap);
-    const float4* cv = reinterpret_cast<const float4*>(a.cval + q * a.cap);
+    auto ci = [&](uint32_t pos) { return *reinterpret_cast<const int4*>(a.cidx + slot_of(a, q, pos)); };
+    auto cv = [&](uint32_t pos) { return *reinterpret_cast<const float4*>(a.cval + slot_of(a, q, pos)); };
     // software pipelined: three batches of 128 candidates are in flight while one is placed
     constexpr int kAhead = 3;
     int4 Iq[kAhead];
@@ -931,8 +1041,8 @@ __global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_i
 #pragma unroll
     for (int h = 0; h < kAhead; ++h) {
       const uint32_t jj = 128 * h + 4 * lane;
-      Iq[h] = jj < cnt ? ci[jj >> 2] : make_int4(0, 0, 0, 0);
-      Xq[h] = jj < cnt ? cv[jj >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+      Iq[h] = jj < cnt ? ci(jj) : make_int4(0, 0, 0, 0);
+      Xq[h] = jj < cnt ? cv(jj) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     for (uint32_t j0 = 0; j0 < cnt; j0 += 128) {
       const uint32_t j = j0 + 4 * lane;
@@ -942,8 +1052,8 @@ __global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_i
       for (int h = 0; h + 1 < kAhead; ++h) { Iq[h] = Iq[h + 1]; Xq[h] = Xq[h + 1]; }
       {
         const uint32_t jj = j + 128 * kAhead;
-        Iq[kAhead - 1] = jj < cnt ? ci[jj >> 2] : make_int4(0, 0, 0, 0);
-        Xq[kAhead - 1] = jj < cnt ? cv[jj >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+        Iq[kAhead - 1] = jj < cnt ? ci(jj) : make_int4(0, 0, 0, 0);
+        Xq[kAhead - 1] = jj < cnt ? cv(jj) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       int32_t iv[4] = {0, 0, 0, 0};
       float xv[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1223,9 +1333,14 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
   a.shist = cv.take<uint32_t>(P * 2 * kBins1);
   a.scount = cv.take<uint32_t>(P);
   a.sdone = cv.take<uint32_t>(2 * (int64_t)T);
+  a.svar = cv.take<unsigned long long>(2 * P);
   const size_t zend = cv.off;
   a.sb1 = cv.take<uint32_t>(P);
+  a.sblo = cv.take<uint32_t>(P);
+  a.ssub = cv.take<uint32_t>(P);
   a.srank = cv.take<int64_t>(P);
+  a.sabove = cv.take<int64_t>(P);
+  a.smcap = cv.take<int64_t>(P);
   L.zero_begin = ws ? (char*)ws + zoff : nullptr;
   L.zero_bytes = zend - zoff;
   if (C == 2) {
@@ -1239,19 +1354,36 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
     L.leaves = cv.take<double>(L.leaf_bound);
     L.partials = cv.take<double>(P * osum_partial_stride(L.per_job_leaf_bound));
   }
+  // pool chunks: a power of two >= 512 slots (one 512-entry chunk of pass 1 never needs more than
+  // one new chunk), with kMaxChunks of them covering a whole piece
+  int32_t shift = 9;
+  while ((kMaxChunks << shift) < L.Lp) ++shift;
+  a.chunk_shift = shift;
+  a.max_chunks = kMaxChunks;
+  a.pchunk = cv.take<int32_t>(L.Q * kMaxChunks);
+  a.pnch = cv.take<uint32_t>(L.Q);
   L.fixed_bytes = cv.off + 512;
   L.cap_rec = rec_cap(L.Lp, C, num, den);
-  int64_t cap;
+  const int64_t csz = (int64_t)1 << shift;
+  int64_t cap, pool;
   if (measure_rec) {
     cap = L.cap_rec;
+    // room for about twice the kept entries beyond the primary stores, as whole chunks
+    pool = cdiv(2 * C * k_bound(n, T, num, den), csz) + 64;
   } else {
+    // the primary stores up to the recommended size (int4-aligned), the rest as pool chunks
     const int64_t room = ws_bytes > L.fixed_bytes ? (int64_t)(ws_bytes - L.fixed_bytes) : 0;
-    cap = (room / (L.Q * 8 > 0 ? L.Q * 8 : 1)) & ~(int64_t)3;  // int4-aligned per-piece stores
+    cap = (room / (L.Q * 8 > 0 ? L.Q * 8 : 1)) & ~(int64_t)3;
+    if (cap > L.cap_rec) cap = L.cap_rec;
     if (cap > L.Lp) cap = L.Lp;
+    pool = (room - L.Q * cap * 8 - 512) / (csz * 8);
+    if (pool < 0) pool = 0;
   }
+  if (pool > INT32_MAX) pool = INT32_MAX;
   L.cap = cap;
-  a.cidx = cv.take<int32_t>(L.Q * cap);
-  a.cval = cv.take<float>(L.Q * cap);
+  a.pool_chunks = pool;
+  a.cidx = cv.take<int32_t>(L.Q * cap + pool * csz);
+  a.cval = cv.take<float>(L.Q * cap + pool * csz);
   L.total_bytes = cv.off;
   a.cap = cap;
   a.Lp = L.Lp;

@@ -100,6 +100,47 @@ def test_topk_sample_threshold_too_high_is_redone():
     assert_topk_equal(gpu_topk(g, r, (1, 60)), oracle.residual_topk(g, r, (1, 60)))
 
 
+def clustered_rows(n, seed, row=512, frac_rows=0.6, tokens=1000):
+    """Embedding-like gradient: rows of `row` entries, only the rows of Zipf-drawn token ids are
+    non-zero (N(0, 1e-2^2)) in the first `frac_rows` of the vector; the rest is dense N(0, 1e-4^2).
+    The large entries come in long runs, so whole pieces of the streaming pass are candidates."""
+    gen = synth.rng(seed, 91)
+    m = int(n * frac_rows) // row
+    g = synth.normal(gen, n, 1e-4)
+    g[:m * row] = 0.0
+    rows = np.unique(synth.zipf_ids(gen, tokens, m, 1.1))
+    for r_ in rows:
+        g[r_ * row:(r_ + 1) * row] = synth.normal(gen, row, 1e-2)
+    return g
+
+
+@pytest.mark.parametrize("pool", [1.0, 0.6, 0.3, 0.0])
+def test_topk_clustered_candidates_pool_and_reread(pool):
+    # candidates concentrated in dense rows overflow the per-piece stores: they continue in pool
+    # chunks, and pieces that find the pool empty are re-read; every split gives the same result
+    n = (1 << 22) + 4321
+    g = clustered_rows(n, 5)
+    r = synth.gaussian(n, 6, sigma=1e-5)
+    seg = np.array([0, 1 << 20, 3 << 20, n], np.int64)
+    for keep, s in [((1, 100), None), ((1, 100), seg), ((1, 20), None)]:
+        T = 1 if s is None else len(s) - 1
+        lo = int(gs.lib().gsparse_residual_topk_workspace_min(n, T))
+        hi = int(gs.lib().gsparse_residual_topk_workspace_size(n, T, *keep))
+        ws = lo + int((hi - lo) * pool) if pool < 1.0 else None
+        assert_topk_equal(gpu_topk(g, r, keep, seg=s, workspace_bytes=ws), oracle.residual_topk(g, r, keep, seg=s))
+
+
+def test_binarize_clustered_candidates():
+    n = (1 << 21) + 77
+    g = clustered_rows(n, 8, frac_rows=0.8)
+    r = np.zeros(n, np.float32)
+    for keep in [(1, 10), (1, 4)]:
+        lo = int(gs.lib().gsparse_binarize_workspace_min(n, 1, *keep))
+        hi = int(gs.lib().gsparse_binarize_workspace_size(n, 1, *keep))
+        for ws in [None, lo + (hi - lo) // 3]:
+            assert_binarize_equal(gpu_binarize(g, r, keep, workspace_bytes=ws), oracle.binarize(g, r, keep))
+
+
 def test_topk_multi_step_residual_carried():
     lay = synth.mlp_layout()
     seg = synth.offsets(lay)
@@ -385,6 +426,37 @@ def test_accumulate_combine_parity(W, n):
             assert np.array_equal(bits(host(dense)), bits(wd))
             out2 = gs.accumulate_combine(lists, n, L, alpha=alpha, beta=beta, mode=mode, own=own)
             assert np.array_equal(bits(host(out2)), bits(want))
+
+
+def test_accumulate_combine_crowded_tiles():
+    # most entries of every worker fall in a few tiles (dense rows), the rest are spread thin:
+    # tiles are taken dynamically and crowded ones walk thousands of entries per worker
+    n = (1 << 22) + 999
+    W = 4
+    gen = np.random.default_rng(4242)
+    host_lists, lists, keep = [], [], []
+    for w in range(W):
+        dense_part = gen.choice(np.arange(50000, 50000 + 40000), 30000, replace=False)
+        sparse_part = gen.choice(n, 20000, replace=False)
+        idx = np.unique(np.concatenate([dense_part, sparse_part])).astype(np.int32)
+        val = synth.gaussian(idx.size, 60 + w, sigma=1e-2)
+        cnt = torch.tensor([idx.size], dtype=torch.int64, device="cuda")
+        t = (dev(idx), cnt, dev(val))
+        keep.append(t)
+        host_lists.append((idx, val))
+        lists.append(gs.make_list(t[0], cnt, val=t[2], capacity=idx.size))
+    Lh = synth.gaussian(n, 9, sigma=1e-2)
+    wd, _, _ = oracle.scatter_accumulate(host_lists, n, merged=False)
+    for mode in (0, 1):
+        own = 1 if mode == 1 else -1
+        kw = {} if mode == 0 else {"own_idx": host_lists[own][0], "own_val": host_lists[own][1]}
+        want = oracle.combine_local(wd, Lh, 1.0, 1.0, mode=mode, **kw)
+        st = gs.status_tensor()
+        dense = torch.empty(n, device="cuda")
+        out = gs.accumulate_combine(lists, n, dev(Lh), mode=mode, own=own, dense_out=dense, d_status=st)
+        assert int(host(st)[0]) == 0
+        assert np.array_equal(bits(host(out)), bits(want))
+        assert np.array_equal(bits(host(dense)), bits(wd))
 
 
 # ------------------------------------------------------------------------------------ pending writes
