@@ -42,6 +42,8 @@ static_assert(kSample % (32 * kSampleCtas) == 0 && kSample / kSampleCtas <= 1024
               "each sample CTA takes whole runs, at most 32 of them");
 constexpr int kWarps = 8;                        // warps (pieces) per CTA
 constexpr int kMaxChunks = 64;                   // pool chunks one piece may claim
+constexpr int kUnitShift = 11;                   // work unit after pass 1: >= 2048 store positions,
+constexpr int kReadUnits = 8;                    // ... or 1/8 of a re-read piece
 constexpr int kThreads = kWarps * 32;
 
 struct Sel {
@@ -56,8 +58,12 @@ struct Sel {
   uint32_t *tlo, *redo, *pfx, *thr;
   int64_t *keff, *krem, *need_eq;
   uint32_t* hist;  // [P][kHist]
-  uint32_t *pcnt, *prsrc, *pgt, *peq, *ptake;
+  uint32_t *pcnt, *prsrc, *pgt, *peq, *ptake;  // pgt..poff: per work unit and class
   int64_t* poff;
+  int64_t* uoff;    // [Q + 1] first work unit of each piece (the last entry: the number of units)
+  int32_t* upiece;  // [units] the piece of each work unit
+  int64_t Ur, units_bound;
+  int32_t ushift;   // a stored piece's unit: 2^ushift store positions
   // candidate stores: Q primary stores of cap slots, then a pool of chunks of 2^chunk_shift slots
   // that a piece claims (at most max_chunks) once its primary store is full
   int32_t* cidx;
@@ -112,6 +118,35 @@ __device__ __forceinline__ int64_t slot_of(const Sel& a, int64_t q, uint32_t pos
   return a.Q * a.cap + (c << a.chunk_shift) + (o & ((1u << a.chunk_shift) - 1u));
 }
 
+// Work units of the steps after pass 1 (histogram levels 2-3, count, scan, emit): a piece with a
+// candidate store is split into units of 2^ushift store positions (at least its primary store,
+// so only pieces that spilled into the pool have more than one), a re-read piece into units of
+// Ur entries, so a piece crowded with candidates is shared by several warps.
+__device__ __forceinline__ int64_t unit_count(const Sel& a) { return a.uoff[total_pieces(a)]; }
+
+__device__ __forceinline__ int64_t unit_piece(const Sel& a, int64_t u) { return a.upiece[u]; }
+
+__device__ __forceinline__ int64_t units_of_piece(const Sel& a, int64_t q) {
+  if (a.prsrc[q]) {
+    const Piece P = piece_of(a, q);
+    return cdiv(P.hi - P.lo, a.Ur);
+  }
+  return cdiv((int64_t)a.pcnt[q], (int64_t)1 << a.ushift);
+}
+
+// The range of unit k of piece q: store positions [b, e), or for a re-read piece entries [b, e).
+__device__ __forceinline__ void unit_range(const Sel& a, int64_t q, const Piece& P, int64_t k,
+                                           int64_t* b, int64_t* e) {
+  if (a.prsrc[q]) {
+    *b = P.lo + k * a.Ur;
+    *e = *b + a.Ur < P.hi ? *b + a.Ur : P.hi;
+  } else {
+    const int64_t cnt = a.pcnt[q];
+    *b = k << a.ushift;
+    *e = *b + ((int64_t)1 << a.ushift) < cnt ? *b + ((int64_t)1 << a.ushift) : cnt;
+  }
+}
+
 // class of an accumulated value: top-k has one class; binarise splits by sign (zeros in none)
 template <int C>
 __device__ __forceinline__ int class_of(float x) {
@@ -135,8 +170,11 @@ struct CtaHist {
     else atomicAdd(hist_of(a, (int64_t)s * C + c, level) + bin, 1u);
   }
   __device__ void init(const Sel& a, int64_t q0) {
+    init_seg(q0 < total_pieces(a) ? piece_of(a, q0).s : -1);
+  }
+  __device__ void init_seg(int64_t seg) {
     for (int i = threadIdx.x; i < C * BINS; i += blockDim.x) sh[i] = 0;
-    if (threadIdx.x == 0) primary = q0 < total_pieces(a) ? piece_of(a, q0).s : -1;
+    if (threadIdx.x == 0) primary = seg;
   }
   // adds the shared counts of bins [0, bins) to the primary segment's histograms
   __device__ void flush(const Sel& a, int level, int bins) {
@@ -736,18 +774,19 @@ __global__ void pending_check_kernel(Sel a) {
 // ------------------------------------------------------------------------------------------
 // candidate iteration for the later steps (order not needed)
 
-// Calls f(x, c, key) for every candidate value of piece q: from the piece's store (values only;
-// four float4 loads per lane in flight), or, for pieces marked to be re-read, from the residual
-// (which then holds acc) filtered by class and T_lo.
+// Calls f(x, c, key) for every candidate value of piece q in [b, e): store positions (values
+// only; four float4 loads per lane in flight), or, for pieces marked to be re-read, entries of
+// the residual (which then holds acc) filtered by class and T_lo. b is a multiple of 4 for the
+// store.
 template <int C, class F>
-__device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, const Piece& P, F f) {
+__device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, const Piece& P,
+                                                   int64_t b, int64_t e, F f) {
   const int lane = threadIdx.x & 31;
   if (!a.prsrc[q]) {
-    // every store region starts 16-byte aligned (cap and the chunk size are multiples of 4):
-    // four per lane
-    const uint32_t cnt = a.pcnt[q];
+    // every store region starts 16-byte aligned (cap and the chunk size are multiples of 4)
+    const uint32_t cnt = (uint32_t)e;
     const uint32_t n4 = (cnt + 3) / 4;
-    for (uint32_t j4 = lane; j4 < n4; j4 += 128) {
+    for (uint32_t j4 = (uint32_t)b / 4 + lane; j4 < n4; j4 += 128) {
       float4 X[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h)
@@ -757,11 +796,11 @@ __device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, cons
       for (int h = 0; h < 4; ++h) {
         const float xv[4] = {X[h].x, X[h].y, X[h].z, X[h].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t j = 4 * (j4 + 32 * h) + e;
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const uint32_t j = 4 * (j4 + 32 * h) + e4;
           if (j < cnt) {
-            const int c = class_of<C>(xv[e]);
-            f(xv[e], c < 0 ? 0 : c, mag_key(xv[e]));
+            const int c = class_of<C>(xv[e4]);
+            f(xv[e4], c < 0 ? 0 : c, mag_key(xv[e4]));
           }
         }
       }
@@ -771,25 +810,25 @@ __device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, cons
   uint32_t tl[C];
 #pragma unroll
   for (int c = 0; c < C; ++c) tl[c] = a.tlo[(int64_t)P.s * C + c];
-  for (int64_t base = P.lo & ~(int64_t)3; base < P.hi; base += 128) {
+  for (int64_t base = b & ~(int64_t)3; base < e; base += 128) {
     const int64_t v = base + lane * 4;
     float x[4] = {0.f, 0.f, 0.f, 0.f};
-    if (v >= P.lo && v + 4 <= P.hi) {
+    if (v >= b && v + 4 <= e) {
       const float4 t = *reinterpret_cast<const float4*>(a.r + v);
       x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
     } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (v + e >= P.lo && v + e < P.hi) x[e] = a.r[v + e];
+      for (int e4 = 0; e4 < 4; ++e4)
+        if (v + e4 >= b && v + e4 < e) x[e4] = a.r[v + e4];
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int64_t i = v + e;
-      if (i < P.lo || i >= P.hi) continue;
-      const int c = class_of<C>(x[e]);
+    for (int e4 = 0; e4 < 4; ++e4) {
+      const int64_t i = v + e4;
+      if (i < b || i >= e) continue;
+      const int c = class_of<C>(x[e4]);
       if (c < 0) continue;
-      const uint32_t key = mag_key(x[e]);
-      if (key >= tl[c]) f(x[e], c, key);
+      const uint32_t key = mag_key(x[e4]);
+      if (key >= tl[c]) f(x[e4], c, key);
     }
   }
 }
@@ -847,7 +886,7 @@ __global__ void __launch_bounds__(kThreads) restore_kernel(Sel a) {
       __syncwarp();
       if (redo) {
         // the redone classes count every member (their T_lo is now 0)
-        for_each_candidate<C>(a, q, P, [&](float, int c, uint32_t key) {
+        for_each_candidate<C>(a, q, P, P.lo, P.hi, [&](float, int c, uint32_t key) {
           if (a.redo[(int64_t)P.s * C + c]) H.add(a, P.s, c, key >> 20, 1);
         });
       }
@@ -861,10 +900,31 @@ __global__ void __launch_bounds__(kThreads) restore_kernel(Sel a) {
 // ------------------------------------------------------------------------------------------
 // 5-7. radix-select levels
 
+// Numbers the work units of every piece (pieces and their stores are final after restore):
+// uoff and the unit -> piece table. One CTA; thread t owns a contiguous run of pieces.
+__device__ void number_units(const Sel& a, int64_t* sh) {
+  const int64_t Qn = total_pieces(a);
+  const int64_t per = cdiv(Qn, (int64_t)blockDim.x);
+  const int64_t q_lo = threadIdx.x * per < Qn ? threadIdx.x * per : Qn;
+  const int64_t q_hi = q_lo + per < Qn ? q_lo + per : Qn;
+  int64_t mine = 0;
+  for (int64_t q = q_lo; q < q_hi; ++q) mine += units_of_piece(a, q);
+  int64_t total;
+  int64_t run = block_exclusive_scan(mine, sh, &total);
+  for (int64_t q = q_lo; q < q_hi; ++q) {
+    const int64_t nu = units_of_piece(a, q);
+    a.uoff[q] = run;
+    for (int64_t k = 0; k < nu; ++k) a.upiece[run + k] = (int32_t)q;
+    run += nu;
+  }
+  if (threadIdx.x == 0) a.uoff[Qn] = total;
+}
+
 __global__ void __launch_bounds__(1024) select_kernel(Sel a, int level) {
   __shared__ uint32_t h[kBins1];
   __shared__ int64_t sh[33];
   if (a.ctl[0]) return;
+  if (level == 1 && blockIdx.x == 0) number_units(a, sh);
   const int64_t p = blockIdx.x;
   const int32_t s = (int32_t)(p / a.C);
   if (level > 1 && a.pfx[p] == kNone) return;
@@ -915,16 +975,20 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(Sel a, int level) {
   constexpr int B = kBins1;  // level 3 uses the first 512 bins
   __shared__ CtaHist<C, B> H;
   if (a.ctl[0]) return;
-  const int64_t q0 = (int64_t)blockIdx.x * kWarps;
-  H.init(a, q0);
+  const int64_t U = unit_count(a);
+  const int64_t u0 = (int64_t)blockIdx.x * kWarps;
+  if (u0 >= U) return;
+  H.init_seg(piece_of(a, unit_piece(a, u0)).s);
   __syncthreads();
-  const int64_t q = q0 + (threadIdx.x >> 5);
-  if (q < total_pieces(a)) {
+  for (int64_t u = u0 + (threadIdx.x >> 5); u < U; u += (int64_t)gridDim.x * kWarps) {
+    const int64_t q = unit_piece(a, u);
     const Piece P = piece_of(a, q);
+    int64_t b, e;
+    unit_range(a, q, P, u - a.uoff[q], &b, &e);
     uint32_t pf[C];
 #pragma unroll
     for (int c = 0; c < C; ++c) pf[c] = a.pfx[(int64_t)P.s * C + c];
-    for_each_candidate<C>(a, q, P, [&](float, int c, uint32_t key) {
+    for_each_candidate<C>(a, q, P, b, e, [&](float, int c, uint32_t key) {
       if (level == 2) {
         if ((key >> 20) == pf[c]) H.add(a, P.s, c, (key >> 9) & 2047u, 2);
       } else {
@@ -942,31 +1006,36 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(Sel a, int level) {
 template <int C>
 __global__ void __launch_bounds__(kThreads) count_kernel(Sel a) {
   if (a.ctl[0]) return;
-  const int64_t q = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (q >= total_pieces(a)) return;
-  const Piece P = piece_of(a, q);
-  uint32_t th[C], gt[C], eq[C];
+  const int64_t U = unit_count(a);
+  for (int64_t u = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); u < U;
+       u += (int64_t)gridDim.x * kWarps) {
+    const int64_t q = unit_piece(a, u);
+    const Piece P = piece_of(a, q);
+    int64_t b, e;
+    unit_range(a, q, P, u - a.uoff[q], &b, &e);
+    uint32_t th[C], gt[C], eq[C];
 #pragma unroll
-  for (int c = 0; c < C; ++c) {
-    th[c] = a.thr[(int64_t)P.s * C + c];
-    gt[c] = 0;
-    eq[c] = 0;
-  }
-  for_each_candidate<C>(a, q, P, [&](float, int c, uint32_t key) {
-#pragma unroll
-    for (int cc = 0; cc < C; ++cc) {
-      if (cc == c) {
-        gt[cc] += key > th[cc] && th[cc] != kNone;
-        eq[cc] += key == th[cc];
-      }
+    for (int c = 0; c < C; ++c) {
+      th[c] = a.thr[(int64_t)P.s * C + c];
+      gt[c] = 0;
+      eq[c] = 0;
     }
-  });
+    for_each_candidate<C>(a, q, P, b, e, [&](float, int c, uint32_t key) {
 #pragma unroll
-  for (int c = 0; c < C; ++c) {
-    const uint32_t G = warp_sum(gt[c]), E = warp_sum(eq[c]);
-    if ((threadIdx.x & 31) == 0) {
-      a.pgt[q * C + c] = G;
-      a.peq[q * C + c] = E;
+      for (int cc = 0; cc < C; ++cc) {
+        if (cc == c) {
+          gt[cc] += key > th[cc] && th[cc] != kNone;
+          eq[cc] += key == th[cc];
+        }
+      }
+    });
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      const uint32_t G = warp_sum(gt[c]), E = warp_sum(eq[c]);
+      if ((threadIdx.x & 31) == 0) {
+        a.pgt[u * C + c] = G;
+        a.peq[u * C + c] = E;
+      }
     }
   }
 }
@@ -977,28 +1046,36 @@ __global__ void __launch_bounds__(1024) scan_kernel(Sel a) {
   const int64_t p = blockIdx.x;
   const int32_t s = (int32_t)(p / a.C);
   const int c = (int)(p % a.C);
-  const int64_t first = a.seg_pbase[s], last = a.seg_pbase[s + 1];
+  // the work units of segment s, in index order; thread t owns a contiguous run of them
+  const int64_t first = a.uoff[a.seg_pbase[s]], last = a.uoff[a.seg_pbase[s + 1]];
   const int64_t need = a.need_eq[p];
-  int64_t eq_carry = 0, sel_carry = 0;
-  for (int64_t base = first; base < last; base += blockDim.x) {
-    const int64_t q = base + threadIdx.x;
-    int64_t eq = 0, gt = 0;
-    if (q < last) {
-      eq = a.peq[q * a.C + c];
-      gt = a.pgt[q * a.C + c];
-    }
-    int64_t teq, tsel;
-    const int64_t eq_before = eq_carry + block_exclusive_scan(eq, sh, &teq);
+  const int64_t per = cdiv(last - first, (int64_t)blockDim.x);
+  const int64_t u_lo = first + threadIdx.x * per < last ? first + threadIdx.x * per : last;
+  const int64_t u_hi = u_lo + per < last ? u_lo + per : last;
+  int64_t eq_mine = 0;
+  for (int64_t u = u_lo; u < u_hi; ++u) eq_mine += a.peq[u * a.C + c];
+  int64_t teq;
+  int64_t eq_before = block_exclusive_scan(eq_mine, sh, &teq);
+  // keys equal to the threshold: the first `need` of them in unit order are taken
+  int64_t sel_mine = 0;
+  for (int64_t u = u_lo; u < u_hi; ++u) {
+    const int64_t eq = a.peq[u * a.C + c];
     int64_t take = need - eq_before;
     take = take < 0 ? 0 : (take > eq ? eq : take);
-    const int64_t sel = gt + take;
-    const int64_t sel_before = sel_carry + block_exclusive_scan(sel, sh, &tsel);
-    if (q < last) {
-      a.poff[q * a.C + c] = sel_before;
-      a.ptake[q * a.C + c] = (uint32_t)take;
-    }
-    eq_carry += teq;
-    sel_carry += tsel;
+    sel_mine += a.pgt[u * a.C + c] + take;
+    eq_before += eq;
+  }
+  int64_t tsel;
+  int64_t sel_before = block_exclusive_scan(sel_mine, sh, &tsel);
+  eq_before -= eq_mine;
+  for (int64_t u = u_lo; u < u_hi; ++u) {
+    const int64_t eq = a.peq[u * a.C + c];
+    int64_t take = need - eq_before;
+    take = take < 0 ? 0 : (take > eq ? eq : take);
+    a.poff[u * a.C + c] = sel_before;
+    a.ptake[u * a.C + c] = (uint32_t)take;
+    sel_before += a.pgt[u * a.C + c] + take;
+    eq_before += eq;
   }
 }
 
@@ -1006,32 +1083,46 @@ __global__ void __launch_bounds__(1024) scan_kernel(Sel a) {
 // 9. emit, in index order
 
 template <int C>
+__device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_idx, float* out_val,
+                                          int64_t limit);
+
+template <int C>
 __global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
                                                         int64_t limit) {
   if (a.ctl[0]) return;
-  const int64_t q = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (q >= total_pieces(a)) return;
+  const int64_t U = unit_count(a);
+  for (int64_t u = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); u < U;
+       u += (int64_t)gridDim.x * kWarps)
+    emit_unit<C>(a, u, out_idx, out_val, limit);
+}
+
+template <int C>
+__device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_idx, float* out_val,
+                                          int64_t limit) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = lanemask_lt();
+  const int64_t q = unit_piece(a, u);
   const Piece P = piece_of(a, q);
+  int64_t ub, ue;
+  unit_range(a, q, P, u - a.uoff[q], &ub, &ue);
   uint32_t th[C], take[C], eq_run[C], sel_run[C];
   int64_t base_out[C];
 #pragma unroll
   for (int c = 0; c < C; ++c) {
     const int64_t p = (int64_t)P.s * C + c;
     th[c] = a.thr[p];
-    take[c] = a.ptake[q * C + c];
+    take[c] = a.ptake[u * C + c];
     eq_run[c] = 0;
     sel_run[c] = 0;
     // top-k: the segment's block of the output; binarise: the class list of the problem
-    base_out[c] = (C == 1 ? a.seg_kbase[P.s] : 2 * a.seg_kbase[P.s] + c * a.seg_k[P.s]) + a.poff[q * C + c];
+    base_out[c] = (C == 1 ? a.seg_kbase[P.s] : 2 * a.seg_kbase[P.s] + c * a.seg_k[P.s]) + a.poff[u * C + c];
   }
   auto is_sel = [&](int c, uint32_t key, bool eq_taken) {
     return c >= 0 && th[c] != kNone && (key > th[c] || eq_taken);
   };
   if (!a.prsrc[q]) {
-    // the store in index order, four consecutive candidates per lane
-    const uint32_t cnt = a.pcnt[q];
+    // the unit's store positions [ub, ue) in index order, four consecutive candidates per lane
+    const uint32_t cnt = (uint32_t)ue, jbeg = (uint32_t)ub;
     auto ci = [&](uint32_t pos) { return *reinterpret_cast<const int4*>(a.cidx + slot_of(a, q, pos)); };
     auto cv = [&](uint32_t pos) { return *reinterpret_cast<const float4*>(a.cval + slot_of(a, q, pos)); };
     // software pipelined: three batches of 128 candidates are in flight while one is placed
@@ -1040,11 +1131,11 @@ __global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_i
     float4 Xq[kAhead];
 #pragma unroll
     for (int h = 0; h < kAhead; ++h) {
-      const uint32_t jj = 128 * h + 4 * lane;
+      const uint32_t jj = jbeg + 128 * h + 4 * lane;
       Iq[h] = jj < cnt ? ci(jj) : make_int4(0, 0, 0, 0);
       Xq[h] = jj < cnt ? cv(jj) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (uint32_t j0 = 0; j0 < cnt; j0 += 128) {
+    for (uint32_t j0 = jbeg; j0 < cnt; j0 += 128) {
       const uint32_t j = j0 + 4 * lane;
       const int4 I = Iq[0];
       const float4 X = Xq[0];
@@ -1114,23 +1205,23 @@ __global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_i
     }
     return;
   }
-  // re-read piece: the residual holds acc; walk it in index order
-  for (int64_t vb = P.lo & ~(int64_t)3; vb < P.hi; vb += 128) {
+  // re-read piece: the residual holds acc; walk the unit's entries [ub, ue) in index order
+  for (int64_t vb = ub & ~(int64_t)3; vb < ue; vb += 128) {
     const int64_t v = vb + lane * 4;
     float x[4] = {0.f, 0.f, 0.f, 0.f};
-    if (v >= P.lo && v + 4 <= P.hi) {
+    if (v >= ub && v + 4 <= ue) {
       const float4 t = *reinterpret_cast<const float4*>(a.r + v);
       x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
     } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (v + e >= P.lo && v + e < P.hi) x[e] = a.r[v + e];
+        if (v + e >= ub && v + e < ue) x[e] = a.r[v + e];
     }
     int cls[4];
     uint32_t key[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const bool in = v + e >= P.lo && v + e < P.hi;
+      const bool in = v + e >= ub && v + e < ue;
       cls[e] = in ? class_of<C>(x[e]) : -1;
       key[e] = mag_key(x[e]);
     }
@@ -1319,10 +1410,16 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
   a.keff = cv.take<int64_t>(P);
   a.krem = cv.take<int64_t>(P);
   a.need_eq = cv.take<int64_t>(P);
-  a.pgt = cv.take<uint32_t>(L.Q * C);
-  a.peq = cv.take<uint32_t>(L.Q * C);
-  a.ptake = cv.take<uint32_t>(L.Q * C);
-  a.poff = cv.take<int64_t>(L.Q * C);
+  a.uoff = cv.take<int64_t>(L.Q + 1);
+  // work units: a stored piece holds at most as many candidates as entries, so at most
+  // n / 2^kUnitShift + Q units; a re-read piece at most kReadUnits
+  a.Ur = round_up(cdiv(L.Lp, kReadUnits), 128);
+  a.units_bound = L.Q * (kReadUnits + 1) + (n >> kUnitShift) + 1;
+  a.upiece = cv.take<int32_t>(a.units_bound);
+  a.pgt = cv.take<uint32_t>(a.units_bound * C);
+  a.peq = cv.take<uint32_t>(a.units_bound * C);
+  a.ptake = cv.take<uint32_t>(a.units_bound * C);
+  a.poff = cv.take<int64_t>(a.units_bound * C);
   // zero-initialised block
   const size_t zoff = (size_t)round_up((int64_t)cv.off, 256);
   a.ctl = cv.take<int32_t>(64);
@@ -1382,6 +1479,11 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
   if (pool > INT32_MAX) pool = INT32_MAX;
   L.cap = cap;
   a.pool_chunks = pool;
+  // a stored piece's work unit covers at least its primary store (pieces that did not spill are
+  // one unit each)
+  int32_t us = kUnitShift;
+  while (((int64_t)1 << us) < cap) ++us;
+  a.ushift = us;
   a.cidx = cv.take<int32_t>(L.Q * cap + pool * csz);
   a.cval = cv.take<float>(L.Q * cap + pool * csz);
   L.total_bytes = cv.off;
@@ -1451,14 +1553,18 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   check_kernel<<<(unsigned)(T * C), 256, 0, st>>>(a);
   if (piece_ctas) restore_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
   select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 1);
-  if (piece_ctas) hist_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a, 2);
+  // the steps after pass 1 run over work units, at most a.units_bound of them
+  int64_t uc = cdiv(a.units_bound, kWarps);
+  if (uc > (int64_t)sm_count() * 8) uc = (int64_t)sm_count() * 8;
+  const unsigned unit_ctas = piece_ctas ? (unsigned)uc : 0u;
+  if (unit_ctas) hist_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a, 2);
   select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 2);
-  if (piece_ctas) hist_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a, 3);
+  if (unit_ctas) hist_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a, 3);
   select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 3);
-  if (piece_ctas) count_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
+  if (unit_ctas) count_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a);
   scan_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a);
-  if (piece_ctas)
-    emit_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a, out_idx, out_val,
+  if (unit_ctas)
+    emit_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a, out_idx, out_val,
                                                     C == 1 ? out_capacity : 2 * L.kbound);
   if (C == 2) {
     bjobs_kernel<<<1, 1024, 0, st>>>(a, L.jobs);
