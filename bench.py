@@ -504,6 +504,32 @@ def run_workload(args):
     compress = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
     receive = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
 
+    # the same step captured once as a CUDA graph and replayed (no host work per step)
+    graph_ms = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(K):
+            graph.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device status {int(st.item())} (graph replay)")
+        graph_ms = g0.elapsed_time(g1) / K
+        del graph
+
     # the oracle on the same step (first step, zero residual), single thread
     t = time.perf_counter()
     if not args.no_oracle:
@@ -523,6 +549,9 @@ def run_workload(args):
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
                          "algorithmic_bytes_per_step": algo},
             "stages_ms": {"compress": round(compress, 4), "receive": round(receive, 4)}, "steps": K,
+            "graph": None if graph_ms is None else {
+                "ms_per_step": round(graph_ms, 4), "value": round(grad / (graph_ms * 1e-3) / 1e9, 2),
+                "what": "the same step captured once as a CUDA graph and replayed"},
             "oracle": None if args.no_oracle else {
                 "ms_per_step": round(oms, 1), "value": round(grad / (oms * 1e-3) / 1e9, 4), "cores": 1,
                 "sample": "the same step on the full workload, zero residual, single-threaded C++ oracle"}}
@@ -611,6 +640,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
                     help="time one of the smaller workloads instead of the default flat 2^30 line")
     ap.add_argument("--no-oracle", action="store_true", help="with --workload: skip the oracle timing")
+    ap.add_argument("--no-graph", action="store_true", help="with --workload: skip the CUDA-graph replay leg")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -44,22 +44,33 @@ __global__ void g_setup_kernel(const int64_t* d_begin, const int64_t* d_end, int
 }
 
 // Gaps of this thread's kPer consecutive codewords (entries j0 .. j0+kPer-1 of the list); an
-// invalid (negative) gap is reported and coded as 0.
+// invalid (negative) gap is reported and coded as 0. Indices are non-negative int32, so a gap
+// fits 32 bits. The eight entries come in as two 16-byte loads when they are aligned.
 __device__ __forceinline__ void thread_gaps(const int32_t* x, int64_t len, int64_t base, int64_t j0,
-                                            int64_t (&d)[kPer], int32_t* d_status) {
+                                            uint32_t (&d)[kPer], int32_t* d_status) {
+  static_assert(kPer == 8, "two int4 loads per thread");
+  int32_t v[kPer];
+  if (j0 + kPer <= len && (reinterpret_cast<uintptr_t>(x + j0) & 15u) == 0) {
+    const int4 a = *reinterpret_cast<const int4*>(x + j0);
+    const int4 c = *reinterpret_cast<const int4*>(x + j0 + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) v[e] = j0 + e < len ? x[j0 + e] : 0;
+  }
   int64_t prev = j0 == 0 ? base - 1 : (j0 - 1 < len ? (int64_t)x[j0 - 1] : 0);
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
-    const int64_t j = j0 + e;
     d[e] = 0;
-    if (j < len) {
-      const int64_t cur = x[j];
-      d[e] = cur - prev - 1;
-      if (d[e] < 0) {
+    if (j0 + e < len) {
+      const int64_t g = (int64_t)v[e] - prev - 1;
+      if (g < 0) {
         if (d_status) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
-        d[e] = 0;
+      } else {
+        d[e] = (uint32_t)g;
       }
-      prev = cur;
+      prev = v[e];
     }
   }
 }
@@ -73,12 +84,12 @@ __global__ void __launch_bounds__(kCodeThreads) g_len_kernel(const int32_t* idx,
   const int64_t len = ctl->len;
   if ((int64_t)blockIdx.x * kBlockCodes >= len) return;
   const int64_t j0 = (int64_t)blockIdx.x * kBlockCodes + (int64_t)threadIdx.x * kPer;
-  int64_t d[kPer];
+  uint32_t d[kPer];
   thread_gaps(idx + ctl->begin, len, base, j0, d, d_status);
   int64_t l = 0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e)
-    if (j0 + e < len) l += (d[e] >> b) + 1 + b;
+    if (j0 + e < len) l += (int64_t)(d[e] >> b) + 1 + b;
   int64_t tot;
   block_exclusive_scan(l, sh, &tot);
   if (threadIdx.x == 0) block_tot[blockIdx.x] = tot;
@@ -171,37 +182,34 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
   const int32_t* x = idx + ctl->begin;
   const int64_t jb = (int64_t)blockIdx.x * kBlockCodes;
   const int64_t j0 = jb + (int64_t)threadIdx.x * kPer;
-  int64_t d[kPer];
+  uint32_t d[kPer];
   thread_gaps(x, len, base, j0, d, nullptr);
   int64_t l = 0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e)
-    if (j0 + e < len) l += (d[e] >> b) + 1 + b;
+    if (j0 + e < len) l += (int64_t)(d[e] >> b) + 1 + b;
   int64_t tot;
   const int64_t o0 = block_pre[blockIdx.x] + block_exclusive_scan(l, sh, &tot);
   if (threadIdx.x == 0) span_lo = (uint64_t)o0;
   if (threadIdx.x == blockDim.x - 1) span_hi = (uint64_t)(o0 + l);   // the block's last bit + 1
-  Code cs[kPer];
-  int64_t o = o0;
-  // position of j0 inside its side-table chunk (one 32-bit division per thread; indices < 2^31)
-  uint32_t in_chunk = table ? (uint32_t)j0 % (uint32_t)chunk : 1u;
+  // side table: bit offset and preceding index at every chunk start (one 32-bit division per
+  // thread; indices < 2^31)
+  if (table) {
+    uint32_t in_chunk = (uint32_t)j0 % (uint32_t)chunk;
+    int64_t o = o0;
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) {
-    const int64_t j = j0 + e;
-    cs[e].o = (uint64_t)o;
-    cs[e].q = (uint64_t)(d[e] >> b);
-    const uint32_t rem = (uint32_t)(d[e] & ((int64_t(1) << b) - 1));
-    cs[e].tail = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
-    cs[e].len_tail = 1u + (uint32_t)b;
-    if (j < len) {
-      if (table && in_chunk == 0) {
-        const int64_t c = (int64_t)((uint32_t)j / (uint32_t)chunk);
-        table[2 * c] = o;
-        table[2 * c + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
+    for (int e = 0; e < kPer; ++e) {
+      const int64_t j = j0 + e;
+      if (j < len) {
+        if (in_chunk == 0) {
+          const int64_t c = (int64_t)((uint32_t)j / (uint32_t)chunk);
+          table[2 * c] = o;
+          table[2 * c + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
+        }
+        o += (int64_t)(d[e] >> b) + 1 + b;
       }
-      o += (int64_t)cs[e].q + cs[e].len_tail;
+      if (++in_chunk == (uint32_t)chunk) in_chunk = 0;
     }
-    if (table && ++in_chunk == (uint32_t)chunk) in_chunk = 0;
   }
   __syncthreads();
   const uint64_t S = span_lo, E = span_hi;
@@ -210,41 +218,63 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
   if (fits) {
     for (int i = threadIdx.x; i < kPackWords; i += blockDim.x) wbuf[i] = 0u;
     __syncthreads();
+    // positions relative to the block's first word: the block spans < 2^17 bits here
+    uint32_t p = (uint32_t)((uint64_t)o0 - 32u * wf);
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      if (j0 + e >= len) break;
+      const uint32_t q = d[e] >> b;
+      const uint32_t rem = d[e] & ((1u << b) - 1u);
+      // terminator 0, then the remainder most significant bit first
+      const uint32_t tail = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
+      if (q + 1u + (uint32_t)b <= 32u) {
+        // the whole codeword as one pattern: at most two words
+        const uint32_t pat = (q ? 0xffffffffu >> (32u - q) : 0u) | (tail << q);
+        const uint64_t v = (uint64_t)pat << (p & 31u);
+        if ((uint32_t)v) atomicOr(&wbuf[p >> 5], (uint32_t)v);
+        if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(p >> 5) + 1], (uint32_t)(v >> 32));
+      } else {
+        uint32_t pp = p, qq = q;
+        while (qq) {  // the unary run of ones
+          const uint32_t sh2 = pp & 31u, nrun = qq < 32u - sh2 ? qq : 32u - sh2;
+          atomicOr(&wbuf[pp >> 5], (nrun == 32u ? 0xffffffffu : ((1u << nrun) - 1u)) << sh2);
+          pp += nrun;
+          qq -= nrun;
+        }
+        const uint64_t v = (uint64_t)tail << (pp & 31u);  // terminator + remainder, <= 32 bits
+        if ((uint32_t)v) atomicOr(&wbuf[pp >> 5], (uint32_t)v);
+        if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(pp >> 5) + 1], (uint32_t)(v >> 32));
+      }
+      p += q + 1u + (uint32_t)b;
+    }
+    __syncthreads();
+    for (uint64_t w = wf + threadIdx.x; w <= wl; w += blockDim.x) {
+      const uint32_t bits = wbuf[w - wf];
+      if ((w == wf && (S & 31)) || (w == wl && (E & 31))) {
+        if (bits) atomicOr(&words[w], bits);   // shared with a neighbouring block
+      } else {
+        words[w] = bits;
+      }
+    }
+    return;
   }
+  // long unary runs: every codeword is OR-ed straight into the zeroed stream
+  int64_t o = o0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     if (j0 + e >= len) break;
-    const Code& c = cs[e];
-    if (fits) {
-      // positions relative to the block's first word: the block spans < 2^17 bits here
-      uint32_t p = (uint32_t)(c.o - 32u * wf);
-      uint32_t q = (uint32_t)c.q;
-      while (q) {  // the unary run of ones
-        const uint32_t sh = p & 31u, nrun = q < 32u - sh ? q : 32u - sh;
-        atomicOr(&wbuf[p >> 5], (nrun == 32u ? 0xffffffffu : ((1u << nrun) - 1u)) << sh);
-        p += nrun;
-        q -= nrun;
-      }
-      const uint64_t v = (uint64_t)c.tail << (p & 31u);  // terminator + remainder, <= 31 bits
-      if ((uint32_t)v) atomicOr(&wbuf[p >> 5], (uint32_t)v);
-      if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(p >> 5) + 1], (uint32_t)(v >> 32));
-    } else {
-      const uint64_t w0 = c.o >> 5, w1 = (c.o + c.q + c.len_tail - 1) >> 5;
-      for (uint64_t w = w0; w <= w1; ++w) {
-        const uint32_t bits = code_bits_in_word(c, w);
-        if (bits) atomicOr(&words[w], bits);
-      }
+    Code c;
+    c.o = (uint64_t)o;
+    c.q = (uint64_t)(d[e] >> b);
+    const uint32_t rem = d[e] & ((1u << b) - 1u);
+    c.tail = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
+    c.len_tail = 1u + (uint32_t)b;
+    const uint64_t w0 = c.o >> 5, w1 = (c.o + c.q + c.len_tail - 1) >> 5;
+    for (uint64_t w = w0; w <= w1; ++w) {
+      const uint32_t bits = code_bits_in_word(c, w);
+      if (bits) atomicOr(&words[w], bits);
     }
-  }
-  if (!fits) return;
-  __syncthreads();
-  for (uint64_t w = wf + threadIdx.x; w <= wl; w += blockDim.x) {
-    const uint32_t bits = wbuf[w - wf];
-    if ((w == wf && (S & 31)) || (w == wl && (E & 31))) {
-      if (bits) atomicOr(&words[w], bits);   // shared with a neighbouring block
-    } else {
-      words[w] = bits;
-    }
+    o += (int64_t)c.q + c.len_tail;
   }
 }
 
@@ -298,36 +328,63 @@ __device__ bool decode_run(const uint32_t* src, int64_t base_w, int64_t lim_w, u
   return true;
 }
 
+// Decodes one codeword from a staged window, word by word (any length): the general path.
+__device__ __forceinline__ bool decode_one_local_slow(const uint32_t* sw, uint32_t nb_rel, uint32_t& t,
+                                                      uint32_t& q_out, uint32_t& rem_out, int b,
+                                                      int32_t* d_status) {
+  uint32_t q = 0;
+  for (;;) {
+    if (t >= nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+    const uint32_t sh = t & 31u;
+    const uint32_t zeros = ~(sw[t >> 5] >> sh) & (0xffffffffu >> sh);
+    if (zeros) {
+      const uint32_t z = (uint32_t)__ffs(zeros) - 1u;
+      q += z;
+      t += z + 1u;
+      break;
+    }
+    q += 32u - sh;
+    t += 32u - sh;
+  }
+  uint32_t rem = 0;
+  if (b > 0) {
+    if (t > nb_rel || nb_rel - t < (uint32_t)b) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+    const uint32_t w = t >> 5;
+    const uint64_t win = (uint64_t)sw[w] | ((uint64_t)sw[w + 1] << 32);
+    rem = __brev((uint32_t)(win >> (t & 31u)) & ((1u << b) - 1u)) >> (32 - b);
+    t += (uint32_t)b;
+  } else if (t > nb_rel) {
+    raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+    return false;
+  }
+  q_out = q;
+  rem_out = rem;
+  return true;
+}
+
 // Decodes `count` codewords from a staged window: sw holds stream words [wa, wa + nwin) (the last
-// one a zero spare), t is the bit position relative to bit 32 * wa, and nb_rel the stream end
-// relative to the same origin (at most 32 * (nwin - 1)). 32-bit positions throughout.
+// two are zero spares), t is the bit position relative to bit 32 * wa, and nb_rel the stream end
+// relative to the same origin (at most 32 * (nwin - 2)). 32-bit positions throughout. A codeword
+// of at most 64 bits (all but pathological gaps) is taken from one 64-bit window: the run of ones
+// ends at the first zero bit, the remainder follows it in the same window.
 __device__ bool decode_run_local(const uint32_t* sw, uint32_t nb_rel, uint32_t& t, int64_t& prev,
                                  int count, int b, int64_t n_limit, int32_t* out, int stride,
                                  int32_t* d_status) {
+  const uint32_t mask = b > 0 ? 0xffffffffu >> (32 - b) : 0u;
   for (int k = 0; k < count; ++k) {
-    uint32_t q = 0;
-    for (;;) {
-      if (t >= nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
-      const uint32_t sh = t & 31u;
-      const uint32_t zeros = ~(sw[t >> 5] >> sh) & (0xffffffffu >> sh);
-      if (zeros) {
-        const uint32_t z = (uint32_t)__ffs(zeros) - 1u;
-        q += z;
-        t += z + 1u;
-        break;
-      }
-      q += 32u - sh;
-      t += 32u - sh;
-    }
-    uint32_t rem = 0;
-    if (b > 0) {
-      if (t > nb_rel || nb_rel - t < (uint32_t)b) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
-      const uint32_t w = t >> 5;
-      const uint64_t win = (uint64_t)sw[w] | ((uint64_t)sw[w + 1] << 32);
-      rem = __brev((uint32_t)(win >> (t & 31u)) & ((1u << b) - 1u)) >> (32 - b);
-      t += (uint32_t)b;
-    } else if (t > nb_rel) {
-      raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
+    if (t >= nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+    const uint32_t w = t >> 5, s = t & 31u;
+    uint64_t win = ((uint64_t)sw[w] | ((uint64_t)sw[w + 1] << 32)) >> s;
+    if (s) win |= (uint64_t)sw[w + 2] << (64u - s);
+    uint32_t q, rem = 0;
+    const uint64_t zeros = ~win;
+    const uint32_t z = zeros ? (uint32_t)__ffsll((long long)zeros) - 1u : 64u;
+    if (z + 1u + (uint32_t)b <= 64u) {
+      q = z;
+      if (b > 0) rem = __brev((uint32_t)(win >> (z + 1u)) & mask) >> (32 - b);
+      t += z + 1u + (uint32_t)b;
+      if (t > nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+    } else if (!decode_one_local_slow(sw, nb_rel, t, q, rem, b, d_status)) {
       return false;
     }
     const int64_t i = prev + 1 + (int64_t)(((uint64_t)q << b) | rem);
@@ -372,7 +429,7 @@ __global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
   ba = ba < nbits ? ba : nbits;
   bz = bz < nbits ? (bz > ba ? bz : ba) : nbits;
   const int64_t nw = cdiv((int64_t)nbits, 32);
-  const int64_t wa = (int64_t)(ba >> 5), wz = cdiv((int64_t)bz, 32) + 1;   // one zero spare word
+  const int64_t wa = (int64_t)(ba >> 5), wz = cdiv((int64_t)bz, 32) + 2;   // two zero spare words
   const bool staged = wz - wa <= kDecWords;
   if (staged) {
     const int span = (int)(wz - wa);

@@ -78,12 +78,29 @@ __global__ void __launch_bounds__(256) sa_starts_kernel(Lists L, int32_t W, int6
 #pragma unroll
     for (int e = 0; e < kStartsPer; ++e) v[e] = j0 + e < c ? ix[j0 + e] : 0;
   }
-  int32_t prev = j0 > 0 ? ix[j0 - 1] : 0;
+  // fast scan: the entries whose tile differs from their predecessor's (or that lie outside
+  // [0, n), or close the list) are marked; the rest start nothing
+  const int32_t p0 = j0 > 0 ? ix[j0 - 1] : -1;
+  const uint32_t un = (uint32_t)(n < INT32_MAX ? n : INT32_MAX);
+  uint32_t mark = 0;
+  int32_t pv = p0;
 #pragma unroll
   for (int e = 0; e < kStartsPer; ++e) {
-    if (j0 + e > c) break;
-    starts_at(ix, j0 + e, c, v[e], prev, ntiles, W, w, start, d_status);
-    prev = v[e];
+    const int64_t j = j0 + e;
+    const bool in = j < c;
+    const bool odd = !in || v[e] < 0 || (uint32_t)v[e] >= un || pv < 0 ||
+                     ((uint32_t)v[e] / (uint32_t)kTile) != ((uint32_t)pv / (uint32_t)kTile);
+    mark |= (uint32_t)(odd && j <= c) << e;
+    pv = v[e];
+  }
+  // the marked entries, in order (rolled loop: the list values come again from L1)
+  while (mark) {
+    const int e = __ffs(mark) - 1;
+    mark &= mark - 1;
+    const int64_t j = j0 + e;
+    const int32_t cur = j < c ? ix[j] : 0;
+    const int32_t prev = j > 0 ? ix[j - 1] : 0;
+    starts_at(ix, j, c, cur, prev, ntiles, W, w, start, d_status);
   }
 }
 

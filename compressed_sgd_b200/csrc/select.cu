@@ -77,7 +77,9 @@ struct Sel {
   uint32_t *shist, *scount, *sdone, *sb1, *sblo, *ssub;
   int64_t *srank, *sabove, *smcap;
   unsigned long long* svar;  // per problem: sum and sum of squares of the per-run counts
-  // pending residual writes applied in the sample and pass 1 (null: none)
+  // pending residual writes applied in the sample and pass 1 (null: none); pstart[q] is the
+  // first write at or after piece q's first entry ([Q + 1])
+  uint32_t* pstart;
   const int32_t* pw_idx;
   const float* pw_val;
   const int64_t* pw_count;
@@ -103,6 +105,15 @@ __device__ __forceinline__ Piece piece_of(const Sel& a, int64_t q) {
   const int64_t end = a.seg_lo[p.s] + a.seg_n[p.s];
   p.hi = p.lo + a.Lp < end ? p.lo + a.Lp : end;
   return p;
+}
+
+// The piece holding entry i (0 <= i < n).
+__device__ __forceinline__ int64_t piece_containing(const Sel& a, int64_t i) {
+  const int64_t s = upper_bound_i64(a.seg_lo, a.T, i) - 1;  // the last segment starting at or before i
+  const int64_t sc = s < 0 ? 0 : s;
+  const int64_t q = a.seg_pbase[sc] + (i - a.seg_lo[sc]) / a.Lp;
+  const int64_t qmax = a.seg_pbase[sc + 1] - 1;
+  return q > qmax ? qmax : q;
 }
 
 // Slots of a piece's candidate store: positions [0, cap) in its primary store, later positions in
@@ -298,6 +309,15 @@ __device__ __forceinline__ uint32_t pending_count(const Sel& a) {
   return (uint32_t)c;
 }
 
+// First pending write at or after entry x: searched only among the writes of x's piece.
+__device__ __forceinline__ uint32_t pending_lower_bound(const Sel& a, int64_t x) {
+  if (x <= 0) return 0;
+  if (x >= a.n) return pending_count(a);
+  const int64_t q = piece_containing(a, x);
+  const uint32_t b = a.pstart[q], e = a.pstart[q + 1];
+  return b + (uint32_t)lower_bound_i32(a.pw_idx + b, e > b ? e - b : 0, x);
+}
+
 // The residual value of entry i with the pending writes applied (the writes in [b, e) of the
 // list, which must hold every write of the caller's range).
 __device__ __forceinline__ float residual_at(const Sel& a, int64_t i, uint32_t b, uint32_t e) {
@@ -372,8 +392,8 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
   if (threadIdx.x == 0) {
     pwb = pwe = 0;
     if (pc && ns <= kSample) {
-      pwb = (uint32_t)lower_bound_i32(a.pw_idx, pc, lo + j0);
-      pwe = (uint32_t)lower_bound_i32(a.pw_idx, pc, lo + j1);
+      pwb = pending_lower_bound(a, lo + j0);
+      pwe = pending_lower_bound(a, lo + j1);
     }
   }
   if (runs && threadIdx.x < 32) {
@@ -381,7 +401,7 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
     uint32_t b = 0, e = 0;
     if (jr < j1) {
       const int64_t start = sample_pos(lo, ns, jr);
-      b = (uint32_t)lower_bound_i32(a.pw_idx, pc, start);
+      b = pending_lower_bound(a, start);
       const uint32_t span = pc - b < 33u ? pc - b : 33u;
       e = b + (uint32_t)lower_bound_i32(a.pw_idx + b, span, start + 32);
     }
@@ -714,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     S.nch = 0;
     S.ch_lo = S.pv_lo = 0;
     S.ch_base = S.pv_base = q * a.cap;
-    if (cend) S.cp = __shfl_sync(kFull, lane == 0 ? (uint32_t)lower_bound_i32(a.pw_idx, cend, lo) : 0u, 0);
+    if (cend) S.cp = a.pstart[q];
     load_window(a, S.cp, cend, lane, S);
     uint32_t base = lo & ~3u;
     float4 gv[4], rv[4];
@@ -752,18 +772,63 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
 }
 
 // The pending residual writes must be strictly ascending indices in [0, n): anything else stops
-// the call before it touches the residual.
-__global__ void pending_check_kernel(Sel a) {
+// the call before it touches the residual. The same pass records pstart: the pieces whose first
+// entry lies in (idx[j-1], idx[j]] start their writes at j. A thread takes kCheckPer consecutive
+// writes and keeps the first entry of the next piece, so it locates a piece only when a write
+// crosses a piece start.
+constexpr int kCheckPer = 16;
+
+__global__ void __launch_bounds__(256) pending_check_kernel(Sel a) {
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (t == 0 && *a.pw_count > a.pw_cap) {
     raise(a.d_status, GSPARSE_DERR_CAPACITY);
     a.ctl[0] = 1;
   }
   const uint32_t c = pending_count(a);
+  const int64_t Qn = total_pieces(a);
+  const int64_t j0 = t * kCheckPer;
   bool bad = false;
-  for (int64_t j = t; j < c; j += (int64_t)gridDim.x * blockDim.x) {
-    const int32_t i = a.pw_idx[j];
-    bad |= i < 0 || (int64_t)i >= a.n || (j > 0 && a.pw_idx[j - 1] >= i);
+  if (j0 <= c) {
+    const int32_t* x = a.pw_idx;
+    int32_t v[kCheckPer];
+    if (j0 + kCheckPer <= c && (reinterpret_cast<uintptr_t>(x + j0) & 15u) == 0) {
+#pragma unroll
+      for (int h = 0; h < kCheckPer / 4; ++h) {
+        const int4 w = *reinterpret_cast<const int4*>(x + j0 + 4 * h);
+        v[4 * h] = w.x; v[4 * h + 1] = w.y; v[4 * h + 2] = w.z; v[4 * h + 3] = w.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kCheckPer; ++e) v[e] = j0 + e < c ? x[j0 + e] : 0;
+    }
+    const int64_t ip0 = j0 > 0 ? x[j0 - 1] : -1;
+    auto clampi = [&](int64_t i) { return i < 0 ? (int64_t)0 : (i < a.n ? i : a.n - 1); };
+    // the last piece already started before this thread's first write, and the next piece's start
+    int64_t q_prev = (ip0 < 0 || Qn == 0) ? -1 : piece_containing(a, clampi(ip0));
+    int64_t next_lo = q_prev + 1 < Qn ? piece_of(a, q_prev + 1).lo : INT64_MAX;
+    // fast scan: validity, and a mark on every write at or beyond the next piece's start
+    uint32_t mark = 0;
+    int64_t ip = ip0;
+#pragma unroll
+    for (int e = 0; e < kCheckPer; ++e) {
+      const int64_t j = j0 + e;
+      const int64_t i = v[e];
+      if (j < c) bad |= i < 0 || i >= a.n || (j > 0 && ip >= i);
+      mark |= (uint32_t)(j <= c && (j == c || i >= next_lo)) << e;
+      ip = i;
+    }
+    // the marked writes, in order (rolled loop)
+    while (mark && Qn > 0) {
+      const int e = __ffs(mark) - 1;
+      mark &= mark - 1;
+      const int64_t j = j0 + e;
+      const int64_t i = j < c ? (int64_t)x[j] : a.n;
+      if (j < c && i < next_lo) continue;
+      const int64_t q_cur = j < c ? piece_containing(a, clampi(i)) : Qn;
+      for (int64_t q = q_prev + 1; q <= q_cur; ++q) a.pstart[q] = (uint32_t)j;
+      if (q_cur > q_prev) q_prev = q_cur;
+      next_lo = q_prev + 1 < Qn ? piece_of(a, q_prev + 1).lo : INT64_MAX;
+    }
   }
   if (__any_sync(kFull, bad) && (threadIdx.x & 31) == 0) {
     raise(a.d_status, GSPARSE_DERR_INDEX_RANGE);
@@ -1338,8 +1403,11 @@ __global__ void bemit_kernel(Sel a, const float* d_mean, const int64_t* out_offs
 // ------------------------------------------------------------------------------------------
 // accumulate only (keep 0): residual <- fl(g + residual)
 
-__global__ void accumulate_kernel(const float* g, float* r, int64_t n, const int32_t* ctl) {
-  if (ctl[0]) return;
+// ctl null: no plan ran (one segment), and the kernel itself reports the empty output offsets.
+__global__ void accumulate_kernel(const float* g, float* r, int64_t n, const int32_t* ctl,
+                                  int64_t* out_offsets) {
+  if (ctl && ctl[0]) return;
+  if (!ctl && out_offsets && blockIdx.x == 0 && threadIdx.x < 2) out_offsets[threadIdx.x] = 0;
   const int64_t nv = n >> 2;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nv; v += stride) {
@@ -1411,6 +1479,7 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
   a.krem = cv.take<int64_t>(P);
   a.need_eq = cv.take<int64_t>(P);
   a.uoff = cv.take<int64_t>(L.Q + 1);
+  a.pstart = cv.take<uint32_t>(L.Q + 1);
   // work units: a stored piece holds at most as many candidates as entries, so at most
   // n / 2^kUnitShift + Q units; a re-read piece at most kReadUnits
   a.Ur = round_up(cdiv(L.Lp, kReadUnits), 128);
@@ -1525,6 +1594,12 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   a.zero_mode = C == 1;
   a.d_status = d_status;
   const bool has_pending = pending && pending->capacity > 0;
+  if (num == 0 && C == 1 && !has_pending && seg == nullptr) {
+    // communication delay step on one segment: accumulate only, nothing to plan
+    const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
+    accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, nullptr, out_offsets);
+    return launch_status();
+  }
   a.pw_idx = has_pending ? pending->idx : nullptr;
   a.pw_val = has_pending ? pending->val : nullptr;
   a.pw_count = has_pending ? pending->d_count : nullptr;
@@ -1532,12 +1607,11 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   if (cudaMemsetAsync(L.zero_begin, 0, L.zero_bytes, st) != cudaSuccess) return GSPARSE_ERR_CUDA;
   plan_kernel<<<1, 1024, 0, st>>>(a, seg, num, den, out_capacity, C == 1 ? out_offsets : nullptr);
   if (has_pending)
-    pending_check_kernel<<<(unsigned)(cdiv(a.pw_cap, 256) < 148 * 8 ? cdiv(a.pw_cap, 256) : 148 * 8), 256, 0,
-                           st>>>(a);
+    pending_check_kernel<<<(unsigned)cdiv(a.pw_cap + 1, 256 * kCheckPer), 256, 0, st>>>(a);
   if (num == 0 && C == 1 && !has_pending) {  // communication delay step: accumulate only
     if (n > 0) {
       const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
-      accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, a.ctl);
+      accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, a.ctl, nullptr);
     }
     return launch_status();
   }
