@@ -569,16 +569,41 @@ __device__ __forceinline__ void load_window(const Sel& a, uint32_t cp, uint32_t 
 
 // One chunk of 512 entries [base, base + 512) of the piece [lo, hi): pending writes, acc, the
 // candidate test and ordered store, the histogram, and the residual write-back. gv/rv hold the
-// chunk (entries outside the piece, as marked by `valid`, are ignored).
-template <int C>
+// chunk (entries outside the piece, as marked by `valid`, are ignored). Ring mode (full chunks
+// only): the chunk is in shared memory instead, g in `gs_`, r in `st`; pending writes go straight
+// into st and gv/rv are read from there.
+template <int C, bool kRing = false>
 __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t base, uint32_t lo,
                                             uint32_t hi, bool full, uint32_t valid,
                                             float4 (&gv)[4], float4 (&rv)[4], P1State& S,
                                             uint32_t cend, const uint32_t (&tl)[C], float* st,
-                                            uint32_t* hsink, int hstride, int lane) {
+                                            uint32_t* hsink, int hstride, int lane,
+                                            const float* gs_ = nullptr) {
   float4* st4 = reinterpret_cast<float4*>(st);
   float* r = a.r;
-  if (S.cp < cend) {
+  if (kRing) {
+    // pending writes that fall in this chunk replace those residual entries in the slot
+    if (S.cp < cend) {
+      const uint32_t lim = base + (uint32_t)kGranule;
+      for (;;) {
+        const bool in = S.win_idx >= (int32_t)base && S.win_idx < (int32_t)lim;
+        const uint32_t mask = __ballot_sync(kFull, in);
+        if (!mask) break;
+        if (in) st[S.win_idx - (int32_t)base] = S.win_val;
+        S.cp += __popc(mask);
+        __syncwarp();
+        load_window(a, S.cp, cend, lane, S);
+        if (mask != kFull) break;
+      }
+    }
+    const float4* g4 = reinterpret_cast<const float4*>(gs_);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      gv[u] = g4[u * 32 + lane];
+      rv[u] = st4[u * 32 + lane];
+    }
+    __syncwarp();
+  } else if (S.cp < cend) {
     // pending residual writes that fall in this chunk replace those residual entries
     const uint32_t lim = base + (uint32_t)kGranule < hi ? base + (uint32_t)kGranule : hi;
     bool staged = false;
@@ -761,6 +786,177 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     if (base < hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
       pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, hsink, hstride, lane);
+    }
+    if (lane == 0) {
+      a.pcnt[q] = S.count;
+      a.pnch[q] = S.nch;
+    }
+  }
+  __syncthreads();
+  H.flush(a, 1, kBins1);
+}
+
+// ------------------------------------------------------------------------------------------
+// 3b. pass 1 through a shared-memory ring (top-k)
+//
+// The same pass, but the interior chunks of a piece reach shared memory by bulk asynchronous
+// copies: one lane issues 2 KB of g and 2 KB of r per chunk, completion is counted on a
+// per-slot mbarrier, and kStages - 1 chunks are in flight ahead of the one being processed. A
+// warp then keeps 8 KB of loads outstanding without holding them in registers. Every wait is
+// bounded (about a second of SM clock); a wait that gives up raises GSPARSE_DERR_TIMEOUT, stops
+// the call and lets the warp's remaining copies land before it exits.
+
+constexpr int kStages = 3;
+constexpr uint32_t kChunkBytes = (uint32_t)kGranule * 4u;
+constexpr long long kWaitCycles = 1ll << 31;
+
+struct __align__(128) RingSlot {
+  float g[kGranule];
+  float r[kGranule];
+};
+constexpr size_t kRingBytes = sizeof(RingSlot) * kStages * kWarps;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits until the barrier's phase with this parity has completed; false after kWaitCycles.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_mbarrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+template <int C>
+__global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
+  extern __shared__ __align__(128) unsigned char ring_mem[];
+  __shared__ CtaHist<C, kBins1> H;
+  __shared__ uint64_t bars[kWarps][kStages];
+  if (a.ctl[0]) return;
+  const int64_t q0 = (int64_t)blockIdx.x * kWarps;
+  H.init(a, q0);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0)
+    for (int k = 0; k < kStages; ++k) mbar_init(&bars[wid][k], 1);
+  fence_mbarrier_init();
+  __syncthreads();
+  const int64_t q = q0 + wid;
+  if (q < total_pieces(a)) {
+    const Piece P = piece_of(a, q);
+    uint32_t tl[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) tl[c] = a.tlo[(int64_t)P.s * C + c];
+    const bool sh_sink = P.s == H.primary;
+    uint32_t* hsink = sh_sink ? H.sh : hist_of(a, (int64_t)P.s * C, 1);
+    const int hstride = sh_sink ? kBins1 : kHist;
+    const uint32_t lo = (uint32_t)P.lo, hi = (uint32_t)P.hi;  // indices are below 2^31
+    RingSlot* ring = reinterpret_cast<RingSlot*>(ring_mem) + wid * kStages;
+    uint64_t* mb = bars[wid];
+    const uint32_t cend = pending_count(a);
+    P1State S;
+    S.count = 0;
+    S.cp = 0;
+    S.room = (uint32_t)a.cap;
+    S.nch = 0;
+    S.ch_lo = S.pv_lo = 0;
+    S.ch_base = S.pv_base = q * a.cap;
+    if (cend) S.cp = a.pstart[q];
+    load_window(a, S.cp, cend, lane, S);
+    uint32_t base = lo & ~3u;
+    float4 gv[4], rv[4];
+    if (base < lo || base + (uint32_t)kGranule > hi) {
+      const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
+      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r, hsink, hstride,
+                     lane);
+      base += (uint32_t)kGranule;
+    }
+    // interior chunks [base, base + nint * 512) through the ring (base is 16-byte aligned)
+    const uint32_t nint = base < hi ? (hi - base) / (uint32_t)kGranule : 0u;
+    auto issue = [&](uint32_t c) {
+      RingSlot& sl = ring[c % kStages];
+      uint64_t* bar = &mb[c % kStages];
+      const size_t off = (size_t)base + (size_t)c * kGranule;
+      mbar_arrive_expect_tx(bar, 2u * kChunkBytes);
+      bulk_load(sl.g, a.g + off, kChunkBytes, bar);
+      bulk_load(sl.r, a.r + off, kChunkBytes, bar);
+    };
+    if (lane == 0)
+      for (uint32_t c = 0; c + 1 < (uint32_t)kStages && c < nint; ++c) issue(c);
+    uint32_t parity = 0;   // bit k: the phase parity slot k waits for next
+    uint32_t issued = nint < (uint32_t)kStages - 1 ? nint : (uint32_t)kStages - 1;
+    bool failed = false;
+    for (uint32_t c = 0; c < nint; ++c) {
+      const uint32_t k = c % kStages;
+      if (issued < nint) {
+        // the slot of chunk c - 1 is free: order this warp's accesses to it before the copy
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) issue(issued);
+        ++issued;
+      }
+      if (!mbar_wait_bounded(&mb[k], (parity >> k) & 1u)) {
+        failed = true;
+        break;
+      }
+      parity ^= 1u << k;
+      pass1_chunk<C, true>(a, q, base + c * (uint32_t)kGranule, lo, hi, true, 0xFFFFu, gv, rv, S, cend,
+                           tl, ring[k].r, hsink, hstride, lane, ring[k].g);
+    }
+    if (failed) {
+      if (lane == 0) {
+        raise(a.d_status, GSPARSE_DERR_TIMEOUT);
+        a.ctl[0] = 1;
+      }
+      // let the copies still in flight land before the warp leaves (bounded as well)
+      for (uint32_t c = 0; c < issued; ++c) {
+        const uint32_t k = c % kStages;
+        if (c + kStages >= issued) mbar_wait_bounded(&mb[k], (parity >> k) & 1u);
+      }
+    } else {
+      base += nint * (uint32_t)kGranule;
+      if (base < hi) {
+        const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
+        pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r, hsink,
+                       hstride, lane);
+      }
     }
     if (lane == 0) {
       a.pcnt[q] = S.count;
@@ -1622,7 +1818,16 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   sample_kernel<C><<<sgrid, 256, 0, st>>>(a, 2, exhaustive);
   const bool timed = g_pass1_before && g_pass1_after;
   if (timed) cudaEventRecord(g_pass1_before, st);
-  if (piece_ctas) pass1_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
+  if (piece_ctas) {
+    if constexpr (C == 1) {
+      if (cudaFuncSetAttribute(pass1_ring_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kRingBytes) != cudaSuccess)
+        return GSPARSE_ERR_CUDA;
+      pass1_ring_kernel<1><<<piece_ctas, kThreads, kRingBytes, st>>>(a);
+    } else {
+      pass1_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
+    }
+  }
   if (timed) cudaEventRecord(g_pass1_after, st);
   check_kernel<<<(unsigned)(T * C), 256, 0, st>>>(a);
   if (piece_ctas) restore_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);

@@ -59,7 +59,9 @@ enum gsparse_device_error {
   GSPARSE_DERR_CAPACITY = 1,       /* an output array is too small for the result */
   GSPARSE_DERR_CORRUPT_STREAM = 2, /* Golomb stream inconsistent with its length or side table */
   GSPARSE_DERR_INDEX_RANGE = 4,    /* an index outside [0, n) or a list not strictly ascending */
-  GSPARSE_DERR_SEGMENTS = 8        /* segment offsets not ascending from 0 to n */
+  GSPARSE_DERR_SEGMENTS = 8,       /* segment offsets not ascending from 0 to n */
+  GSPARSE_DERR_TIMEOUT = 16        /* a bounded wait for an asynchronous copy gave up (about a
+                                      second); the call stopped and its outputs are not valid */
 };
 
 /* Flags for gsparse_residual_topk / gsparse_binarize. */
