@@ -53,13 +53,14 @@ def _L():
         _lib.orc_golomb_b_star.argtypes = [f64]
         _lib.orc_golomb_b_star.restype = i32
         _lib.orc_residual_topk.argtypes = [vp, vp, i64, vp, i32, i64, i64, vp, vp, vp, i64]
+        _lib.orc_residual_topk_momentum.argtypes = [vp, vp, f32, vp, i64, vp, i32, i64, i64, vp, vp, vp, i64]
         _lib.orc_quantize.argtypes = [vp, vp, i64, vp, i64, vp, vp, i32]
         _lib.orc_binarize.argtypes = [vp, vp, i64, vp, i32, i64, i64, vp, vp, vp, vp, i64]
         _lib.orc_golomb_encode.argtypes = [vp, i64, i64, i32, vp, i64, vp, i64, vp]
         _lib.orc_golomb_decode.argtypes = [vp, ctypes.c_uint64, i64, i64, i32, i64, vp]
         _lib.orc_scatter_accumulate.argtypes = [i32, vp, vp, vp, vp, i64, vp, vp, vp, vp, i64]
         _lib.orc_combine_local.argtypes = [vp, vp, vp, i64, f32, f32, i32, vp, vp, i64]
-        for name in ("orc_residual_topk", "orc_quantize", "orc_binarize", "orc_golomb_encode",
+        for name in ("orc_residual_topk", "orc_residual_topk_momentum", "orc_quantize", "orc_binarize", "orc_golomb_encode",
                      "orc_golomb_decode", "orc_scatter_accumulate", "orc_combine_local"):
             getattr(_lib, name).restype = ctypes.c_int
     return _lib
@@ -99,6 +100,24 @@ def residual_topk(g: np.ndarray, r: np.ndarray, keep=(1, 100), seg=None):
     off = np.empty(T + 1, np.int64)
     _check(_L().orc_residual_topk(_p(g), _p(r), n, _p(s), T, keep[0], keep[1], _p(idx), _p(val), _p(off), cap))
     return idx[:cap], val[:cap], off, r
+
+
+def residual_topk_momentum(g: np.ndarray, u: np.ndarray, m: float, r: np.ndarray, keep=(1, 100), seg=None):
+    """Momentum-corrected residual top-k with momentum masking.
+    Returns (idx, val, offsets, new residual, new momentum)."""
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    u = np.array(u, dtype=np.float32, copy=True)
+    r = np.array(r, dtype=np.float32, copy=True)
+    n = g.size
+    s = _segments(n, seg)
+    T = s.size - 1
+    cap = sum(k_for(int(s[t + 1] - s[t]), *keep) for t in range(T))
+    idx = np.empty(max(cap, 1), np.int32)
+    val = np.empty(max(cap, 1), np.float32)
+    off = np.empty(T + 1, np.int64)
+    _check(_L().orc_residual_topk_momentum(_p(g), _p(u), float(m), _p(r), n, _p(s), T, keep[0], keep[1], _p(idx),
+                                           _p(val), _p(off), cap))
+    return idx[:cap], val[:cap], off, r, u
 
 
 def quantize(idx: np.ndarray, val: np.ndarray, residual: Optional[np.ndarray] = None,

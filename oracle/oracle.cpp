@@ -169,6 +169,33 @@ int orc_residual_topk(const float* g, float* r, int64_t n, const int64_t* seg, i
   return kOk;
 }
 
+// Residual top-k with momentum correction and momentum masking ([SBC] §II "Momentum Correction,
+// Warm-up Training and Momentum Masking" and Appendix A: the momentum-corrected gradient is added
+// to the residual; the momentum of the entries that were sent is set to zero). READING of the
+// arithmetic, one fp32 operation at a time:
+//   v_i = fl(fl(m * u_i) + g_i)        the momentum-corrected gradient; u_i <- v_i
+//   acc_i = fl(r_i + v_i)              then the residual top-k above on acc
+//   for the sent i: r_i <- 0 and u_i <- 0 (masking); all other entries keep r_i = acc_i.
+// With m = 0 this is orc_residual_topk plus u <- g with the sent entries zeroed.
+int orc_residual_topk_momentum(const float* g, float* u, float m, float* r, int64_t n,
+                               const int64_t* seg, int32_t T, int64_t num, int64_t den,
+                               int32_t* out_idx, float* out_val, int64_t* out_off,
+                               int64_t capacity) {
+  if (n < 0 || n > INT32_MAX || !valid_segments(n, seg, T) || num < 0 || den <= 0 || num > den)
+    return kBadArg;
+  std::vector<float> v(n);
+  for (int64_t i = 0; i < n; ++i) {
+    const float mu = m * u[i];
+    v[i] = mu + g[i];
+  }
+  const int st = orc_residual_topk(v.data(), r, n, seg, T, num, den, out_idx, out_val, out_off,
+                                   capacity);
+  if (st != kOk) return st;
+  for (int64_t i = 0; i < n; ++i) u[i] = v[i];
+  for (int64_t j = 0; j < out_off[T]; ++j) u[out_idx[j]] = 0.0f;
+  return kOk;
+}
+
 // 2-bit quantisation of a kept list ([AH17] Abstract: sparsification "can be combined with
 // quantization"). READING of the rule: every positive kept value becomes m+ = mean of the positive
 // kept values, every negative one m- = mean of the negative kept values (a negative number), a

@@ -161,6 +161,65 @@ def test_topk_special_cases():
     assert idx.size == 0 and off.tolist() == [0, 0]
 
 
+# ------------------------------------------------------------------ momentum correction and masking
+# "Sparse Binary Compression", §II and Appendix A: the momentum-corrected gradient goes into the
+# residual, and the momentum of the sent entries is zeroed.
+
+def test_momentum_delay_only_closed_form():
+    # keep 0 (nothing sent), m = 1/2, g = 1, u = r = 0 at the start: after t steps
+    # u_t = 2 - 2^(1-t) and r_t = sum_{s<=t} u_s = 2t - 2 + 2^(1-t), all exact in fp32
+    n = 7
+    g = np.ones(n, np.float32)
+    u = np.zeros(n, np.float32)
+    r = np.zeros(n, np.float32)
+    for t in range(1, 13):
+        idx, _, off, r, u = oracle.residual_topk_momentum(g, u, 0.5, r, keep=(0, 1))
+        assert idx.size == 0 and off.tolist() == [0, 0]
+        assert np.all(u == np.float32(2.0 - 2.0 ** (1 - t)))
+        assert np.all(r == np.float32(2.0 * t - 2.0 + 2.0 ** (1 - t)))
+
+
+def test_momentum_send_all_masks_everything():
+    # keep 1 (everything sent every step): the residual and the momentum are zeroed each step, so
+    # the sent values are the raw gradient at every step whatever m is
+    n = 50
+    u = np.zeros(n, np.float32)
+    r = np.zeros(n, np.float32)
+    for t in range(4):
+        g = synth.gaussian(n, 70 + t)
+        idx, val, _, r, u = oracle.residual_topk_momentum(g, u, 0.9, r, keep=(1, 1))
+        assert idx.tolist() == list(range(n))
+        assert np.array_equal(val.view(np.uint32), g.view(np.uint32))
+        assert np.all(r.view(np.uint32) == 0) and np.all(u.view(np.uint32) == 0)
+
+
+def test_momentum_zero_reduces_to_plain_topk():
+    n = 1000
+    for step in range(3):
+        g = synth.gaussian(n, 80 + step)
+        r0 = synth.gaussian(n, 90 + step, sigma=1e-4)
+        u0 = synth.gaussian(n, 95 + step)
+        idx, val, off, rn, un = oracle.residual_topk_momentum(g, u0, 0.0, r0, keep=(1, 10))
+        pi, pv, po, pr = oracle.residual_topk(g, r0, keep=(1, 10))
+        assert np.array_equal(idx, pi) and np.array_equal(val.view(np.uint32), pv.view(np.uint32))
+        assert np.array_equal(off, po) and np.array_equal(rn.view(np.uint32), pr.view(np.uint32))
+        want_u = g.copy()
+        want_u[idx] = 0.0
+        assert np.array_equal(un.view(np.uint32), want_u.view(np.uint32))
+
+
+def test_momentum_small_exact_case():
+    # integer-valued inputs, m = 1/2: v = (u / 2) + g exactly; the two largest |r + v| are sent
+    g = np.array([1, -4, 2, 0, 3], np.float32)
+    u = np.array([4, 2, -6, 8, 0], np.float32)
+    r = np.array([0, 1, 0, -1, 0], np.float32)
+    # v = [3, -3, -1, 4, 3]; acc = [3, -2, -1, 3, 3]; k = 2 -> indices 0 and 3 (ties -> lower)
+    idx, val, _, rn, un = oracle.residual_topk_momentum(g, u, 0.5, r, keep=(2, 5))
+    assert idx.tolist() == [0, 3] and val.tolist() == [3.0, 3.0]
+    assert rn.tolist() == [0.0, -2.0, -1.0, 0.0, 3.0]
+    assert un.tolist() == [0.0, -3.0, -1.0, 0.0, 3.0]
+
+
 def test_topk_negative_zero_ties_positive_zero():
     g = np.array([-0.0, 0.0, -0.0, 1.0], np.float32)
     r = np.array([-0.0, -0.0, 0.0, 0.0], np.float32)
