@@ -170,6 +170,8 @@ def run_ours(args, rank, world, dist):
         g_host.append(t)
     g = [t.to(dev) for t in g_host]
     r = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)]
+    mom = args.momentum
+    u = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(W)] if mom is not None else None
     # sent lists alternate between two buffers: step t applies step t-1's quantisation error
     idx2 = [[torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(W)] for _ in range(2)]
     val2 = [[torch.empty(cap, dtype=torch.float32, device=dev) for _ in range(W)] for _ in range(2)]
@@ -216,7 +218,8 @@ def run_ours(args, rank, world, dist):
             if p1 is not None:
                 gs.set_pass1_events(p1[w][0], p1[w][1])
             gs.residual_topk(g[w], r[w], keep, out_idx=idx, out_val=val, out_offsets=off, workspace=ws_t[w],
-                             d_status=st, capacity=cap, pending=pend2[prev][w])
+                             d_status=st, capacity=cap, pending=pend2[prev][w],
+                             momentum=None if u is None else (u[w], mom))
             if p1 is not None:
                 gs.set_pass1_events(None, None)
             rec()
@@ -320,18 +323,20 @@ def run_ours(args, rank, world, dist):
     grad_bytes = world * W * 4 * n
     value = grad_bytes / (ms * 1e-3) / 1e9
     p1 = statistics.mean(pass1_ms)
-    p1_bytes = 12 * n
+    per_entry = 12 if mom is None else 20     # g, r read + r written (+ u read and written)
+    p1_bytes = per_entry * n
     achieved = p1_bytes / (p1 * 1e-3) / 1e9
     topk_ms = statistics.mean(stage_ms["residual_topk"])
-    topk_bytes = 12 * n + 8 * cap
+    topk_bytes = per_entry * n + 8 * cap
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(n, W, args.drop, b, {"parallelism": f"replicas x{world}"}),
+        "config": workload_config(n, W, args.drop, b, {"parallelism": f"replicas x{world}"}
+                                  if mom is None else {"parallelism": f"replicas x{world}", "momentum": mom}),
         "roofline": {"bound": "hbm", "kernel": "pass1_kernel (streaming pass of residual top-k)",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(n),
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(n) if mom is None else None,
                      "algorithmic_bytes_per_launch": p1_bytes, "launch_ms": round(p1, 4)},
         "residual_topk_call": {"ms": round(topk_ms, 4), "algorithmic_bytes": topk_bytes,
                                "gbs": round(topk_bytes / (topk_ms * 1e-3) / 1e9, 1),
@@ -560,11 +565,15 @@ def run_workload(args):
 # ---------------------------------------------------------------------------------------------
 # the CPU oracle (reference arm and cpu_baseline)
 
-def oracle_step(gs_list, rs, keep, b, n):
+def oracle_step(gs_list, rs, keep, b, n, us=None, mom=None):
     import oracle
     lists = []
-    for g, r in zip(gs_list, rs):
-        idx, val, off, r2 = oracle.residual_topk(g, r, keep)
+    for w, (g, r) in enumerate(zip(gs_list, rs)):
+        if us is None:
+            idx, val, off, r2 = oracle.residual_topk(g, r, keep)
+        else:
+            idx, val, off, r2, u2 = oracle.residual_topk_momentum(g, us[w], mom, r, keep)
+            us[w][:] = u2
         bits, means, val, r2 = oracle.quantize(idx, val, residual=r2, write_dequantized=True)
         words, nb, table = oracle.golomb_encode(idx, b, chunk=64)
         dec = oracle.golomb_decode(words, nb, idx.size, b, n_limit=n)
@@ -583,11 +592,12 @@ def cpu_baseline(args, n_s):
     b = oracle.golomb_b_star(1.0 - args.drop)
     gsl = [synth.laplace_outliers(w, n_s) for w in range(args.workers)]
     rs = [np.zeros(n_s, np.float32) for _ in range(args.workers)]
-    oracle_step(gsl, rs, keep, b, n_s)          # warm
+    us = None if args.momentum is None else [np.zeros(n_s, np.float32) for _ in range(args.workers)]
+    oracle_step(gsl, rs, keep, b, n_s, us, args.momentum)          # warm
     t = time.perf_counter()
     reps = 0
     while True:
-        oracle_step(gsl, rs, keep, b, n_s)
+        oracle_step(gsl, rs, keep, b, n_s, us, args.momentum)
         reps += 1
         if time.perf_counter() - t > 8.0 or reps >= 5:
             break
@@ -606,11 +616,12 @@ def run_reference(args):
     n_s = args.ref_n
     gsl = [synth.laplace_outliers(w, n_s) for w in range(args.workers)]
     rs = [np.zeros(n_s, np.float32) for _ in range(args.workers)]
+    us = None if args.momentum is None else [np.zeros(n_s, np.float32) for _ in range(args.workers)]
     for _ in range(args.warmup):
-        oracle_step(gsl, rs, keep, b, n_s)
+        oracle_step(gsl, rs, keep, b, n_s, us, args.momentum)
     t = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(gsl, rs, keep, b, n_s)
+        oracle_step(gsl, rs, keep, b, n_s, us, args.momentum)
     dt = (time.perf_counter() - t) / args.steps
     value = round(args.workers * 4 * n_s / dt / 1e9, 4)
     sample = (f"each step the full hot path on {n_s} entries per worker ({args.workers} workers) instead of "
@@ -640,6 +651,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
                     help="time one of the smaller workloads instead of the default flat 2^30 line")
     ap.add_argument("--no-oracle", action="store_true", help="with --workload: skip the oracle timing")
+    ap.add_argument("--momentum", type=float, default=None,
+                    help="momentum correction and masking in the residual top-k (e.g. 0.9); off by default")
     ap.add_argument("--no-graph", action="store_true", help="with --workload: skip the CUDA-graph replay leg")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

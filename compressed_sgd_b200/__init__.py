@@ -50,6 +50,9 @@ _SIGNATURES = {
     "gsparse_residual_topk_workspace_min": (_sz, [_i64, _i32]),
     "gsparse_residual_topk": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _i64,
                                              ctypes.POINTER(GsparsePending), _u32, _vp, _sz, _vp, _vp]),
+    "gsparse_residual_topk_momentum": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _vp, _i64, _vp, _i32, _i64, _i64,
+                                                      _vp, _vp, _vp, _i64, ctypes.POINTER(GsparsePending), _u32,
+                                                      _vp, _sz, _vp, _vp]),
     "gsparse_residual_topk_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp]),
     "gsparse_quantize_workspace_size": (_sz, [_i64]),
     "gsparse_quantize": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _sz, _vp,
@@ -156,10 +159,11 @@ def residual_topk(g: torch.Tensor, residual: torch.Tensor, keep=(1, 100), seg_of
                   out_idx: Optional[torch.Tensor] = None, out_val: Optional[torch.Tensor] = None,
                   out_offsets: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                   flags: int = 0, d_status: Optional[torch.Tensor] = None, capacity: Optional[int] = None,
-                  pending: Optional[GsparsePending] = None):
+                  pending: Optional[GsparsePending] = None, momentum: Optional[Tuple[torch.Tensor, float]] = None):
     """residual <- acc with the sent entries zeroed. Returns (idx, val, offsets) device tensors;
     idx/val hold `capacity` slots of which offsets[-1] are used. `pending` (make_pending) are
-    residual writes applied first."""
+    residual writes applied first. `momentum` = (u, m): momentum correction and masking
+    (v = m u + g replaces g, u <- v, sent entries of u zeroed)."""
     _dev(g, torch.float32, "g")
     _dev(residual, torch.float32, "residual")
     n = g.numel()
@@ -178,6 +182,15 @@ def residual_topk(g: torch.Tensor, residual: torch.Tensor, keep=(1, 100), seg_of
     if workspace is None:
         workspace = _workspace(residual_topk_workspace_size(n, T, keep), dev)
     pend = ctypes.byref(pending) if pending is not None else None
+    if momentum is not None:
+        u, m = momentum
+        _dev(u, torch.float32, "momentum buffer")
+        st = lib().gsparse_residual_topk_momentum(_ptr(g), _ptr(u), float(m), _ptr(residual), n, _ptr(seg_offsets), T,
+                                                  keep[0], keep[1], _ptr(out_idx), _ptr(out_val), _ptr(out_offsets),
+                                                  capacity, pend, flags, _ptr(workspace), workspace.numel(),
+                                                  _ptr(d_status), _stream(dev))
+        _check(st, "gsparse_residual_topk_momentum")
+        return out_idx, out_val, out_offsets
     st = lib().gsparse_residual_topk(_ptr(g), _ptr(residual), n, _ptr(seg_offsets), T, keep[0], keep[1],
                                      _ptr(out_idx), _ptr(out_val), _ptr(out_offsets), capacity, pend, flags,
                                      _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev))

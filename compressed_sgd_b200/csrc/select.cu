@@ -24,6 +24,8 @@
 // Ties: keys equal to T are taken in ascending index order, so the lowest indices win.
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "osum.cuh"
 
@@ -49,6 +51,8 @@ constexpr int kThreads = kWarps * 32;
 struct Sel {
   const float* g;
   float* r;
+  float* u;    // momentum (null: none): v = fl(fl(mom * u) + g) replaces g, u <- v, sent u <- 0
+  float mom;
   int64_t n;
   int32_t T, C;       // segments; classes: 1 = |x| (top-k), 2 = x > 0 and x < 0 (binarise)
   int32_t zero_mode;  // top-k: write +0 for candidates in pass 1
@@ -309,6 +313,16 @@ __device__ __forceinline__ uint32_t pending_count(const Sel& a) {
   return (uint32_t)c;
 }
 
+// The gradient term of entry i: g_i, or with momentum v_i = fl(fl(mom * u_i) + g_i).
+__device__ __forceinline__ float grad_at(const Sel& a, int64_t i) {
+  return a.u ? __fadd_rn(__fmul_rn(a.mom, a.u[i]), a.g[i]) : a.g[i];
+}
+
+__device__ __forceinline__ float4 momentum4(float m, float4 u, float4 g) {
+  return make_float4(__fadd_rn(__fmul_rn(m, u.x), g.x), __fadd_rn(__fmul_rn(m, u.y), g.y),
+                     __fadd_rn(__fmul_rn(m, u.z), g.z), __fadd_rn(__fmul_rn(m, u.w), g.w));
+}
+
 // First pending write at or after entry x: searched only among the writes of x's piece.
 __device__ __forceinline__ uint32_t pending_lower_bound(const Sel& a, int64_t x) {
   if (x <= 0) return 0;
@@ -413,7 +427,7 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
     const int64_t i = sample_pos(lo, ns, j);
     const uint32_t cb = runs ? run_b[(j - j0) >> 5] : pwb;
     const uint32_t ce = runs ? run_e[(j - j0) >> 5] : pwe;
-    const float x = __fadd_rn(a.g[i], residual_at(a, i, cb, ce));
+    const float x = __fadd_rn(grad_at(a, i), residual_at(a, i, cb, ce));
     const int c = class_of<C>(x);
     const uint32_t key = mag_key(x);
     if (level == 2 && sparse) {
@@ -578,7 +592,7 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
                                             float4 (&gv)[4], float4 (&rv)[4], P1State& S,
                                             uint32_t cend, const uint32_t (&tl)[C], float* st,
                                             uint32_t* hsink, int hstride, int lane,
-                                            const float* gs_ = nullptr) {
+                                            const float* gs_ = nullptr, const float* us_ = nullptr) {
   float4* st4 = reinterpret_cast<float4*>(st);
   float* r = a.r;
   if (kRing) {
@@ -601,6 +615,15 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
     for (int u = 0; u < 4; ++u) {
       gv[u] = g4[u * 32 + lane];
       rv[u] = st4[u * 32 + lane];
+    }
+    if (us_) {
+      // momentum correction: v = fl(fl(m u) + g) stands in for g and becomes the new momentum
+      const float4* u4 = reinterpret_cast<const float4*>(us_);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        gv[u] = momentum4(a.mom, u4[u * 32 + lane], gv[u]);
+        st_stream(a.u + base + u * 128 + lane * 4, gv[u]);
+      }
     }
     __syncwarp();
   } else if (S.cp < cend) {
@@ -814,7 +837,15 @@ struct __align__(128) RingSlot {
   float g[kGranule];
   float r[kGranule];
 };
+// with momentum a slot also holds the chunk of u, and the ring is one stage shorter (same bytes)
+struct __align__(128) RingSlotM {
+  float g[kGranule];
+  float r[kGranule];
+  float u[kGranule];
+};
+constexpr int kStagesM = 2;
 constexpr size_t kRingBytes = sizeof(RingSlot) * kStages * kWarps;
+constexpr size_t kRingBytesM = sizeof(RingSlotM) * kStagesM * kWarps;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -865,17 +896,37 @@ __device__ __forceinline__ void fence_mbarrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-template <int C>
+// Momentum correction of an edge chunk held in registers: gv <- v, and u <- v for the entries
+// inside the piece.
+__device__ __forceinline__ void momentum_edge(const Sel& a, uint32_t base, uint32_t valid, int lane,
+                                              float4 (&gv)[4]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    float gx[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (!((valid >> (4 * u + e)) & 1u)) continue;
+      const uint32_t i = base + u * 128 + lane * 4 + e;
+      gx[e] = __fadd_rn(__fmul_rn(a.mom, a.u[i]), gx[e]);
+      a.u[i] = gx[e];
+    }
+    gv[u] = make_float4(gx[0], gx[1], gx[2], gx[3]);
+  }
+}
+
+template <int C, bool kMom>
 __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
+  using Slot = typename std::conditional<kMom, RingSlotM, RingSlot>::type;
+  constexpr int kSt = kMom ? kStagesM : kStages;
   extern __shared__ __align__(128) unsigned char ring_mem[];
   __shared__ CtaHist<C, kBins1> H;
-  __shared__ uint64_t bars[kWarps][kStages];
+  __shared__ uint64_t bars[kWarps][kSt];
   if (a.ctl[0]) return;
   const int64_t q0 = (int64_t)blockIdx.x * kWarps;
   H.init(a, q0);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   if (lane == 0)
-    for (int k = 0; k < kStages; ++k) mbar_init(&bars[wid][k], 1);
+    for (int k = 0; k < kSt; ++k) mbar_init(&bars[wid][k], 1);
   fence_mbarrier_init();
   __syncthreads();
   const int64_t q = q0 + wid;
@@ -888,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
     uint32_t* hsink = sh_sink ? H.sh : hist_of(a, (int64_t)P.s * C, 1);
     const int hstride = sh_sink ? kBins1 : kHist;
     const uint32_t lo = (uint32_t)P.lo, hi = (uint32_t)P.hi;  // indices are below 2^31
-    RingSlot* ring = reinterpret_cast<RingSlot*>(ring_mem) + wid * kStages;
+    Slot* ring = reinterpret_cast<Slot*>(ring_mem) + wid * kSt;
     uint64_t* mb = bars[wid];
     const uint32_t cend = pending_count(a);
     P1State S;
@@ -904,6 +955,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
     float4 gv[4], rv[4];
     if (base < lo || base + (uint32_t)kGranule > hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
+      if (kMom) momentum_edge(a, base, valid, lane, gv);
       pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r, hsink, hstride,
                      lane);
       base += (uint32_t)kGranule;
@@ -911,20 +963,21 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
     // interior chunks [base, base + nint * 512) through the ring (base is 16-byte aligned)
     const uint32_t nint = base < hi ? (hi - base) / (uint32_t)kGranule : 0u;
     auto issue = [&](uint32_t c) {
-      RingSlot& sl = ring[c % kStages];
-      uint64_t* bar = &mb[c % kStages];
+      Slot& sl = ring[c % kSt];
+      uint64_t* bar = &mb[c % kSt];
       const size_t off = (size_t)base + (size_t)c * kGranule;
-      mbar_arrive_expect_tx(bar, 2u * kChunkBytes);
+      mbar_arrive_expect_tx(bar, (kMom ? 3u : 2u) * kChunkBytes);
       bulk_load(sl.g, a.g + off, kChunkBytes, bar);
       bulk_load(sl.r, a.r + off, kChunkBytes, bar);
+      if constexpr (kMom) bulk_load(sl.u, a.u + off, kChunkBytes, bar);
     };
     if (lane == 0)
-      for (uint32_t c = 0; c + 1 < (uint32_t)kStages && c < nint; ++c) issue(c);
+      for (uint32_t c = 0; c + 1 < (uint32_t)kSt && c < nint; ++c) issue(c);
     uint32_t parity = 0;   // bit k: the phase parity slot k waits for next
-    uint32_t issued = nint < (uint32_t)kStages - 1 ? nint : (uint32_t)kStages - 1;
+    uint32_t issued = nint < (uint32_t)kSt - 1 ? nint : (uint32_t)kSt - 1;
     bool failed = false;
     for (uint32_t c = 0; c < nint; ++c) {
-      const uint32_t k = c % kStages;
+      const uint32_t k = c % kSt;
       if (issued < nint) {
         // the slot of chunk c - 1 is free: order this warp's accesses to it before the copy
         fence_proxy_async_smem();
@@ -937,8 +990,10 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
         break;
       }
       parity ^= 1u << k;
+      const float* us_ = nullptr;
+      if constexpr (kMom) us_ = ring[k].u;
       pass1_chunk<C, true>(a, q, base + c * (uint32_t)kGranule, lo, hi, true, 0xFFFFu, gv, rv, S, cend,
-                           tl, ring[k].r, hsink, hstride, lane, ring[k].g);
+                           tl, ring[k].r, hsink, hstride, lane, ring[k].g, us_);
     }
     if (failed) {
       if (lane == 0) {
@@ -947,13 +1002,14 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
       }
       // let the copies still in flight land before the warp leaves (bounded as well)
       for (uint32_t c = 0; c < issued; ++c) {
-        const uint32_t k = c % kStages;
-        if (c + kStages >= issued) mbar_wait_bounded(&mb[k], (parity >> k) & 1u);
+        const uint32_t k = c % kSt;
+        if (c + kSt >= issued) mbar_wait_bounded(&mb[k], (parity >> k) & 1u);
       }
     } else {
       base += nint * (uint32_t)kGranule;
       if (base < hi) {
         const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
+        if (kMom) momentum_edge(a, base, valid, lane, gv);
         pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r, hsink,
                        hstride, lane);
       }
@@ -1449,8 +1505,11 @@ __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_
             if ((sm >> e) & 1u) {
               const int64_t o = o0 + __popc(sm & ((1u << e) - 1u));
               if (o >= limit) raise(a.d_status, GSPARSE_DERR_CAPACITY);
-              else if (C == 1) { out_idx[o] = iv[e]; out_val[o] = xv[e]; }
-              else { a.lidx[o] = iv[e]; a.lval[o] = xv[e]; }
+              else if (C == 1) {
+                out_idx[o] = iv[e];
+                out_val[o] = xv[e];
+                if (a.u) a.u[iv[e]] = 0.0f;  // momentum masking of the sent entry
+              } else { a.lidx[o] = iv[e]; a.lval[o] = xv[e]; }
             }
           }
         }
@@ -1508,8 +1567,11 @@ __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_
         if ((sm >> e) & 1u) {
           const int64_t o = base_out[cc] + sel_run[cc] + pre_sel + __popc(sm & ((1u << e) - 1u));
           if (o >= limit) raise(a.d_status, GSPARSE_DERR_CAPACITY);
-          else if (C == 1) { out_idx[o] = (int32_t)(v + e); out_val[o] = x[e]; }
-          else { a.lidx[o] = (int32_t)(v + e); a.lval[o] = x[e]; }
+          else if (C == 1) {
+            out_idx[o] = (int32_t)(v + e);
+            out_val[o] = x[e];
+            if (a.u) a.u[v + e] = 0.0f;  // momentum masking of the sent entry
+          } else { a.lidx[o] = (int32_t)(v + e); a.lval[o] = x[e]; }
         }
       }
       eq_run[cc] += teq;
@@ -1600,19 +1662,33 @@ __global__ void bemit_kernel(Sel a, const float* d_mean, const int64_t* out_offs
 // accumulate only (keep 0): residual <- fl(g + residual)
 
 // ctl null: no plan ran (one segment), and the kernel itself reports the empty output offsets.
+// With momentum (u non-null) the gradient term is v = fl(fl(mom * u) + g), and u <- v.
 __global__ void accumulate_kernel(const float* g, float* r, int64_t n, const int32_t* ctl,
-                                  int64_t* out_offsets) {
+                                  int64_t* out_offsets, float* u, float mom) {
   if (ctl && ctl[0]) return;
   if (!ctl && out_offsets && blockIdx.x == 0 && threadIdx.x < 2) out_offsets[threadIdx.x] = 0;
   const int64_t nv = n >> 2;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nv; v += stride) {
-    const float4 a = ld_stream(g + 4 * v), b = ld_stream(r + 4 * v);
+    float4 a = ld_stream(g + 4 * v);
+    const float4 b = ld_stream(r + 4 * v);
+    if (u) {
+      a = momentum4(mom, ld_stream(u + 4 * v), a);
+      st_stream(u + 4 * v, a);
+    }
     st_stream(r + 4 * v, make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z),
                                      __fadd_rn(a.w, b.w)));
   }
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t < (n & 3)) r[4 * nv + t] = __fadd_rn(g[4 * nv + t], r[4 * nv + t]);
+  if (t < (n & 3)) {
+    const int64_t i = 4 * nv + t;
+    float gi = g[i];
+    if (u) {
+      gi = __fadd_rn(__fmul_rn(mom, u[i]), gi);
+      u[i] = gi;
+    }
+    r[i] = __fadd_rn(gi, r[i]);
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1769,7 +1845,8 @@ template <int C>
 int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t T, int64_t num,
                int64_t den, int32_t* out_idx, float* out_val, float* d_mean, int64_t* out_offsets,
                int64_t out_capacity, const gsparse_pending* pending, uint32_t flags, void* ws,
-               size_t ws_bytes, int32_t* d_status, cudaStream_t st) {
+               size_t ws_bytes, int32_t* d_status, cudaStream_t st, float* u = nullptr,
+               float mom = 0.0f) {
   if (pending && (!pending->d_count || pending->capacity < 0 ||
                   (pending->capacity > 0 && (!pending->idx || !pending->val))))
     return GSPARSE_ERR_INVALID_ARG;
@@ -1778,6 +1855,8 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
     return GSPARSE_ERR_INVALID_ARG;
   if (n > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
   if (n > 0 && (!g || !r || !aligned16(g) || !aligned16(r))) return GSPARSE_ERR_INVALID_ARG;
+  if (u && (C != 1 || !aligned16(u) || u == r || u == g)) return GSPARSE_ERR_INVALID_ARG;
+  if (n == 0) u = nullptr;
   if (out_capacity > 0 && !out_idx) return GSPARSE_ERR_INVALID_ARG;
   if (C == 1 && out_capacity > 0 && !out_val) return GSPARSE_ERR_INVALID_ARG;
   if (C == 2 && !d_mean) return GSPARSE_ERR_INVALID_ARG;
@@ -1787,13 +1866,16 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   Sel a = L.a;
   a.g = g;
   a.r = r;
+  a.u = u;
+  a.mom = mom;
   a.zero_mode = C == 1;
   a.d_status = d_status;
   const bool has_pending = pending && pending->capacity > 0;
   if (num == 0 && C == 1 && !has_pending && seg == nullptr) {
     // communication delay step on one segment: accumulate only, nothing to plan
     const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
-    accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, nullptr, out_offsets);
+    accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, nullptr, out_offsets,
+                                                                          u, mom);
     return launch_status();
   }
   a.pw_idx = has_pending ? pending->idx : nullptr;
@@ -1807,7 +1889,8 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   if (num == 0 && C == 1 && !has_pending) {  // communication delay step: accumulate only
     if (n > 0) {
       const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
-      accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, a.ctl, nullptr);
+      accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, a.ctl, nullptr, u,
+                                                                            mom);
     }
     return launch_status();
   }
@@ -1820,10 +1903,17 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   if (timed) cudaEventRecord(g_pass1_before, st);
   if (piece_ctas) {
     if constexpr (C == 1) {
-      if (cudaFuncSetAttribute(pass1_ring_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kRingBytes) != cudaSuccess)
-        return GSPARSE_ERR_CUDA;
-      pass1_ring_kernel<1><<<piece_ctas, kThreads, kRingBytes, st>>>(a);
+      if (a.u) {
+        if (cudaFuncSetAttribute(pass1_ring_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kRingBytesM) != cudaSuccess)
+          return GSPARSE_ERR_CUDA;
+        pass1_ring_kernel<1, true><<<piece_ctas, kThreads, kRingBytesM, st>>>(a);
+      } else {
+        if (cudaFuncSetAttribute(pass1_ring_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kRingBytes) != cudaSuccess)
+          return GSPARSE_ERR_CUDA;
+        pass1_ring_kernel<1, false><<<piece_ctas, kThreads, kRingBytes, st>>>(a);
+      }
     } else {
       pass1_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
     }
@@ -1895,6 +1985,19 @@ size_t gsparse_residual_topk_workspace_size(int64_t n, int32_t T, int64_t num, i
 size_t gsparse_residual_topk_workspace_min(int64_t n, int32_t T) {
   if (n < 0 || T < 1) return 0;
   return carve(n, T, 1, 1, 1, nullptr, 0, false).fixed_bytes;
+}
+
+int gsparse_residual_topk_momentum(const float* g, float* momentum_buf, float momentum,
+                                   float* residual, int64_t n, const int64_t* seg_offsets,
+                                   int32_t num_segments, int64_t keep_num, int64_t keep_den,
+                                   int32_t* out_idx, float* out_val, int64_t* out_offsets,
+                                   int64_t out_capacity, const gsparse_pending* pending,
+                                   uint32_t flags, void* workspace, size_t workspace_bytes,
+                                   int32_t* d_status, gsparse_stream stream) {
+  if (n > 0 && !momentum_buf) return GSPARSE_ERR_INVALID_ARG;
+  return run_select<1>(g, residual, n, seg_offsets, num_segments, keep_num, keep_den, out_idx,
+                       out_val, nullptr, out_offsets, out_capacity, pending, flags, workspace,
+                       workspace_bytes, d_status, (cudaStream_t)stream, momentum_buf, momentum);
 }
 
 int gsparse_residual_topk(const float* g, float* residual, int64_t n, const int64_t* seg_offsets,

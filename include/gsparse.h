@@ -143,6 +143,28 @@ int gsparse_residual_topk(const float* g, float* residual, int64_t n, const int6
                           const gsparse_pending* pending, uint32_t flags, void* workspace,
                           size_t workspace_bytes, int32_t* d_status, gsparse_stream stream);
 
+/* Residual top-k with momentum correction and momentum masking ("Sparse Binary Compression",
+ * §II "Momentum Correction, Warm-up Training and Momentum Masking" and Appendix A: the
+ * momentum-corrected gradient is added to the residual, and the momentum of the entries that
+ * were sent is set to zero):
+ *
+ *   v_i = fl(fl(momentum * u_i) + g_i);   u_i <- v_i
+ *   then gsparse_residual_topk on v in place of g (acc_i = fl(v_i + residual_i));
+ *   u_i <- +0.0f for every sent entry.
+ *
+ * momentum_buf   u, fp32[n], 16-byte aligned, read and overwritten in place; must not alias g or
+ *                residual. keep_num == 0 only accumulates (u <- v, residual <- fl(v + residual)).
+ * All other arguments, the workspace (same size queries) and the errors are those of
+ * gsparse_residual_topk. One streaming pass moves 20 bytes per entry (g, u, r read; u, r written).
+ */
+int gsparse_residual_topk_momentum(const float* g, float* momentum_buf, float momentum,
+                                   float* residual, int64_t n, const int64_t* seg_offsets,
+                                   int32_t num_segments, int64_t keep_num, int64_t keep_den,
+                                   int32_t* out_idx, float* out_val, int64_t* out_offsets,
+                                   int64_t out_capacity, const gsparse_pending* pending,
+                                   uint32_t flags, void* workspace, size_t workspace_bytes,
+                                   int32_t* d_status, gsparse_stream stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Residual top-k without caller-provided scratch  (no counterpart in the pages: this entry point
  * exists for callers, not for the method)

@@ -158,6 +158,103 @@ def test_topk_multi_step_residual_carried():
         assert np.array_equal(bits(host(rd)), bits(r_o))
 
 
+# --------------------------------------------------------- momentum correction and momentum masking
+
+def gpu_topk_momentum(g, u, m, r, keep, seg=None, flags=0, workspace_bytes=None):
+    gd, ud, rd = dev(g), dev(u), dev(r)
+    segd = None if seg is None else dev(np.asarray(seg, np.int64))
+    st = gs.status_tensor()
+    ws = None
+    if workspace_bytes is not None:
+        ws = torch.empty(max(workspace_bytes, 256), dtype=torch.uint8, device="cuda")
+    idx, val, off = gs.residual_topk(gd, rd, keep, seg_offsets=segd, flags=flags, workspace=ws, d_status=st,
+                                     momentum=(ud, m))
+    offh = host(off)
+    K = int(offh[-1])
+    return host(idx)[:K], host(val)[:K], offh, host(rd), host(ud), int(host(st)[0])
+
+
+def assert_momentum_equal(got, want):
+    gi, gv, go, gr, gu, st = got
+    wi, wv, wo, wr, wu = want
+    assert st == 0
+    assert np.array_equal(go, wo)
+    assert np.array_equal(gi, wi)
+    assert np.array_equal(bits(gv), bits(wv))
+    assert np.array_equal(bits(gr), bits(wr))
+    assert np.array_equal(bits(gu), bits(wu))
+
+
+@pytest.mark.parametrize("n", [1, 1000, 300001, (1 << 21) + 3])
+def test_topk_momentum_multi_step(n):
+    for m, keep in [(0.9, (1, 100)), (0.5, (1, 10)), (0.0, (1, 100)), (0.9, (1, 1)), (0.9, (0, 1))]:
+        u = np.zeros(n, np.float32)
+        r = np.zeros(n, np.float32)
+        for step in range(3):
+            g = synth.flat_mixture(n, seed=10 + step)
+            want = oracle.residual_topk_momentum(g, u, m, r, keep)
+            got = gpu_topk_momentum(g, u, m, r, keep)
+            assert_momentum_equal(got, want)
+            r, u = want[3], want[4]
+
+
+@pytest.mark.parametrize("route", ["default", "exhaustive", "min_workspace", "clustered"])
+def test_topk_momentum_segments_and_routes(route):
+    n = (1 << 20) + 77
+    g = clustered_rows(n, 21) if route == "clustered" else synth.flat_mixture(n, seed=21)
+    u = synth.gaussian(n, 22, sigma=1e-3)
+    r = synth.gaussian(n, 23, sigma=1e-4)
+    seg = np.array([0, 5000, 600000, n], np.int64)
+    for keep, s in [((1, 100), None), ((1, 50), seg)]:
+        T = 1 if s is None else len(s) - 1
+        kw = {}
+        if route == "exhaustive":
+            kw["flags"] = gs.GSPARSE_SELECT_EXHAUSTIVE
+        elif route == "min_workspace":
+            kw["workspace_bytes"] = int(gs.lib().gsparse_residual_topk_workspace_min(n, T))
+        assert_momentum_equal(gpu_topk_momentum(g, u, 0.9, r, keep, seg=s, **kw),
+                              oracle.residual_topk_momentum(g, u, 0.9, r, keep, seg=s))
+
+
+def test_topk_momentum_with_pending_writes():
+    # the quantisation error of the previous step arrives as pending writes to the residual
+    n = 500003
+    keep = (1, 100)
+    u = np.zeros(n, np.float32)
+    r = np.zeros(n, np.float32)
+    ud, rd = dev(u), dev(r)
+    st = gs.status_tensor()
+    pend = None
+    keep_alive = []
+    for step in range(3):
+        g = synth.flat_mixture(n, seed=40 + step)
+        idx, val, off, r_o, u_o = oracle.residual_topk_momentum(g, u, 0.9, r, keep)
+        _, _, qv, r_o = oracle.quantize(idx, val, residual=r_o, write_dequantized=True)
+        gi, gv, go = gs.residual_topk(dev(g), rd, keep, d_status=st, pending=pend, momentum=(ud, 0.9))
+        K = int(host(go)[-1])
+        fb = torch.empty(max(K, 1), device="cuda")
+        gs.quantize(gi, gv, go[1:2], write_dequantized=True, feedback_out=fb, d_status=st, capacity=gi.numel())
+        pend = gs.make_pending(gi, fb, go[1:2], capacity=gi.numel())
+        keep_alive.append((gi, gv, go, fb))
+        assert int(host(st)[0]) == 0
+        assert np.array_equal(host(gi)[:K], idx) and np.array_equal(bits(host(gv)[:K]), bits(qv))
+        assert np.array_equal(bits(host(ud)), bits(u_o))
+        u, r = u_o, r_o
+    # the last feedback is still pending: applying it must give the oracle's residual
+    gs.residual_topk(torch.zeros(n, device="cuda"), rd, (0, 1), d_status=st, pending=pend)
+    assert np.array_equal(bits(host(rd)), bits(r))
+
+
+def test_topk_momentum_argument_errors():
+    n = 1024
+    g = torch.zeros(n, device="cuda")
+    r = torch.zeros(n, device="cuda")
+    with pytest.raises(RuntimeError):
+        gs.residual_topk(g, r, (1, 100), momentum=(r, 0.9))   # u aliases the residual
+    with pytest.raises(RuntimeError):
+        gs.residual_topk(g, r, (1, 100), momentum=(torch.zeros(n + 1, device="cuda")[1:], 0.9))  # misaligned
+
+
 def test_topk_bad_segments_and_capacity_flagged():
     n = 1000
     g = synth.gaussian(n, 1)
