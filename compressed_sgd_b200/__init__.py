@@ -46,6 +46,7 @@ _SIGNATURES = {
     "gsparse_set_pass1_events": (None, [_vp, _vp]),
     "gsparse_k_for": (_i64, [_i64, _i64, _i64]),
     "gsparse_golomb_b_star": (_i32, [_f64]),
+    "gsparse_warmup_keep_num": (_i64, [_i64, _i64, _f64, _f64, _i64]),
     "gsparse_residual_topk_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_residual_topk_workspace_min": (_sz, [_i64, _i32]),
     "gsparse_residual_topk": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _i64,
@@ -127,6 +128,11 @@ def k_for(n_s: int, keep: Tuple[int, int]) -> int:
 
 def golomb_b_star(p: float) -> int:
     return int(lib().gsparse_golomb_b_star(p))
+
+
+def warmup_keep(t: int, T: int, start: float = 0.25, end: float = 0.001, den: int = 1_000_000) -> Tuple[int, int]:
+    """Keep fraction (num, den) at step t of a warm-up of T steps (exponential from start to end)."""
+    return int(lib().gsparse_warmup_keep_num(t, T, start, end, den)), den
 
 
 def set_pass1_events(before: Optional[torch.cuda.Event], after: Optional[torch.cuda.Event]):

@@ -46,4 +46,14 @@ int32_t gsparse_golomb_b_star(double p) {
   return 1 + (int32_t)floor(log2(log(phi - 1.0) / log(1.0 - p)));
 }
 
+int64_t gsparse_warmup_keep_num(int64_t t, int64_t T, double start, double end, int64_t den) {
+  if (den <= 0 || t < 0 || T < 0 || !(start > 0.0) || !(start <= 1.0) || !(end > 0.0) || !(end <= 1.0))
+    return -1;
+  const double f = (T == 0 || t >= T) ? end : start * pow(end / start, (double)t / (double)T);
+  int64_t num = llround(f * (double)den);
+  if (num < 1) num = 1;
+  if (num > den) num = den;
+  return num;
+}
+
 }  // extern "C"

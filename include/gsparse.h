@@ -95,6 +95,14 @@ int64_t gsparse_k_for(int64_t n_s, int64_t keep_num, int64_t keep_den);
  * al., §II Optimal Position Encoding, names Golomb coding of the distances). -1 if p not in (0,1). */
 int32_t gsparse_golomb_b_star(double p);
 
+/* Warm-up sparsity schedule ("Sparse Binary Compression", Appendix A: warm-up training raises the
+ * sparsity exponentially from 25% to 0.1% kept during the first epochs). READING: the keep
+ * fraction at step t of a warm-up of T steps is start * (end / start)^(t / T), and end from step T
+ * on. Returned as the numerator of keep = num / den (rounded to nearest, clamped to [1, den]), so
+ * the step's selection is gsparse_residual_topk with keep (num, den). -1 for bad arguments
+ * (den <= 0, fractions outside (0, 1], negative t or T). */
+int64_t gsparse_warmup_keep_num(int64_t t, int64_t T, double start, double end, int64_t den);
+
 /* ---------------------------------------------------------------------------------------------
  * Residual top-k  (Aji & Heafield 2017, Abstract; Sattler et al. §II Residual Accumulation and
  * Communication Delay)

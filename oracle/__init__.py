@@ -52,15 +52,19 @@ def _L():
         _lib.orc_k_for.restype = i64
         _lib.orc_golomb_b_star.argtypes = [f64]
         _lib.orc_golomb_b_star.restype = i32
+        _lib.orc_warmup_keep_num.argtypes = [i64, i64, f64, f64, i64]
+        _lib.orc_warmup_keep_num.restype = i64
         _lib.orc_residual_topk.argtypes = [vp, vp, i64, vp, i32, i64, i64, vp, vp, vp, i64]
         _lib.orc_residual_topk_momentum.argtypes = [vp, vp, f32, vp, i64, vp, i32, i64, i64, vp, vp, vp, i64]
         _lib.orc_quantize.argtypes = [vp, vp, i64, vp, i64, vp, vp, i32]
         _lib.orc_binarize.argtypes = [vp, vp, i64, vp, i32, i64, i64, vp, vp, vp, vp, i64]
+        _lib.orc_binarize_magnitude.argtypes = [vp, vp, i64, vp, i32, i64, i64, vp, vp, vp, vp, i64]
         _lib.orc_golomb_encode.argtypes = [vp, i64, i64, i32, vp, i64, vp, i64, vp]
         _lib.orc_golomb_decode.argtypes = [vp, ctypes.c_uint64, i64, i64, i32, i64, vp]
         _lib.orc_scatter_accumulate.argtypes = [i32, vp, vp, vp, vp, i64, vp, vp, vp, vp, i64]
         _lib.orc_combine_local.argtypes = [vp, vp, vp, i64, f32, f32, i32, vp, vp, i64]
-        for name in ("orc_residual_topk", "orc_residual_topk_momentum", "orc_quantize", "orc_binarize", "orc_golomb_encode",
+        for name in ("orc_residual_topk", "orc_residual_topk_momentum", "orc_quantize", "orc_binarize",
+                     "orc_binarize_magnitude", "orc_golomb_encode",
                      "orc_golomb_decode", "orc_scatter_accumulate", "orc_combine_local"):
             getattr(_lib, name).restype = ctypes.c_int
     return _lib
@@ -85,6 +89,11 @@ def k_for(n_s: int, num: int, den: int) -> int:
 
 def golomb_b_star(p: float) -> int:
     return int(_L().orc_golomb_b_star(p))
+
+
+def warmup_keep(t: int, T: int, start: float = 0.25, end: float = 0.001, den: int = 1_000_000):
+    """Keep fraction (num, den) at step t of a warm-up of T steps."""
+    return int(_L().orc_warmup_keep_num(t, T, start, end, den)), den
 
 
 def residual_topk(g: np.ndarray, r: np.ndarray, keep=(1, 100), seg=None):
@@ -134,8 +143,9 @@ def quantize(idx: np.ndarray, val: np.ndarray, residual: Optional[np.ndarray] = 
     return bits[:(K + 31) // 32], means, val, res
 
 
-def binarize(g: np.ndarray, r: np.ndarray, keep=(1, 1000), seg=None):
-    """Returns (idx int32[K'], val float32[K'], mean float32[T], offsets int64[T+1], new residual)."""
+def binarize(g: np.ndarray, r: np.ndarray, keep=(1, 1000), seg=None, by_magnitude: bool = False):
+    """Returns (idx int32[K'], val float32[K'], mean float32[T], offsets int64[T+1], new residual).
+    by_magnitude: the magnitude-first reading (top-k by |acc|, then the sign with the larger mean)."""
     g = np.ascontiguousarray(g, dtype=np.float32)
     r = np.array(r, dtype=np.float32, copy=True)
     n = g.size
@@ -146,7 +156,8 @@ def binarize(g: np.ndarray, r: np.ndarray, keep=(1, 1000), seg=None):
     val = np.empty(max(cap, 1), np.float32)
     mean = np.empty(T, np.float32)
     off = np.empty(T + 1, np.int64)
-    _check(_L().orc_binarize(_p(g), _p(r), n, _p(s), T, keep[0], keep[1], _p(idx), _p(val), _p(mean), _p(off), cap))
+    fn = _L().orc_binarize_magnitude if by_magnitude else _L().orc_binarize
+    _check(fn(_p(g), _p(r), n, _p(s), T, keep[0], keep[1], _p(idx), _p(val), _p(mean), _p(off), cap))
     K = int(off[-1])
     return idx[:K], val[:K], mean, off, r
 

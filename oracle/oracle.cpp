@@ -130,6 +130,18 @@ int32_t orc_golomb_b_star(double p) {
   return 1 + (int32_t)std::floor(std::log2(std::log(phi - 1.0) / std::log(1.0 - p)));
 }
 
+// Warm-up schedule ([SBC] Appendix A: sparsity raised exponentially from 25% to 0.1% kept during
+// the first epochs). READING: keep(t) = start * (end/start)^(t/T) for t < T, end afterwards;
+// returned as a numerator over den, rounded to nearest and clamped to [1, den].
+int64_t orc_warmup_keep_num(int64_t t, int64_t T, double start, double end, int64_t den) {
+  if (den <= 0 || t < 0 || T < 0 || !(start > 0.0) || !(start <= 1.0) || !(end > 0.0) || !(end <= 1.0))
+    return -1;
+  double keep = end;
+  if (T > 0 && t < T) keep = start * std::exp(std::log(end / start) * (double)t / (double)T);
+  int64_t num = (int64_t)std::llround(keep * (double)den);
+  return std::min<int64_t>(std::max<int64_t>(num, 1), den);
+}
+
 // Residual top-k ([AH17] Abstract; [SBC] §II Residual Accumulation).
 //   acc_i = fl(g_i + r_i)                                   (fp32, round to nearest even)
 //   per segment s: send the k_s entries of largest |acc| (ties to the lower index), ascending;
@@ -277,6 +289,60 @@ int orc_binarize(const float* g, float* r, int64_t n, const int64_t* seg, int32_
         r[i] = acc[i] - m;
         ++o;
       }
+    }
+    out_off[s + 1] = o;
+  }
+  return kOk;
+}
+
+// Sparse binarisation, the magnitude-first reading ([SBC] §II Sparse Binarization: only the
+// largest-magnitude fraction p is retained, its nonzero values are represented by one mean, and
+// the sign with the larger absolute mean decides which values remain). READING, per segment:
+//   S = the k_s entries of largest |acc| (ties to the lower index), ascending;
+//   mu+ = mean of the positive members of S, mu- = mean of |acc| over its negative members, both
+//   with the fixed-order sum over the positions of S (blocks of 256 positions, members only);
+//   send the positive members with +mu+ if mu+ >= mu- (and any exist), else the negative members
+//   with -mu-; residual <- fl(acc - m) on the sent entries and acc everywhere else (the unsent
+//   members of S keep their value in the residual).
+int orc_binarize_magnitude(const float* g, float* r, int64_t n, const int64_t* seg, int32_t T,
+                           int64_t num, int64_t den, int32_t* out_idx, float* out_val, float* mean,
+                           int64_t* out_off, int64_t capacity) {
+  if (n < 0 || n > INT32_MAX || !valid_segments(n, seg, T) || num < 0 || den <= 0 || num > den)
+    return kBadArg;
+  std::vector<float> acc(n);
+  for (int64_t i = 0; i < n; ++i) acc[i] = g[i] + r[i];
+  for (int64_t i = 0; i < n; ++i) r[i] = acc[i];
+  int64_t o = 0;
+  out_off[0] = 0;
+  for (int32_t s = 0; s < T; ++s) {
+    std::vector<uint64_t> packed(seg[s + 1] - seg[s]);
+    for (int64_t i = seg[s]; i < seg[s + 1]; ++i) packed[i - seg[s]] = pack(mag_key(acc[i]), i);
+    const std::vector<int64_t> S = top_k_packed(packed, kept_count(seg[s + 1] - seg[s], num, den));
+    std::vector<double> vp(S.size()), vn(S.size());
+    std::vector<char> isp(S.size()), isn(S.size());
+    for (size_t j = 0; j < S.size(); ++j) {
+      const float x = acc[S[j]];
+      vp[j] = (double)x;
+      vn[j] = -(double)x;
+      isp[j] = x > 0.0f;
+      isn[j] = x < 0.0f;
+    }
+    const int64_t np = std::count(isp.begin(), isp.end(), 1);
+    const int64_t nn = std::count(isn.begin(), isn.end(), 1);
+    const float mu_pos = ordered_mean(vp, isp);
+    const float mu_neg = ordered_mean(vn, isn);
+    const bool take_pos = np > 0 && mu_pos >= mu_neg;
+    const bool take_neg = !take_pos && nn > 0;
+    const float m = take_pos ? mu_pos : (take_neg ? -mu_neg : 0.0f);
+    mean[s] = m;
+    for (size_t j = 0; j < S.size(); ++j) {
+      if (!((take_pos && isp[j]) || (take_neg && isn[j]))) continue;
+      if (o >= capacity) return kCapacity;
+      const int64_t i = S[j];
+      out_idx[o] = (int32_t)i;
+      if (out_val) out_val[o] = m;
+      r[i] = acc[i] - m;
+      ++o;
     }
     out_off[s + 1] = o;
   }

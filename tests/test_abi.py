@@ -49,6 +49,10 @@ def test_host_helpers_match_oracle(gs):
     for p in [0.1, 0.01, 0.001, 0.5, 1e-6]:
         assert gs.golomb_b_star(p) == oracle.golomb_b_star(p)
     assert gs.k_for(10, (2, 1)) == -1 and gs.golomb_b_star(1.0) == -1
+    for T in [0, 1, 4, 10]:
+        for t in range(T + 2):
+            for start, end in [(0.25, 0.001), (0.5, 0.01), (1.0, 1.0)]:
+                assert gs.warmup_keep(t, T, start, end) == oracle.warmup_keep(t, T, start, end)
 
 
 def test_workspace_queries(gs):

@@ -255,6 +255,19 @@ def test_topk_momentum_argument_errors():
         gs.residual_topk(g, r, (1, 100), momentum=(torch.zeros(n + 1, device="cuda")[1:], 0.9))  # misaligned
 
 
+def test_topk_warmup_schedule_carried_residual():
+    # keep fractions 25% -> 0.1% over the warm-up (large k first), residual carried
+    n = (1 << 21) + 11
+    r = np.zeros(n, np.float32)
+    for t in range(6):
+        keep = gs.warmup_keep(t, 4)
+        assert keep == oracle.warmup_keep(t, 4)
+        g = synth.flat_mixture(n, seed=60 + t)
+        want = oracle.residual_topk(g, r, keep)
+        assert_topk_equal(gpu_topk(g, r, keep), want)
+        r = want[3]
+
+
 def test_topk_bad_segments_and_capacity_flagged():
     n = 1000
     g = synth.gaussian(n, 1)

@@ -220,6 +220,83 @@ def test_momentum_small_exact_case():
     assert un.tolist() == [0.0, -3.0, -1.0, 0.0, 3.0]
 
 
+def test_warmup_schedule_endpoints_and_ratio():
+    # "Sparse Binary Compression", Appendix A: sparsity raised exponentially from 25% to 0.1% kept
+    T = 4
+    nums = [oracle.warmup_keep(t, T)[0] for t in range(T + 3)]
+    assert nums[0] == 250000 and all(x == 1000 for x in nums[T:])
+    # geometric: each step multiplies the keep fraction by (0.001 / 0.25)^(1/4) = 0.2515 (4 steps)
+    q = (0.001 / 0.25) ** 0.25
+    for t in range(1, T + 1):
+        assert abs(nums[t] - nums[t - 1] * q) <= 1.0
+    assert nums[1] in (62872, 62873) and nums[2] == 15811
+    assert oracle.warmup_keep(0, 0)[0] == 1000          # no warm-up: the final fraction at once
+    assert oracle.warmup_keep(3, 4, 0.5, 0.5)[0] == 500000
+    assert oracle.warmup_keep(1, 4, 0.0, 0.1)[0] == -1
+
+
+# ------------------------------------------- sparse binarisation, magnitude-first reading
+# "Sparse Binary Compression", §II Sparse Binarization: keep the largest-magnitude fraction, then
+# the sign with the larger absolute mean decides which values remain.
+
+def test_binarize_magnitude_hand_worked():
+    g = np.array([3, -5, 1, -4, 2, 0, -1], np.float32)
+    r = np.zeros(7, np.float32)
+    # k = 3: S = {0, 1, 3} (|3|, |-5|, |-4|); mu+ = 3, mu- = 4.5 -> the negatives, mean -4.5
+    idx, val, mean, off, rn = oracle.binarize(g, r, (3, 7), by_magnitude=True)
+    assert idx.tolist() == [1, 3] and val.tolist() == [-4.5, -4.5] and mean.tolist() == [-4.5]
+    assert off.tolist() == [0, 2] and rn.tolist() == [3.0, -0.5, 1.0, 0.5, 2.0, 0.0, -1.0]
+
+
+def test_binarize_magnitude_equal_means_take_positive():
+    # mu+ = mu- = 1.5 with everything kept: the positive set is sent (ties go to the positive sign)
+    g = np.array([2, -2, 1, -1], np.float32)
+    idx, val, mean, off, rn = oracle.binarize(g, np.zeros(4, np.float32), (1, 1), by_magnitude=True)
+    assert idx.tolist() == [0, 2] and mean.tolist() == [1.5] and rn.tolist() == [0.5, -2.0, -0.5, -1.0]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_binarize_magnitude_brute_force(seed):
+    # integer-valued inputs: every mean is an exact rational, rounded once to fp32
+    gen = np.random.default_rng(500 + seed)
+    n = int(gen.integers(1, 40))
+    g = gen.integers(-9, 10, n).astype(np.float32)
+    r = gen.integers(-3, 4, n).astype(np.float32)
+    keep = (int(gen.integers(0, 5)), 4)
+    acc = g + r
+    k = math.ceil(n * keep[0] / keep[1])
+    S = sorted(sorted(range(n), key=lambda i: (-abs(float(acc[i])), i))[:k])
+    P = [i for i in S if acc[i] > 0]
+    N = [i for i in S if acc[i] < 0]
+    mp = float(np.float32(Fraction(int(sum(acc[i] for i in P))) / len(P))) if P else 0.0
+    mn = float(np.float32(Fraction(int(-sum(acc[i] for i in N))) / len(N))) if N else 0.0
+    if P and mp >= mn:
+        sent, m = P, mp
+    elif N:
+        sent, m = N, -mn
+    else:
+        sent, m = [], 0.0
+    idx, val, mean, off, rn = oracle.binarize(g, r, keep, by_magnitude=True)
+    assert idx.tolist() == sent and mean.tolist() == [np.float32(m)]
+    assert all(v == np.float32(m) for v in val)
+    want_r = acc.copy()
+    for i in sent:
+        want_r[i] = acc[i] - np.float32(m)
+    assert np.array_equal(rn, want_r)
+
+
+def test_binarize_magnitude_keep_all_equals_sign_sets():
+    # k = n: S is everything, so both readings compare all positives against all negatives
+    n = 301
+    gen = np.random.default_rng(9)
+    g = gen.integers(-50, 51, n).astype(np.float32)
+    r = np.zeros(n, np.float32)
+    a = oracle.binarize(g, r, (1, 1), by_magnitude=True)
+    b = oracle.binarize(g, r, (1, 1))
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
 def test_topk_negative_zero_ties_positive_zero():
     g = np.array([-0.0, 0.0, -0.0, 1.0], np.float32)
     r = np.array([-0.0, -0.0, 0.0, 0.0], np.float32)
