@@ -20,6 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libgsparse.so")
 
 GSPARSE_SELECT_EXHAUSTIVE = 1
+GSPARSE_BINARIZE_BY_MAGNITUDE = 2
 DERR_CAPACITY, DERR_CORRUPT_STREAM, DERR_INDEX_RANGE, DERR_SEGMENTS = 1, 2, 4, 8
 MAX_WORKERS = 64
 
@@ -275,8 +276,11 @@ def binarize_workspace_size(n: int, num_segments: int = 1, keep=(1, 1000)) -> in
 
 def binarize(g: torch.Tensor, residual: torch.Tensor, keep=(1, 1000), seg_offsets: Optional[torch.Tensor] = None,
              out_idx=None, out_val=None, mean=None, out_offsets=None, workspace=None, flags: int = 0,
-             d_status=None, capacity: Optional[int] = None, want_values: bool = True):
-    """Returns (idx, val or None, mean[T], offsets[T+1])."""
+             d_status=None, capacity: Optional[int] = None, want_values: bool = True, by_magnitude: bool = False):
+    """Returns (idx, val or None, mean[T], offsets[T+1]). by_magnitude: the magnitude-first reading
+    (top fraction by |acc|, then the sign with the larger mean)."""
+    if by_magnitude:
+        flags |= GSPARSE_BINARIZE_BY_MAGNITUDE
     _dev(g, torch.float32, "g")
     _dev(residual, torch.float32, "residual")
     n = g.numel()

@@ -1659,6 +1659,150 @@ __global__ void bemit_kernel(Sel a, const float* d_mean, const int64_t* out_offs
 }
 
 // ------------------------------------------------------------------------------------------
+// binarise, magnitude-first reading: the top-k list S of each segment (residual top-k), then the
+// means of its positive and of its negative members (fixed-order sums over the positions of S),
+// the choice per segment, and an ordered compaction of the chosen members
+
+constexpr int kMagBlock = 1024;  // list positions per compaction block (4 per thread)
+
+__global__ void __launch_bounds__(1024) mjobs_kernel(const float* lval, const int64_t* loff, int32_t T,
+                                                     SumJob* jobs, const int32_t* abort_flag) {
+  __shared__ int64_t sh[33];
+  if (*abort_flag) return;
+  const int64_t P = (int64_t)T * 2;
+  int64_t carry = 0;
+  for (int64_t base = 0; base < P; base += blockDim.x) {
+    const int64_t p = base + threadIdx.x;
+    const int64_t s = p >> 1;
+    const int64_t len = p < P ? loff[s + 1] - loff[s] : 0;
+    int64_t tot;
+    const int64_t ex = block_exclusive_scan(cdiv(len, kSumBlock), sh, &tot);
+    if (p < P) {
+      SumJob J;
+      J.vals = lval + loff[s];
+      J.len = len;
+      J.mode = (p & 1) ? kSumNegative : kSumPositive;
+      J.pad = 0;
+      J.leaf_base = carry + ex;
+      J.count = 0;
+      J.sum = 0.0;
+      J.mean = 0.0f;
+      J.done_blocks = 0;
+      jobs[p] = J;
+    }
+    carry += tot;
+  }
+}
+
+// mu+ = mean of the positive members, mu- = -(mean of the negative members); the larger is sent
+// (ties to positive), with the signed mean.
+__global__ void __launch_bounds__(1024) mchoose_kernel(const SumJob* jobs, int32_t T, int32_t* bsel,
+                                                       float* d_mean, int64_t* out_offsets,
+                                                       const int32_t* abort_flag) {
+  __shared__ int64_t sh[33];
+  if (*abort_flag) return;
+  int64_t carry = 0;
+  for (int64_t base = 0; base < T; base += blockDim.x) {
+    const int64_t s = base + threadIdx.x;
+    int64_t cnt = 0;
+    if (s < T) {
+      const int64_t np = (int64_t)jobs[2 * s].count, nn = (int64_t)jobs[2 * s + 1].count;
+      const float mp = jobs[2 * s].mean, mn = -jobs[2 * s + 1].mean;
+      const bool pos = np > 0 && mp >= mn;
+      const bool neg = !pos && nn > 0;
+      bsel[s] = pos ? 0 : (neg ? 1 : -1);
+      d_mean[s] = pos ? mp : (neg ? -mn : 0.0f);
+      cnt = pos ? np : (neg ? nn : 0);
+    }
+    int64_t tot;
+    const int64_t ex = block_exclusive_scan(cnt, sh, &tot);
+    if (s < T) out_offsets[s] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) out_offsets[T] = carry;
+}
+
+__device__ __forceinline__ bool mag_chosen(const int32_t* bsel, const int64_t* loff, int32_t T,
+                                           const float* lval, int64_t j, int32_t* seg_out) {
+  const int32_t s = (int32_t)(upper_bound_i64(loff, T + 1, j) - 1);
+  *seg_out = s;
+  const int c = bsel[s];
+  return c == 0 ? lval[j] > 0.0f : (c == 1 ? lval[j] < 0.0f : false);
+}
+
+__global__ void __launch_bounds__(256) mcount_kernel(const int32_t* bsel, const int64_t* loff, int32_t T,
+                                                     const float* lval, int64_t* bcnt,
+                                                     const int32_t* abort_flag) {
+  __shared__ int64_t sh[33];
+  if (*abort_flag) return;
+  const int64_t K = loff[T];
+  const int64_t j0 = (int64_t)blockIdx.x * kMagBlock + 4 * threadIdx.x;
+  int64_t mine = 0;
+  for (int e = 0; e < 4; ++e) {
+    int32_t s;
+    if (j0 + e < K && mag_chosen(bsel, loff, T, lval, j0 + e, &s)) ++mine;
+  }
+  int64_t tot;
+  block_exclusive_scan(mine, sh, &tot);
+  if (threadIdx.x == 0) bcnt[blockIdx.x] = tot;
+}
+
+__global__ void __launch_bounds__(1024) mscan_kernel(int64_t* bcnt, int64_t nblk, const int32_t* abort_flag) {
+  __shared__ int64_t sh[33];
+  if (*abort_flag) return;
+  int64_t carry = 0;
+  for (int64_t base = 0; base < nblk; base += blockDim.x) {
+    const int64_t b = base + threadIdx.x;
+    const int64_t v = b < nblk ? bcnt[b] : 0;
+    int64_t tot;
+    const int64_t ex = block_exclusive_scan(v, sh, &tot);
+    if (b < nblk) bcnt[b] = carry + ex;
+    carry += tot;
+  }
+}
+
+// The chosen members of S leave in list order (their global rank among the chosen is their output
+// position, since the segments' outputs are consecutive); every member of S gets its residual:
+// fl(acc - m_s) when sent, acc otherwise (the top-k left +0 there).
+__global__ void __launch_bounds__(256) memit_kernel(const int32_t* bsel, const int64_t* loff, int32_t T,
+                                                    const int32_t* lidx, const float* lval,
+                                                    const int64_t* bcnt, const float* d_mean, float* r,
+                                                    int32_t* out_idx, float* out_val, int64_t out_capacity,
+                                                    int32_t* d_status, const int32_t* abort_flag) {
+  __shared__ int64_t sh[33];
+  if (*abort_flag) return;
+  const int64_t K = loff[T];
+  const int64_t j0 = (int64_t)blockIdx.x * kMagBlock + 4 * threadIdx.x;
+  bool ch[4];
+  int32_t sg[4];
+  int64_t mine = 0;
+  for (int e = 0; e < 4; ++e) {
+    ch[e] = j0 + e < K && mag_chosen(bsel, loff, T, lval, j0 + e, &sg[e]);
+    mine += ch[e];
+  }
+  int64_t tot;
+  int64_t o = bcnt[blockIdx.x] + block_exclusive_scan(mine, sh, &tot);
+  for (int e = 0; e < 4; ++e) {
+    const int64_t j = j0 + e;
+    if (j >= K) break;
+    const int32_t i = lidx[j];
+    if (ch[e]) {
+      const float m = d_mean[sg[e]];
+      if (o >= out_capacity) {
+        raise(d_status, GSPARSE_DERR_CAPACITY);
+      } else {
+        out_idx[o] = i;
+        if (out_val) out_val[o] = m;
+      }
+      r[i] = __fsub_rn(lval[j], m);
+      ++o;
+    } else {
+      r[i] = lval[j];
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
 // accumulate only (keep 0): residual <- fl(g + residual)
 
 // ctl null: no plan ran (one segment), and the kernel itself reports the empty output offsets.
@@ -1946,6 +2090,72 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   return launch_status();
 }
 
+// Magnitude-first binarisation: its own lists and sums at the front of the workspace, the
+// residual top-k's workspace behind them.
+struct MagLayout {
+  int32_t* lidx;
+  float* lval;
+  int64_t* loff;
+  SumJob* jobs;
+  double* leaves;
+  double* partials;
+  int32_t* bsel;
+  int64_t* bcnt;
+  int64_t kb, leaf_bound, per_job, nblk;
+  size_t bytes;
+};
+
+MagLayout mag_carve(int64_t n, int32_t T, int64_t num, int64_t den, void* ws) {
+  MagLayout M;
+  Carver cv(ws);
+  M.kb = k_bound(n, T, num, den);
+  M.lidx = cv.take<int32_t>(M.kb);
+  M.lval = cv.take<float>(M.kb);
+  M.loff = cv.take<int64_t>((int64_t)T + 1);
+  M.per_job = cdiv(M.kb, kSumBlock);
+  M.leaf_bound = 2 * (M.per_job + T);
+  M.jobs = cv.take<SumJob>(2 * (int64_t)T);
+  M.leaves = cv.take<double>(M.leaf_bound);
+  M.partials = cv.take<double>(2 * (int64_t)T * osum_partial_stride(M.per_job));
+  M.bsel = cv.take<int32_t>(T);
+  M.nblk = cdiv(M.kb > 0 ? M.kb : 1, kMagBlock);
+  M.bcnt = cv.take<int64_t>(M.nblk + 1);
+  M.bytes = (size_t)round_up((int64_t)cv.off, 256);
+  return M;
+}
+
+int run_binarize_magnitude(const float* g, float* r, int64_t n, const int64_t* seg, int32_t T,
+                           int64_t num, int64_t den, int32_t* out_idx, float* out_val, float* d_mean,
+                           int64_t* out_offsets, int64_t out_capacity, uint32_t flags, void* ws,
+                           size_t ws_bytes, int32_t* d_status, cudaStream_t st) {
+  if (n < 0 || T < 1 || bad_keep(num, den) || !d_mean || !out_offsets || out_capacity < 0)
+    return GSPARSE_ERR_INVALID_ARG;
+  if (n > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
+  if (out_capacity > 0 && !out_idx) return GSPARSE_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return GSPARSE_ERR_WORKSPACE;
+  const MagLayout M = mag_carve(n, T, num, den, ws);
+  if (ws_bytes < M.bytes) return GSPARSE_ERR_WORKSPACE;
+  void* tws = static_cast<char*>(ws) + M.bytes;
+  const size_t tws_bytes = ws_bytes - M.bytes;
+  // S: the residual top-k into the internal lists (the caller's capacity bounds sum k_s, as for
+  // the two-set reading)
+  const int rc = run_select<1>(g, r, n, seg, T, num, den, M.lidx, M.lval, nullptr, M.loff,
+                               out_capacity < M.kb ? out_capacity : M.kb, nullptr,
+                               flags & GSPARSE_SELECT_EXHAUSTIVE, tws, tws_bytes, d_status, st);
+  if (rc != GSPARSE_OK) return rc;
+  const int32_t* abort_flag = carve(n, T, 1, num, den, tws, tws_bytes, false).a.ctl;
+  mjobs_kernel<<<1, 1024, 0, st>>>(M.lval, M.loff, T, M.jobs, abort_flag);
+  osum_launch(M.jobs, 2 * T, M.leaves, M.leaf_bound, M.per_job, M.partials, abort_flag, st);
+  mchoose_kernel<<<1, 1024, 0, st>>>(M.jobs, T, M.bsel, d_mean, out_offsets, abort_flag);
+  if (M.kb > 0) {
+    mcount_kernel<<<(unsigned)M.nblk, 256, 0, st>>>(M.bsel, M.loff, T, M.lval, M.bcnt, abort_flag);
+    mscan_kernel<<<1, 1024, 0, st>>>(M.bcnt, M.nblk, abort_flag);
+    memit_kernel<<<(unsigned)M.nblk, 256, 0, st>>>(M.bsel, M.loff, T, M.lidx, M.lval, M.bcnt, d_mean, r,
+                                                   out_idx, out_val, out_capacity, d_status, abort_flag);
+  }
+  return launch_status();
+}
+
 // Scratch of gsparse_residual_topk_noalloc: one array per device, in the library's own memory.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GSPARSE_NOALLOC_SCRATCH_BYTES];
 
@@ -2012,12 +2222,18 @@ int gsparse_residual_topk(const float* g, float* residual, int64_t n, const int6
 
 size_t gsparse_binarize_workspace_size(int64_t n, int32_t T, int64_t num, int64_t den) {
   if (n < 0 || T < 1 || bad_keep(num, den)) return 0;
-  return carve(n, T, 2, num, den, nullptr, 0, true).total_bytes + 256;
+  const size_t two_sets = carve(n, T, 2, num, den, nullptr, 0, true).total_bytes + 256;
+  const size_t by_mag = mag_carve(n, T, num, den, nullptr).bytes +
+                        carve(n, T, 1, num, den, nullptr, 0, true).total_bytes + 256;
+  return two_sets > by_mag ? two_sets : by_mag;
 }
 
 size_t gsparse_binarize_workspace_min(int64_t n, int32_t T, int64_t num, int64_t den) {
   if (n < 0 || T < 1 || bad_keep(num, den)) return 0;
-  return carve(n, T, 2, num, den, nullptr, 0, false).fixed_bytes;
+  const size_t two_sets = carve(n, T, 2, num, den, nullptr, 0, false).fixed_bytes;
+  const size_t by_mag = mag_carve(n, T, num, den, nullptr).bytes +
+                        carve(n, T, 1, num, den, nullptr, 0, false).fixed_bytes;
+  return two_sets > by_mag ? two_sets : by_mag;
 }
 
 int gsparse_residual_topk_noalloc(const float* g, float* residual, int64_t n, int64_t keep_num,
@@ -2038,6 +2254,10 @@ int gsparse_binarize(const float* g, float* residual, int64_t n, const int64_t* 
                      float* out_val, float* d_mean, int64_t* out_offsets, int64_t out_capacity,
                      uint32_t flags, void* workspace, size_t workspace_bytes, int32_t* d_status,
                      gsparse_stream stream) {
+  if (flags & GSPARSE_BINARIZE_BY_MAGNITUDE)
+    return run_binarize_magnitude(g, residual, n, seg_offsets, num_segments, keep_num, keep_den,
+                                  out_idx, out_val, d_mean, out_offsets, out_capacity, flags, workspace,
+                                  workspace_bytes, d_status, (cudaStream_t)stream);
   return run_select<2>(g, residual, n, seg_offsets, num_segments, keep_num, keep_den, out_idx,
                        out_val, d_mean, out_offsets, out_capacity, nullptr, flags, workspace,
                        workspace_bytes, d_status, (cudaStream_t)stream);

@@ -69,7 +69,9 @@ enum gsparse_select_flags {
   GSPARSE_SELECT_DEFAULT = 0,
   /* Skip the sampled candidate threshold: every entry is a candidate and the exact threshold is
      found from the full data. Same result, more memory traffic. */
-  GSPARSE_SELECT_EXHAUSTIVE = 1
+  GSPARSE_SELECT_EXHAUSTIVE = 1,
+  /* gsparse_binarize only: the magnitude-first reading of sparse binarisation (see there). */
+  GSPARSE_BINARIZE_BY_MAGNITUDE = 2
 };
 
 const char* gsparse_status_string(int status);
@@ -244,6 +246,14 @@ int gsparse_quantize(const int32_t* idx, float* val, const int64_t* d_begin, con
  * d_mean    fp32[num_segments] device: m_s.
  * out_val   fp32[out_capacity] or NULL: m_s for every sent entry.
  * out_offsets  exclusive offsets of the compacted per-segment outputs (counts vary).
+ *
+ * flags & GSPARSE_BINARIZE_BY_MAGNITUDE: the magnitude-first reading of the same section (only
+ * the largest-magnitude fraction is retained, and the sign with the larger absolute mean decides
+ * which values remain): S = the k_s entries of largest |acc| (gsparse_residual_topk's selection);
+ * mu+ = mean of the positive members of S, mu- = mean of |acc| over its negative members (the
+ * fixed-order sums over the positions of S, as gsparse_quantize's means); the members of the
+ * larger-mean sign are sent with the signed mean (ties to positive); residual_i <- fl(acc_i - m_s)
+ * on them and acc_i everywhere else, the unsent members of S included. Same workspace queries.
  */
 size_t gsparse_binarize_workspace_size(int64_t n, int32_t num_segments, int64_t keep_num,
                                        int64_t keep_den);

@@ -37,14 +37,15 @@ def gpu_topk(g, r, keep, seg=None, flags=0, workspace_bytes=None, capacity=None)
     return host(idx)[:K], host(val)[:K], offh, host(rd), int(host(st)[0])
 
 
-def gpu_binarize(g, r, keep, seg=None, flags=0, workspace_bytes=None):
+def gpu_binarize(g, r, keep, seg=None, flags=0, workspace_bytes=None, by_magnitude=False):
     gd, rd = dev(g), dev(r)
     segd = None if seg is None else dev(np.asarray(seg, np.int64))
     st = gs.status_tensor()
     ws = None
     if workspace_bytes is not None:
         ws = torch.empty(max(workspace_bytes, 256), dtype=torch.uint8, device="cuda")
-    idx, val, mean, off = gs.binarize(gd, rd, keep, seg_offsets=segd, flags=flags, workspace=ws, d_status=st)
+    idx, val, mean, off = gs.binarize(gd, rd, keep, seg_offsets=segd, flags=flags, workspace=ws, d_status=st,
+                                      by_magnitude=by_magnitude)
     offh = host(off)
     K = int(offh[-1])
     return host(idx)[:K], host(val)[:K], host(mean), offh, host(rd), int(host(st)[0])

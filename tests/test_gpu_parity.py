@@ -362,6 +362,38 @@ def test_binarize_skewed_ties_segments_and_routes():
         assert_binarize_equal(gpu_binarize(g, r, keep, seg=seg, workspace_bytes=mn), want)
 
 
+@pytest.mark.parametrize("n", [1, 2, 1000, 300001, (1 << 21) + 9])
+def test_binarize_by_magnitude(n):
+    # the magnitude-first reading: top fraction by |acc|, then the sign with the larger mean
+    r = np.zeros(n, np.float32)
+    for step, keep in enumerate([(1, 1000), (1, 100), (1, 10), (1, 1)]):
+        g = synth.gaussian(n, 300 + step, sigma=1e-2) + np.float32(2e-3)   # a sign imbalance
+        want = oracle.binarize(g, r, keep, by_magnitude=True)
+        assert_binarize_equal(gpu_binarize(g, r, keep, by_magnitude=True), want)
+        r = want[4]
+
+
+@pytest.mark.parametrize("route", ["segments", "exhaustive", "min_workspace", "ties"])
+def test_binarize_by_magnitude_routes(route):
+    n = 400009
+    g = synth.gaussian(n, 310, sigma=1e-2)
+    r = synth.gaussian(n, 311, sigma=1e-3)
+    seg = None
+    kw = {}
+    if route == "segments":
+        seg = np.array([0, 17, 1000, 250000, 250000, n], np.int64)
+    elif route == "exhaustive":
+        kw["flags"] = gs.GSPARSE_SELECT_EXHAUSTIVE
+    elif route == "ties":
+        g = synth.tied_values(n, 312, levels=4) * np.float32(1e-2)
+        r = np.zeros(n, np.float32)
+    for keep in [(1, 100), (1, 7)]:
+        if route == "min_workspace":
+            kw["workspace_bytes"] = int(gs.lib().gsparse_binarize_workspace_min(n, 1, *keep))
+        assert_binarize_equal(gpu_binarize(g, r, keep, seg=seg, by_magnitude=True, **kw),
+                              oracle.binarize(g, r, keep, seg=seg, by_magnitude=True))
+
+
 def test_binarize_one_sign_only():
     n = 5000
     g = np.abs(synth.gaussian(n, 1))
