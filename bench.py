@@ -38,7 +38,7 @@ import numpy as np  # noqa: E402
 
 METRIC = "gradient GB/s compressed (top-1% residual select+compact)"
 UNIT = "GB/s"
-PROFILE = os.path.join(ROOT, "profiles", "pass1_ring_kernel_flat_fp32.md")
+PROFILE = os.path.join(ROOT, "profiles", "pass1_kernel_flat_fp32.md")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -334,7 +334,7 @@ def run_ours(args, rank, world, dist):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(n, W, args.drop, b, {"parallelism": f"replicas x{world}"}
                                   if mom is None else {"parallelism": f"replicas x{world}", "momentum": mom}),
-        "roofline": {"bound": "hbm", "kernel": "pass1_ring_kernel (streaming pass of residual top-k)",
+        "roofline": {"bound": "hbm", "kernel": ("pass1_kernel" if mom is None else "pass1_ring_kernel") + " (streaming pass of residual top-k)",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": profiled_traffic(n) if mom is None else None,
                      "algorithmic_bytes_per_launch": p1_bytes, "launch_ms": round(p1, 4)},
