@@ -68,3 +68,30 @@ def test_reference_arm_json_line():
     assert line["metric"] == bench.METRIC and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["cpu_baseline"]["cores"] == 1 and line["warmup"] >= 3
+
+
+def test_workload_oracle_small_workloads():
+    # the oracle leg of `bench.py --workload`: one step of the two small workloads end to end
+    import numpy as np
+    import oracle
+    import synth
+    n = 1 << 20
+    g = [synth.flat_mixture(n, seed=0)]
+    b = oracle.golomb_b_star(0.01)
+    dense, outs = bench.workload_oracle("flat2e20", g, n, None, (1, 100), b)
+    assert outs is None and np.count_nonzero(dense) == oracle.k_for(n, 1, 100)
+    seg = synth.offsets(synth.mlp_layout())
+    n = int(seg[-1])
+    g = [synth.mlp_gradient(w, 0) for w in range(4)]
+    dense, _ = bench.workload_oracle("mlp", g, n, seg, (1, 100), None)
+    kept = sum(oracle.k_for(int(seg[t + 1] - seg[t]), 1, 100) for t in range(len(seg) - 1))
+    assert kept <= np.count_nonzero(dense) <= 4 * kept
+
+
+def test_reference_arm_with_momentum():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "1", "--ref-n", "4096", "--momentum", "0.9"],
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
