@@ -78,7 +78,8 @@ const char* gsparse_status_string(int status);
 const char* gsparse_version(void);
 
 /* Measurement hook, off by default and not thread-safe: while both events are non-NULL, every
- * gsparse_residual_topk and gsparse_binarize call records `before` on its stream right before
+ * gsparse_residual_topk, gsparse_residual_topk_momentum and gsparse_binarize call records
+ * `before` on its stream right before
  * its streaming pass over g and the residual, and `after` right after it, so that pass can be
  * timed alone with cudaEventElapsedTime. Passing NULLs turns it off. */
 void gsparse_set_pass1_events(gsparse_event before, gsparse_event after);
