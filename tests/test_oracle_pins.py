@@ -396,6 +396,48 @@ def test_fixed_order_sum_keeps_a_later_block_whole():
     assert np.float32(seq / 512) == np.float32(1.0 + 2.0 ** -23)
 
 
+def test_fixed_order_sum_pairs_four_block_sums_as_a_tree():
+    # Four blocks of 256 positions. Members: 4 and 2^-22 in block 0 (block sum A = 4 + 2^-22, exact
+    # in fp64), none in block 1 (sum +0), 2^-51 in block 2, 2^-51 in block 3. In fp64 one ulp of A
+    # is 2^-50, so adding 2^-51 to A alone is an exact tie, which goes to A (its last mantissa bit
+    # is 0). Pairwise tree: (A + 0) + (2^-51 + 2^-51) = A + 2^-50 exactly; mean over 4 members
+    # 1 + 2^-24 + 2^-52, just above the fp32 midpoint of 1 and 1 + 2^-23, rounds up to 1 + 2^-23.
+    # Left to right: ((A + 0) + 2^-51) + 2^-51 = A; mean 1 + 2^-24 is the midpoint itself and ties
+    # to the even 1.0. So this case fails a block-sum combination that runs left to right.
+    val = np.zeros(4 * 256, np.float32)
+    val[0], val[1], val[512], val[768] = 4.0, 2.0 ** -22, 2.0 ** -51, 2.0 ** -51
+    _, means, _, _ = oracle.quantize(np.arange(val.size, dtype=np.int32), val)
+    assert means[0] == np.float32(1.0 + 2.0 ** -23)
+    assert means[0].view(np.uint32) == np.uint32(0x3F800001)
+    A = 4.0 + 2.0 ** -22
+    assert A + 2.0 ** -51 == A and A + 2.0 ** -50 == 4.0 + 2.0 ** -22 + 2.0 ** -50   # the fp64 facts used
+    blocks = [A, 0.0, 2.0 ** -51, 2.0 ** -51]
+    tree = (blocks[0] + blocks[1]) + (blocks[2] + blocks[3])
+    left_to_right = ((blocks[0] + blocks[1]) + blocks[2]) + blocks[3]
+    assert np.float32(tree / 4) == np.float32(1.0 + 2.0 ** -23)
+    assert np.float32(left_to_right / 4) == np.float32(1.0)
+
+
+def test_fixed_order_sum_lifts_an_odd_last_block_unchanged():
+    # Five blocks: 4 | 2^-22 | (none) | 2^-51 | 2^-51, one member each where present. Level 1 of the
+    # tree pairs (b0 + b1) = A = 4 + 2^-22 and (b2 + b3) = 2^-51; b4 moves up alone. Level 2:
+    # A + 2^-51 = A (an exact tie to even, as above); b4 moves up. Level 3: A + 2^-51 = A. Mean over
+    # 4 members 1 + 2^-24 ties to 1.0. Pairing from the right end instead (b0 alone, (b1 + b2),
+    # (b3 + b4) = 2^-50) gives A + 2^-50 and 1 + 2^-23, as does the exact sum; folding the odd
+    # block into the last pair, (b2 + b3 + b4), gives 2^-50 there and 1 + 2^-23 as well.
+    val = np.zeros(5 * 256, np.float32)
+    val[0], val[256], val[768], val[1024] = 4.0, 2.0 ** -22, 2.0 ** -51, 2.0 ** -51
+    _, means, _, _ = oracle.quantize(np.arange(val.size, dtype=np.int32), val)
+    assert means[0] == np.float32(1.0)
+    b = [4.0, 2.0 ** -22, 0.0, 2.0 ** -51, 2.0 ** -51]
+    from_right = (b[0] + (b[1] + b[2])) + (b[3] + b[4])
+    folded = (b[0] + b[1]) + ((b[2] + b[3]) + b[4])
+    assert np.float32(from_right / 4) == np.float32(1.0 + 2.0 ** -23)
+    assert np.float32(folded / 4) == np.float32(1.0 + 2.0 ** -23)
+    exact = sum(Fraction(x) for x in b) / 4
+    assert round_f32_exact(exact) == np.float32(1.0 + 2.0 ** -23)
+
+
 # ------------------------------------------------------------------------------------ binarise
 
 def brute_binarize(acc, k):
