@@ -215,13 +215,10 @@ def run_ours(args, rank, world, dist):
             idx, val, off, fb = idx2[cur][w], val2[cur][w], off2[cur][w], fb2[cur][w]
             end = off[1:2]
             rec()
-            if p1 is not None:
-                gs.set_pass1_events(p1[w][0], p1[w][1])
             gs.residual_topk(g[w], r[w], keep, out_idx=idx, out_val=val, out_offsets=off, workspace=ws_t[w],
                              d_status=st, capacity=cap, pending=pend2[prev][w],
-                             momentum=None if u is None else (u[w], mom))
-            if p1 is not None:
-                gs.set_pass1_events(None, None)
+                             momentum=None if u is None else (u[w], mom),
+                             pass_events=None if p1 is None else (p1[w][0], p1[w][1]))
             rec()
             gs.quantize(idx, val, end, write_dequantized=True, feedback_out=fb, sign_bits=sb[w], means=means[w],
                         workspace=ws_q[w], d_status=st, capacity=cap)

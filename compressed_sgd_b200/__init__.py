@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libgsparse.so")
 
 GSPARSE_SELECT_EXHAUSTIVE = 1
 GSPARSE_BINARIZE_BY_MAGNITUDE = 2
-DERR_CAPACITY, DERR_CORRUPT_STREAM, DERR_INDEX_RANGE, DERR_SEGMENTS = 1, 2, 4, 8
+GSPARSE_SELECT_TEST_EXPIRE_WAIT = 4
+DERR_CAPACITY, DERR_CORRUPT_STREAM, DERR_INDEX_RANGE, DERR_SEGMENTS, DERR_TIMEOUT = 1, 2, 4, 8, 16
 MAX_WORKERS = 64
 
 _i64, _i32, _u32, _vp, _f32, _f64, _sz = (ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_void_p,
@@ -40,21 +41,25 @@ class GsparseList(ctypes.Structure):
     _fields_ = [("idx", _vp), ("val", _vp), ("uniform_val", _vp), ("d_count", _vp), ("capacity", _i64)]
 
 
+class GsparsePassEvents(ctypes.Structure):
+    _fields_ = [("before", _vp), ("after", _vp)]
+
+
 # name -> (restype, argtypes)
 _SIGNATURES = {
     "gsparse_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gsparse_version": (ctypes.c_char_p, []),
-    "gsparse_set_pass1_events": (None, [_vp, _vp]),
     "gsparse_k_for": (_i64, [_i64, _i64, _i64]),
     "gsparse_golomb_b_star": (_i32, [_f64]),
     "gsparse_warmup_keep_num": (_i64, [_i64, _i64, _f64, _f64, _i64]),
     "gsparse_residual_topk_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_residual_topk_workspace_min": (_sz, [_i64, _i32]),
     "gsparse_residual_topk": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _i64,
-                                             ctypes.POINTER(GsparsePending), _u32, _vp, _sz, _vp, _vp]),
+                                             ctypes.POINTER(GsparsePending), _u32, _vp, _sz, _vp, _vp,
+                                             ctypes.POINTER(GsparsePassEvents)]),
     "gsparse_residual_topk_momentum": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _vp, _i64, _vp, _i32, _i64, _i64,
                                                       _vp, _vp, _vp, _i64, ctypes.POINTER(GsparsePending), _u32,
-                                                      _vp, _sz, _vp, _vp]),
+                                                      _vp, _sz, _vp, _vp, ctypes.POINTER(GsparsePassEvents)]),
     "gsparse_residual_topk_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp]),
     "gsparse_quantize_workspace_size": (_sz, [_i64]),
     "gsparse_quantize": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _sz, _vp,
@@ -62,7 +67,7 @@ _SIGNATURES = {
     "gsparse_binarize_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_binarize_workspace_min": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_binarize": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _u32,
-                                        _vp, _sz, _vp, _vp]),
+                                        _vp, _sz, _vp, _vp, ctypes.POINTER(GsparsePassEvents)]),
     "gsparse_golomb_encode_workspace_size": (_sz, [_i64]),
     "gsparse_golomb_encode": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i32, _vp, _i64, _vp, _vp, _i32, _vp,
                                              _sz, _vp, _vp]),
@@ -136,13 +141,12 @@ def warmup_keep(t: int, T: int, start: float = 0.25, end: float = 0.001, den: in
     return int(lib().gsparse_warmup_keep_num(t, T, start, end, den)), den
 
 
-def set_pass1_events(before: Optional[torch.cuda.Event], after: Optional[torch.cuda.Event]):
-    """Measurement hook: record these events around the streaming pass of every following
-    residual_topk / binarize call (None, None turns it off)."""
-    if before is None or after is None:
-        lib().gsparse_set_pass1_events(None, None)
-    else:
-        lib().gsparse_set_pass1_events(before.cuda_event, after.cuda_event)
+def _pass_events(events):
+    """(before, after) torch.cuda.Event pair -> a by-reference gsparse_pass_events, or None."""
+    if events is None:
+        return None
+    before, after = events
+    return ctypes.byref(GsparsePassEvents(before.cuda_event, after.cuda_event))
 
 
 def status_tensor(device="cuda") -> torch.Tensor:
@@ -166,11 +170,13 @@ def residual_topk(g: torch.Tensor, residual: torch.Tensor, keep=(1, 100), seg_of
                   out_idx: Optional[torch.Tensor] = None, out_val: Optional[torch.Tensor] = None,
                   out_offsets: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                   flags: int = 0, d_status: Optional[torch.Tensor] = None, capacity: Optional[int] = None,
-                  pending: Optional[GsparsePending] = None, momentum: Optional[Tuple[torch.Tensor, float]] = None):
+                  pending: Optional[GsparsePending] = None, momentum: Optional[Tuple[torch.Tensor, float]] = None,
+                  pass_events: Optional[Tuple[torch.cuda.Event, torch.cuda.Event]] = None):
     """residual <- acc with the sent entries zeroed. Returns (idx, val, offsets) device tensors;
     idx/val hold `capacity` slots of which offsets[-1] are used. `pending` (make_pending) are
     residual writes applied first. `momentum` = (u, m): momentum correction and masking
-    (v = m u + g replaces g, u <- v, sent entries of u zeroed)."""
+    (v = m u + g replaces g, u <- v, sent entries of u zeroed). `pass_events` = (before, after):
+    CUDA events this call records around its streaming pass."""
     _dev(g, torch.float32, "g")
     _dev(residual, torch.float32, "residual")
     n = g.numel()
@@ -195,12 +201,13 @@ def residual_topk(g: torch.Tensor, residual: torch.Tensor, keep=(1, 100), seg_of
         st = lib().gsparse_residual_topk_momentum(_ptr(g), _ptr(u), float(m), _ptr(residual), n, _ptr(seg_offsets), T,
                                                   keep[0], keep[1], _ptr(out_idx), _ptr(out_val), _ptr(out_offsets),
                                                   capacity, pend, flags, _ptr(workspace), workspace.numel(),
-                                                  _ptr(d_status), _stream(dev))
+                                                  _ptr(d_status), _stream(dev), _pass_events(pass_events))
         _check(st, "gsparse_residual_topk_momentum")
         return out_idx, out_val, out_offsets
     st = lib().gsparse_residual_topk(_ptr(g), _ptr(residual), n, _ptr(seg_offsets), T, keep[0], keep[1],
                                      _ptr(out_idx), _ptr(out_val), _ptr(out_offsets), capacity, pend, flags,
-                                     _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev))
+                                     _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev),
+                                     _pass_events(pass_events))
     _check(st, "gsparse_residual_topk")
     return out_idx, out_val, out_offsets
 
@@ -276,7 +283,8 @@ def binarize_workspace_size(n: int, num_segments: int = 1, keep=(1, 1000)) -> in
 
 def binarize(g: torch.Tensor, residual: torch.Tensor, keep=(1, 1000), seg_offsets: Optional[torch.Tensor] = None,
              out_idx=None, out_val=None, mean=None, out_offsets=None, workspace=None, flags: int = 0,
-             d_status=None, capacity: Optional[int] = None, want_values: bool = True, by_magnitude: bool = False):
+             d_status=None, capacity: Optional[int] = None, want_values: bool = True, by_magnitude: bool = False,
+             pass_events=None):
     """Returns (idx, val or None, mean[T], offsets[T+1]). by_magnitude: the magnitude-first reading
     (top fraction by |acc|, then the sign with the larger mean)."""
     if by_magnitude:
@@ -300,7 +308,7 @@ def binarize(g: torch.Tensor, residual: torch.Tensor, keep=(1, 1000), seg_offset
         workspace = _workspace(binarize_workspace_size(n, T, keep), dev)
     st = lib().gsparse_binarize(_ptr(g), _ptr(residual), n, _ptr(seg_offsets), T, keep[0], keep[1], _ptr(out_idx),
                                 _ptr(out_val), _ptr(mean), _ptr(out_offsets), capacity, flags, _ptr(workspace),
-                                workspace.numel(), _ptr(d_status), _stream(dev))
+                                workspace.numel(), _ptr(d_status), _stream(dev), _pass_events(pass_events))
     _check(st, "gsparse_binarize")
     return out_idx, out_val, mean, out_offsets
 

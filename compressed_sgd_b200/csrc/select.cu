@@ -24,6 +24,7 @@
 // Ties: keys equal to T are taken in ascending index order, so the lowest indices win.
 #include <math.h>
 
+#include <atomic>
 #include <type_traits>
 
 #include "common.cuh"
@@ -56,7 +57,7 @@ struct Sel {
   int64_t n;
   int32_t T, C;       // segments; classes: 1 = |x| (top-k), 2 = x > 0 and x < 0 (binarise)
   int32_t zero_mode;  // top-k: write +0 for candidates in pass 1
-  int32_t pad;
+  int32_t wait_test;  // test hook: the first ring wait of every warp is on a barrier nothing completes
   int64_t Lp, Q, cap;
   int64_t *seg_lo, *seg_n, *seg_k, *seg_kbase, *seg_pbase;
   uint32_t *tlo, *redo, *pfx, *thr;
@@ -833,6 +834,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
 constexpr int kStages = 3;
 constexpr uint32_t kChunkBytes = (uint32_t)kGranule * 4u;
 constexpr long long kWaitCycles = 1ll << 31;
+constexpr long long kTestWaitCycles = 1ll << 16;   // the test hook's wait (about 33 us)
 
 struct __align__(128) RingSlot {
   float g[kGranule];
@@ -871,12 +873,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits until the barrier's phase with this parity has completed; false after kWaitCycles.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+// Waits until the barrier's phase with this parity has completed; false after `limit` SM cycles.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   return true;
 }
 
@@ -920,13 +923,14 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
   constexpr int kSt = kMom ? kStagesM : kStages;
   extern __shared__ __align__(128) unsigned char ring_mem[];
   __shared__ CtaHist<C, kBins1> H;
-  __shared__ uint64_t bars[kWarps][kSt];
+  // per warp: one barrier per ring slot, and one that nothing ever arrives at (the test hook's)
+  __shared__ uint64_t bars[kWarps][kSt + 1];
   if (a.ctl[0]) return;
   const int64_t q0 = (int64_t)blockIdx.x * kWarps;
   H.init(a, q0);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   if (lane == 0)
-    for (int k = 0; k < kSt; ++k) mbar_init(&bars[wid][k], 1);
+    for (int k = 0; k <= kSt; ++k) mbar_init(&bars[wid][k], 1);
   fence_mbarrier_init();
   __syncthreads();
   const int64_t q = q0 + wid;
@@ -976,6 +980,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
     uint32_t parity = 0;   // bit k: the phase parity slot k waits for next
     uint32_t issued = nint < (uint32_t)kSt - 1 ? nint : (uint32_t)kSt - 1;
     bool failed = false;
+    uint32_t c_fail = 0;
     for (uint32_t c = 0; c < nint; ++c) {
       const uint32_t k = c % kSt;
       if (issued < nint) {
@@ -985,8 +990,12 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
         if (lane == 0) issue(issued);
         ++issued;
       }
-      if (!mbar_wait_bounded(&mb[k], (parity >> k) & 1u)) {
+      // test hook: the first wait is on the extra barrier, which never completes, with a short limit
+      const bool ok = (a.wait_test && c == 0) ? mbar_wait_bounded(&mb[kSt], 0u, kTestWaitCycles)
+                                              : mbar_wait_bounded(&mb[k], (parity >> k) & 1u);
+      if (!ok) {
         failed = true;
+        c_fail = c;
         break;
       }
       parity ^= 1u << k;
@@ -1000,10 +1009,11 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
         raise(a.d_status, GSPARSE_DERR_TIMEOUT);
         a.ctl[0] = 1;
       }
-      // let the copies still in flight land before the warp leaves (bounded as well)
-      for (uint32_t c = 0; c < issued; ++c) {
+      // let the copies still in flight land before the warp leaves (bounded as well): chunks
+      // c_fail .. issued - 1, at most one per slot, each still waiting for its slot's next phase
+      for (uint32_t c = c_fail; c < issued; ++c) {
         const uint32_t k = c % kSt;
-        if (c + kSt >= issued) mbar_wait_bounded(&mb[k], (parity >> k) & 1u);
+        mbar_wait_bounded(&mb[k], (parity >> k) & 1u);
       }
     } else {
       base += nint * (uint32_t)kGranule;
@@ -1983,14 +1993,12 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
 
 bool bad_keep(int64_t num, int64_t den) { return den <= 0 || num < 0 || num > den; }
 
-cudaEvent_t g_pass1_before = nullptr, g_pass1_after = nullptr;
-
 template <int C>
 int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t T, int64_t num,
                int64_t den, int32_t* out_idx, float* out_val, float* d_mean, int64_t* out_offsets,
                int64_t out_capacity, const gsparse_pending* pending, uint32_t flags, void* ws,
-               size_t ws_bytes, int32_t* d_status, cudaStream_t st, float* u = nullptr,
-               float mom = 0.0f) {
+               size_t ws_bytes, int32_t* d_status, cudaStream_t st,
+               const gsparse_pass_events* events, float* u = nullptr, float mom = 0.0f) {
   if (pending && (!pending->d_count || pending->capacity < 0 ||
                   (pending->capacity > 0 && (!pending->idx || !pending->val))))
     return GSPARSE_ERR_INVALID_ARG;
@@ -2013,6 +2021,7 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   a.u = u;
   a.mom = mom;
   a.zero_mode = C == 1;
+  a.wait_test = (flags & GSPARSE_SELECT_TEST_EXPIRE_WAIT) ? 1 : 0;
   a.d_status = d_status;
   const bool has_pending = pending && pending->capacity > 0;
   if (num == 0 && C == 1 && !has_pending && seg == nullptr) {
@@ -2043,8 +2052,8 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   const dim3 sgrid(kSampleCtas, (unsigned)T);
   sample_kernel<C><<<sgrid, 256, 0, st>>>(a, 1, exhaustive);
   sample_kernel<C><<<sgrid, 256, 0, st>>>(a, 2, exhaustive);
-  const bool timed = g_pass1_before && g_pass1_after;
-  if (timed) cudaEventRecord(g_pass1_before, st);
+  const bool timed = events && events->before && events->after;
+  if (timed) cudaEventRecord((cudaEvent_t)events->before, st);
   if (piece_ctas) {
     if constexpr (C == 1) {
       if (a.u) {
@@ -2061,7 +2070,7 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
       pass1_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
     }
   }
-  if (timed) cudaEventRecord(g_pass1_after, st);
+  if (timed) cudaEventRecord((cudaEvent_t)events->after, st);
   check_kernel<<<(unsigned)(T * C), 256, 0, st>>>(a);
   if (piece_ctas) restore_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
   select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 1);
@@ -2126,7 +2135,8 @@ MagLayout mag_carve(int64_t n, int32_t T, int64_t num, int64_t den, void* ws) {
 int run_binarize_magnitude(const float* g, float* r, int64_t n, const int64_t* seg, int32_t T,
                            int64_t num, int64_t den, int32_t* out_idx, float* out_val, float* d_mean,
                            int64_t* out_offsets, int64_t out_capacity, uint32_t flags, void* ws,
-                           size_t ws_bytes, int32_t* d_status, cudaStream_t st) {
+                           size_t ws_bytes, int32_t* d_status, cudaStream_t st,
+                           const gsparse_pass_events* events) {
   if (n < 0 || T < 1 || bad_keep(num, den) || !d_mean || !out_offsets || out_capacity < 0)
     return GSPARSE_ERR_INVALID_ARG;
   if (n > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
@@ -2140,7 +2150,7 @@ int run_binarize_magnitude(const float* g, float* r, int64_t n, const int64_t* s
   // the two-set reading)
   const int rc = run_select<1>(g, r, n, seg, T, num, den, M.lidx, M.lval, nullptr, M.loff,
                                out_capacity < M.kb ? out_capacity : M.kb, nullptr,
-                               flags & GSPARSE_SELECT_EXHAUSTIVE, tws, tws_bytes, d_status, st);
+                               flags & GSPARSE_SELECT_EXHAUSTIVE, tws, tws_bytes, d_status, st, events);
   if (rc != GSPARSE_OK) return rc;
   const int32_t* abort_flag = carve(n, T, 1, num, den, tws, tws_bytes, false).a.ctl;
   mjobs_kernel<<<1, 1024, 0, st>>>(M.lval, M.loff, T, M.jobs, abort_flag);
@@ -2159,18 +2169,25 @@ int run_binarize_magnitude(const float* g, float* r, int64_t n, const int64_t* s
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GSPARSE_NOALLOC_SCRATCH_BYTES];
 
 // Device address of the array on the current device, looked up once per device. In host code
-// the symbol itself is only a host-side stand-in, never a device address.
+// the symbol itself is only a host-side stand-in, never a device address. Several host threads
+// may look it up at once: each writes the same address, published with release ordering.
 int noalloc_scratch(void** out) {
-  static void* addr[64] = {};
+  static std::atomic<void*> addr[64];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GSPARSE_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return GSPARSE_ERR_UNSUPPORTED;
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GSPARSE_ERR_CUDA;
-    addr[dev] = p;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GSPARSE_ERR_CUDA;
   }
-  *out = addr[dev];
+  if (dev < 0 || dev >= 64) return GSPARSE_ERR_UNSUPPORTED;
+  void* p = addr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();   // leave no error behind for the caller's next launch check
+      return GSPARSE_ERR_CUDA;
+    }
+    addr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
   return GSPARSE_OK;
 }
 
@@ -2180,11 +2197,6 @@ int noalloc_scratch(void** out) {
 using namespace gs;
 
 extern "C" {
-
-void gsparse_set_pass1_events(gsparse_event before, gsparse_event after) {
-  g_pass1_before = (cudaEvent_t)before;
-  g_pass1_after = (cudaEvent_t)after;
-}
 
 size_t gsparse_residual_topk_workspace_size(int64_t n, int32_t T, int64_t num, int64_t den) {
   if (n < 0 || T < 1 || bad_keep(num, den)) return 0;
@@ -2202,21 +2214,24 @@ int gsparse_residual_topk_momentum(const float* g, float* momentum_buf, float mo
                                    int32_t* out_idx, float* out_val, int64_t* out_offsets,
                                    int64_t out_capacity, const gsparse_pending* pending,
                                    uint32_t flags, void* workspace, size_t workspace_bytes,
-                                   int32_t* d_status, gsparse_stream stream) {
+                                   int32_t* d_status, gsparse_stream stream,
+                                   const gsparse_pass_events* pass_events) {
   if (n > 0 && !momentum_buf) return GSPARSE_ERR_INVALID_ARG;
   return run_select<1>(g, residual, n, seg_offsets, num_segments, keep_num, keep_den, out_idx,
                        out_val, nullptr, out_offsets, out_capacity, pending, flags, workspace,
-                       workspace_bytes, d_status, (cudaStream_t)stream, momentum_buf, momentum);
+                       workspace_bytes, d_status, (cudaStream_t)stream, pass_events, momentum_buf,
+                       momentum);
 }
 
 int gsparse_residual_topk(const float* g, float* residual, int64_t n, const int64_t* seg_offsets,
                           int32_t num_segments, int64_t keep_num, int64_t keep_den, int32_t* out_idx,
                           float* out_val, int64_t* out_offsets, int64_t out_capacity,
                           const gsparse_pending* pending, uint32_t flags, void* workspace,
-                          size_t workspace_bytes, int32_t* d_status, gsparse_stream stream) {
+                          size_t workspace_bytes, int32_t* d_status, gsparse_stream stream,
+                          const gsparse_pass_events* pass_events) {
   return run_select<1>(g, residual, n, seg_offsets, num_segments, keep_num, keep_den, out_idx,
                        out_val, nullptr, out_offsets, out_capacity, pending, flags, workspace,
-                       workspace_bytes, d_status, (cudaStream_t)stream);
+                       workspace_bytes, d_status, (cudaStream_t)stream, pass_events);
 }
 
 size_t gsparse_binarize_workspace_size(int64_t n, int32_t T, int64_t num, int64_t den) {
@@ -2245,21 +2260,21 @@ int gsparse_residual_topk_noalloc(const float* g, float* residual, int64_t n, in
   if (st != GSPARSE_OK) return st;
   return run_select<1>(g, residual, n, nullptr, 1, keep_num, keep_den, out_idx, out_val, nullptr,
                        out_offsets, out_capacity, nullptr, 0, scratch, GSPARSE_NOALLOC_SCRATCH_BYTES,
-                       d_status, (cudaStream_t)stream);
+                       d_status, (cudaStream_t)stream, nullptr);
 }
 
 int gsparse_binarize(const float* g, float* residual, int64_t n, const int64_t* seg_offsets,
                      int32_t num_segments, int64_t keep_num, int64_t keep_den, int32_t* out_idx,
                      float* out_val, float* d_mean, int64_t* out_offsets, int64_t out_capacity,
                      uint32_t flags, void* workspace, size_t workspace_bytes, int32_t* d_status,
-                     gsparse_stream stream) {
+                     gsparse_stream stream, const gsparse_pass_events* pass_events) {
   if (flags & GSPARSE_BINARIZE_BY_MAGNITUDE)
     return run_binarize_magnitude(g, residual, n, seg_offsets, num_segments, keep_num, keep_den,
                                   out_idx, out_val, d_mean, out_offsets, out_capacity, flags, workspace,
-                                  workspace_bytes, d_status, (cudaStream_t)stream);
+                                  workspace_bytes, d_status, (cudaStream_t)stream, pass_events);
   return run_select<2>(g, residual, n, seg_offsets, num_segments, keep_num, keep_den, out_idx,
                        out_val, d_mean, out_offsets, out_capacity, nullptr, flags, workspace,
-                       workspace_bytes, d_status, (cudaStream_t)stream);
+                       workspace_bytes, d_status, (cudaStream_t)stream, pass_events);
 }
 
 }  // extern "C"

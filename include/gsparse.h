@@ -20,7 +20,10 @@
  *    The library allocates and frees nothing; scratch memory is the caller's `workspace`, whose
  *    required size the matching *_workspace_size() function returns.
  *  - Calls are asynchronous on `stream` (NULL = the legacy default stream). No call
- *    synchronises the host. Calls that use separate workspaces may run concurrently.
+ *    synchronises the host. Calls that use separate workspaces may run concurrently. The library
+ *    keeps no state between calls, with one exception: gsparse_residual_topk_noalloc uses a fixed
+ *    scratch array owned by the library, shared by all its calls on a device, so calls of it
+ *    that overlap on the GPU must be serialised.
  *  - The return value is a gsparse_status for errors found on the host before any launch (bad
  *    arguments, short workspace, launch failure). Errors that depend on device data are OR-ed as
  *    GSPARSE_DERR_* bits into *d_status (device int32; may be NULL to ignore them). The library
@@ -71,18 +74,27 @@ enum gsparse_select_flags {
      found from the full data. Same result, more memory traffic. */
   GSPARSE_SELECT_EXHAUSTIVE = 1,
   /* gsparse_binarize only: the magnitude-first reading of sparse binarisation (see there). */
-  GSPARSE_BINARIZE_BY_MAGNITUDE = 2
+  GSPARSE_BINARIZE_BY_MAGNITUDE = 2,
+  /* Test hook for the failure path, never for production use: in gsparse_residual_topk_momentum
+     the first bounded wait of every warp of the streaming pass waits on a barrier that nothing
+     completes, with a limit of 2^16 SM cycles. The wait runs out, GSPARSE_DERR_TIMEOUT is
+     raised, the rest of the call does nothing, and residual, momentum buffer and outputs are
+     left partly updated (not valid); the context stays usable. No effect on the other calls. */
+  GSPARSE_SELECT_TEST_EXPIRE_WAIT = 4
 };
 
 const char* gsparse_status_string(int status);
 const char* gsparse_version(void);
 
-/* Measurement hook, off by default and not thread-safe: while both events are non-NULL, every
- * gsparse_residual_topk, gsparse_residual_topk_momentum and gsparse_binarize call records
- * `before` on its stream right before
- * its streaming pass over g and the residual, and `after` right after it, so that pass can be
- * timed alone with cudaEventElapsedTime. Passing NULLs turns it off. */
-void gsparse_set_pass1_events(gsparse_event before, gsparse_event after);
+/* Per-call measurement events (HOST struct, optional): a call of gsparse_residual_topk,
+ * gsparse_residual_topk_momentum or gsparse_binarize given a non-NULL pointer with both events
+ * set records `before` on its stream right before its streaming pass over g and the residual,
+ * and `after` right after it, so that pass can be timed alone with cudaEventElapsedTime. The
+ * events are created by the caller (cudaEventCreate); NULL records nothing. */
+typedef struct {
+  gsparse_event before;
+  gsparse_event after;
+} gsparse_pass_events;
 
 /* ---------------------------------------------------------------------------------------------
  * Host helpers.
@@ -135,6 +147,7 @@ int64_t gsparse_warmup_keep_num(int64_t t, int64_t T, double start, double end, 
  * workspace        256-byte aligned, at least gsparse_residual_topk_workspace_min(); the
  *                  recommended size is gsparse_residual_topk_workspace_size(). Less room only
  *                  costs speed.
+ * pass_events      HOST pointer or NULL: events recorded around the streaming pass (above).
  * Data errors: GSPARSE_DERR_SEGMENTS, GSPARSE_DERR_CAPACITY, GSPARSE_DERR_INDEX_RANGE (a pending
  * list that is not strictly ascending in [0, n)); on any of them nothing is written.
  */
@@ -152,7 +165,8 @@ int gsparse_residual_topk(const float* g, float* residual, int64_t n, const int6
                           int32_t num_segments, int64_t keep_num, int64_t keep_den, int32_t* out_idx,
                           float* out_val, int64_t* out_offsets, int64_t out_capacity,
                           const gsparse_pending* pending, uint32_t flags, void* workspace,
-                          size_t workspace_bytes, int32_t* d_status, gsparse_stream stream);
+                          size_t workspace_bytes, int32_t* d_status, gsparse_stream stream,
+                          const gsparse_pass_events* pass_events);
 
 /* Residual top-k with momentum correction and momentum masking ("Sparse Binary Compression",
  * §II "Momentum Correction, Warm-up Training and Momentum Masking" and Appendix A: the
@@ -174,7 +188,8 @@ int gsparse_residual_topk_momentum(const float* g, float* momentum_buf, float mo
                                    int32_t* out_idx, float* out_val, int64_t* out_offsets,
                                    int64_t out_capacity, const gsparse_pending* pending,
                                    uint32_t flags, void* workspace, size_t workspace_bytes,
-                                   int32_t* d_status, gsparse_stream stream);
+                                   int32_t* d_status, gsparse_stream stream,
+                                   const gsparse_pass_events* pass_events);
 
 /* ---------------------------------------------------------------------------------------------
  * Residual top-k without caller-provided scratch  (no counterpart in the pages: this entry point
@@ -184,8 +199,11 @@ int gsparse_residual_topk_momentum(const float* g, float* momentum_buf, float mo
  * framework whose caching allocator owns the whole device and budgets every byte (an allocation
  * of our own would fail or fight that allocator), or code invoked from that allocator's own hooks
  * (allocating there would re-enter it). This call needs neither: its scratch is a fixed array of
- * GSPARSE_NOALLOC_SCRATCH_BYTES in the library's own device memory, created when the library is
- * loaded and held by every GPU that loads it until the process exits. It allocates nothing.
+ * GSPARSE_NOALLOC_SCRATCH_BYTES in the library's own device memory. The array comes into
+ * existence when the library's top-k module is first used on a device (with CUDA's lazy module
+ * loading, the default, that is the first top-k, binarise or noalloc call on that device, which
+ * may be this call itself) and stays until the process exits. A caller whose allocator reserves
+ * the whole device should make one call (any size) before the reservation. It allocates nothing.
  *
  * Same result as gsparse_residual_topk with seg_offsets = NULL and num_segments = 1 (one global
  * selection) and flags = 0, bit for bit. The caller still owns g, residual and the outputs.
@@ -194,7 +212,9 @@ int gsparse_residual_topk_momentum(const float* g, float* momentum_buf, float mo
  *   that device current; make that first call before any stream capture on the device.
  * - All calls on a device share the one array and it keeps the last call's contents; each call
  *   clears the parts that must start at zero. Calls whose kernels overlap on the GPU (concurrent
- *   streams, or several host threads) race on the array: serialise them.
+ *   streams, or several host threads) race on the array: serialise them. The host-side lookup
+ *   of the address is itself safe from several threads.
+ * - If the lookup fails the call returns GSPARSE_ERR_CUDA and clears the runtime's last error.
  */
 #define GSPARSE_NOALLOC_MAX_N (1 << 24)
 #define GSPARSE_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -264,7 +284,7 @@ int gsparse_binarize(const float* g, float* residual, int64_t n, const int64_t* 
                      int32_t num_segments, int64_t keep_num, int64_t keep_den, int32_t* out_idx,
                      float* out_val, float* d_mean, int64_t* out_offsets, int64_t out_capacity,
                      uint32_t flags, void* workspace, size_t workspace_bytes, int32_t* d_status,
-                     gsparse_stream stream);
+                     gsparse_stream stream, const gsparse_pass_events* pass_events);
 
 /* ---------------------------------------------------------------------------------------------
  * Golomb position coding  (Sattler et al. §II Optimal Position Encoding; Appendix A)
