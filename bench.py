@@ -13,6 +13,7 @@ Metric: gradient GB/s compressed = W * 4 * n bytes per step / step time (whole j
 ranks), with the residual-top-k call's share of HBM bandwidth reported beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--drop 0.99]
+  python bench.py --exchange [--gpus N] ...   one worker per GPU, payloads all-gathered (NCCL)
 
 With N > 1 (torchrun, one process per GPU) every rank runs an independent replica of the step:
 the path has no exchange on one node's simulated workers, so there is no collective in the data
@@ -355,6 +356,130 @@ def run_ours(args, rank, world, dist):
 
 
 # ---------------------------------------------------------------------------------------------
+# exchange between ranks: one worker per GPU
+
+def run_exchange(args, rank, world, dist):
+    """One worker per rank. Step per rank: residual top-k (with the previous step's quantisation
+    error as pending writes) -> 2-bit quantisation (dequantised values sent) -> Golomb encode ->
+    all-gather of the fixed-capacity payloads (NCCL; lengths travel in a device header, no host
+    synchronisation) -> decode of every rank's stream -> fused receive of all ranks' updates in
+    rank order combined with the rank's own gradient."""
+    import torch
+    import compressed_sgd_b200 as gs
+    from compressed_sgd_b200 import exchange
+    import synth
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    n = args.n
+    keep = keep_of(args.drop)
+    b = gs.golomb_b_star(1.0 - args.drop)
+    cap = gs.k_for(n, keep)
+    chunk = 64
+    nch = (cap + chunk - 1) // chunk
+    nwords = gs.golomb_word_capacity(cap, b, n)
+    g = torch.from_numpy(synth.laplace_outliers(rank, n)).to(dev)
+    r = torch.zeros(n, dtype=torch.float32, device=dev)
+    out = torch.empty(n, dtype=torch.float32, device=dev)
+    # two sets of send buffers: step t applies step t-1's quantisation error
+    idx = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(2)]
+    val = [torch.empty(cap, dtype=torch.float32, device=dev) for _ in range(2)]
+    fb = [torch.empty(cap, dtype=torch.float32, device=dev) for _ in range(2)]
+    # header: [0] stream bits (written by the encoder), [1:3] the top-k's offsets {0, K}
+    meta = [torch.zeros(3, dtype=torch.int64, device=dev) for _ in range(2)]
+    words = [torch.zeros(nwords, dtype=torch.int32, device=dev) for _ in range(2)]
+    table = [torch.zeros(nch * 2, dtype=torch.int64, device=dev) for _ in range(2)]
+    pend = [gs.make_pending(idx[p], fb[p], meta[p][2:3], capacity=cap) for p in range(2)]
+    sb = torch.empty((cap + 31) // 32, dtype=torch.int32, device=dev)
+    means = torch.empty(2, dtype=torch.float32, device=dev)
+    ws_t = torch.empty(gs.residual_topk_workspace_size(n, 1, keep), dtype=torch.uint8, device=dev)
+    ws_q = torch.empty(gs.lib().gsparse_quantize_workspace_size(cap), dtype=torch.uint8, device=dev)
+    ws_g = torch.empty(gs.lib().gsparse_golomb_encode_workspace_size(cap), dtype=torch.uint8, device=dev)
+    ws_s = torch.empty(gs.lib().gsparse_accumulate_combine_workspace_size(world, n), dtype=torch.uint8,
+                       device=dev)
+    st = gs.status_tensor(dev)
+    dec = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(world)]
+    recv = [exchange.gather_buffers([words[p], table[p], val[p], meta[p]], world) for p in range(2)]
+    parity = [0]
+
+    def step(ev=None):
+        rec = (lambda k: ev[k].record()) if ev is not None else (lambda k: None)
+        cur, prev = parity[0], 1 - parity[0]
+        parity[0] = prev
+        rec(0)
+        gs.residual_topk(g, r, keep, out_idx=idx[cur], out_val=val[cur], out_offsets=meta[cur][1:3],
+                         workspace=ws_t, d_status=st, capacity=cap, pending=pend[prev])
+        end = meta[cur][2:3]
+        gs.quantize(idx[cur], val[cur], end, write_dequantized=True, feedback_out=fb[cur], sign_bits=sb,
+                    means=means, workspace=ws_q, d_status=st, capacity=cap)
+        gs.golomb_encode(idx[cur], end, b, n, chunk=chunk, words=words[cur], nbits=meta[cur][0:1],
+                         table=table[cur].view(nch, 2), workspace=ws_g, d_status=st, capacity=cap)
+        rec(1)
+        rows = exchange.all_gather_fixed([words[cur], table[cur], val[cur], meta[cur]],
+                                         dist if world > 1 else None, out=recv[cur])
+        rec(2)
+        lists = []
+        for q in range(world):
+            w_q, t_q, v_q, m_q = rows[q]
+            gs.golomb_decode(w_q, m_q[0:1], m_q[2:3], cap, b, table=t_q.view(nch, 2), chunk=chunk, n_limit=n,
+                             out_idx=dec[q], d_status=st)
+            lists.append(gs.make_list(dec[q], m_q[2:3], val=v_q, capacity=cap))
+        rec(3)
+        gs.accumulate_combine(lists, n, g, out=out, workspace=ws_s, d_status=st)
+        rec(4)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} after warm-up")
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(dev.index if dev.index is not None else 0)
+    barrier()
+    clocks.start()
+    t0.record()
+    for k in range(K):
+        step(evs[k])
+    t1.record()
+    barrier()
+    clk = clocks.stop()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the timed region")
+    ms = t0.elapsed_time(t1) / K
+    names = ["compress", "all_gather", "decode", "receive"]
+    stages = {nm: statistics.median(e[i].elapsed_time(e[i + 1]) for e in evs) for i, nm in enumerate(names)}
+    # bytes of this rank's payload (used part) and of the padded buffers that cross the interconnect
+    p = 1 - parity[0]
+    m = [int(x) for x in meta[p].tolist()]
+    used = ((m[0] + 31) // 32) * 4 + ((m[2] + chunk - 1) // chunk) * 16 + m[2] * 4 + 24
+    padded = sum(t.numel() * t.element_size() for t in (words[p], table[p], val[p], meta[p]))
+    vals = max_over_ranks([ms] + [stages[nm] for nm in names], dist if world > 1 else None, dev)
+    if rank != 0:
+        return None
+    ms = vals[0]
+    grad_bytes = world * 4 * n
+    return {"metric": METRIC, "mode": "exchange", "value": round(grad_bytes / (ms * 1e-3) / 1e9, 2), "unit": UNIT,
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"flat fp32 gradient of {n} entries per rank (one worker per GPU), Laplace(0,1e-3) "
+                                   f"with 0.1% Laplace(0,1e-1) outliers, residual carried",
+                       "n": n, "drop": args.drop, "keep": f"1/{keep[1]}", "golomb_b": b,
+                       "step": "per rank: topk+quantise+golomb encode; all-gather of fixed-capacity payloads; decode "
+                               "of every rank's stream; fused receive of all ranks' updates + own gradient",
+                       "parallelism": f"data parallel x{world}, NCCL all-gather" if world > 1 else "one rank"},
+            "stages_ms": {nm: round(v, 4) for nm, v in zip(names, vals[1:])},
+            "payload_bytes_per_rank": used, "padded_bytes_per_rank": padded,
+            "clocks": clk}
+
+
+# ---------------------------------------------------------------------------------------------
 # the other workloads (one JSON line each; not the default line)
 
 WORKLOADS = {
@@ -651,6 +776,8 @@ def main():
     ap.add_argument("--momentum", type=float, default=None,
                     help="momentum correction and masking in the residual top-k (e.g. 0.9); off by default")
     ap.add_argument("--no-graph", action="store_true", help="with --workload: skip the CUDA-graph replay leg")
+    ap.add_argument("--exchange", action="store_true",
+                    help="one worker per GPU with the compressed payloads all-gathered between ranks")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -672,7 +799,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     try:
-        line = run_ours(args, rank, world, dist)
+        line = run_exchange(args, rank, world, dist) if args.exchange else run_ours(args, rank, world, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()

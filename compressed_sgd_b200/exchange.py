@@ -10,8 +10,13 @@ section is padded to the longest and all-gathered, and every rank trims the rece
 their own lengths. With CUDA tensors and the NCCL backend the transfers run over NVLink; with CPU
 tensors and gloo the same code runs on the host. Decoding and the worker-ordered sum then use the
 library's calls on the gathered payloads (rank order = worker order).
+
+all_gather_payloads learns the lengths on the host (one small gather and a synchronisation per
+call). all_gather_fixed instead gathers buffers of a fixed capacity whose used lengths travel
+inside them (the stream's bit count and the entry count in a device header), so a training loop
+can run the exchange with no host synchronisation; the decoder reads the lengths on the device.
 """
-from typing import Dict, List, Sequence
+from typing import Dict, List, Optional, Sequence
 
 import torch
 
@@ -66,3 +71,30 @@ def all_gather_payloads(payload: Dict[str, torch.Tensor], dist, group=None) -> L
 def payload_bytes(payloads: Sequence[Dict[str, torch.Tensor]]) -> int:
     """Bytes that cross the interconnect per rank and step (before padding)."""
     return sum(t.numel() * t.element_size() for p in payloads for t in p.values())
+
+
+def gather_buffers(sections: Sequence[torch.Tensor], world: int) -> List[torch.Tensor]:
+    """Receive buffers for all_gather_fixed: one tensor of world x numel per section."""
+    return [torch.empty(world * t.numel(), dtype=t.dtype, device=t.device) for t in sections]
+
+
+def all_gather_fixed(sections: Sequence[torch.Tensor], dist, group=None,
+                     out: Optional[Sequence[torch.Tensor]] = None) -> List[List[torch.Tensor]]:
+    """Gathers same-shaped buffers from every rank, one collective per section. sections: 1-D
+    contiguous tensors of the same length and dtype on every rank (fixed capacities, e.g. the
+    Golomb word buffer, the side table, the values and an int64 header holding the bit count and
+    the entry count). out: receive buffers from gather_buffers (allocated here if None). With
+    dist None there is one rank and its sections are returned as they are.
+    Returns rows[r][k] = section k of rank r (views into the receive buffers)."""
+    if dist is None:
+        return [list(sections)]
+    world = dist.get_world_size(group)
+    if out is None:
+        out = gather_buffers(sections, world)
+    per_rank: List[List[torch.Tensor]] = [[] for _ in range(world)]
+    for t, gathered in zip(sections, out):
+        dist.all_gather_into_tensor(gathered, t, group=group)
+        rows = gathered.view(world, t.numel())
+        for r in range(world):
+            per_rank[r].append(rows[r])
+    return per_rank
