@@ -573,12 +573,12 @@ def run_workload(args):
     none_i = torch.empty(1, dtype=torch.int32, device=dev)
     none_v = torch.empty(1, device=dev)
     none_o = torch.zeros(2, dtype=torch.int64, device=dev)
-    ws_q = torch.empty(gs.lib().gsparse_quantize_workspace_size(cap), dtype=torch.uint8, device=dev)
+    ws_q = torch.empty(gs.lib().gsparse_quantize_segments_workspace_size(cap, T), dtype=torch.uint8, device=dev)
     ws_g = torch.empty(gs.lib().gsparse_golomb_encode_workspace_size(cap), dtype=torch.uint8, device=dev)
     ws_s = torch.empty(max(gs.lib().gsparse_scatter_accumulate_workspace_size(W, n),
                            gs.lib().gsparse_accumulate_combine_workspace_size(W, n)), dtype=torch.uint8, device=dev)
     sb = [torch.empty((cap + 31) // 32, dtype=torch.int32, device=dev) for _ in range(W)]
-    means = [torch.empty(2, device=dev) for _ in range(W)]
+    means = [torch.empty(2 * T, device=dev) for _ in range(W)]
 
     def step(ev=None):
         rec = (lambda k: ev[k].record()) if ev is not None else (lambda k: None)
@@ -594,10 +594,9 @@ def run_workload(args):
                 gs.residual_topk(g[w], r[w], keep, seg_offsets=seg_d, out_idx=idx[w], out_val=val[w],
                                  out_offsets=off[w], workspace=ws_t, d_status=st, capacity=cap)
             if name == "mlp":
-                for s_ in range(T):
-                    gs.quantize(idx[w], val[w], off[w][s_ + 1:s_ + 2], d_begin=off[w][s_:s_ + 1], residual=r[w],
-                                write_dequantized=True, sign_bits=sb[w], means=means[w], workspace=ws_q,
-                                d_status=st, capacity=cap)
+                # per-tensor means, all tensors in one call
+                gs.quantize_segments(idx[w], val[w], off[w], residual=r[w], write_dequantized=True, sign_bits=sb[w],
+                                     means=means[w], workspace=ws_q, d_status=st, capacity=cap)
             if name in ("flat2e20", "resnet50"):
                 end = off[w][T:T + 1]
                 gs.golomb_encode(idx[w], end, b, n, chunk=64, words=words[w], nbits=nbits[w], table=table[w],

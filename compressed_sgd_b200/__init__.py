@@ -64,6 +64,9 @@ _SIGNATURES = {
     "gsparse_quantize_workspace_size": (_sz, [_i64]),
     "gsparse_quantize": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _sz, _vp,
                                         _vp]),
+    "gsparse_quantize_segments_workspace_size": (_sz, [_i64, _i32]),
+    "gsparse_quantize_segments": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i64, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _sz,
+                                                 _vp, _vp]),
     "gsparse_binarize_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_binarize_workspace_min": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_binarize": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _u32,
@@ -146,6 +149,9 @@ def _pass_events(events):
     if events is None:
         return None
     before, after = events
+    for e in (before, after):
+        if not e.cuda_event:   # torch creates the CUDA event on its first record
+            e.record()
     return ctypes.byref(GsparsePassEvents(before.cuda_event, after.cuda_event))
 
 
@@ -271,6 +277,31 @@ def quantize(idx: torch.Tensor, val: torch.Tensor, d_end: torch.Tensor, d_begin:
                                 _ptr(feedback_out), _ptr(sign_bits), _ptr(means), int(write_dequantized),
                                 _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev))
     _check(st, "gsparse_quantize")
+    return sign_bits, means
+
+
+def quantize_segments(idx: torch.Tensor, val: torch.Tensor, offsets: torch.Tensor,
+                      residual: Optional[torch.Tensor] = None, write_dequantized: bool = False,
+                      feedback_out: Optional[torch.Tensor] = None, sign_bits: Optional[torch.Tensor] = None,
+                      means: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                      d_status: Optional[torch.Tensor] = None, capacity: Optional[int] = None):
+    """2-bit quantisation of the T sub-lists [offsets[s], offsets[s+1]) in one call (per-segment
+    means). Returns (sign_bits, means float32[2T])."""
+    dev = val.device
+    _dev(offsets, torch.int64, "offsets")
+    T = offsets.numel() - 1
+    capacity = val.numel() if capacity is None else capacity
+    if sign_bits is None:
+        sign_bits = torch.zeros(max((capacity + 31) // 32, 1), dtype=torch.int32, device=dev)
+    if means is None:
+        means = torch.empty(2 * T, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = _workspace(lib().gsparse_quantize_segments_workspace_size(capacity, T), dev)
+    n = 0 if residual is None else residual.numel()
+    st = lib().gsparse_quantize_segments(_ptr(idx), _ptr(val), _ptr(offsets), T, capacity, _ptr(residual), n,
+                                         _ptr(feedback_out), _ptr(sign_bits), _ptr(means), int(write_dequantized),
+                                         _ptr(workspace), workspace.numel(), _ptr(d_status), _stream(dev))
+    _check(st, "gsparse_quantize_segments")
     return sign_bits, means
 
 

@@ -4,10 +4,11 @@
 // Codeword of gap d: q = d >> b one-bits, a zero-bit, then d mod 2^b in b bits, most significant
 // first; stream bit t is bit t % 32 of word t / 32.
 //
-// Encoder: codeword lengths -> device-wide exclusive scan (bit offsets) -> zero the stream ->
-// pack. A warp packs 32 codewords: it stages their offsets in shared memory and writes every
-// word that lies wholly inside its bit range with one plain store; only the two words it shares
-// with neighbouring warps are OR-ed atomically.
+// Encoder, one pass over the indices: a block of 2048 codewords sums its codeword lengths, finds
+// its first bit by a decoupled look-back over the blocks before it (bounded waits; blocks are
+// numbered in the order they start, so a block only waits on running blocks), packs its
+// codewords into a shared word buffer and writes each of its words once. The two words a block
+// may share with its neighbours go to a side array and a small fix-up kernel merges them.
 // Decoder: with the side table, one thread per chunk of codewords decodes sequentially from its
 // recorded bit offset and checks that it ends where the next chunk starts.
 #include "common.cuh"
@@ -15,32 +16,39 @@
 namespace gs {
 namespace {
 
-constexpr int kScanThreads = 1024;
 constexpr int kPer = 8;                      // codewords per thread
 constexpr int kCodeThreads = 256;
-constexpr int kBlockCodes = kPer * kCodeThreads;  // codewords per block of the length and pack passes
-constexpr int kPackWords = 4096;             // shared word buffer of the pack pass (128 Kbit)
+constexpr int kBlockCodes = kPer * kCodeThreads;  // codewords per block
+constexpr int kPackWords = 4096;             // shared word buffer of a block (128 Kbit)
+constexpr long long kLookbackCycles = 1ll << 31;  // bound of one block's look-back (about a second)
 
-struct GCtl {
-  int64_t begin, len;
-  int32_t abort;
-  int32_t pad;
+// Look-back descriptors: flag in the top two bits, a bit count below.
+constexpr uint64_t kFlagAgg = 1ull << 62;    // the block's own total is published
+constexpr uint64_t kFlagInc = 2ull << 62;    // the total of this block and all before it
+constexpr uint64_t kValMask = (1ull << 62) - 1ull;
+
+struct GState {
+  uint32_t next_block;  // dynamic block numbering (blocks start in this order)
+  int32_t abort;        // a look-back gave up
 };
 
-__global__ void g_setup_kernel(const int64_t* d_begin, const int64_t* d_end, int64_t capacity,
-                               GCtl* ctl, GCtl* wctl, int32_t* d_status) {
+__device__ __forceinline__ uint64_t ld_relaxed(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// The list [begin, begin + len) from the device bounds; false (len 0) if they are invalid.
+__device__ __forceinline__ bool list_bounds(const int64_t* d_begin, const int64_t* d_end,
+                                            int64_t capacity, int64_t* begin, int64_t* len) {
   const int64_t b = d_begin ? *d_begin : 0;
-  const int64_t len = *d_end - b;
-  if (b < 0 || len < 0 || len > capacity) {
-    raise(d_status, GSPARSE_DERR_CAPACITY);
-    ctl->abort = 1;
-    ctl->len = 0;
-  } else {
-    ctl->abort = 0;
-    ctl->len = len;
-  }
-  ctl->begin = b;
-  wctl->abort = 0;
+  const int64_t l = *d_end - b;
+  *begin = b;
+  *len = (b < 0 || l < 0 || l > capacity) ? 0 : l;
+  return !(b < 0 || l < 0 || l > capacity);
 }
 
 // Gaps of this thread's kPer consecutive codewords (entries j0 .. j0+kPer-1 of the list); an
@@ -60,79 +68,18 @@ __device__ __forceinline__ void thread_gaps(const int32_t* x, int64_t len, int64
     for (int e = 0; e < kPer; ++e) v[e] = j0 + e < len ? x[j0 + e] : 0;
   }
   int64_t prev = j0 == 0 ? base - 1 : (j0 - 1 < len ? (int64_t)x[j0 - 1] : 0);
+  bool bad = false;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     d[e] = 0;
     if (j0 + e < len) {
       const int64_t g = (int64_t)v[e] - prev - 1;
-      if (g < 0) {
-        if (d_status) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
-      } else {
-        d[e] = (uint32_t)g;
-      }
+      if (g < 0) bad = true;
+      else d[e] = (uint32_t)g;
       prev = v[e];
     }
   }
-}
-
-// per-block totals of the codeword lengths
-__global__ void __launch_bounds__(kCodeThreads) g_len_kernel(const int32_t* idx, const GCtl* ctl,
-                                                              int64_t base, int b, int64_t* block_tot,
-                                                              int32_t* d_status) {
-  __shared__ int64_t sh[33];
-  if (ctl->abort) return;
-  const int64_t len = ctl->len;
-  if ((int64_t)blockIdx.x * kBlockCodes >= len) return;
-  const int64_t j0 = (int64_t)blockIdx.x * kBlockCodes + (int64_t)threadIdx.x * kPer;
-  uint32_t d[kPer];
-  thread_gaps(idx + ctl->begin, len, base, j0, d, d_status);
-  int64_t l = 0;
-#pragma unroll
-  for (int e = 0; e < kPer; ++e)
-    if (j0 + e < len) l += (int64_t)(d[e] >> b) + 1 + b;
-  int64_t tot;
-  block_exclusive_scan(l, sh, &tot);
-  if (threadIdx.x == 0) block_tot[blockIdx.x] = tot;
-}
-
-// exclusive scan of the block totals (one CTA), total = stream length
-__global__ void __launch_bounds__(kScanThreads) g_scan_blocks_kernel(int64_t* block_tot,
-                                                                      const GCtl* ctl,
-                                                                      int64_t word_capacity,
-                                                                      uint64_t* d_nbits,
-                                                                      GCtl* wctl,
-                                                                      int32_t* d_status) {
-  __shared__ int64_t sh[33];
-  if (ctl->abort) {
-    if (threadIdx.x == 0) *d_nbits = 0;
-    return;
-  }
-  const int64_t nblk = cdiv(ctl->len, kBlockCodes);
-  int64_t carry = 0;
-  for (int64_t base = 0; base < nblk; base += blockDim.x) {
-    const int64_t i = base + threadIdx.x;
-    const int64_t v = i < nblk ? block_tot[i] : 0;
-    int64_t tot;
-    const int64_t ex = block_exclusive_scan(v, sh, &tot);
-    if (i < nblk) block_tot[i] = carry + ex;
-    carry += tot;
-  }
-  if (threadIdx.x == 0) {
-    *d_nbits = (uint64_t)carry;
-    if (cdiv(carry, 32) > word_capacity) {
-      raise(d_status, GSPARSE_DERR_CAPACITY);
-      wctl->abort = 1;
-    }
-  }
-}
-
-__global__ void g_zero_kernel(uint32_t* words, const uint64_t* d_nbits, int64_t bound,
-                              const GCtl* ctl, const GCtl* wctl) {
-  if (ctl->abort || wctl->abort) return;
-  const int64_t nw = cdiv((int64_t)*d_nbits, 32);
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < nw && w < bound; w += stride)
-    words[w] = 0u;
+  if (bad) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
 }
 
 struct Code {
@@ -163,35 +110,104 @@ __device__ __forceinline__ uint32_t code_bits_in_word(const Code& c, uint64_t w)
   return bits;
 }
 
-// Offsets of this block's codewords (block prefix + in-block scan), the side table, and the
-// packing: when the block's bits fit the shared word buffer, each thread ORs its codewords in
-// with shared atomics and the words go out in one coalesced sweep (the first and last word, which
-// the block may share with its neighbours, are OR-ed into the zeroed stream). Otherwise (long
-// unary runs) every codeword is OR-ed straight into the zeroed stream.
-__global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx, const GCtl* ctl,
-                                                               const GCtl* wctl, int64_t base, int b,
-                                                               const int64_t* block_pre,
-                                                               int64_t* table, int32_t chunk,
-                                                               uint32_t* words) {
+// Exclusive prefix of block vb (the bits of all blocks before it), by warp 0 looking back over
+// the descriptors of blocks vb-1, vb-2, ... 32 at a time: aggregates are added until a block
+// whose inclusive total is published. Blocks are numbered in the order they start, so every
+// block waited on is already running and publishes its aggregate without waiting itself.
+// Returns false if a descriptor stayed unpublished for kLookbackCycles.
+__device__ bool lookback(const uint64_t* flags, uint32_t vb, int lane, uint64_t* prefix) {
+  uint64_t acc = 0;
+  int64_t p = (int64_t)vb - 1;
+  const long long t0 = clock64();
+  while (p >= 0) {
+    const int64_t q = p - lane;
+    uint64_t f = q >= 0 ? ld_relaxed(flags + q) : kFlagInc;   // before block 0: an inclusive 0
+    for (;;) {
+      const bool missing = (f >> 62) == 0;
+      if (!__any_sync(kFull, missing)) break;
+      const bool late = lane == 0 && clock64() - t0 > kLookbackCycles;
+      if (__any_sync(kFull, late)) return false;
+      if (missing) f = ld_relaxed(flags + q);
+    }
+    const uint32_t inc = __ballot_sync(kFull, (f >> 62) == 2u);
+    const int first = inc ? __ffs(inc) - 1 : 32;   // the nearest block with an inclusive total
+    acc += warp_sum(lane <= first ? (f & kValMask) : 0ull);
+    if (inc) break;
+    p -= 32;
+  }
+  *prefix = acc;
+  return true;
+}
+
+// One pass: codeword lengths and the block's bit count, look-back for the block's first bit,
+// side table, packing into a shared word buffer and one write per word. The first and the last
+// word of a block may hold bits of the neighbouring block: those two go to head[]/tail[] and the
+// fix-up kernel merges them; every other word is written here with a plain store. A block whose
+// bits do not fit the shared buffer (very long unary runs) zeroes its interior words and ORs its
+// codewords into them.
+__global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
+    const int32_t* idx, const int64_t* d_begin, const int64_t* d_end, int64_t capacity, int64_t base,
+    int b, uint32_t* words, int64_t word_capacity, uint64_t* d_nbits, int64_t* table, int32_t chunk,
+    GState* state, uint64_t* flags, uint32_t* head, uint32_t* tail, int32_t* d_status) {
   __shared__ uint32_t wbuf[kPackWords];
   __shared__ int64_t sh[33];
-  __shared__ uint64_t span_lo, span_hi;
-  if (ctl->abort || wctl->abort) return;
-  const int64_t len = ctl->len;
-  if ((int64_t)blockIdx.x * kBlockCodes >= len) return;
-  const int32_t* x = idx + ctl->begin;
-  const int64_t jb = (int64_t)blockIdx.x * kBlockCodes;
+  __shared__ uint32_t s_vb;
+  __shared__ uint64_t s_prefix;
+  __shared__ int s_ok;
+  __shared__ uint32_t s_head, s_tail;
+  if (threadIdx.x == 0) s_vb = atomicAdd(&state->next_block, 1u);
+  int64_t lb, len;
+  const bool valid = list_bounds(d_begin, d_end, capacity, &lb, &len);
+  __syncthreads();
+  const uint32_t vb = s_vb;
+  if (!valid) {
+    if (vb == 0 && threadIdx.x == 0) {
+      raise(d_status, GSPARSE_DERR_CAPACITY);
+      *d_nbits = 0;
+    }
+    return;
+  }
+  const int64_t nact = cdiv(len, kBlockCodes);
+  if (len == 0) {
+    if (vb == 0 && threadIdx.x == 0) *d_nbits = 0;
+    return;
+  }
+  if ((int64_t)vb >= nact) return;
+  const int32_t* x = idx + lb;
+  const int64_t jb = (int64_t)vb * kBlockCodes;
   const int64_t j0 = jb + (int64_t)threadIdx.x * kPer;
   uint32_t d[kPer];
-  thread_gaps(x, len, base, j0, d, nullptr);
+  thread_gaps(x, len, base, j0, d, d_status);
   int64_t l = 0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e)
     if (j0 + e < len) l += (int64_t)(d[e] >> b) + 1 + b;
   int64_t tot;
-  const int64_t o0 = block_pre[blockIdx.x] + block_exclusive_scan(l, sh, &tot);
-  if (threadIdx.x == 0) span_lo = (uint64_t)o0;
-  if (threadIdx.x == blockDim.x - 1) span_hi = (uint64_t)(o0 + l);   // the block's last bit + 1
+  const int64_t ex = block_exclusive_scan(l, sh, &tot);
+  // publish the aggregate, then look back (warp 0)
+  if (threadIdx.x == 0) st_relaxed(flags + vb, (vb == 0 ? kFlagInc : kFlagAgg) | (uint64_t)tot);
+  if (threadIdx.x < 32) {
+    uint64_t prefix = 0;
+    const bool ok = vb == 0 ? true : lookback(flags, vb, (int)threadIdx.x, &prefix);
+    if (threadIdx.x == 0) {
+      s_ok = ok;
+      s_prefix = prefix;
+      if (ok && vb > 0) st_relaxed(flags + vb, kFlagInc | (prefix + (uint64_t)tot));
+      if (!ok) {
+        raise(d_status, GSPARSE_DERR_TIMEOUT);
+        state->abort = 1;
+      }
+    }
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  const uint64_t S = s_prefix, E = S + (uint64_t)tot;
+  const bool last = (int64_t)vb == nact - 1;
+  if (last && threadIdx.x == 0) {
+    *d_nbits = E;
+    if ((int64_t)cdiv((int64_t)E, 32) > word_capacity) raise(d_status, GSPARSE_DERR_CAPACITY);
+  }
+  const int64_t o0 = (int64_t)S + ex;
   // side table: bit offset and preceding index at every chunk start (one 32-bit division per
   // thread; indices < 2^31)
   if (table) {
@@ -211,12 +227,15 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
       if (++in_chunk == (uint32_t)chunk) in_chunk = 0;
     }
   }
-  __syncthreads();
-  const uint64_t S = span_lo, E = span_hi;
   const uint64_t wf = S >> 5, wl = (E - 1) >> 5;
-  const bool fits = wl - wf + 1 <= (uint64_t)kPackWords;
-  if (fits) {
-    for (int i = threadIdx.x; i < kPackWords; i += blockDim.x) wbuf[i] = 0u;
+  if ((int64_t)wl >= word_capacity) return;   // capacity raised by the last block
+  // the first word is shared with the block before when the block starts inside it, the last
+  // with the block after when it ends inside it (the last block's final word is its own)
+  const bool head_shared = vb > 0 && (S & 31);
+  const bool tail_shared = !last && (E & 31);
+  const uint32_t span = (uint32_t)(wl - wf + 1);
+  if (span <= (uint32_t)kPackWords) {
+    for (uint32_t i = threadIdx.x; i < span; i += blockDim.x) wbuf[i] = 0u;
     __syncthreads();
     // positions relative to the block's first word: the block spans < 2^17 bits here
     uint32_t p = (uint32_t)((uint64_t)o0 - 32u * wf);
@@ -226,39 +245,41 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
       const uint32_t q = d[e] >> b;
       const uint32_t rem = d[e] & ((1u << b) - 1u);
       // terminator 0, then the remainder most significant bit first
-      const uint32_t tail = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
+      const uint32_t tl = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
       if (q + 1u + (uint32_t)b <= 32u) {
         // the whole codeword as one pattern: at most two words
-        const uint32_t pat = (q ? 0xffffffffu >> (32u - q) : 0u) | (tail << q);
+        const uint32_t pat = (q ? 0xffffffffu >> (32u - q) : 0u) | (tl << q);
         const uint64_t v = (uint64_t)pat << (p & 31u);
         if ((uint32_t)v) atomicOr(&wbuf[p >> 5], (uint32_t)v);
         if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(p >> 5) + 1], (uint32_t)(v >> 32));
       } else {
         uint32_t pp = p, qq = q;
         while (qq) {  // the unary run of ones
-          const uint32_t sh2 = pp & 31u, nrun = qq < 32u - sh2 ? qq : 32u - sh2;
-          atomicOr(&wbuf[pp >> 5], (nrun == 32u ? 0xffffffffu : ((1u << nrun) - 1u)) << sh2);
+          const uint32_t s2 = pp & 31u, nrun = qq < 32u - s2 ? qq : 32u - s2;
+          atomicOr(&wbuf[pp >> 5], (nrun == 32u ? 0xffffffffu : ((1u << nrun) - 1u)) << s2);
           pp += nrun;
           qq -= nrun;
         }
-        const uint64_t v = (uint64_t)tail << (pp & 31u);  // terminator + remainder, <= 32 bits
+        const uint64_t v = (uint64_t)tl << (pp & 31u);  // terminator + remainder, <= 32 bits
         if ((uint32_t)v) atomicOr(&wbuf[pp >> 5], (uint32_t)v);
         if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(pp >> 5) + 1], (uint32_t)(v >> 32));
       }
       p += q + 1u + (uint32_t)b;
     }
     __syncthreads();
-    for (uint64_t w = wf + threadIdx.x; w <= wl; w += blockDim.x) {
-      const uint32_t bits = wbuf[w - wf];
-      if ((w == wf && (S & 31)) || (w == wl && (E & 31))) {
-        if (bits) atomicOr(&words[w], bits);   // shared with a neighbouring block
-      } else {
-        words[w] = bits;
-      }
+    for (uint32_t i = threadIdx.x; i < span; i += blockDim.x) {
+      const uint32_t bits = wbuf[i];
+      if (i == 0 && head_shared) head[vb] = bits;
+      else if (i == span - 1 && tail_shared) tail[vb] = bits;
+      else words[wf + i] = bits;
     }
     return;
   }
-  // long unary runs: every codeword is OR-ed straight into the zeroed stream
+  // long unary runs: interior words zeroed, then every codeword OR-ed in; the two edge words
+  // are gathered in shared memory
+  if (threadIdx.x == 0) { s_head = 0u; s_tail = 0u; }
+  for (uint64_t w = wf + 1 + threadIdx.x; w < wl; w += blockDim.x) words[w] = 0u;
+  __syncthreads();
   int64_t o = o0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
@@ -272,10 +293,33 @@ __global__ void __launch_bounds__(kCodeThreads) g_pack_kernel(const int32_t* idx
     const uint64_t w0 = c.o >> 5, w1 = (c.o + c.q + c.len_tail - 1) >> 5;
     for (uint64_t w = w0; w <= w1; ++w) {
       const uint32_t bits = code_bits_in_word(c, w);
-      if (bits) atomicOr(&words[w], bits);
+      if (!bits) continue;
+      if (w == wf) atomicOr(&s_head, bits);
+      else if (w == wl) atomicOr(&s_tail, bits);
+      else atomicOr(&words[w], bits);
     }
     o += (int64_t)c.q + c.len_tail;
   }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (head_shared) head[vb] = s_head; else words[wf] = s_head;
+    if (tail_shared) tail[vb] = s_tail; else words[wl] = s_tail;
+  }
+}
+
+// The words shared by two blocks: word (S_j >> 5) for every block j > 0 that starts inside a
+// word holds the end of block j - 1 (its tail) and the start of block j (its head).
+__global__ void g_fix_kernel(const int64_t* d_begin, const int64_t* d_end, int64_t capacity,
+                             const GState* state, const uint64_t* flags, const uint32_t* head,
+                             const uint32_t* tail, uint32_t* words, int64_t word_capacity) {
+  int64_t lb, len;
+  if (!list_bounds(d_begin, d_end, capacity, &lb, &len) || state->abort) return;
+  const int64_t nact = cdiv(len, kBlockCodes);
+  const int64_t j = 1 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= nact) return;
+  const uint64_t S = flags[j - 1] & kValMask;   // inclusive total of the blocks before j
+  const int64_t w = (int64_t)(S >> 5);
+  if ((S & 31) && w < word_capacity) words[w] = tail[j - 1] | head[j];
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -494,18 +538,24 @@ __global__ void g_decode_serial_kernel(const uint32_t* words, int64_t word_capac
 }
 
 struct GLayout {
-  GCtl* ctl;
-  GCtl* wctl;
-  int64_t* block_tot;
+  GState* state;
+  uint64_t* flags;
+  uint32_t* head;
+  uint32_t* tail;
+  int64_t nblk;
+  size_t zero_bytes;   // state and flags, cleared per call
   size_t bytes;
 };
 
 GLayout g_carve(int64_t capacity, void* ws) {
   GLayout L;
   Carver cv(ws);
-  L.ctl = cv.take<GCtl>(1);
-  L.wctl = cv.take<GCtl>(1);
-  L.block_tot = cv.take<int64_t>(cdiv(capacity, kBlockCodes) + 1);
+  L.nblk = cdiv(capacity > 0 ? capacity : 1, kBlockCodes);
+  L.state = cv.take<GState>(1);
+  L.flags = cv.take<uint64_t>(L.nblk);
+  L.zero_bytes = cv.off;
+  L.head = cv.take<uint32_t>(L.nblk);
+  L.tail = cv.take<uint32_t>(L.nblk);
   L.bytes = cv.off + 256;
   return L;
 }
@@ -535,16 +585,13 @@ int gsparse_golomb_encode(const int32_t* idx, const int64_t* d_begin, const int6
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GSPARSE_ERR_WORKSPACE;
   GLayout L = g_carve(capacity, workspace);
   if (workspace_bytes < L.bytes) return GSPARSE_ERR_WORKSPACE;
-  g_setup_kernel<<<1, 1, 0, st>>>(d_begin, d_end, capacity, L.ctl, L.wctl, d_status);
-  const unsigned nblk = (unsigned)cdiv(capacity > 0 ? capacity : 1, kBlockCodes);
-  g_len_kernel<<<nblk, kCodeThreads, 0, st>>>(idx, L.ctl, base, b, L.block_tot, d_status);
-  g_scan_blocks_kernel<<<1, kScanThreads, 0, st>>>(L.block_tot, L.ctl, word_capacity, d_nbits,
-                                                    L.wctl, d_status);
-  const int64_t zb = cdiv(word_capacity > 0 ? word_capacity : 1, 256);
-  g_zero_kernel<<<(unsigned)(zb < 148 * 16 ? zb : 148 * 16), 256, 0, st>>>(words, d_nbits,
-                                                                            word_capacity, L.ctl, L.wctl);
-  g_pack_kernel<<<nblk, kCodeThreads, 0, st>>>(idx, L.ctl, L.wctl, base, b, L.block_tot, chunk_table,
-                                               chunk, words);
+  if (cudaMemsetAsync(workspace, 0, L.zero_bytes, st) != cudaSuccess) return GSPARSE_ERR_CUDA;
+  g_encode_kernel<<<(unsigned)L.nblk, kCodeThreads, 0, st>>>(idx, d_begin, d_end, capacity, base, b, words,
+                                                             word_capacity, d_nbits, chunk_table, chunk,
+                                                             L.state, L.flags, L.head, L.tail, d_status);
+  if (L.nblk > 1)
+    g_fix_kernel<<<(unsigned)cdiv(L.nblk - 1, 256), 256, 0, st>>>(d_begin, d_end, capacity, L.state, L.flags,
+                                                                 L.head, L.tail, words, word_capacity);
   return launch_status();
 }
 

@@ -87,6 +87,88 @@ __global__ void __launch_bounds__(kLeafWarps * 32) osum_leaves_kernel(SumJob* jo
   if (job >= 0 && (int)(threadIdx.x & 31) == __ffs(same) - 1 && grp) atomicAdd(&jobs[job].count, grp);
 }
 
+// Paired leaves: jobs 2p (positive members) and 2p + 1 (negative members) of the same list. One
+// lane per 256-position block reads the block once and forms both sequential fp64 sums; leaf t of
+// the pair numbering (pair p owns leaves [jobs[2p].leaf_base, + its leaf count)) is leaf
+// t - jobs[2p].leaf_base of both jobs.
+__global__ void __launch_bounds__(kLeafWarps * 32) osum_pair_leaves_kernel(SumJob* jobs, int32_t npairs,
+                                                                           double* leaves,
+                                                                           int64_t pair_leaf_bound,
+                                                                           const int32_t* abort_flag) {
+  __shared__ float tile[kLeafWarps][32][kLeafRound + 1];
+  __shared__ const float* lptr[kLeafWarps][32];
+  __shared__ int lcnt[kLeafWarps][32];
+  if (abort_flag && *abort_flag) return;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t t = ((int64_t)blockIdx.x * kLeafWarps + wid) * 32 + lane;
+  int32_t pair = -1, cnt = 0;
+  int64_t leaf = 0;
+  const float* ptr = nullptr;
+  if (t < pair_leaf_bound) {
+    int32_t lo = 0, hi = npairs;
+    while (lo < hi) {
+      const int32_t mid = (lo + hi) >> 1;
+      if (jobs[2 * mid].leaf_base <= t) lo = mid + 1; else hi = mid;
+    }
+    pair = lo - 1;
+    if (pair >= 0) {
+      const SumJob& J = jobs[2 * pair];
+      leaf = t - J.leaf_base;
+      if (leaf < cdiv(J.len, kSumBlock)) {
+        const int64_t b = leaf * kSumBlock;
+        cnt = (int)((J.len - b) < kSumBlock ? (J.len - b) : kSumBlock);
+        ptr = J.vals + b;
+      } else {
+        pair = -1;
+      }
+    }
+  }
+  lptr[wid][lane] = ptr;
+  lcnt[wid][lane] = cnt;
+  __syncwarp();
+  double sp = 0.0, sn = 0.0;
+  uint32_t np = 0, nn = 0;
+  for (int base = 0; base < kSumBlock; base += kLeafRound) {
+    float v0[32], v1[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const float* pc = lptr[wid][c];
+      const int nc = lcnt[wid][c];
+      v0[c] = base + lane < nc ? pc[base + lane] : 0.0f;
+      v1[c] = base + 32 + lane < nc ? pc[base + 32 + lane] : 0.0f;
+    }
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      tile[wid][c][lane] = v0[c];
+      tile[wid][c][32 + lane] = v1[c];
+    }
+    __syncwarp();
+    const int m = cnt - base < kLeafRound ? cnt - base : kLeafRound;
+    for (int j = 0; j < m; ++j) {
+      const float x = tile[wid][lane][j];
+      if (x > 0.0f) { sp = __dadd_rn(sp, (double)x); ++np; }
+      else if (x < 0.0f) { sn = __dadd_rn(sn, (double)x); ++nn; }
+    }
+    __syncwarp();
+  }
+  if (pair >= 0) {
+    leaves[jobs[2 * pair].leaf_base + leaf] = sp;
+    leaves[jobs[2 * pair + 1].leaf_base + leaf] = sn;
+  }
+  // member counts: the lowest lane of each group of lanes on the same pair adds the group's total
+  const uint32_t same = __match_any_sync(kFull, pair);
+  unsigned long long gp = 0, gn = 0;
+  for (int l = 0; l < 32; ++l) {
+    const unsigned long long a = __shfl_sync(kFull, (unsigned long long)np, l);
+    const unsigned long long b = __shfl_sync(kFull, (unsigned long long)nn, l);
+    if ((same >> l) & 1u) { gp += a; gn += b; }
+  }
+  if (pair >= 0 && lane == __ffs(same) - 1) {
+    if (gp) atomicAdd(&jobs[2 * pair].count, gp);
+    if (gn) atomicAdd(&jobs[2 * pair + 1].count, gn);
+  }
+}
+
 // Pairwise reduction of m values held in a[] (shared), ping-ponging with b[]. Returns the result
 // in thread 0's view via the returned pointer's element 0 after the final barrier.
 __device__ double* tree_reduce_shared(double* a, double* b, int m) {
@@ -154,6 +236,20 @@ __global__ void __launch_bounds__(1024) osum_tree_kernel(SumJob* jobs, int32_t n
     J.mean = J.count ? __double2float_rn(__ddiv_rn(s, (double)J.count)) : 0.0f;
     J.done_blocks = 0;
   }
+}
+
+void osum_launch_pairs(SumJob* jobs, int32_t npairs, double* leaves, int64_t pair_leaf_bound,
+                       int64_t per_job_leaf_bound, double* partials, const int32_t* abort_flag,
+                       cudaStream_t s) {
+  if (npairs <= 0) return;
+  if (pair_leaf_bound > 0) {
+    const int threads = kLeafWarps * 32;
+    osum_pair_leaves_kernel<<<(unsigned)cdiv(pair_leaf_bound, threads), threads, 0, s>>>(
+        jobs, npairs, leaves, pair_leaf_bound, abort_flag);
+  }
+  const int64_t stride = osum_partial_stride(per_job_leaf_bound);
+  dim3 grid((unsigned)stride, (unsigned)(2 * npairs));
+  osum_tree_kernel<<<grid, 1024, 0, s>>>(jobs, 2 * npairs, leaves, partials, stride, abort_flag);
 }
 
 void osum_launch(SumJob* jobs, int32_t njobs, double* leaves, int64_t leaf_bound,

@@ -48,6 +48,13 @@ void osum_launch(SumJob* jobs, int32_t njobs, double* leaves, int64_t leaf_bound
                  int64_t per_job_leaf_bound, double* partials, const int32_t* abort_flag,
                  cudaStream_t s);
 
+// Paired jobs: jobs[2p] (positive members) and jobs[2p + 1] (negative members) of one list, with
+// jobs[2p].leaf_base the pair's first leaf in a numbering of pair_leaf_bound leaves and
+// jobs[2p + 1].leaf_base its own leaf range; the list is read once per pair.
+void osum_launch_pairs(SumJob* jobs, int32_t npairs, double* leaves, int64_t pair_leaf_bound,
+                       int64_t per_job_leaf_bound, double* partials, const int32_t* abort_flag,
+                       cudaStream_t s);
+
 inline int64_t osum_partial_stride(int64_t per_job_leaf_bound) {
   return cdiv(per_job_leaf_bound > 0 ? per_job_leaf_bound : 1, kTreeLeaves);
 }

@@ -94,7 +94,30 @@ struct Sel {
   int32_t* lidx;
   float* lval;
   int32_t* bsel;
+  // few problems: the select levels and the unit scan run in the last CTA of the kernel before
+  // them instead of as launches of their own
+  int32_t fuse_tail;
+  int32_t pad2;
 };
+
+// ctl words: [0] abort, [1] any redo, [2] next free pool chunk, [8 + k] done-CTA counters of the
+// kernels that end in a fused tail (k: 0 restore, 1 histogram level 2, 2 level 3, 3 count)
+constexpr int kCtlDone = 8;
+constexpr int kFuseProblems = 8;
+
+// True in every thread of the CTA that finishes the kernel last (counter ctl[kCtlDone + k]); its
+// earlier global writes and atomics, and those of all other CTAs, are then visible to it.
+__device__ __forceinline__ bool last_cta(const Sel& a, int k) {
+  __shared__ int is_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    is_last = atomicAdd(reinterpret_cast<uint32_t*>(a.ctl + kCtlDone + k), 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (is_last) __threadfence();
+  return is_last != 0;
+}
 
 struct Piece {
   int64_t lo, hi;
@@ -592,7 +615,7 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
                                             uint32_t hi, bool full, uint32_t valid,
                                             float4 (&gv)[4], float4 (&rv)[4], P1State& S,
                                             uint32_t cend, const uint32_t (&tl)[C], float* st,
-                                            uint32_t* hsink, int hstride, int lane,
+                                            uint16_t* cs, uint32_t* hsink, int hstride, int lane,
                                             const float* gs_ = nullptr, const float* us_ = nullptr) {
   float4* st4 = reinterpret_cast<float4*>(st);
   float* r = a.r;
@@ -670,38 +693,47 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
   const uint32_t tot = __shfl_sync(kFull, incl, 31);
   bool from_stage = false;
   if (tot) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = av[u];
-    __syncwarp();
     const uint32_t excl = incl - packed;
     const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu;
-    p1_reserve(a, q, t0 + t1 + t2 + (tot >> 24), S, lane);
-    uint32_t stored = 0;
+    const uint32_t ntot = t0 + t1 + t2 + (tot >> 24);
+    p1_reserve(a, q, ntot, S, lane);
+    // candidates that find a slot: ranks below `lim` (the store fills in rank order)
+    const uint32_t lim = S.room > S.count ? S.room - S.count : 0u;
+    // the chunk in shared memory (entry base + o at offset o); its candidates' offsets compacted in
+    // index order (rank r = store position - count) in the warp's staging row
+#pragma unroll
+    for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = av[u];
     for (uint32_t m = m16; m; m &= m - 1) {
       const int b = __ffs(m) - 1;
       const int u = b >> 2, e = b & 3;
       const uint32_t before = (u >= 1 ? t0 : 0u) + (u >= 2 ? t1 : 0u) + (u >= 3 ? t2 : 0u);
-      const uint32_t pos = S.count + before + ((excl >> (8 * u)) & 0xFFu) +
-                           __popc(m16 & ((1u << b) - 1u) & (0xFu << (4 * u)));
-      const float x = st[(u * 32 + lane) * 4 + e];
-      if (pos < S.room) {
+      const uint32_t r = before + ((excl >> (8 * u)) & 0xFFu) +
+                         __popc(m16 & ((1u << b) - 1u) & (0xFu << (4 * u)));
+      cs[r] = (uint16_t)(u * 128 + lane * 4 + e);
+    }
+    __syncwarp();
+    // rows to the store (consecutive ranks -> consecutive slots of the newest regions) and the
+    // histogram, one shared atomic per distinct bin of each row; stored candidates leave the
+    // residual as +0 (the not-sent ones get acc back later)
+    for (uint32_t j0 = 0; j0 < ntot; j0 += 32) {
+      const uint32_t r = j0 + (uint32_t)lane;
+      const bool in = r < ntot;
+      const uint32_t o = in ? cs[r] : 0u;
+      const float x = in ? st[o] : 0.0f;
+      const uint32_t bin = in ? (uint32_t)cand_class<C>(x) * (uint32_t)hstride + (mag_key(x) >> 20) : 0xFFFFFFFFu;
+      const uint32_t peers = __match_any_sync(kFull, bin);
+      if (in && lane == __ffs(peers) - 1) atomicAdd(hsink + bin, (uint32_t)__popc(peers));
+      if (in && r < lim) {
+        const uint32_t pos = S.count + r;
         const int64_t slot = pos >= S.ch_lo ? S.ch_base + (pos - S.ch_lo) : S.pv_base + (pos - S.pv_lo);
-        a.cidx[slot] = (int32_t)(base + u * 128 + lane * 4 + e);
+        a.cidx[slot] = (int32_t)(base + o);
         a.cval[slot] = x;
-        stored |= 1u << b;
+        if (a.zero_mode) st[o] = 0.0f;
       }
-      atomicAdd(hsink + cand_class<C>(x) * hstride + (mag_key(x) >> 20), 1u);
     }
-    S.count += t0 + t1 + t2 + (tot >> 24);
-    if (a.zero_mode) {
-      // stored candidates leave the residual as +0 (the not-sent ones get acc back later)
-      for (uint32_t m = stored; m; m &= m - 1) {
-        const int b = __ffs(m) - 1;
-        st[((b >> 2) * 32 + lane) * 4 + (b & 3)] = 0.0f;
-      }
-      __syncwarp();
-      from_stage = true;
-    }
+    from_stage = a.zero_mode != 0;
+    __syncwarp();
+    S.count += ntot;
   }
   if (full) {
 #pragma unroll
@@ -757,6 +789,7 @@ template <int C>
 __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
   __shared__ CtaHist<C, kBins1> H;
   __shared__ __align__(16) float stage[kWarps * kGranule];  // per warp: one chunk, entry order
+  __shared__ uint16_t cstage[kWarps * kGranule];            // per warp: a chunk's candidate offsets
   if (a.ctl[0]) return;
   const int64_t q0 = (int64_t)blockIdx.x * kWarps;
   H.init(a, q0);
@@ -774,6 +807,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     const int hstride = sh_sink ? kBins1 : kHist;
     const uint32_t lo = (uint32_t)P.lo, hi = (uint32_t)P.hi;  // indices are below 2^31
     float* st = stage + wid * kGranule;
+    uint16_t* cs = cstage + wid * kGranule;
     // pending residual writes of this piece start at the first index >= lo
     const uint32_t cend = pending_count(a);
     P1State S;
@@ -789,7 +823,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     float4 gv[4], rv[4];
     if (base < lo || base + (uint32_t)kGranule > hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
-      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, hsink, hstride, lane);
+      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, cs, hsink, hstride, lane);
       base += (uint32_t)kGranule;
     }
     if (base < hi && base + (uint32_t)kGranule <= hi) {
@@ -801,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
         const uint32_t nb = base + (uint32_t)kGranule;
         const bool more = nb + (uint32_t)kGranule <= hi;
         if (more) load_full(a, nb, lane, gn, rn);
-        pass1_chunk<C>(a, q, base, lo, hi, true, 0xFFFFu, gv, rv, S, cend, tl, st, hsink, hstride,
+        pass1_chunk<C>(a, q, base, lo, hi, true, 0xFFFFu, gv, rv, S, cend, tl, st, cs, hsink, hstride,
                        lane);
         base = nb;
         if (!more) break;
@@ -809,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     }
     if (base < hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
-      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, hsink, hstride, lane);
+      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, cs, hsink, hstride, lane);
     }
     if (lane == 0) {
       a.pcnt[q] = S.count;
@@ -960,8 +994,8 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
     if (base < lo || base + (uint32_t)kGranule > hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
       if (kMom) momentum_edge(a, base, valid, lane, gv);
-      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r, hsink, hstride,
-                     lane);
+      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r,
+                     reinterpret_cast<uint16_t*>(ring[0].g), hsink, hstride, lane);
       base += (uint32_t)kGranule;
     }
     // interior chunks [base, base + nint * 512) through the ring (base is 16-byte aligned)
@@ -1001,8 +1035,10 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
       parity ^= 1u << k;
       const float* us_ = nullptr;
       if constexpr (kMom) us_ = ring[k].u;
+      // the slot's g rows are read into registers first, then reused as the staging row
       pass1_chunk<C, true>(a, q, base + c * (uint32_t)kGranule, lo, hi, true, 0xFFFFu, gv, rv, S, cend,
-                           tl, ring[k].r, hsink, hstride, lane, ring[k].g, us_);
+                           tl, ring[k].r, reinterpret_cast<uint16_t*>(ring[k].g), hsink,
+                           hstride, lane, ring[k].g, us_);
     }
     if (failed) {
       if (lane == 0) {
@@ -1020,8 +1056,8 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
       if (base < hi) {
         const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
         if (kMom) momentum_edge(a, base, valid, lane, gv);
-        pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r, hsink,
-                       hstride, lane);
+        pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r,
+                       reinterpret_cast<uint16_t*>(ring[0].g), hsink, hstride, lane);
       }
     }
     if (lane == 0) {
@@ -1222,6 +1258,7 @@ __global__ void __launch_bounds__(kThreads) restore_kernel(Sel a) {
   __syncthreads();
   // only redone problems received counts here
   H.flush(a, 1, kBins1);
+  if (a.fuse_tail && last_cta(a, 0)) select_tail(a, 1, H.sh);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1247,19 +1284,18 @@ __device__ void number_units(const Sel& a, int64_t* sh) {
   if (threadIdx.x == 0) a.uoff[Qn] = total;
 }
 
-__global__ void __launch_bounds__(1024) select_kernel(Sel a, int level) {
-  __shared__ uint32_t h[kBins1];
-  __shared__ int64_t sh[33];
-  if (a.ctl[0]) return;
-  if (level == 1 && blockIdx.x == 0) number_units(a, sh);
-  const int64_t p = blockIdx.x;
+// One radix-select level of problem p by the whole CTA (any block size): the bin holding the
+// remaining rank, narrowing the prefix (levels 1-2) or fixing the threshold (level 3). h: the
+// CTA's shared scratch of kBins1 counts. The histogram is read through L2 (written by atomics of
+// other CTAs of the same or the previous kernel).
+__device__ void select_problem(const Sel& a, int64_t p, int level, uint32_t* h, int64_t* sh) {
   const int32_t s = (int32_t)(p / a.C);
-  if (level > 1 && a.pfx[p] == kNone) return;
+  if (level > 1 && a.pfx[p] == kNone) return;   // CTA-uniform
   const int B = level == 3 ? kBins3 : kBins1;
   const uint32_t* src = hist_of(a, p, level);
   int64_t mine = 0;
   for (int i = threadIdx.x; i < B; i += blockDim.x) {
-    h[i] = src[i];
+    h[i] = __ldcg(src + i);
     mine += h[i];
   }
   int64_t total;
@@ -1274,6 +1310,7 @@ __global__ void __launch_bounds__(1024) select_kernel(Sel a, int level) {
         a.thr[p] = kNone;
         a.need_eq[p] = 0;
       }
+      __syncthreads();
       return;
     }
     rank = k;
@@ -1295,6 +1332,24 @@ __global__ void __launch_bounds__(1024) select_kernel(Sel a, int level) {
       a.need_eq[p] = rank - above;
     }
   }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(1024) select_kernel(Sel a, int level) {
+  __shared__ uint32_t h[kBins1];
+  __shared__ int64_t sh[33];
+  if (a.ctl[0]) return;
+  if (level == 1 && blockIdx.x == 0) number_units(a, sh);
+  select_problem(a, blockIdx.x, level, h, sh);
+}
+
+// The fused tail of a kernel that ran with a.fuse_tail: every problem's select at this level (and
+// before level 1, the numbering of the work units), in the last CTA to finish.
+__device__ void select_tail(const Sel& a, int level, uint32_t* h) {
+  __shared__ int64_t sh[33];
+  if (level == 1) number_units(a, sh);
+  __syncthreads();
+  for (int64_t p = 0; p < (int64_t)a.T * a.C; ++p) select_problem(a, p, level, h, sh);
 }
 
 template <int C>
@@ -1304,8 +1359,7 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(Sel a, int level) {
   if (a.ctl[0]) return;
   const int64_t U = unit_count(a);
   const int64_t u0 = (int64_t)blockIdx.x * kWarps;
-  if (u0 >= U) return;
-  H.init_seg(piece_of(a, unit_piece(a, u0)).s);
+  H.init_seg(u0 < U ? piece_of(a, unit_piece(a, u0)).s : -1);
   __syncthreads();
   for (int64_t u = u0 + (threadIdx.x >> 5); u < U; u += (int64_t)gridDim.x * kWarps) {
     const int64_t q = unit_piece(a, u);
@@ -1325,10 +1379,13 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(Sel a, int level) {
   }
   __syncthreads();
   H.flush(a, level, level == 2 ? kBins2 : kBins3);
+  if (a.fuse_tail && last_cta(a, level - 1)) select_tail(a, level, H.sh);
 }
 
 // ------------------------------------------------------------------------------------------
 // 8. count + scan
+
+__device__ void scan_problem(const Sel& a, int64_t p, int64_t* sh);
 
 template <int C>
 __global__ void __launch_bounds__(kThreads) count_kernel(Sel a) {
@@ -1365,12 +1422,19 @@ __global__ void __launch_bounds__(kThreads) count_kernel(Sel a) {
       }
     }
   }
+  if (a.fuse_tail && last_cta(a, 3)) {
+    __shared__ int64_t sh[33];
+    for (int64_t p = 0; p < (int64_t)a.T * a.C; ++p) {
+      scan_problem(a, p, sh);
+      __syncthreads();
+    }
+  }
 }
 
-__global__ void __launch_bounds__(1024) scan_kernel(Sel a) {
-  __shared__ int64_t sh[33];
-  if (a.ctl[0]) return;
-  const int64_t p = blockIdx.x;
+// Offsets of every work unit's selected entries within problem p's output, and how many keys
+// equal to the threshold it takes (the first need_eq of them in unit order), by the whole CTA.
+// The per-unit counts are read through L2.
+__device__ void scan_problem(const Sel& a, int64_t p, int64_t* sh) {
   const int32_t s = (int32_t)(p / a.C);
   const int c = (int)(p % a.C);
   // the work units of segment s, in index order; thread t owns a contiguous run of them
@@ -1380,52 +1444,65 @@ __global__ void __launch_bounds__(1024) scan_kernel(Sel a) {
   const int64_t u_lo = first + threadIdx.x * per < last ? first + threadIdx.x * per : last;
   const int64_t u_hi = u_lo + per < last ? u_lo + per : last;
   int64_t eq_mine = 0;
-  for (int64_t u = u_lo; u < u_hi; ++u) eq_mine += a.peq[u * a.C + c];
+  for (int64_t u = u_lo; u < u_hi; ++u) eq_mine += __ldcg(a.peq + u * a.C + c);
   int64_t teq;
   int64_t eq_before = block_exclusive_scan(eq_mine, sh, &teq);
   // keys equal to the threshold: the first `need` of them in unit order are taken
   int64_t sel_mine = 0;
   for (int64_t u = u_lo; u < u_hi; ++u) {
-    const int64_t eq = a.peq[u * a.C + c];
+    const int64_t eq = __ldcg(a.peq + u * a.C + c);
     int64_t take = need - eq_before;
     take = take < 0 ? 0 : (take > eq ? eq : take);
-    sel_mine += a.pgt[u * a.C + c] + take;
+    sel_mine += __ldcg(a.pgt + u * a.C + c) + take;
     eq_before += eq;
   }
   int64_t tsel;
   int64_t sel_before = block_exclusive_scan(sel_mine, sh, &tsel);
   eq_before -= eq_mine;
   for (int64_t u = u_lo; u < u_hi; ++u) {
-    const int64_t eq = a.peq[u * a.C + c];
+    const int64_t eq = __ldcg(a.peq + u * a.C + c);
     int64_t take = need - eq_before;
     take = take < 0 ? 0 : (take > eq ? eq : take);
     a.poff[u * a.C + c] = sel_before;
     a.ptake[u * a.C + c] = (uint32_t)take;
-    sel_before += a.pgt[u * a.C + c] + take;
+    sel_before += __ldcg(a.pgt + u * a.C + c) + take;
     eq_before += eq;
   }
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(Sel a) {
+  __shared__ int64_t sh[33];
+  if (a.ctl[0]) return;
+  scan_problem(a, blockIdx.x, sh);
 }
 
 // ------------------------------------------------------------------------------------------
 // 9. emit, in index order
 
+// A warp's staging rows for the ordered output: the selected entries of 128 candidates, compacted.
+struct EmitStage {
+  int32_t idx[128];
+  float val[128];
+};
+
 template <int C>
 __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_idx, float* out_val,
-                                          int64_t limit);
+                                          int64_t limit, EmitStage& stg);
 
 template <int C>
 __global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
                                                         int64_t limit) {
+  __shared__ EmitStage stage[kWarps];
   if (a.ctl[0]) return;
   const int64_t U = unit_count(a);
   for (int64_t u = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); u < U;
        u += (int64_t)gridDim.x * kWarps)
-    emit_unit<C>(a, u, out_idx, out_val, limit);
+    emit_unit<C>(a, u, out_idx, out_val, limit, stage[threadIdx.x >> 5]);
 }
 
 template <int C>
 __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_idx, float* out_val,
-                                          int64_t limit) {
+                                          int64_t limit, EmitStage& stg) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = lanemask_lt();
   const int64_t q = unit_piece(a, u);
@@ -1508,20 +1585,26 @@ __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_
         }
         uint32_t tsel;
         const uint32_t pre_sel = warp_prefix_small(__popc(sm), &tsel);
-        if (sm) {
-          const int64_t o0 = base_out[cc] + sel_run[cc] + pre_sel;
+        if (tsel) {
+          // the selected entries of these 128 candidates, compacted in index order, leave as one
+          // contiguous run of output positions (coalesced rows)
+          uint32_t k = pre_sel;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if ((sm >> e) & 1u) {
-              const int64_t o = o0 + __popc(sm & ((1u << e) - 1u));
-              if (o >= limit) raise(a.d_status, GSPARSE_DERR_CAPACITY);
-              else if (C == 1) {
-                out_idx[o] = iv[e];
-                out_val[o] = xv[e];
-                if (a.u) a.u[iv[e]] = 0.0f;  // momentum masking of the sent entry
-              } else { a.lidx[o] = iv[e]; a.lval[o] = xv[e]; }
-            }
+          for (int e = 0; e < 4; ++e)
+            if ((sm >> e) & 1u) { stg.idx[k] = iv[e]; stg.val[k] = xv[e]; ++k; }
+          __syncwarp();
+          const int64_t o0 = base_out[cc] + sel_run[cc];
+          int32_t* oi = C == 1 ? out_idx : a.lidx;
+          float* ov = C == 1 ? out_val : a.lval;
+          for (uint32_t t = (uint32_t)lane; t < tsel; t += 32) {
+            const int64_t o = o0 + t;
+            const int32_t i = stg.idx[t];
+            if (o >= limit) { raise(a.d_status, GSPARSE_DERR_CAPACITY); continue; }
+            oi[o] = i;
+            ov[o] = stg.val[t];
+            if (C == 1 && a.u) a.u[i] = 0.0f;  // momentum masking of the sent entry
           }
+          __syncwarp();
         }
         sel_run[cc] += tsel;
         selm |= sm;
@@ -1675,30 +1758,32 @@ __global__ void bemit_kernel(Sel a, const float* d_mean, const int64_t* out_offs
 
 constexpr int kMagBlock = 1024;  // list positions per compaction block (4 per thread)
 
+// Two sum jobs per segment over the members of S: positive (job 2s) and negative (job 2s + 1),
+// summed as a pair (the list is read once): the pair's leaves are leaves [pb_s, pb_s + L_s) of the
+// positive job and [pair_bound + pb_s, ...) of the negative job.
 __global__ void __launch_bounds__(1024) mjobs_kernel(const float* lval, const int64_t* loff, int32_t T,
-                                                     SumJob* jobs, const int32_t* abort_flag) {
+                                                     int64_t pair_bound, SumJob* jobs,
+                                                     const int32_t* abort_flag) {
   __shared__ int64_t sh[33];
   if (*abort_flag) return;
-  const int64_t P = (int64_t)T * 2;
   int64_t carry = 0;
-  for (int64_t base = 0; base < P; base += blockDim.x) {
-    const int64_t p = base + threadIdx.x;
-    const int64_t s = p >> 1;
-    const int64_t len = p < P ? loff[s + 1] - loff[s] : 0;
+  for (int64_t base = 0; base < (int64_t)T; base += blockDim.x) {
+    const int64_t s = base + threadIdx.x;
+    const int64_t len = s < T ? loff[s + 1] - loff[s] : 0;
     int64_t tot;
     const int64_t ex = block_exclusive_scan(cdiv(len, kSumBlock), sh, &tot);
-    if (p < P) {
+    for (int c = 0; c < 2 && s < T; ++c) {
       SumJob J;
       J.vals = lval + loff[s];
       J.len = len;
-      J.mode = (p & 1) ? kSumNegative : kSumPositive;
+      J.mode = c ? kSumNegative : kSumPositive;
       J.pad = 0;
-      J.leaf_base = carry + ex;
+      J.leaf_base = carry + ex + (c ? pair_bound : 0);
       J.count = 0;
       J.sum = 0.0;
       J.mean = 0.0f;
       J.done_blocks = 0;
-      jobs[p] = J;
+      jobs[2 * s + c] = J;
     }
     carry += tot;
   }
@@ -2072,18 +2157,21 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   }
   if (timed) cudaEventRecord((cudaEvent_t)events->after, st);
   check_kernel<<<(unsigned)(T * C), 256, 0, st>>>(a);
-  if (piece_ctas) restore_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
-  select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 1);
   // the steps after pass 1 run over work units, at most a.units_bound of them
   int64_t uc = cdiv(a.units_bound, kWarps);
   if (uc > (int64_t)sm_count() * 8) uc = (int64_t)sm_count() * 8;
   const unsigned unit_ctas = piece_ctas ? (unsigned)uc : 0u;
+  // with few problems each select level (and the scan) runs as the tail of the kernel before it
+  const bool fuse = piece_ctas && (int64_t)T * C <= kFuseProblems;
+  a.fuse_tail = fuse ? 1 : 0;
+  if (piece_ctas) restore_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
+  if (!fuse) select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 1);
   if (unit_ctas) hist_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a, 2);
-  select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 2);
+  if (!fuse) select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 2);
   if (unit_ctas) hist_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a, 3);
-  select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 3);
+  if (!fuse) select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 3);
   if (unit_ctas) count_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a);
-  scan_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a);
+  if (!fuse) scan_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a);
   if (unit_ctas)
     emit_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a, out_idx, out_val,
                                                     C == 1 ? out_capacity : 2 * L.kbound);
@@ -2121,9 +2209,9 @@ MagLayout mag_carve(int64_t n, int32_t T, int64_t num, int64_t den, void* ws) {
   M.lval = cv.take<float>(M.kb);
   M.loff = cv.take<int64_t>((int64_t)T + 1);
   M.per_job = cdiv(M.kb, kSumBlock);
-  M.leaf_bound = 2 * (M.per_job + T);
+  M.leaf_bound = M.per_job + T;   // leaves of the pair numbering (each sign has this many)
   M.jobs = cv.take<SumJob>(2 * (int64_t)T);
-  M.leaves = cv.take<double>(M.leaf_bound);
+  M.leaves = cv.take<double>(2 * M.leaf_bound);
   M.partials = cv.take<double>(2 * (int64_t)T * osum_partial_stride(M.per_job));
   M.bsel = cv.take<int32_t>(T);
   M.nblk = cdiv(M.kb > 0 ? M.kb : 1, kMagBlock);
@@ -2153,8 +2241,8 @@ int run_binarize_magnitude(const float* g, float* r, int64_t n, const int64_t* s
                                flags & GSPARSE_SELECT_EXHAUSTIVE, tws, tws_bytes, d_status, st, events);
   if (rc != GSPARSE_OK) return rc;
   const int32_t* abort_flag = carve(n, T, 1, num, den, tws, tws_bytes, false).a.ctl;
-  mjobs_kernel<<<1, 1024, 0, st>>>(M.lval, M.loff, T, M.jobs, abort_flag);
-  osum_launch(M.jobs, 2 * T, M.leaves, M.leaf_bound, M.per_job, M.partials, abort_flag, st);
+  mjobs_kernel<<<1, 1024, 0, st>>>(M.lval, M.loff, T, M.leaf_bound, M.jobs, abort_flag);
+  osum_launch_pairs(M.jobs, T, M.leaves, M.leaf_bound, M.per_job, M.partials, abort_flag, st);
   mchoose_kernel<<<1, 1024, 0, st>>>(M.jobs, T, M.bsel, d_mean, out_offsets, abort_flag);
   if (M.kb > 0) {
     mcount_kernel<<<(unsigned)M.nblk, 256, 0, st>>>(M.bsel, M.loff, T, M.lval, M.bcnt, abort_flag);

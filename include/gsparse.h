@@ -253,6 +253,22 @@ int gsparse_quantize(const int32_t* idx, float* val, const int64_t* d_begin, con
                      void* workspace, size_t workspace_bytes, int32_t* d_status,
                      gsparse_stream stream);
 
+/* Segmented 2-bit quantisation: the sub-lists [off[s], off[s+1]) of idx/val for s = 0..T-1
+ * (off = d_offsets, device int64[T+1], ascending, 0 <= off[0], off[T] <= capacity; e.g. the
+ * out_offsets of a per-tensor gsparse_residual_topk) are quantised as by gsparse_quantize with
+ * d_begin = &off[s] and d_end = &off[s+1], each with its own two means, in one call:
+ * d_means     fp32[2T] device: {m+_s, m-_s} for each segment s.
+ * sign_bits, feedback_out   positions counted from off[0] (bit (j % 32) of word j / 32 is the
+ *             sign of entry off[0] + j); residual, write_dequantized as for gsparse_quantize.
+ * Offsets that are not ascending within [0, capacity] raise GSPARSE_DERR_CAPACITY and nothing is
+ * written. */
+size_t gsparse_quantize_segments_workspace_size(int64_t capacity, int32_t num_segments);
+int gsparse_quantize_segments(const int32_t* idx, float* val, const int64_t* d_offsets,
+                              int32_t num_segments, int64_t capacity, float* residual, int64_t n,
+                              float* feedback_out, uint32_t* sign_bits, float* d_means,
+                              int32_t write_dequantized, void* workspace, size_t workspace_bytes,
+                              int32_t* d_status, gsparse_stream stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Sparse binarisation  (Sattler et al. §II Sparse Binarization)
  *

@@ -93,24 +93,35 @@ def test_config2_mlp_50_steps_4_workers(mode, quantise):
         lists, keepalive = [], []
         for w in range(W):
             idx, val, off = gs.residual_topk(dev(grads[w]), r_dev[w], keep, seg_offsets=seg_d, d_status=st)
-            if quantise:
+            segmented = quantise and step % 2 == 1   # odd steps: all tensors in one call
+            if quantise and not segmented:
                 qparts = []
                 for s in range(T):
                     sb, mm = gs.quantize(idx, val, off[s + 1:s + 2], d_begin=off[s:s + 1], residual=r_dev[w],
                                          write_dequantized=True, d_status=st, capacity=idx.numel())
                     qparts.append((sb, mm))
+            elif segmented:
+                sb_all, mm_all = gs.quantize_segments(idx, val, off, residual=r_dev[w], write_dequantized=True,
+                                                      d_status=st, capacity=idx.numel())
             oi, ov, oo, parts = want[w]
             K = int(oo[-1])
             assert np.array_equal(host(off), oo), (step, w)
             assert np.array_equal(host(idx)[:K], oi), (step, w)
             assert np.array_equal(bits(host(val)[:K]), bits(ov)), (step, w)
             assert np.array_equal(bits(host(r_dev[w])), bits(r_host[w])), (step, w)
-            if quantise:
+            if quantise and not segmented:
                 for s in range(T):
                     sb, mm = qparts[s]
                     wb, wm = parts[s]
                     assert np.array_equal(bits(host(mm)), bits(wm))
                     assert np.array_equal(host(sb)[:wb.size].view(np.uint32), wb)
+            elif segmented:
+                wm_all = np.concatenate([parts[s][1] for s in range(T)])
+                assert np.array_equal(bits(host(mm_all)), bits(wm_all))
+                neg = np.zeros(((K + 31) // 32) * 32, bool)
+                neg[:K] = ov < 0
+                want_words = np.packbits(neg.reshape(-1, 32)[:, ::-1], axis=1).view(">u4").ravel().astype(np.uint32)
+                assert np.array_equal(host(sb_all)[:want_words.size].view(np.uint32), want_words)
             cnt = off[T:T + 1]
             lists.append(gs.make_list(idx, cnt, val=val))
             keepalive.append((idx, val, off))

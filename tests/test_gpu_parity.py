@@ -652,3 +652,57 @@ def test_pending_writes_must_be_ascending():
                      pending=gs.make_pending(pidx, pval, torch.tensor([3], device="cuda")))
     assert int(host(st)[0]) & gs.DERR_INDEX_RANGE
     assert bool((r == 0).all())                       # nothing written
+
+
+# ------------------------------------------------------------------- segmented quantisation
+
+@pytest.mark.parametrize("layout", [[1000], [37, 0, 5000, 256, 1, 70001], [0], [300, 0, 0]])
+def test_quantize_segments_parity(layout):
+    # one call over T sub-lists equals T separate quantisations of the oracle, each with its own
+    # two means; sign bits and feedback over positions from the first offset
+    off = np.concatenate([[0], np.cumsum(layout)]).astype(np.int64)
+    K = int(off[-1])
+    n = max(3 * K, 1)
+    gen = np.random.default_rng(K + len(layout))
+    idx = np.sort(gen.choice(n, K, replace=False)).astype(np.int32)
+    val = synth.gaussian(K, K + 7, sigma=1e-2)
+    if K > 20:
+        val[::17] = 0.0
+        val[3::19] = -0.0
+    res = synth.gaussian(n, 9, sigma=1e-4)
+    want_res = res.copy()
+    want_val = val.copy()
+    want_bits = np.zeros(max((K + 31) // 32, 1), np.uint32)
+    want_means = np.zeros(2 * len(layout), np.float32)
+    for s in range(len(layout)):
+        b, e = int(off[s]), int(off[s + 1])
+        wb, wm, wv, want_res = oracle.quantize(idx[b:e], val[b:e], residual=want_res, write_dequantized=True)
+        want_val[b:e] = wv
+        want_means[2 * s:2 * s + 2] = wm
+        for j in range(b, e):
+            if val[j] < 0:
+                want_bits[j // 32] |= np.uint32(1 << (j % 32))
+    vd, rd = dev(val), dev(res)
+    fb = torch.zeros(max(K, 1), device="cuda")
+    st = gs.status_tensor()
+    sb, means = gs.quantize_segments(dev(idx), vd, dev(off), residual=rd, write_dequantized=True, feedback_out=fb,
+                                     d_status=st, capacity=K)
+    assert int(host(st)[0]) == 0
+    assert np.array_equal(bits(host(means)), bits(want_means))
+    assert np.array_equal(host(sb)[:(K + 31) // 32].view(np.uint32), want_bits[:(K + 31) // 32])
+    assert np.array_equal(bits(host(vd)), bits(want_val))
+    assert np.array_equal(bits(host(rd)), bits(want_res))
+    # the feedback list holds the same errors the residual received
+    got_fb = host(fb)[:K]
+    assert np.array_equal(bits(got_fb), bits(want_res[idx])) if K else True
+
+
+def test_quantize_segments_bad_offsets_flagged():
+    idx = dev(np.arange(100, dtype=np.int32))
+    val = dev(synth.gaussian(100, 1))
+    st = gs.status_tensor()
+    gs.quantize_segments(idx, val, dev(np.array([0, 60, 40, 100], np.int64)), d_status=st, capacity=100)
+    assert int(host(st)[0]) & gs.DERR_CAPACITY
+    st = gs.status_tensor()
+    gs.quantize_segments(idx, val, dev(np.array([0, 101], np.int64)), d_status=st, capacity=100)
+    assert int(host(st)[0]) & gs.DERR_CAPACITY
