@@ -406,52 +406,84 @@ __device__ __forceinline__ bool decode_one_local_slow(const uint32_t* sw, uint32
   return true;
 }
 
-// Decodes `count` codewords from a staged window: sw holds stream words [wa, wa + nwin) (the last
-// two are zero spares), t is the bit position relative to bit 32 * wa, and nb_rel the stream end
-// relative to the same origin (at most 32 * (nwin - 2)). 32-bit positions throughout. A codeword
-// of at most 64 bits (all but pathological gaps) is taken from one 64-bit window: the run of ones
-// ends at the first zero bit, the remainder follows it in the same window.
-__device__ bool decode_run_local(const uint32_t* sw, uint32_t nb_rel, uint32_t& t, int64_t& prev,
-                                 int count, int b, int64_t n_limit, int32_t* out, int stride,
-                                 int32_t* d_status) {
+// Decodes `count` codewords of one chunk from a staged window with a 64-bit register bit buffer:
+// sw holds stream words [wa, ...) (two zero spares past the window), t0 is the chunk's first bit
+// relative to bit 32 * wa and nb_rel the window's end. The buffer holds `avail` unread bits, LSB
+// first, and takes the next stream word whenever 32 or fewer remain, so one codeword of up to
+// 33 - b bits needs no refill; a longer one is finished word by word from the window. Outputs go
+// out four at a time when the chunk's output row is 16-byte aligned. Returns false (and raises)
+// on a corrupt stream; on success t0 is the bit after the last codeword.
+__device__ bool decode_chunk_buffered(const uint32_t* sw, uint32_t nb_rel, uint32_t& t0, int64_t& prev,
+                                      int count, int b, int64_t n_limit, int32_t* out, int32_t* d_status) {
   const uint32_t mask = b > 0 ? 0xffffffffu >> (32 - b) : 0u;
+  uint32_t wi = t0 >> 5;                      // next word to take into the buffer
+  const uint32_t s0 = t0 & 31u;
+  uint64_t buf = ((uint64_t)sw[wi] | ((uint64_t)sw[wi + 1] << 32)) >> s0;
+  uint32_t avail = 64u - s0;
+  wi += 2;
+  const bool vec = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+  int4 ov = make_int4(0, 0, 0, 0);
   for (int k = 0; k < count; ++k) {
-    if (t >= nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
-    const uint32_t w = t >> 5, s = t & 31u;
-    uint64_t win = ((uint64_t)sw[w] | ((uint64_t)sw[w + 1] << 32)) >> s;
-    if (s) win |= (uint64_t)sw[w + 2] << (64u - s);
+    if (avail <= 32u) {
+      buf |= (uint64_t)sw[wi] << avail;
+      avail += 32u;
+      ++wi;
+    }
+    const uint32_t pos = 32u * wi - avail;    // relative bit of this codeword
+    if (pos >= nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+    const uint64_t nz = ~buf;
+    const uint32_t z = nz ? (uint32_t)__ffsll((long long)nz) - 1u : 64u;   // ones before the first zero
     uint32_t q, rem = 0;
-    const uint64_t zeros = ~win;
-    const uint32_t z = zeros ? (uint32_t)__ffsll((long long)zeros) - 1u : 64u;
-    if (z + 1u + (uint32_t)b <= 64u) {
+    if (z + 1u + (uint32_t)b <= avail) {
       q = z;
-      if (b > 0) rem = __brev((uint32_t)(win >> (z + 1u)) & mask) >> (32 - b);
-      t += z + 1u + (uint32_t)b;
-      if (t > nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
-    } else if (!decode_one_local_slow(sw, nb_rel, t, q, rem, b, d_status)) {
-      return false;
+      if (b > 0) rem = __brev((uint32_t)(buf >> (z + 1u)) & mask) >> (32 - b);
+      const uint32_t used = z + 1u + (uint32_t)b;
+      buf = used == 64u ? 0ull : buf >> used;
+      avail -= used;
+      if (32u * wi - avail > nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+    } else {
+      // a long unary run: finish this codeword from the window, then restart the buffer after it
+      uint32_t t = pos;
+      if (!decode_one_local_slow(sw, nb_rel, t, q, rem, b, d_status)) return false;
+      wi = t >> 5;
+      const uint32_t s = t & 31u;
+      buf = ((uint64_t)sw[wi] | ((uint64_t)sw[wi + 1] << 32)) >> s;
+      avail = 64u - s;
+      wi += 2;
     }
     const int64_t i = prev + 1 + (int64_t)(((uint64_t)q << b) | rem);
     if (i >= n_limit || i > INT32_MAX) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); return false; }
-    out[k * stride] = (int32_t)i;
     prev = i;
+    if (vec) {
+      const int e = k & 3;
+      if (e == 0) ov.x = (int32_t)i; else if (e == 1) ov.y = (int32_t)i; else if (e == 2) ov.z = (int32_t)i;
+      else ov.w = (int32_t)i;
+      if (e == 3) *reinterpret_cast<int4*>(out + k - 3) = ov;
+    } else {
+      out[k] = (int32_t)i;
+    }
   }
+  if (vec) {
+    const int e = count & 3;   // the last partial group of four
+    if (e > 0) out[count - e] = ov.x;
+    if (e > 1) out[count - e + 1] = ov.y;
+    if (e > 2) out[count - e + 2] = ov.z;
+  }
+  t0 = 32u * wi - avail;
   return true;
 }
 
 // One thread per chunk of codewords, kDecThreads chunks per CTA. The CTA's stream words (a
-// contiguous bit range given by the side table) are staged in shared memory when they fit, and
-// decoded there with 32-bit positions; otherwise the thread reads global memory.
-constexpr int kDecThreads = 64;
-constexpr int kDecWords = 2048;   // 64 Kbit of staged stream per CTA
-constexpr int kDecMaxChunk = 64;  // outputs staged when the chunk is at most this long
+// contiguous bit range given by the side table) are staged in shared memory when they fit and
+// decoded there through a register bit buffer; otherwise the thread reads global memory.
+constexpr int kDecThreads = 128;
+constexpr int kDecWords = 4096;   // 128 Kbit of staged stream per CTA
 
 __global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
     const uint32_t* words, int64_t word_capacity, const uint64_t* d_nbits, const int64_t* d_count,
     int64_t capacity, int b, const int64_t* table, int32_t chunk, int64_t n_limit, int32_t* out,
     int32_t* d_status) {
   __shared__ uint32_t sw[kDecWords];
-  __shared__ int32_t so[kDecMaxChunk * (kDecThreads + 1)];  // [codeword][chunk], padded
   const int64_t K = *d_count;
   if (K < 0 || K > capacity) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise(d_status, GSPARSE_DERR_CAPACITY);
@@ -473,52 +505,36 @@ __global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
   ba = ba < nbits ? ba : nbits;
   bz = bz < nbits ? (bz > ba ? bz : ba) : nbits;
   const int64_t nw = cdiv((int64_t)nbits, 32);
-  const int64_t wa = (int64_t)(ba >> 5), wz = cdiv((int64_t)bz, 32) + 2;   // two zero spare words
+  const int64_t wa = (int64_t)(ba >> 5), wz = cdiv((int64_t)bz, 32) + 3;   // three zero spare words
   const bool staged = wz - wa <= kDecWords;
   if (staged) {
     const int span = (int)(wz - wa);
-#pragma unroll 4
     for (int k = threadIdx.x; k < span; k += kDecThreads) sw[k] = wa + k < nw ? words[wa + k] : 0u;
     __syncthreads();
   }
-  // outputs go through shared memory when staged, so they leave as whole rows (coalesced)
-  const bool stage_out = staged && chunk <= kDecMaxChunk;
-  if (c < nch) {
-    uint64_t t = (uint64_t)table[2 * c];
-    int64_t prev = table[2 * c + 1];
-    const int64_t first = c * chunk;
-    const int count = (int)((K - first) < chunk ? (K - first) : chunk);
-    if (t > nbits || (staged && (t < ba || t > bz))) {
-      raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);   // the side table does not fit the stream
-    } else {
-      bool ok;
-      if (staged) {
-        // the window's end: this CTA's range, so a chunk cannot run into the next CTA's bits
-        uint32_t tl = (uint32_t)(t - 32u * (uint64_t)wa);
-        const uint32_t nb_rel = (uint32_t)(bz - 32u * (uint64_t)wa);
-        if (stage_out)
-          ok = decode_run_local(sw, nb_rel, tl, prev, count, b, n_limit, so + threadIdx.x,
-                               kDecThreads + 1, d_status);
-        else
-          ok = decode_run_local(sw, nb_rel, tl, prev, count, b, n_limit, out + first, 1, d_status);
-        t = 32u * (uint64_t)wa + tl;
-      } else {
-        ok = decode_run(words, 0, nw, nbits, t, prev, count, b, n_limit, out + first, d_status);
-      }
-      if (ok) {
-        const bool last = c + 1 == nch;
-        const uint64_t end = last ? nbits : (uint64_t)table[2 * (c + 1)];
-        if (t != end || (!last && prev != table[2 * (c + 1) + 1])) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
-      }
-    }
+  if (c >= nch) return;
+  uint64_t t = (uint64_t)table[2 * c];
+  int64_t prev = table[2 * c + 1];
+  const int64_t first = c * chunk;
+  const int count = (int)((K - first) < chunk ? (K - first) : chunk);
+  if (t > nbits || (staged && (t < ba || t > bz))) {
+    raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);   // the side table does not fit the stream
+    return;
   }
-  if (stage_out) {
-    __syncthreads();
-    for (int cc = 0; cc < (int)(c1 - c0); ++cc) {
-      const int64_t first = (c0 + cc) * chunk;
-      const int cnt = (int)((K - first) < chunk ? (K - first) : chunk);
-      if ((int)threadIdx.x < cnt) out[first + threadIdx.x] = so[threadIdx.x * (kDecThreads + 1) + cc];
-    }
+  bool ok;
+  if (staged) {
+    // the window's end: this CTA's range, so a chunk cannot run into the next CTA's bits
+    uint32_t tl = (uint32_t)(t - 32u * (uint64_t)wa);
+    const uint32_t nb_rel = (uint32_t)(bz - 32u * (uint64_t)wa);
+    ok = decode_chunk_buffered(sw, nb_rel, tl, prev, count, b, n_limit, out + first, d_status);
+    t = 32u * (uint64_t)wa + tl;
+  } else {
+    ok = decode_run(words, 0, nw, nbits, t, prev, count, b, n_limit, out + first, d_status);
+  }
+  if (ok) {
+    const bool last = c + 1 == nch;
+    const uint64_t end = last ? nbits : (uint64_t)table[2 * (c + 1)];
+    if (t != end || (!last && prev != table[2 * (c + 1) + 1])) raise(d_status, GSPARSE_DERR_CORRUPT_STREAM);
   }
 }
 

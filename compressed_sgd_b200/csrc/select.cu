@@ -85,6 +85,7 @@ struct Sel {
   // pending residual writes applied in the sample and pass 1 (null: none); pstart[q] is the
   // first write at or after piece q's first entry ([Q + 1])
   uint32_t* pstart;
+  uint32_t* srun;   // [T][kSampleRuns][2]: each sampled run's range of pending writes (level 1 -> 2)
   const int32_t* pw_idx;
   const float* pw_val;
   const int64_t* pw_count;
@@ -438,10 +439,18 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
     const int64_t jr = j0 + 32 * threadIdx.x;       // j0 is a multiple of 32 here
     uint32_t b = 0, e = 0;
     if (jr < j1) {
-      const int64_t start = sample_pos(lo, ns, jr);
-      b = pending_lower_bound(a, start);
-      const uint32_t span = pc - b < 33u ? pc - b : 33u;
-      e = b + (uint32_t)lower_bound_i32(a.pw_idx + b, span, start + 32);
+      uint32_t* rr = a.srun + 2 * ((int64_t)s * kSampleRuns + (jr >> 5));
+      if (level == 1) {
+        const int64_t start = sample_pos(lo, ns, jr);
+        b = pending_lower_bound(a, start);
+        const uint32_t span = pc - b < 33u ? pc - b : 33u;
+        e = b + (uint32_t)lower_bound_i32(a.pw_idx + b, span, start + 32);
+        rr[0] = b;
+        rr[1] = e;
+      } else {
+        b = rr[0];   // found by level 1 (same runs, same CTA split)
+        e = rr[1];
+      }
     }
     run_b[threadIdx.x] = b;
     run_e[threadIdx.x] = e;
@@ -1991,6 +2000,7 @@ Layout carve(int64_t n, int32_t T, int32_t C, int64_t num, int64_t den, void* ws
   a.need_eq = cv.take<int64_t>(P);
   a.uoff = cv.take<int64_t>(L.Q + 1);
   a.pstart = cv.take<uint32_t>(L.Q + 1);
+  a.srun = cv.take<uint32_t>((int64_t)T * kSampleRuns * 2);
   // work units: a stored piece holds at most as many candidates as entries, so at most
   // n / 2^kUnitShift + Q units; a re-read piece at most kReadUnits
   a.Ur = round_up(cdiv(L.Lp, kReadUnits), 128);
