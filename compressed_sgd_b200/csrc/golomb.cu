@@ -139,17 +139,18 @@ __device__ bool lookback(const uint64_t* flags, uint32_t vb, int lane, uint64_t*
   return true;
 }
 
-// One pass: codeword lengths and the block's bit count, look-back for the block's first bit,
-// side table, packing into a shared word buffer and one write per word. The first and the last
-// word of a block may hold bits of the neighbouring block: those two go to head[]/tail[] and the
-// fix-up kernel merges them; every other word is written here with a plain store. A block whose
-// bits do not fit the shared buffer (very long unary runs) zeroes its interior words and ORs its
-// codewords into them.
+// One pass: codeword lengths and the block's bit count (published at once), packing into a shared
+// word buffer relative to the block's own first bit, then the look-back for that bit's stream
+// position (by warp 0, after the packing, so the blocks before have had time to publish) and one
+// write per word, shifted into place with a funnel shift. The first and the last word of a block
+// may hold bits of the neighbouring block: those two go to head[]/tail[] and the fix-up kernel
+// merges them. A block whose bits do not fit the shared buffer (very long unary runs) looks back
+// first, zeroes its interior words and ORs its codewords into them.
 __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
     const int32_t* idx, const int64_t* d_begin, const int64_t* d_end, int64_t capacity, int64_t base,
     int b, uint32_t* words, int64_t word_capacity, uint64_t* d_nbits, int64_t* table, int32_t chunk,
     GState* state, uint64_t* flags, uint32_t* head, uint32_t* tail, int32_t* d_status) {
-  __shared__ uint32_t wbuf[kPackWords];
+  __shared__ uint32_t wbuf[kPackWords + 1];
   __shared__ int64_t sh[33];
   __shared__ uint32_t s_vb;
   __shared__ uint64_t s_prefix;
@@ -183,26 +184,65 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
   for (int e = 0; e < kPer; ++e)
     if (j0 + e < len) l += (int64_t)(d[e] >> b) + 1 + b;
   int64_t tot;
-  const int64_t ex = block_exclusive_scan(l, sh, &tot);
-  // publish the aggregate, then look back (warp 0)
+  const int64_t ex = block_exclusive_scan(l, sh, &tot);   // this thread's first bit in the block
   if (threadIdx.x == 0) st_relaxed(flags + vb, (vb == 0 ? kFlagInc : kFlagAgg) | (uint64_t)tot);
-  if (threadIdx.x < 32) {
-    uint64_t prefix = 0;
-    const bool ok = vb == 0 ? true : lookback(flags, vb, (int)threadIdx.x, &prefix);
-    if (threadIdx.x == 0) {
-      s_ok = ok;
-      s_prefix = prefix;
-      if (ok && vb > 0) st_relaxed(flags + vb, kFlagInc | (prefix + (uint64_t)tot));
-      if (!ok) {
-        raise(d_status, GSPARSE_DERR_TIMEOUT);
-        state->abort = 1;
+  const bool last = (int64_t)vb == nact - 1;
+  // relative words [0, nrel): the block's bits from its own first bit
+  const int64_t nrel = cdiv(tot, 32);
+  const bool fits = nrel + 1 <= kPackWords;
+  auto find_prefix = [&]() {
+    if (threadIdx.x < 32) {
+      uint64_t prefix = 0;
+      const bool ok = vb == 0 ? true : lookback(flags, vb, (int)threadIdx.x, &prefix);
+      if (threadIdx.x == 0) {
+        s_ok = ok;
+        s_prefix = prefix;
+        if (ok && vb > 0) st_relaxed(flags + vb, kFlagInc | (prefix + (uint64_t)tot));
+        if (!ok) {
+          raise(d_status, GSPARSE_DERR_TIMEOUT);
+          state->abort = 1;
+        }
       }
     }
+    __syncthreads();
+  };
+  if (fits) {
+    for (int64_t i = threadIdx.x; i <= nrel; i += blockDim.x) wbuf[i] = 0u;
+    __syncthreads();
+    uint32_t p = (uint32_t)ex;   // relative bit position (< 2^17 here)
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      if (j0 + e >= len) break;
+      const uint32_t q = d[e] >> b;
+      const uint32_t rem = d[e] & ((1u << b) - 1u);
+      // terminator 0, then the remainder most significant bit first
+      const uint32_t tl = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
+      if (q + 1u + (uint32_t)b <= 32u) {
+        // the whole codeword as one pattern: at most two words
+        const uint32_t pat = (q ? 0xffffffffu >> (32u - q) : 0u) | (tl << q);
+        const uint64_t v = (uint64_t)pat << (p & 31u);
+        if ((uint32_t)v) atomicOr(&wbuf[p >> 5], (uint32_t)v);
+        if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(p >> 5) + 1], (uint32_t)(v >> 32));
+      } else {
+        uint32_t pp = p, qq = q;
+        while (qq) {  // the unary run of ones
+          const uint32_t s2 = pp & 31u, nrun = qq < 32u - s2 ? qq : 32u - s2;
+          atomicOr(&wbuf[pp >> 5], (nrun == 32u ? 0xffffffffu : ((1u << nrun) - 1u)) << s2);
+          pp += nrun;
+          qq -= nrun;
+        }
+        const uint64_t v = (uint64_t)tl << (pp & 31u);  // terminator + remainder, <= 32 bits
+        if ((uint32_t)v) atomicOr(&wbuf[pp >> 5], (uint32_t)v);
+        if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(pp >> 5) + 1], (uint32_t)(v >> 32));
+      }
+      p += q + 1u + (uint32_t)b;
+    }
+    find_prefix();   // includes the barrier that completes the packing
+  } else {
+    find_prefix();
   }
-  __syncthreads();
   if (!s_ok) return;
   const uint64_t S = s_prefix, E = S + (uint64_t)tot;
-  const bool last = (int64_t)vb == nact - 1;
   if (last && threadIdx.x == 0) {
     *d_nbits = E;
     if ((int64_t)cdiv((int64_t)E, 32) > word_capacity) raise(d_status, GSPARSE_DERR_CAPACITY);
@@ -234,41 +274,13 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
   const bool head_shared = vb > 0 && (S & 31);
   const bool tail_shared = !last && (E & 31);
   const uint32_t span = (uint32_t)(wl - wf + 1);
-  if (span <= (uint32_t)kPackWords) {
-    for (uint32_t i = threadIdx.x; i < span; i += blockDim.x) wbuf[i] = 0u;
-    __syncthreads();
-    // positions relative to the block's first word: the block spans < 2^17 bits here
-    uint32_t p = (uint32_t)((uint64_t)o0 - 32u * wf);
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-      if (j0 + e >= len) break;
-      const uint32_t q = d[e] >> b;
-      const uint32_t rem = d[e] & ((1u << b) - 1u);
-      // terminator 0, then the remainder most significant bit first
-      const uint32_t tl = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
-      if (q + 1u + (uint32_t)b <= 32u) {
-        // the whole codeword as one pattern: at most two words
-        const uint32_t pat = (q ? 0xffffffffu >> (32u - q) : 0u) | (tl << q);
-        const uint64_t v = (uint64_t)pat << (p & 31u);
-        if ((uint32_t)v) atomicOr(&wbuf[p >> 5], (uint32_t)v);
-        if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(p >> 5) + 1], (uint32_t)(v >> 32));
-      } else {
-        uint32_t pp = p, qq = q;
-        while (qq) {  // the unary run of ones
-          const uint32_t s2 = pp & 31u, nrun = qq < 32u - s2 ? qq : 32u - s2;
-          atomicOr(&wbuf[pp >> 5], (nrun == 32u ? 0xffffffffu : ((1u << nrun) - 1u)) << s2);
-          pp += nrun;
-          qq -= nrun;
-        }
-        const uint64_t v = (uint64_t)tl << (pp & 31u);  // terminator + remainder, <= 32 bits
-        if ((uint32_t)v) atomicOr(&wbuf[pp >> 5], (uint32_t)v);
-        if ((uint32_t)(v >> 32)) atomicOr(&wbuf[(pp >> 5) + 1], (uint32_t)(v >> 32));
-      }
-      p += q + 1u + (uint32_t)b;
-    }
-    __syncthreads();
+  if (fits) {
+    // stream word wf + i holds relative bits [32 i - sh, 32 i - sh + 32): a funnel shift of
+    // relative words i - 1 and i (span <= nrel + 1, and wbuf[nrel] is zero)
+    const uint32_t shf = (uint32_t)(S & 31);
     for (uint32_t i = threadIdx.x; i < span; i += blockDim.x) {
-      const uint32_t bits = wbuf[i];
+      const uint32_t hi = wbuf[i], lo = i ? wbuf[i - 1] : 0u;
+      const uint32_t bits = __funnelshift_l(lo, hi, shf);
       if (i == 0 && head_shared) head[vb] = bits;
       else if (i == span - 1 && tail_shared) tail[vb] = bits;
       else words[wf + i] = bits;
@@ -303,7 +315,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
   __syncthreads();
   if (threadIdx.x == 0) {
     if (head_shared) head[vb] = s_head; else words[wf] = s_head;
-    if (tail_shared) tail[vb] = s_tail; else words[wl] = s_tail;
+    if (tail_shared) tail[vb] = s_tail; else if (wl != wf) words[wl] = s_tail;
   }
 }
 
@@ -421,29 +433,29 @@ __device__ bool decode_chunk_buffered(const uint32_t* sw, uint32_t nb_rel, uint3
   uint64_t buf = ((uint64_t)sw[wi] | ((uint64_t)sw[wi + 1] << 32)) >> s0;
   uint32_t avail = 64u - s0;
   wi += 2;
-  const bool vec = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
-  int4 ov = make_int4(0, 0, 0, 0);
-  for (int k = 0; k < count; ++k) {
+  // one codeword; false on a corrupt stream or an index out of range
+  auto next = [&](int32_t& outv) -> bool {
     if (avail <= 32u) {
       buf |= (uint64_t)sw[wi] << avail;
       avail += 32u;
       ++wi;
     }
-    const uint32_t pos = 32u * wi - avail;    // relative bit of this codeword
-    if (pos >= nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
-    const uint64_t nz = ~buf;
-    const uint32_t z = nz ? (uint32_t)__ffsll((long long)nz) - 1u : 64u;   // ones before the first zero
+    const uint32_t lo = (uint32_t)buf, hi = (uint32_t)(buf >> 32);
+    uint32_t z;                                // ones before the first zero bit
+    if (~lo) z = (uint32_t)__ffs(~lo) - 1u;
+    else z = ~hi ? 31u + (uint32_t)__ffs(~hi) : 64u;
     uint32_t q, rem = 0;
-    if (z + 1u + (uint32_t)b <= avail) {
+    const uint32_t used = z + 1u + (uint32_t)b;
+    if (used <= avail) {
       q = z;
       if (b > 0) rem = __brev((uint32_t)(buf >> (z + 1u)) & mask) >> (32 - b);
-      const uint32_t used = z + 1u + (uint32_t)b;
       buf = used == 64u ? 0ull : buf >> used;
       avail -= used;
       if (32u * wi - avail > nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
     } else {
       // a long unary run: finish this codeword from the window, then restart the buffer after it
-      uint32_t t = pos;
+      uint32_t t = 32u * wi - avail;
+      if (t >= nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
       if (!decode_one_local_slow(sw, nb_rel, t, q, rem, b, d_status)) return false;
       wi = t >> 5;
       const uint32_t s = t & 31u;
@@ -454,20 +466,21 @@ __device__ bool decode_chunk_buffered(const uint32_t* sw, uint32_t nb_rel, uint3
     const int64_t i = prev + 1 + (int64_t)(((uint64_t)q << b) | rem);
     if (i >= n_limit || i > INT32_MAX) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); return false; }
     prev = i;
-    if (vec) {
-      const int e = k & 3;
-      if (e == 0) ov.x = (int32_t)i; else if (e == 1) ov.y = (int32_t)i; else if (e == 2) ov.z = (int32_t)i;
-      else ov.w = (int32_t)i;
-      if (e == 3) *reinterpret_cast<int4*>(out + k - 3) = ov;
-    } else {
-      out[k] = (int32_t)i;
+    outv = (int32_t)i;
+    return true;
+  };
+  int k = 0;
+  if ((reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+    for (; k + 4 <= count; k += 4) {
+      int32_t v0, v1, v2, v3;
+      if (!next(v0) || !next(v1) || !next(v2) || !next(v3)) return false;
+      *reinterpret_cast<int4*>(out + k) = make_int4(v0, v1, v2, v3);
     }
   }
-  if (vec) {
-    const int e = count & 3;   // the last partial group of four
-    if (e > 0) out[count - e] = ov.x;
-    if (e > 1) out[count - e + 1] = ov.y;
-    if (e > 2) out[count - e + 2] = ov.z;
+  for (; k < count; ++k) {
+    int32_t v;
+    if (!next(v)) return false;
+    out[k] = v;
   }
   t0 = 32u * wi - avail;
   return true;

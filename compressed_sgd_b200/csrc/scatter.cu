@@ -285,11 +285,6 @@ __global__ void __launch_bounds__(kCombThreads, 4) sa_combine_kernel(Lists L, in
         }
       }
     }
-    // a tile with many entries clears its whole accumulator afterwards; a sparse one records the
-    // entries it touches (bitmap) and clears only those
-    int64_t tile_entries = 0;
-    for (int w = 0; w < W; ++w) tile_entries += re[w] - rb[w];
-    const bool dense_tile = tile_entries > kTile / 8;
     for (int w = 0; w < W; ++w) {
       const int32_t* ix = L.idx[w];
       const float* vv = L.val[w];
@@ -313,15 +308,12 @@ __global__ void __launch_bounds__(kCombThreads, 4) sa_combine_kernel(Lists L, in
 #pragma unroll
         for (int k = 0; k < kCombPer; ++k) {
           const int64_t j = jb + k * kCombThreads + threadIdx.x;
-          // the predecessor entry's index: from the neighbouring lane, or loaded by lane 0
-          int32_t pv = __shfl_up_sync(kFull, iv[k], 1);
-          if ((threadIdx.x & 31) == 0) pv = (j > 0 && j <= e) ? ix[j - 1] : INT32_MIN;
           if (j >= e) continue;
-          if (j > 0 && pv >= iv[k]) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); continue; }
+          if (j > 0 && ix[j - 1] >= iv[k]) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); continue; }
           const int off = (int)(iv[k] - t0);
           if (off < 0 || off >= kTile) continue;  // out of range, reported by the bounds pass
           acc[off] = __fadd_rn(acc[off], xv[k]);
-          if (!dense_tile) atomicOr(&touched[off >> 5], 1u << (off & 31));
+          atomicOr(&touched[off >> 5], 1u << (off & 31));
         }
       }
       __syncthreads();  // worker order: all of worker w before any of worker w + 1
@@ -366,19 +358,14 @@ __global__ void __launch_bounds__(kCombThreads, 4) sa_combine_kernel(Lists L, in
         out[t0 + i] = __fadd_rn(__fmul_rn(alpha, acc[i]), __fmul_rn(beta, Lg[t0 + i]));
     }
     __syncthreads();
-    if (dense_tile) {
-      for (int v = threadIdx.x; v < kTile / 4; v += blockDim.x)
-        reinterpret_cast<float4*>(acc)[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-      // clear what this tile touched (thread k owns bitmap word k)
-      for (int k = threadIdx.x; k < kTile / 32; k += blockDim.x) {
-        uint32_t word = touched[k];
-        touched[k] = 0u;
-        while (word) {
-          const int bit = __ffs(word) - 1;
-          word &= word - 1;
-          acc[k * 32 + bit] = 0.0f;
-        }
+    // clear what this tile touched (thread k owns bitmap word k)
+    for (int k = threadIdx.x; k < kTile / 32; k += blockDim.x) {
+      uint32_t word = touched[k];
+      touched[k] = 0u;
+      while (word) {
+        const int bit = __ffs(word) - 1;
+        word &= word - 1;
+        acc[k * 32 + bit] = 0.0f;
       }
     }
     if (threadIdx.x < W) {
