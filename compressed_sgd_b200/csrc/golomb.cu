@@ -496,7 +496,7 @@ __global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
     const uint32_t* words, int64_t word_capacity, const uint64_t* d_nbits, const int64_t* d_count,
     int64_t capacity, int b, const int64_t* table, int32_t chunk, int64_t n_limit, int32_t* out,
     int32_t* d_status) {
-  __shared__ uint32_t sw[kDecWords];
+  __shared__ __align__(16) uint32_t sw[kDecWords];
   const int64_t K = *d_count;
   if (K < 0 || K > capacity) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise(d_status, GSPARSE_DERR_CAPACITY);
@@ -521,8 +521,33 @@ __global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
   const int64_t wa = (int64_t)(ba >> 5), wz = cdiv((int64_t)bz, 32) + 3;   // three zero spare words
   const bool staged = wz - wa <= kDecWords;
   if (staged) {
+    // the window with 16-byte loads (the stream's words only; zero past its end), all of a
+    // thread's loads issued before any is stored
     const int span = (int)(wz - wa);
-    for (int k = threadIdx.x; k < span; k += kDecThreads) sw[k] = wa + k < nw ? words[wa + k] : 0u;
+    const bool vec = (reinterpret_cast<uintptr_t>(words + wa) & 15u) == 0;
+    constexpr int kStageIt = kDecWords / (4 * kDecThreads);
+    uint4 vbuf[kStageIt];
+#pragma unroll
+    for (int it = 0; it < kStageIt; ++it) {
+      const int k = 4 * (threadIdx.x + it * kDecThreads);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (k < span) {
+        if (vec && wa + k + 3 < nw) {
+          v = *reinterpret_cast<const uint4*>(words + wa + k);
+        } else {
+          v.x = wa + k < nw ? words[wa + k] : 0u;
+          v.y = wa + k + 1 < nw ? words[wa + k + 1] : 0u;
+          v.z = wa + k + 2 < nw ? words[wa + k + 2] : 0u;
+          v.w = wa + k + 3 < nw ? words[wa + k + 3] : 0u;
+        }
+      }
+      vbuf[it] = v;
+    }
+#pragma unroll
+    for (int it = 0; it < kStageIt; ++it) {
+      const int k = 4 * (threadIdx.x + it * kDecThreads);
+      if (k < span) *reinterpret_cast<uint4*>(sw + k) = vbuf[it];
+    }
     __syncthreads();
   }
   if (c >= nch) return;
