@@ -139,4 +139,31 @@ inline int launch_status() {
 // SM count of the current device, cached per device.
 int sm_count();
 
+// Programmatic dependent launch (sm_90 and later). Every kernel of the library is launched with
+// launch(), which lets it start while the kernel before it in the stream is finishing, and begins
+// with pdl_begin(): griddepcontrol.wait blocks until every earlier grid it depends on has completed
+// and its memory is visible, so nothing is read or written before that; the kernel then allows
+// the next kernel to launch at once. Only the launch latency overlaps. A kernel whose
+// predecessor was launched without this attribute (a memset, another library's kernel) simply
+// starts after it.
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... P, typename... A>
+inline void launch(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, static_cast<A&&>(args)...);
+}
+
 }  // namespace gs

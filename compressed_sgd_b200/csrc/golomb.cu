@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
     const int32_t* idx, const int64_t* d_begin, const int64_t* d_end, int64_t capacity, int64_t base,
     int b, uint32_t* words, int64_t word_capacity, uint64_t* d_nbits, int64_t* table, int32_t chunk,
     GState* state, uint64_t* flags, uint32_t* head, uint32_t* tail, int32_t* d_status) {
+  pdl_begin();
   __shared__ uint32_t wbuf[kPackWords + 1];
   __shared__ int64_t sh[33];
   __shared__ uint32_t s_vb;
@@ -179,10 +180,13 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
   const int64_t j0 = jb + (int64_t)threadIdx.x * kPer;
   uint32_t d[kPer];
   thread_gaps(x, len, base, j0, d, d_status);
-  int64_t l = 0;
+  // codewords of this thread: entries j0 .. j0 + nv - 1 of the list
+  const int nv = len - j0 >= kPer ? kPer : (len > j0 ? (int)(len - j0) : 0);
+  uint64_t lu = 0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e)
-    if (j0 + e < len) l += (int64_t)(d[e] >> b) + 1 + b;
+    if (e < nv) lu += (uint64_t)(d[e] >> b) + 1u + (uint32_t)b;
+  const int64_t l = (int64_t)lu;
   int64_t tot;
   const int64_t ex = block_exclusive_scan(l, sh, &tot);   // this thread's first bit in the block
   if (threadIdx.x == 0) st_relaxed(flags + vb, (vb == 0 ? kFlagInc : kFlagAgg) | (uint64_t)tot);
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
     uint32_t p = (uint32_t)ex;   // relative bit position (< 2^17 here)
 #pragma unroll
     for (int e = 0; e < kPer; ++e) {
-      if (j0 + e >= len) break;
+      if (e >= nv) break;
       const uint32_t q = d[e] >> b;
       const uint32_t rem = d[e] & ((1u << b) - 1u);
       // terminator 0, then the remainder most significant bit first
@@ -251,20 +255,23 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
   // side table: bit offset and preceding index at every chunk start (one 32-bit division per
   // thread; indices < 2^31)
   if (table) {
-    uint32_t in_chunk = (uint32_t)j0 % (uint32_t)chunk;
-    int64_t o = o0;
+    // the chunk starts among this thread's codewords: e = e0, e0 + chunk, ... below nv
+    const uint32_t e0 = (uint32_t)((chunk - (int64_t)((uint32_t)j0 % (uint32_t)chunk)) % chunk);
+    if (e0 < (uint32_t)nv) {
+      int64_t o = o0;
+      uint32_t next = e0;
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-      const int64_t j = j0 + e;
-      if (j < len) {
-        if (in_chunk == 0) {
+      for (int e = 0; e < kPer; ++e) {
+        if (e >= nv) break;
+        if ((uint32_t)e == next) {
+          next += (uint32_t)chunk;
+          const int64_t j = j0 + e;
           const int64_t c = (int64_t)((uint32_t)j / (uint32_t)chunk);
           table[2 * c] = o;
           table[2 * c + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
         }
         o += (int64_t)(d[e] >> b) + 1 + b;
       }
-      if (++in_chunk == (uint32_t)chunk) in_chunk = 0;
     }
   }
   const uint64_t wf = S >> 5, wl = (E - 1) >> 5;
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
   int64_t o = o0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
-    if (j0 + e >= len) break;
+    if (e >= nv) break;
     Code c;
     c.o = (uint64_t)o;
     c.q = (uint64_t)(d[e] >> b);
@@ -324,6 +331,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
 __global__ void g_fix_kernel(const int64_t* d_begin, const int64_t* d_end, int64_t capacity,
                              const GState* state, const uint64_t* flags, const uint32_t* head,
                              const uint32_t* tail, uint32_t* words, int64_t word_capacity) {
+  pdl_begin();
   int64_t lb, len;
   if (!list_bounds(d_begin, d_end, capacity, &lb, &len) || state->abort) return;
   const int64_t nact = cdiv(len, kBlockCodes);
@@ -425,9 +433,14 @@ __device__ __forceinline__ bool decode_one_local_slow(const uint32_t* sw, uint32
 // 33 - b bits needs no refill; a longer one is finished word by word from the window. Outputs go
 // out four at a time when the chunk's output row is 16-byte aligned. Returns false (and raises)
 // on a corrupt stream; on success t0 is the bit after the last codeword.
-__device__ bool decode_chunk_buffered(const uint32_t* sw, uint32_t nb_rel, uint32_t& t0, int64_t& prev,
-                                      int count, int b, int64_t n_limit, int32_t* out, int32_t* d_status) {
+__device__ bool decode_chunk_buffered(const uint32_t* sw, uint32_t nb_rel, uint32_t wlim, uint32_t& t0,
+                                      int64_t& prev64, int count, int b, int64_t n_limit, int32_t* out,
+                                      int32_t* d_status) {
   const uint32_t mask = b > 0 ? 0xffffffffu >> (32 - b) : 0u;
+  // indices live in [0, 2^31): 32-bit arithmetic; qmax keeps (q << b) below 2^31
+  const uint32_t qmax = 0x7fffffffu >> b;
+  const uint32_t lim = (uint32_t)(n_limit < (int64_t)INT32_MAX ? n_limit : (int64_t)INT32_MAX);
+  uint32_t prev1 = (uint32_t)(prev64 + 1);   // the index after the previous one (>= 0)
   uint32_t wi = t0 >> 5;                      // next word to take into the buffer
   const uint32_t s0 = t0 & 31u;
   uint64_t buf = ((uint64_t)sw[wi] | ((uint64_t)sw[wi + 1] << 32)) >> s0;
@@ -436,14 +449,15 @@ __device__ bool decode_chunk_buffered(const uint32_t* sw, uint32_t nb_rel, uint3
   // one codeword; false on a corrupt stream or an index out of range
   auto next = [&](int32_t& outv) -> bool {
     if (avail <= 32u) {
+      if (wi >= wlim) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }   // ran off the window
       buf |= (uint64_t)sw[wi] << avail;
       avail += 32u;
       ++wi;
     }
-    const uint32_t lo = (uint32_t)buf, hi = (uint32_t)(buf >> 32);
+    const uint32_t lo = (uint32_t)buf;
     uint32_t z;                                // ones before the first zero bit
     if (~lo) z = (uint32_t)__ffs(~lo) - 1u;
-    else z = ~hi ? 31u + (uint32_t)__ffs(~hi) : 64u;
+    else z = ~(uint32_t)(buf >> 32) ? 31u + (uint32_t)__ffs(~(uint32_t)(buf >> 32)) : 64u;
     uint32_t q, rem = 0;
     const uint32_t used = z + 1u + (uint32_t)b;
     if (used <= avail) {
@@ -451,7 +465,6 @@ __device__ bool decode_chunk_buffered(const uint32_t* sw, uint32_t nb_rel, uint3
       if (b > 0) rem = __brev((uint32_t)(buf >> (z + 1u)) & mask) >> (32 - b);
       buf = used == 64u ? 0ull : buf >> used;
       avail -= used;
-      if (32u * wi - avail > nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
     } else {
       // a long unary run: finish this codeword from the window, then restart the buffer after it
       uint32_t t = 32u * wi - avail;
@@ -463,26 +476,31 @@ __device__ bool decode_chunk_buffered(const uint32_t* sw, uint32_t nb_rel, uint3
       avail = 64u - s;
       wi += 2;
     }
-    const int64_t i = prev + 1 + (int64_t)(((uint64_t)q << b) | rem);
-    if (i >= n_limit || i > INT32_MAX) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); return false; }
-    prev = i;
+    if (q > qmax) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); return false; }
+    const uint32_t i = prev1 + ((q << b) | rem);   // < 2^32: prev1 <= 2^31, gap < 2^31
+    if (i >= lim) { raise(d_status, GSPARSE_DERR_INDEX_RANGE); return false; }
+    prev1 = i + 1u;
     outv = (int32_t)i;
     return true;
   };
   int k = 0;
+  bool ok = true;
   if ((reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
     for (; k + 4 <= count; k += 4) {
       int32_t v0, v1, v2, v3;
-      if (!next(v0) || !next(v1) || !next(v2) || !next(v3)) return false;
+      if (!next(v0) || !next(v1) || !next(v2) || !next(v3)) { ok = false; break; }
       *reinterpret_cast<int4*>(out + k) = make_int4(v0, v1, v2, v3);
     }
   }
-  for (; k < count; ++k) {
+  for (; ok && k < count; ++k) {
     int32_t v;
-    if (!next(v)) return false;
+    if (!next(v)) { ok = false; break; }
     out[k] = v;
   }
+  if (!ok) return false;
   t0 = 32u * wi - avail;
+  if (t0 > nb_rel) { raise(d_status, GSPARSE_DERR_CORRUPT_STREAM); return false; }
+  prev64 = (int64_t)prev1 - 1;
   return true;
 }
 
@@ -496,6 +514,7 @@ __global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
     const uint32_t* words, int64_t word_capacity, const uint64_t* d_nbits, const int64_t* d_count,
     int64_t capacity, int b, const int64_t* table, int32_t chunk, int64_t n_limit, int32_t* out,
     int32_t* d_status) {
+  pdl_begin();
   __shared__ __align__(16) uint32_t sw[kDecWords];
   const int64_t K = *d_count;
   if (K < 0 || K > capacity) {
@@ -564,7 +583,9 @@ __global__ void __launch_bounds__(kDecThreads) g_decode_chunks_kernel(
     // the window's end: this CTA's range, so a chunk cannot run into the next CTA's bits
     uint32_t tl = (uint32_t)(t - 32u * (uint64_t)wa);
     const uint32_t nb_rel = (uint32_t)(bz - 32u * (uint64_t)wa);
-    ok = decode_chunk_buffered(sw, nb_rel, tl, prev, count, b, n_limit, out + first, d_status);
+    // refills stop two words short of the staged span (the last words are zero spares)
+    ok = decode_chunk_buffered(sw, nb_rel, (uint32_t)(wz - wa) - 1u, tl, prev, count, b, n_limit, out + first,
+                               d_status);
     t = 32u * (uint64_t)wa + tl;
   } else {
     ok = decode_run(words, 0, nw, nbits, t, prev, count, b, n_limit, out + first, d_status);
@@ -580,6 +601,7 @@ __global__ void g_decode_serial_kernel(const uint32_t* words, int64_t word_capac
                                        const uint64_t* d_nbits,
                                        const int64_t* d_count, int64_t capacity, int64_t base,
                                        int b, int64_t n_limit, int32_t* out, int32_t* d_status) {
+  pdl_begin();
   const int64_t K = *d_count;
   if (K < 0 || K > capacity) { raise(d_status, GSPARSE_DERR_CAPACITY); return; }
   const uint64_t nbits = *d_nbits;
@@ -640,11 +662,11 @@ int gsparse_golomb_encode(const int32_t* idx, const int64_t* d_begin, const int6
   GLayout L = g_carve(capacity, workspace);
   if (workspace_bytes < L.bytes) return GSPARSE_ERR_WORKSPACE;
   if (cudaMemsetAsync(workspace, 0, L.zero_bytes, st) != cudaSuccess) return GSPARSE_ERR_CUDA;
-  g_encode_kernel<<<(unsigned)L.nblk, kCodeThreads, 0, st>>>(idx, d_begin, d_end, capacity, base, b, words,
+  launch(g_encode_kernel, (unsigned)L.nblk, kCodeThreads, 0, st, idx, d_begin, d_end, capacity, base, b, words,
                                                              word_capacity, d_nbits, chunk_table, chunk,
                                                              L.state, L.flags, L.head, L.tail, d_status);
   if (L.nblk > 1)
-    g_fix_kernel<<<(unsigned)cdiv(L.nblk - 1, 256), 256, 0, st>>>(d_begin, d_end, capacity, L.state, L.flags,
+    launch(g_fix_kernel, (unsigned)cdiv(L.nblk - 1, 256), 256, 0, st, d_begin, d_end, capacity, L.state, L.flags,
                                                                  L.head, L.tail, words, word_capacity);
   return launch_status();
 }
@@ -660,11 +682,11 @@ int gsparse_golomb_decode(const uint32_t* words, int64_t word_capacity, const ui
   if (b < 0 || b > 30 || capacity > INT32_MAX) return GSPARSE_ERR_UNSUPPORTED;
   if (chunk_table) {
     const int64_t nch = cdiv(capacity > 0 ? capacity : 1, chunk);
-    g_decode_chunks_kernel<<<(unsigned)cdiv(nch, kDecThreads), kDecThreads, 0, st>>>(
+    launch(g_decode_chunks_kernel, (unsigned)cdiv(nch, kDecThreads), kDecThreads, 0, st, 
         words, word_capacity, d_nbits, d_count, capacity, b, chunk_table, chunk, n_limit, out_idx,
         d_status);
   } else {
-    g_decode_serial_kernel<<<1, 1, 0, st>>>(words, word_capacity, d_nbits, d_count, capacity, base,
+    launch(g_decode_serial_kernel, 1, 1, 0, st, words, word_capacity, d_nbits, d_count, capacity, base,
                                             b, n_limit, out_idx, d_status);
   }
   return launch_status();

@@ -12,6 +12,7 @@ constexpr int kLeafRound = 64;
 __global__ void __launch_bounds__(kLeafWarps * 32) osum_leaves_kernel(SumJob* jobs, int32_t njobs,
                                                                       double* leaves, int64_t leaf_bound,
                                                                       const int32_t* abort_flag) {
+  pdl_begin();
   __shared__ float tile[kLeafWarps][32][kLeafRound + 1];
   __shared__ const float* lptr[kLeafWarps][32];
   __shared__ int lcnt[kLeafWarps][32];
@@ -95,6 +96,7 @@ __global__ void __launch_bounds__(kLeafWarps * 32) osum_pair_leaves_kernel(SumJo
                                                                            double* leaves,
                                                                            int64_t pair_leaf_bound,
                                                                            const int32_t* abort_flag) {
+  pdl_begin();
   __shared__ float tile[kLeafWarps][32][kLeafRound + 1];
   __shared__ const float* lptr[kLeafWarps][32];
   __shared__ int lcnt[kLeafWarps][32];
@@ -187,6 +189,7 @@ __device__ double* tree_reduce_shared(double* a, double* b, int m) {
 __global__ void __launch_bounds__(1024) osum_tree_kernel(SumJob* jobs, int32_t njobs, const double* leaves,
                                  double* partials, int64_t partial_stride,
                                  const int32_t* abort_flag) {
+  pdl_begin();
   if (abort_flag && *abort_flag) return;
   __shared__ double sa[kTreeLeaves], sb[kTreeLeaves];
   __shared__ int is_last;
@@ -244,12 +247,12 @@ void osum_launch_pairs(SumJob* jobs, int32_t npairs, double* leaves, int64_t pai
   if (npairs <= 0) return;
   if (pair_leaf_bound > 0) {
     const int threads = kLeafWarps * 32;
-    osum_pair_leaves_kernel<<<(unsigned)cdiv(pair_leaf_bound, threads), threads, 0, s>>>(
+    launch(osum_pair_leaves_kernel, (unsigned)cdiv(pair_leaf_bound, threads), threads, 0, s, 
         jobs, npairs, leaves, pair_leaf_bound, abort_flag);
   }
   const int64_t stride = osum_partial_stride(per_job_leaf_bound);
   dim3 grid((unsigned)stride, (unsigned)(2 * npairs));
-  osum_tree_kernel<<<grid, 1024, 0, s>>>(jobs, 2 * npairs, leaves, partials, stride, abort_flag);
+  launch(osum_tree_kernel, grid, 1024, 0, s, jobs, 2 * npairs, leaves, partials, stride, abort_flag);
 }
 
 void osum_launch(SumJob* jobs, int32_t njobs, double* leaves, int64_t leaf_bound,
@@ -258,12 +261,12 @@ void osum_launch(SumJob* jobs, int32_t njobs, double* leaves, int64_t leaf_bound
   if (njobs <= 0) return;
   if (leaf_bound > 0) {
     const int threads = kLeafWarps * 32;
-    osum_leaves_kernel<<<(unsigned)cdiv(leaf_bound, threads), threads, 0, s>>>(jobs, njobs, leaves,
+    launch(osum_leaves_kernel, (unsigned)cdiv(leaf_bound, threads), threads, 0, s, jobs, njobs, leaves,
                                                                                leaf_bound, abort_flag);
   }
   const int64_t stride = osum_partial_stride(per_job_leaf_bound);
   dim3 grid((unsigned)stride, (unsigned)njobs);
-  osum_tree_kernel<<<grid, 1024, 0, s>>>(jobs, njobs, leaves, partials, stride, abort_flag);
+  launch(osum_tree_kernel, grid, 1024, 0, s, jobs, njobs, leaves, partials, stride, abort_flag);
 }
 
 }  // namespace gs

@@ -13,6 +13,7 @@ namespace {
 
 __global__ void q_setup_kernel(const float* val, const int64_t* d_begin, const int64_t* d_end,
                                int64_t capacity, SumJob* jobs, int32_t* ctl, int32_t* d_status) {
+  pdl_begin();
   const int64_t b = d_begin ? *d_begin : 0;
   const int64_t e = *d_end;
   int64_t len = e - b;
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(kApplyThreads) q_apply_kernel(
     const int32_t* idx, float* val, const int64_t* d_begin, const int64_t* d_end, const SumJob* jobs,
     float* residual, int64_t n, float* feedback, uint32_t* sign_bits, float* d_means,
     int32_t write_deq, const int32_t* ctl, int32_t* d_status) {
+  pdl_begin();
   if (ctl[0]) return;
   const int64_t b = d_begin ? *d_begin : 0;
   const int64_t len = *d_end - b;
@@ -93,6 +95,7 @@ __global__ void __launch_bounds__(kApplyThreads) q_apply_kernel(
 __global__ void __launch_bounds__(1024) q_setup_seg_kernel(const float* val, const int64_t* off, int32_t T,
                                                            int64_t capacity, int64_t pair_bound, SumJob* jobs,
                                                            int32_t* ctl, int32_t* d_status) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
@@ -141,6 +144,7 @@ __global__ void __launch_bounds__(kApplyThreads) q_apply_seg_kernel(
     const int32_t* idx, float* val, const int64_t* off, int32_t T, const SumJob* jobs, float* residual,
     int64_t n, float* feedback, uint32_t* sign_bits, float* d_means, int32_t write_deq, const int32_t* ctl,
     int32_t* d_status) {
+  pdl_begin();
   if (ctl[0]) return;
   const int64_t b = off[0];
   const int64_t len = off[T] - b;
@@ -248,10 +252,10 @@ int gsparse_quantize(const int32_t* idx, float* val, const int64_t* d_begin, con
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GSPARSE_ERR_WORKSPACE;
   QLayout L = q_carve(capacity, workspace);
   if (workspace_bytes < L.bytes) return GSPARSE_ERR_WORKSPACE;
-  q_setup_kernel<<<1, 1, 0, st>>>(val, d_begin, d_end, capacity, L.jobs, L.ctl, d_status);
+  launch(q_setup_kernel, 1, 1, 0, st, val, d_begin, d_end, capacity, L.jobs, L.ctl, d_status);
   osum_launch_pairs(L.jobs, 1, L.leaves, L.per_job, L.per_job, L.partials, L.ctl, st);
   const int64_t blocks = cdiv(capacity > 0 ? capacity : 1, kApplyThreads * kApplyPer);
-  q_apply_kernel<<<(unsigned)blocks, kApplyThreads, 0, st>>>(
+  launch(q_apply_kernel, (unsigned)blocks, kApplyThreads, 0, st, 
       idx, val, d_begin, d_end, L.jobs, residual, n, feedback_out, sign_bits, d_means,
       write_dequantized, L.ctl, d_status);
   return launch_status();
@@ -276,10 +280,10 @@ int gsparse_quantize_segments(const int32_t* idx, float* val, const int64_t* d_o
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GSPARSE_ERR_WORKSPACE;
   QSegLayout L = qs_carve(capacity, T, workspace);
   if (workspace_bytes < L.bytes) return GSPARSE_ERR_WORKSPACE;
-  q_setup_seg_kernel<<<1, 1024, 0, st>>>(val, d_offsets, T, capacity, L.leaf_bound, L.jobs, L.ctl, d_status);
+  launch(q_setup_seg_kernel, 1, 1024, 0, st, val, d_offsets, T, capacity, L.leaf_bound, L.jobs, L.ctl, d_status);
   osum_launch_pairs(L.jobs, T, L.leaves, L.leaf_bound, L.per_job, L.partials, L.ctl, st);
   const int64_t blocks = cdiv(capacity > 0 ? capacity : 1, kApplyThreads * kApplyPer);
-  q_apply_seg_kernel<<<(unsigned)blocks, kApplyThreads, 0, st>>>(idx, val, d_offsets, T, L.jobs, residual, n,
+  launch(q_apply_seg_kernel, (unsigned)blocks, kApplyThreads, 0, st, idx, val, d_offsets, T, L.jobs, residual, n,
                                                                  feedback_out, sign_bits, d_means,
                                                                  write_dequantized, L.ctl, d_status);
   return launch_status();

@@ -57,6 +57,7 @@ constexpr int kStartsPer = 16;
 __global__ void __launch_bounds__(256) sa_starts_kernel(Lists L, int32_t W, int64_t n, int64_t ntiles,
                                                         int64_t* start, uint32_t* next_tile,
                                                         int32_t* d_status) {
+  pdl_begin();
   const int w = blockIdx.y;
   const int64_t c = list_count(L, w);
   const int32_t* ix = L.idx[w];
@@ -140,6 +141,7 @@ __global__ void __launch_bounds__(kTileThreads) sa_tile_kernel(Lists L, int32_t 
                                                                const int64_t* start, float* dense,
                                                                int64_t* tile_count,
                                                                int32_t* d_status) {
+  pdl_begin();
   __shared__ __align__(16) float acc[kTile];
   __shared__ uint32_t touched[kTile / 32];
   const int64_t t = blockIdx.x;
@@ -170,6 +172,7 @@ __global__ void __launch_bounds__(kTileThreads) sa_tile_kernel(Lists L, int32_t 
 __global__ void __launch_bounds__(1024) sa_scan_kernel(int64_t* tile_count, int64_t ntiles,
                                                        int64_t* d_merged_count, int64_t capacity,
                                                        int32_t* ctl, int32_t* d_status) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   int64_t carry = 0;
   for (int64_t base = 0; base < ntiles; base += blockDim.x) {
@@ -191,6 +194,7 @@ __global__ void __launch_bounds__(kTileThreads) sa_merge_kernel(Lists L, int32_t
                                                                 const int64_t* tile_off,
                                                                 int32_t* merged_idx, float* merged_val,
                                                                 const int32_t* ctl) {
+  pdl_begin();
   __shared__ float acc[kTile];
   __shared__ uint32_t touched[kTile / 32];
   __shared__ int64_t sh[33];
@@ -243,6 +247,7 @@ __global__ void __launch_bounds__(kCombThreads, 4) sa_combine_kernel(Lists L, in
                                                                   float alpha, float beta,
                                                                   int32_t own, float* dense,
                                                                   int32_t* d_status) {
+  pdl_begin();
   constexpr int kVec = kTile / 4 / kCombThreads;  // float4s of a tile per thread
   __shared__ __align__(16) float acc[kTile];
   __shared__ uint32_t touched[kTile / 32];
@@ -381,6 +386,7 @@ __global__ void __launch_bounds__(kCombThreads, 4) sa_combine_kernel(Lists L, in
 
 __global__ void combine_kernel(const float* G, const float* Lg, float* out, int64_t n, float alpha,
                                float beta) {
+  pdl_begin();
   const int64_t nv = n >> 2;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nv; v += stride) {
@@ -403,6 +409,7 @@ __global__ void combine_partial_kernel(const float* G, const float* Lg, float* o
                                        float alpha, float beta, const int32_t* own_idx,
                                        const float* own_val, const int64_t* d_count,
                                        int64_t capacity, int32_t* d_status) {
+  pdl_begin();
   int64_t K = *d_count;
   if (K > capacity) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise(d_status, GSPARSE_DERR_CAPACITY);
@@ -428,7 +435,7 @@ void launch_starts(const Lists& L, int32_t W, int64_t n, int64_t ntiles, int64_t
   int64_t most = 0;
   for (int w = 0; w < W; ++w) most = L.cap[w] > most ? L.cap[w] : most;
   const int64_t bx = cdiv(most + 1, kStartsPer * 256);  // entries 0..count of every list
-  sa_starts_kernel<<<dim3((unsigned)bx, (unsigned)W), 256, 0, st>>>(L, W, n, ntiles, start, next_tile,
+  launch(sa_starts_kernel, dim3((unsigned)bx, (unsigned)W), 256, 0, st, L, W, n, ntiles, start, next_tile,
                                                                       d_status);
 }
 
@@ -486,12 +493,12 @@ int gsparse_scatter_accumulate(const gsparse_list* lists, int32_t W, int64_t n, 
     return launch_status();
   }
   launch_starts(L, W, n, ntiles, S.start, nullptr, d_status, st);
-  sa_tile_kernel<<<(unsigned)ntiles, kTileThreads, 0, st>>>(L, W, n, S.start, dense_out,
+  launch(sa_tile_kernel, (unsigned)ntiles, kTileThreads, 0, st, L, W, n, S.start, dense_out,
                                                             merged ? S.tile_count : nullptr, d_status);
   if (merged) {
-    sa_scan_kernel<<<1, 1024, 0, st>>>(S.tile_count, ntiles, d_merged_count, merged_capacity, S.ctl,
+    launch(sa_scan_kernel, 1, 1024, 0, st, S.tile_count, ntiles, d_merged_count, merged_capacity, S.ctl,
                                        d_status);
-    sa_merge_kernel<<<(unsigned)ntiles, kTileThreads, 0, st>>>(L, W, S.start, S.tile_count,
+    launch(sa_merge_kernel, (unsigned)ntiles, kTileThreads, 0, st, L, W, S.start, S.tile_count,
                                                                merged_idx, merged_val, S.ctl);
   }
   return launch_status();
@@ -530,7 +537,7 @@ int gsparse_accumulate_combine(const gsparse_list* lists, int32_t W, int64_t n, 
   uint32_t* next_tile = reinterpret_cast<uint32_t*>(S.ctl + 1);
   launch_starts(Ls, W, n, ntiles, S.start, next_tile, d_status, st);
   const int64_t ctas = (int64_t)sm_count() * 4 < ntiles ? (int64_t)sm_count() * 4 : ntiles;
-  sa_combine_kernel<<<(unsigned)ctas, kCombThreads, 0, st>>>(
+  launch(sa_combine_kernel, (unsigned)ctas, kCombThreads, 0, st, 
       Ls, W, n, S.start, next_tile, L, out, alpha, beta, mode == 1 ? own : -1, dense_out, d_status);
   return launch_status();
 }
@@ -548,10 +555,10 @@ int gsparse_combine_local(const float* G, const float* L, float* out, int64_t n,
   if (mode == 1 && (out == G || out == L)) return GSPARSE_ERR_INVALID_ARG;
   if (n > 0) {
     const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
-    combine_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(G, L, out, n, alpha, beta);
+    launch(combine_kernel, (unsigned)(blocks > 0 ? blocks : 1), 256, 0, st, G, L, out, n, alpha, beta);
   }
   if (mode == 1 && own_capacity > 0)
-    combine_partial_kernel<<<(unsigned)cdiv(own_capacity, 256), 256, 0, st>>>(
+    launch(combine_partial_kernel, (unsigned)cdiv(own_capacity, 256), 256, 0, st, 
         G, L, out, n, alpha, beta, own_idx, own_val, d_own_count, own_capacity, d_status);
   return launch_status();
 }

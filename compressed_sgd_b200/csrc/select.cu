@@ -104,7 +104,7 @@ struct Sel {
 // ctl words: [0] abort, [1] any redo, [2] next free pool chunk, [8 + k] done-CTA counters of the
 // kernels that end in a fused tail (k: 0 restore, 1 histogram level 2, 2 level 3, 3 count)
 constexpr int kCtlDone = 8;
-constexpr int kFuseProblems = 8;
+constexpr int kFuseProblems = 2;
 
 // True in every thread of the CTA that finishes the kernel last (counter ctl[kCtlDone + k]); its
 // earlier global writes and atomics, and those of all other CTAs, are then visible to it.
@@ -266,6 +266,7 @@ __device__ void block_find_bin(const uint32_t* h, int B, int64_t rank, uint32_t*
 
 __global__ void __launch_bounds__(1024) plan_kernel(Sel a, const int64_t* seg, int64_t knum, int64_t kden,
                             int64_t out_capacity, int64_t* out_offsets) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
@@ -381,6 +382,7 @@ __device__ __forceinline__ uint32_t ceil_log2(uint32_t v) { return v <= 1 ? 0u :
 
 template <int C>
 __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhaustive) {
+  pdl_begin();
   __shared__ uint32_t h[C * kBins1];
   __shared__ uint32_t cnt[C];
   __shared__ unsigned long long vsum[C], vsq[C];
@@ -809,6 +811,7 @@ __device__ __forceinline__ void load_full(const Sel& a, uint32_t base, int lane,
 // processed.
 template <int C>
 __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
+  pdl_begin();
   __shared__ CtaHist<C, kBins1> H;
   __shared__ __align__(16) float stage[kWarps * kGranule];  // per warp: one chunk, entry order
   __shared__ uint16_t cstage[kWarps * kGranule];            // per warp: a chunk's candidate offsets
@@ -975,6 +978,7 @@ __device__ __forceinline__ void momentum_edge(const Sel& a, uint32_t base, uint3
 
 template <int C, bool kMom>
 __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
+  pdl_begin();
   using Slot = typename std::conditional<kMom, RingSlotM, RingSlot>::type;
   constexpr int kSt = kMom ? kStagesM : kStages;
   extern __shared__ __align__(128) unsigned char ring_mem[];
@@ -1099,6 +1103,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
 constexpr int kCheckPer = 16;
 
 __global__ void __launch_bounds__(256) pending_check_kernel(Sel a) {
+  pdl_begin();
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (t == 0 && *a.pw_count > a.pw_cap) {
     raise(a.d_status, GSPARSE_DERR_CAPACITY);
@@ -1222,6 +1227,7 @@ __device__ __forceinline__ void for_each_candidate(const Sel& a, int64_t q, cons
 // 4. check + restore
 
 __global__ void check_kernel(Sel a) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   if (a.ctl[0]) return;
   const int64_t p = blockIdx.x;
@@ -1244,6 +1250,7 @@ __global__ void check_kernel(Sel a) {
 
 template <int C>
 __global__ void __launch_bounds__(kThreads) restore_kernel(Sel a) {
+  pdl_begin();
   __shared__ CtaHist<C, kBins1> H;
   if (a.ctl[0]) return;
   const int64_t q0 = (int64_t)blockIdx.x * kWarps;
@@ -1372,6 +1379,7 @@ __device__ void select_problem(const Sel& a, int64_t p, int level, uint32_t* h, 
 }
 
 __global__ void __launch_bounds__(1024) select_kernel(Sel a, int level) {
+  pdl_begin();
   __shared__ uint32_t h[kBins1];
   __shared__ int64_t sh[33];
   if (a.ctl[0]) return;
@@ -1390,6 +1398,7 @@ __device__ void select_tail(const Sel& a, int level, uint32_t* h) {
 
 template <int C>
 __global__ void __launch_bounds__(kThreads) hist_kernel(Sel a, int level) {
+  pdl_begin();
   constexpr int B = kBins1;  // level 3 uses the first 512 bins
   __shared__ CtaHist<C, B> H;
   if (a.ctl[0]) return;
@@ -1425,6 +1434,7 @@ __device__ void scan_problem(const Sel& a, int64_t p, int64_t* sh);
 
 template <int C>
 __global__ void __launch_bounds__(kThreads) count_kernel(Sel a) {
+  pdl_begin();
   if (a.ctl[0]) return;
   const int64_t U = unit_count(a);
   for (int64_t u = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); u < U;
@@ -1532,6 +1542,7 @@ __device__ void scan_problem(const Sel& a, int64_t p, int64_t* sh) {
 }
 
 __global__ void __launch_bounds__(1024) scan_kernel(Sel a) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   if (a.ctl[0]) return;
   scan_problem(a, blockIdx.x, sh);
@@ -1553,6 +1564,7 @@ __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_
 template <int C>
 __global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
                                                         int64_t limit) {
+  pdl_begin();
   __shared__ EmitStage stage[kWarps];
   if (a.ctl[0]) return;
   const int64_t U = unit_count(a);
@@ -1744,6 +1756,7 @@ __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_
 // binarise: means, choice, output
 
 __global__ void __launch_bounds__(1024) bjobs_kernel(Sel a, SumJob* jobs) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   if (a.ctl[0]) return;
   const int64_t P = (int64_t)a.T * 2;
@@ -1774,6 +1787,7 @@ __global__ void __launch_bounds__(1024) bjobs_kernel(Sel a, SumJob* jobs) {
 }
 
 __global__ void __launch_bounds__(1024) bchoose_kernel(Sel a, const SumJob* jobs, float* d_mean, int64_t* out_offsets) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   if (a.ctl[0]) return;
   int64_t carry = 0;
@@ -1799,6 +1813,7 @@ __global__ void __launch_bounds__(1024) bchoose_kernel(Sel a, const SumJob* jobs
 
 __global__ void bemit_kernel(Sel a, const float* d_mean, const int64_t* out_offsets,
                              int64_t bound, int32_t* out_idx, float* out_val) {
+  pdl_begin();
   if (a.ctl[0]) return;
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= bound || j >= out_offsets[a.T]) return;
@@ -1825,6 +1840,7 @@ constexpr int kMagBlock = 1024;  // list positions per compaction block (4 per t
 __global__ void __launch_bounds__(1024) mjobs_kernel(const float* lval, const int64_t* loff, int32_t T,
                                                      int64_t pair_bound, SumJob* jobs,
                                                      const int32_t* abort_flag) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   if (*abort_flag) return;
   int64_t carry = 0;
@@ -1855,6 +1871,7 @@ __global__ void __launch_bounds__(1024) mjobs_kernel(const float* lval, const in
 __global__ void __launch_bounds__(1024) mchoose_kernel(const SumJob* jobs, int32_t T, int32_t* bsel,
                                                        float* d_mean, int64_t* out_offsets,
                                                        const int32_t* abort_flag) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   if (*abort_flag) return;
   int64_t carry = 0;
@@ -1889,6 +1906,7 @@ __device__ __forceinline__ bool mag_chosen(const int32_t* bsel, const int64_t* l
 __global__ void __launch_bounds__(256) mcount_kernel(const int32_t* bsel, const int64_t* loff, int32_t T,
                                                      const float* lval, int64_t* bcnt,
                                                      const int32_t* abort_flag) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   if (*abort_flag) return;
   const int64_t K = loff[T];
@@ -1904,6 +1922,7 @@ __global__ void __launch_bounds__(256) mcount_kernel(const int32_t* bsel, const 
 }
 
 __global__ void __launch_bounds__(1024) mscan_kernel(int64_t* bcnt, int64_t nblk, const int32_t* abort_flag) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   if (*abort_flag) return;
   int64_t carry = 0;
@@ -1925,6 +1944,7 @@ __global__ void __launch_bounds__(256) memit_kernel(const int32_t* bsel, const i
                                                     const int64_t* bcnt, const float* d_mean, float* r,
                                                     int32_t* out_idx, float* out_val, int64_t out_capacity,
                                                     int32_t* d_status, const int32_t* abort_flag) {
+  pdl_begin();
   __shared__ int64_t sh[33];
   if (*abort_flag) return;
   const int64_t K = loff[T];
@@ -1965,6 +1985,7 @@ __global__ void __launch_bounds__(256) memit_kernel(const int32_t* bsel, const i
 // With momentum (u non-null) the gradient term is v = fl(fl(mom * u) + g), and u <- v.
 __global__ void accumulate_kernel(const float* g, float* r, int64_t n, const int32_t* ctl,
                                   int64_t* out_offsets, float* u, float mom) {
+  pdl_begin();
   if (ctl && ctl[0]) return;
   if (!ctl && out_offsets && blockIdx.x == 0 && threadIdx.x < 2) out_offsets[threadIdx.x] = 0;
   const int64_t nv = n >> 2;
@@ -2174,7 +2195,7 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   if (num == 0 && C == 1 && !has_pending && seg == nullptr) {
     // communication delay step on one segment: accumulate only, nothing to plan
     const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
-    accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, nullptr, out_offsets,
+    launch(accumulate_kernel, (unsigned)(blocks > 0 ? blocks : 1), 256, 0, st, g, r, n, nullptr, out_offsets,
                                                                           u, mom);
     return launch_status();
   }
@@ -2183,13 +2204,13 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   a.pw_count = has_pending ? pending->d_count : nullptr;
   a.pw_cap = has_pending ? pending->capacity : 0;
   if (cudaMemsetAsync(L.zero_begin, 0, L.zero_bytes, st) != cudaSuccess) return GSPARSE_ERR_CUDA;
-  plan_kernel<<<1, 1024, 0, st>>>(a, seg, num, den, out_capacity, C == 1 ? out_offsets : nullptr);
+  launch(plan_kernel, 1, 1024, 0, st, a, seg, num, den, out_capacity, C == 1 ? out_offsets : nullptr);
   if (has_pending)
-    pending_check_kernel<<<(unsigned)cdiv(a.pw_cap + 1, 256 * kCheckPer), 256, 0, st>>>(a);
+    launch(pending_check_kernel, (unsigned)cdiv(a.pw_cap + 1, 256 * kCheckPer), 256, 0, st, a);
   if (num == 0 && C == 1 && !has_pending) {  // communication delay step: accumulate only
     if (n > 0) {
       const int64_t blocks = cdiv(n, 4 * 256) < 148 * 8 ? cdiv(n, 4 * 256) : 148 * 8;
-      accumulate_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, st>>>(g, r, n, a.ctl, nullptr, u,
+      launch(accumulate_kernel, (unsigned)(blocks > 0 ? blocks : 1), 256, 0, st, g, r, n, a.ctl, nullptr, u,
                                                                             mom);
     }
     return launch_status();
@@ -2197,8 +2218,8 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   const unsigned piece_ctas = (unsigned)cdiv(L.Q, kWarps);
   const int exhaustive = (flags & GSPARSE_SELECT_EXHAUSTIVE) ? 1 : 0;
   const dim3 sgrid(kSampleCtas, (unsigned)T);
-  sample_kernel<C><<<sgrid, 256, 0, st>>>(a, 1, exhaustive);
-  sample_kernel<C><<<sgrid, 256, 0, st>>>(a, 2, exhaustive);
+  launch(sample_kernel<C>, sgrid, 256, 0, st, a, 1, exhaustive);
+  launch(sample_kernel<C>, sgrid, 256, 0, st, a, 2, exhaustive);
   const bool timed = events && events->before && events->after;
   if (timed) cudaEventRecord((cudaEvent_t)events->before, st);
   if (piece_ctas) {
@@ -2207,7 +2228,7 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
         if (cudaFuncSetAttribute(pass1_ring_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kRingBytesM) != cudaSuccess)
           return GSPARSE_ERR_CUDA;
-        pass1_ring_kernel<1, true><<<piece_ctas, kThreads, kRingBytesM, st>>>(a);
+        launch(pass1_ring_kernel<1, true>, piece_ctas, kThreads, kRingBytesM, st, a);
       } else {
         // two streams through the 3-stage ring: faster than the register pipeline on flat
         // gradients (2% at a 99% drop, 9% at 90%), 4% slower when candidates cluster
@@ -2215,14 +2236,14 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
         if (cudaFuncSetAttribute(pass1_ring_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kRingBytes) != cudaSuccess)
           return GSPARSE_ERR_CUDA;
-        pass1_ring_kernel<1, false><<<piece_ctas, kThreads, kRingBytes, st>>>(a);
+        launch(pass1_ring_kernel<1, false>, piece_ctas, kThreads, kRingBytes, st, a);
       }
     } else {
-      pass1_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
+      launch(pass1_kernel<C>, piece_ctas, kThreads, 0, st, a);
     }
   }
   if (timed) cudaEventRecord((cudaEvent_t)events->after, st);
-  check_kernel<<<(unsigned)(T * C), 256, 0, st>>>(a);
+  launch(check_kernel, (unsigned)(T * C), 256, 0, st, a);
   // the steps after pass 1 run over work units, at most a.units_bound of them
   int64_t uc = cdiv(a.units_bound, kWarps);
   if (uc > (int64_t)sm_count() * 8) uc = (int64_t)sm_count() * 8;
@@ -2230,23 +2251,23 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   // with few problems each select level (and the scan) runs as the tail of the kernel before it
   const bool fuse = piece_ctas && (int64_t)T * C <= kFuseProblems;
   a.fuse_tail = fuse ? 1 : 0;
-  if (piece_ctas) restore_kernel<C><<<piece_ctas, kThreads, 0, st>>>(a);
-  if (!fuse) select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 1);
-  if (unit_ctas) hist_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a, 2);
-  if (!fuse) select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 2);
-  if (unit_ctas) hist_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a, 3);
-  if (!fuse) select_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a, 3);
-  if (unit_ctas) count_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a);
-  if (!fuse) scan_kernel<<<(unsigned)(T * C), 1024, 0, st>>>(a);
+  if (piece_ctas) launch(restore_kernel<C>, piece_ctas, kThreads, 0, st, a);
+  if (!fuse) launch(select_kernel, (unsigned)(T * C), 1024, 0, st, a, 1);
+  if (unit_ctas) launch(hist_kernel<C>, unit_ctas, kThreads, 0, st, a, 2);
+  if (!fuse) launch(select_kernel, (unsigned)(T * C), 1024, 0, st, a, 2);
+  if (unit_ctas) launch(hist_kernel<C>, unit_ctas, kThreads, 0, st, a, 3);
+  if (!fuse) launch(select_kernel, (unsigned)(T * C), 1024, 0, st, a, 3);
+  if (unit_ctas) launch(count_kernel<C>, unit_ctas, kThreads, 0, st, a);
+  if (!fuse) launch(scan_kernel, (unsigned)(T * C), 1024, 0, st, a);
   if (unit_ctas)
-    emit_kernel<C><<<unit_ctas, kThreads, 0, st>>>(a, out_idx, out_val,
+    launch(emit_kernel<C>, unit_ctas, kThreads, 0, st, a, out_idx, out_val,
                                                     C == 1 ? out_capacity : 2 * L.kbound);
   if (C == 2) {
-    bjobs_kernel<<<1, 1024, 0, st>>>(a, L.jobs);
+    launch(bjobs_kernel, 1, 1024, 0, st, a, L.jobs);
     osum_launch(L.jobs, T * 2, L.leaves, L.leaf_bound, L.per_job_leaf_bound, L.partials, a.ctl, st);
-    bchoose_kernel<<<1, 1024, 0, st>>>(a, L.jobs, d_mean, out_offsets);
+    launch(bchoose_kernel, 1, 1024, 0, st, a, L.jobs, d_mean, out_offsets);
     if (L.kbound > 0)
-      bemit_kernel<<<(unsigned)cdiv(L.kbound, 256), 256, 0, st>>>(a, d_mean, out_offsets, L.kbound,
+      launch(bemit_kernel, (unsigned)cdiv(L.kbound, 256), 256, 0, st, a, d_mean, out_offsets, L.kbound,
                                                                   out_idx, out_val);
   }
   return launch_status();
@@ -2307,13 +2328,13 @@ int run_binarize_magnitude(const float* g, float* r, int64_t n, const int64_t* s
                                flags & GSPARSE_SELECT_EXHAUSTIVE, tws, tws_bytes, d_status, st, events);
   if (rc != GSPARSE_OK) return rc;
   const int32_t* abort_flag = carve(n, T, 1, num, den, tws, tws_bytes, false).a.ctl;
-  mjobs_kernel<<<1, 1024, 0, st>>>(M.lval, M.loff, T, M.leaf_bound, M.jobs, abort_flag);
+  launch(mjobs_kernel, 1, 1024, 0, st, M.lval, M.loff, T, M.leaf_bound, M.jobs, abort_flag);
   osum_launch_pairs(M.jobs, T, M.leaves, M.leaf_bound, M.per_job, M.partials, abort_flag, st);
-  mchoose_kernel<<<1, 1024, 0, st>>>(M.jobs, T, M.bsel, d_mean, out_offsets, abort_flag);
+  launch(mchoose_kernel, 1, 1024, 0, st, M.jobs, T, M.bsel, d_mean, out_offsets, abort_flag);
   if (M.kb > 0) {
-    mcount_kernel<<<(unsigned)M.nblk, 256, 0, st>>>(M.bsel, M.loff, T, M.lval, M.bcnt, abort_flag);
-    mscan_kernel<<<1, 1024, 0, st>>>(M.bcnt, M.nblk, abort_flag);
-    memit_kernel<<<(unsigned)M.nblk, 256, 0, st>>>(M.bsel, M.loff, T, M.lidx, M.lval, M.bcnt, d_mean, r,
+    launch(mcount_kernel, (unsigned)M.nblk, 256, 0, st, M.bsel, M.loff, T, M.lval, M.bcnt, abort_flag);
+    launch(mscan_kernel, 1, 1024, 0, st, M.bcnt, M.nblk, abort_flag);
+    launch(memit_kernel, (unsigned)M.nblk, 256, 0, st, M.bsel, M.loff, T, M.lidx, M.lval, M.bcnt, d_mean, r,
                                                    out_idx, out_val, out_capacity, d_status, abort_flag);
   }
   return launch_status();

@@ -75,11 +75,12 @@ enum gsparse_select_flags {
   GSPARSE_SELECT_EXHAUSTIVE = 1,
   /* gsparse_binarize only: the magnitude-first reading of sparse binarisation (see there). */
   GSPARSE_BINARIZE_BY_MAGNITUDE = 2,
-  /* Test hook for the failure path, never for production use: in gsparse_residual_topk_momentum
-     the first bounded wait of every warp of the streaming pass waits on a barrier that nothing
-     completes, with a limit of 2^16 SM cycles. The wait runs out, GSPARSE_DERR_TIMEOUT is
-     raised, the rest of the call does nothing, and residual, momentum buffer and outputs are
-     left partly updated (not valid); the context stays usable. No effect on the other calls. */
+  /* Test hook for the failure path, never for production use: in gsparse_residual_topk and
+     gsparse_residual_topk_momentum the first bounded wait of every warp of the streaming pass
+     waits on a barrier that nothing completes, with a limit of 2^16 SM cycles. The wait runs
+     out, GSPARSE_DERR_TIMEOUT is raised, the rest of the call does nothing, and residual,
+     momentum buffer and outputs are left partly updated (not valid); the context stays usable.
+     No effect on gsparse_binarize (its streaming pass has no waits). */
   GSPARSE_SELECT_TEST_EXPIRE_WAIT = 4
 };
 

@@ -48,18 +48,40 @@ def test_expired_wait_reports_timeout_and_the_next_call_is_exact():
     assert np.array_equal(bits(host(ud)), bits(wu))
 
 
-def test_the_hook_does_nothing_outside_the_momentum_pass():
-    # plain top-k streams through registers (no waits): the flag changes nothing
-    n, keep = 300001, (1, 100)
-    g = synth.flat_mixture(n, seed=73)
-    r = synth.gaussian(n, 74, sigma=1e-4)
-    rd = dev(r)
+def test_expired_wait_in_plain_topk_reports_timeout():
+    # plain top-k streams through the same ring: the hook makes its first waits run out too, and
+    # the next call (residual restored) equals the oracle
+    n, keep = (1 << 22) + 9, (1, 100)
+    g = synth.flat_mixture(n, seed=75)
+    r = synth.gaussian(n, 76, sigma=1e-4)
+    gd, rd = dev(g), dev(r)
     st = gs.status_tensor()
-    gi, gv, go = gs.residual_topk(dev(g), rd, keep, d_status=st, flags=gs.GSPARSE_SELECT_TEST_EXPIRE_WAIT)
+    gs.residual_topk(gd, rd, keep, d_status=st, flags=gs.GSPARSE_SELECT_TEST_EXPIRE_WAIT)
+    torch.cuda.synchronize()
+    assert int(st.item()) & gs.DERR_TIMEOUT
+    rd.copy_(dev(r))
+    st2 = gs.status_tensor()
+    gi, gv, go = gs.residual_topk(gd, rd, keep, d_status=st2)
     wi, wv, wo, wr = oracle.residual_topk(g, r, keep)
     K = int(host(go)[-1])
+    assert int(host(st2)[0]) == 0
+    assert np.array_equal(host(gi)[:K], wi) and np.array_equal(bits(host(gv)[:K]), bits(wv))
+    assert np.array_equal(bits(host(rd)), bits(wr))
+
+
+def test_the_hook_does_nothing_in_binarize():
+    # sparse binarisation streams through registers (no waits): the flag changes nothing
+    n, keep = 300001, (1, 1000)
+    g = synth.gaussian(n, 73, sigma=1e-2)
+    r = synth.gaussian(n, 74, sigma=1e-3)
+    rd = dev(r)
+    st = gs.status_tensor()
+    gi, gv, gm, go = gs.binarize(dev(g), rd, keep, d_status=st, flags=gs.GSPARSE_SELECT_TEST_EXPIRE_WAIT)
+    wi, wv, wm, wo, wr = oracle.binarize(g, r, keep)
+    K = int(host(go)[-1])
     assert int(host(st)[0]) == 0
-    assert np.array_equal(host(gi)[:K], wi) and np.array_equal(bits(host(rd)), bits(wr))
+    assert np.array_equal(host(gi)[:K], wi) and np.array_equal(bits(host(gm)), bits(wm))
+    assert np.array_equal(bits(host(rd)), bits(wr))
 
 
 def test_pass_events_are_per_call():
