@@ -593,8 +593,9 @@ __device__ __forceinline__ int cand_class(float x) {
 struct P1State {
   uint32_t count;   // candidates found so far
   uint32_t cp;      // next pending write of this piece
-  int32_t win_idx;  // pending window (entry cp + lane), loaded one chunk ahead
-  float win_val;
+  // pending window of 64 writes (entries cp + lane and cp + 32 + lane), loaded one chunk ahead
+  int32_t win_idx, win_idx2;
+  float win_val, win_val2;
   // the store: positions below `room` have slots; the newest region (primary store or pool
   // chunk) starts at position ch_lo, slot ch_base; the one before it at pv_lo, pv_base
   uint32_t room, nch, ch_lo, pv_lo;
@@ -627,6 +628,8 @@ __device__ __forceinline__ void load_window(const Sel& a, uint32_t cp, uint32_t 
   const uint32_t j = cp + lane;
   S.win_idx = j < cend ? a.pw_idx[j] : INT32_MAX;
   S.win_val = j < cend ? a.pw_val[j] : 0.0f;
+  S.win_idx2 = j + 32 < cend ? a.pw_idx[j + 32] : INT32_MAX;
+  S.win_val2 = j + 32 < cend ? a.pw_val[j + 32] : 0.0f;
 }
 
 // One chunk of 512 entries [base, base + 512) of the piece [lo, hi): pending writes, acc, the
@@ -639,7 +642,7 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
                                             uint32_t hi, bool full, uint32_t valid,
                                             float4 (&gv)[4], float4 (&rv)[4], P1State& S,
                                             uint32_t cend, const uint32_t (&tl)[C], float* st,
-                                            uint16_t* cs, uint32_t* hsink, int hstride, int lane,
+                                            uint32_t* hsink, int hstride, int lane,
                                             const float* gs_ = nullptr, const float* us_ = nullptr) {
   float4* st4 = reinterpret_cast<float4*>(st);
   float* r = a.r;
@@ -648,14 +651,17 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
     if (S.cp < cend) {
       const uint32_t lim = base + (uint32_t)kGranule;
       for (;;) {
+        // the window's writes inside the chunk are a prefix of it (the list ascends)
         const bool in = S.win_idx >= (int32_t)base && S.win_idx < (int32_t)lim;
-        const uint32_t mask = __ballot_sync(kFull, in);
+        const bool in2 = S.win_idx2 >= (int32_t)base && S.win_idx2 < (int32_t)lim;
+        const uint32_t mask = __ballot_sync(kFull, in), mask2 = __ballot_sync(kFull, in2);
         if (!mask) break;
         if (in) st[S.win_idx - (int32_t)base] = S.win_val;
-        S.cp += __popc(mask);
+        if (in2) st[S.win_idx2 - (int32_t)base] = S.win_val2;
+        S.cp += __popc(mask) + __popc(mask2);
         __syncwarp();
         load_window(a, S.cp, cend, lane, S);
-        if (mask != kFull) break;
+        if (mask2 != kFull) break;
       }
     }
     const float4* g4 = reinterpret_cast<const float4*>(gs_);
@@ -679,8 +685,10 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
     const uint32_t lim = base + (uint32_t)kGranule < hi ? base + (uint32_t)kGranule : hi;
     bool staged = false;
     for (;;) {
+      // the window's writes inside the chunk are a prefix of it (the list ascends)
       const bool in = S.win_idx >= (int32_t)base && S.win_idx < (int32_t)lim;
-      const uint32_t mask = __ballot_sync(kFull, in);
+      const bool in2 = S.win_idx2 >= (int32_t)base && S.win_idx2 < (int32_t)lim;
+      const uint32_t mask = __ballot_sync(kFull, in), mask2 = __ballot_sync(kFull, in2);
       if (!mask) break;
       if (!staged) {
 #pragma unroll
@@ -689,10 +697,11 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
         staged = true;
       }
       if (in) st[S.win_idx - (int32_t)base] = S.win_val;
-      S.cp += __popc(mask);
+      if (in2) st[S.win_idx2 - (int32_t)base] = S.win_val2;
+      S.cp += __popc(mask) + __popc(mask2);
       __syncwarp();
       load_window(a, S.cp, cend, lane, S);   // the next window (for this chunk if it was full)
-      if (mask != kFull) break;
+      if (mask2 != kFull) break;
     }
     if (staged) {
 #pragma unroll
@@ -717,47 +726,38 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
   const uint32_t tot = __shfl_sync(kFull, incl, 31);
   bool from_stage = false;
   if (tot) {
-    const uint32_t excl = incl - packed;
-    const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu;
-    const uint32_t ntot = t0 + t1 + t2 + (tot >> 24);
-    p1_reserve(a, q, ntot, S, lane);
-    // candidates that find a slot: ranks below `lim` (the store fills in rank order)
-    const uint32_t lim = S.room > S.count ? S.room - S.count : 0u;
-    // the chunk in shared memory (entry base + o at offset o); its candidates' offsets compacted in
-    // index order (rank r = store position - count) in the warp's staging row
 #pragma unroll
     for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = av[u];
+    __syncwarp();
+    const uint32_t excl = incl - packed;
+    const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu;
+    p1_reserve(a, q, t0 + t1 + t2 + (tot >> 24), S, lane);
+    uint32_t stored = 0;
     for (uint32_t m = m16; m; m &= m - 1) {
       const int b = __ffs(m) - 1;
       const int u = b >> 2, e = b & 3;
       const uint32_t before = (u >= 1 ? t0 : 0u) + (u >= 2 ? t1 : 0u) + (u >= 3 ? t2 : 0u);
-      const uint32_t r = before + ((excl >> (8 * u)) & 0xFFu) +
-                         __popc(m16 & ((1u << b) - 1u) & (0xFu << (4 * u)));
-      cs[r] = (uint16_t)(u * 128 + lane * 4 + e);
-    }
-    __syncwarp();
-    // rows to the store (consecutive ranks -> consecutive slots of the newest regions) and the
-    // histogram, one shared atomic per distinct bin of each row; stored candidates leave the
-    // residual as +0 (the not-sent ones get acc back later)
-    for (uint32_t j0 = 0; j0 < ntot; j0 += 32) {
-      const uint32_t r = j0 + (uint32_t)lane;
-      const bool in = r < ntot;
-      const uint32_t o = in ? cs[r] : 0u;
-      const float x = in ? st[o] : 0.0f;
-      const uint32_t bin = in ? (uint32_t)cand_class<C>(x) * (uint32_t)hstride + (mag_key(x) >> 20) : 0xFFFFFFFFu;
-      const uint32_t peers = __match_any_sync(kFull, bin);
-      if (in && lane == __ffs(peers) - 1) atomicAdd(hsink + bin, (uint32_t)__popc(peers));
-      if (in && r < lim) {
-        const uint32_t pos = S.count + r;
+      const uint32_t pos = S.count + before + ((excl >> (8 * u)) & 0xFFu) +
+                           __popc(m16 & ((1u << b) - 1u) & (0xFu << (4 * u)));
+      const float x = st[(u * 32 + lane) * 4 + e];
+      if (pos < S.room) {
         const int64_t slot = pos >= S.ch_lo ? S.ch_base + (pos - S.ch_lo) : S.pv_base + (pos - S.pv_lo);
-        a.cidx[slot] = (int32_t)(base + o);
+        a.cidx[slot] = (int32_t)(base + u * 128 + lane * 4 + e);
         a.cval[slot] = x;
-        if (a.zero_mode) st[o] = 0.0f;
+        stored |= 1u << b;
       }
+      atomicAdd(hsink + cand_class<C>(x) * hstride + (mag_key(x) >> 20), 1u);
     }
-    from_stage = a.zero_mode != 0;
-    __syncwarp();
-    S.count += ntot;
+    S.count += t0 + t1 + t2 + (tot >> 24);
+    if (a.zero_mode) {
+      // stored candidates leave the residual as +0 (the not-sent ones get acc back later)
+      for (uint32_t m = stored; m; m &= m - 1) {
+        const int b = __ffs(m) - 1;
+        st[((b >> 2) * 32 + lane) * 4 + (b & 3)] = 0.0f;
+      }
+      __syncwarp();
+      from_stage = true;
+    }
   }
   if (full) {
 #pragma unroll
@@ -814,7 +814,6 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
   pdl_begin();
   __shared__ CtaHist<C, kBins1> H;
   __shared__ __align__(16) float stage[kWarps * kGranule];  // per warp: one chunk, entry order
-  __shared__ uint16_t cstage[kWarps * kGranule];            // per warp: a chunk's candidate offsets
   if (a.ctl[0]) return;
   const int64_t q0 = (int64_t)blockIdx.x * kWarps;
   H.init(a, q0);
@@ -832,7 +831,6 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     const int hstride = sh_sink ? kBins1 : kHist;
     const uint32_t lo = (uint32_t)P.lo, hi = (uint32_t)P.hi;  // indices are below 2^31
     float* st = stage + wid * kGranule;
-    uint16_t* cs = cstage + wid * kGranule;
     // pending residual writes of this piece start at the first index >= lo
     const uint32_t cend = pending_count(a);
     P1State S;
@@ -848,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     float4 gv[4], rv[4];
     if (base < lo || base + (uint32_t)kGranule > hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
-      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, cs, hsink, hstride, lane);
+      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, hsink, hstride, lane);
       base += (uint32_t)kGranule;
     }
     if (base < hi && base + (uint32_t)kGranule <= hi) {
@@ -860,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
         const uint32_t nb = base + (uint32_t)kGranule;
         const bool more = nb + (uint32_t)kGranule <= hi;
         if (more) load_full(a, nb, lane, gn, rn);
-        pass1_chunk<C>(a, q, base, lo, hi, true, 0xFFFFu, gv, rv, S, cend, tl, st, cs, hsink, hstride,
+        pass1_chunk<C>(a, q, base, lo, hi, true, 0xFFFFu, gv, rv, S, cend, tl, st, hsink, hstride,
                        lane);
         base = nb;
         if (!more) break;
@@ -868,7 +866,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     }
     if (base < hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
-      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, cs, hsink, hstride, lane);
+      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, st, hsink, hstride, lane);
     }
     if (lane == 0) {
       a.pcnt[q] = S.count;
@@ -1020,8 +1018,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
     if (base < lo || base + (uint32_t)kGranule > hi) {
       const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
       if (kMom) momentum_edge(a, base, valid, lane, gv);
-      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r,
-                     reinterpret_cast<uint16_t*>(ring[0].g), hsink, hstride, lane);
+      pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r, hsink, hstride, lane);
       base += (uint32_t)kGranule;
     }
     // interior chunks [base, base + nint * 512) through the ring (base is 16-byte aligned)
@@ -1061,10 +1058,8 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
       parity ^= 1u << k;
       const float* us_ = nullptr;
       if constexpr (kMom) us_ = ring[k].u;
-      // the slot's g rows are read into registers first, then reused as the staging row
       pass1_chunk<C, true>(a, q, base + c * (uint32_t)kGranule, lo, hi, true, 0xFFFFu, gv, rv, S, cend,
-                           tl, ring[k].r, reinterpret_cast<uint16_t*>(ring[k].g), hsink,
-                           hstride, lane, ring[k].g, us_);
+                           tl, ring[k].r, hsink, hstride, lane, ring[k].g, us_);
     }
     if (failed) {
       if (lane == 0) {
@@ -1082,8 +1077,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
       if (base < hi) {
         const uint32_t valid = load_edge(a, base, lo, hi, lane, gv, rv);
         if (kMom) momentum_edge(a, base, valid, lane, gv);
-        pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r,
-                       reinterpret_cast<uint16_t*>(ring[0].g), hsink, hstride, lane);
+        pass1_chunk<C>(a, q, base, lo, hi, false, valid, gv, rv, S, cend, tl, ring[0].r, hsink, hstride, lane);
       }
     }
     if (lane == 0) {
@@ -1562,7 +1556,7 @@ __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_
                                           int64_t limit, EmitStage& stg);
 
 template <int C>
-__global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
+__global__ void __launch_bounds__(kThreads, 3) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
                                                         int64_t limit) {
   pdl_begin();
   __shared__ EmitStage stage[kWarps];
@@ -1667,14 +1661,16 @@ __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_
             if ((sm >> e) & 1u) { stg.idx[k] = iv[e]; stg.val[k] = xv[e]; ++k; }
           __syncwarp();
           const int64_t o0 = base_out[cc] + sel_run[cc];
-          int32_t* oi = C == 1 ? out_idx : a.lidx;
-          float* ov = C == 1 ? out_val : a.lval;
-          for (uint32_t t = (uint32_t)lane; t < tsel; t += 32) {
-            const int64_t o = o0 + t;
+          int32_t* oi = (C == 1 ? out_idx : a.lidx) + o0;
+          float* ov = (C == 1 ? out_val : a.lval) + o0;
+          // positions past the output's capacity are dropped (and reported)
+          const int64_t room = limit - o0;
+          const uint32_t nfit = room <= 0 ? 0u : (room < (int64_t)tsel ? (uint32_t)room : tsel);
+          if (nfit < tsel && lane == 0) raise(a.d_status, GSPARSE_DERR_CAPACITY);
+          for (uint32_t t = (uint32_t)lane; t < nfit; t += 32) {
             const int32_t i = stg.idx[t];
-            if (o >= limit) { raise(a.d_status, GSPARSE_DERR_CAPACITY); continue; }
-            oi[o] = i;
-            ov[o] = stg.val[t];
+            oi[t] = i;
+            ov[t] = stg.val[t];
             if (C == 1 && a.u) a.u[i] = 0.0f;  // momentum masking of the sent entry
           }
           __syncwarp();
