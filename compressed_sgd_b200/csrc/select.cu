@@ -95,30 +95,7 @@ struct Sel {
   int32_t* lidx;
   float* lval;
   int32_t* bsel;
-  // few problems: the select levels and the unit scan run in the last CTA of the kernel before
-  // them instead of as launches of their own
-  int32_t fuse_tail;
-  int32_t pad2;
 };
-
-// ctl words: [0] abort, [1] any redo, [2] next free pool chunk, [8 + k] done-CTA counters of the
-// kernels that end in a fused tail (k: 0 restore, 1 histogram level 2, 2 level 3, 3 count)
-constexpr int kCtlDone = 8;
-constexpr int kFuseProblems = 2;
-
-// True in every thread of the CTA that finishes the kernel last (counter ctl[kCtlDone + k]); its
-// earlier global writes and atomics, and those of all other CTAs, are then visible to it.
-__device__ __forceinline__ bool last_cta(const Sel& a, int k) {
-  __shared__ int is_last;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    is_last = atomicAdd(reinterpret_cast<uint32_t*>(a.ctl + kCtlDone + k), 1u) == gridDim.x - 1;
-  }
-  __syncthreads();
-  if (is_last) __threadfence();
-  return is_last != 0;
-}
 
 struct Piece {
   int64_t lo, hi;
@@ -1281,7 +1258,6 @@ __global__ void __launch_bounds__(kThreads) restore_kernel(Sel a) {
   __syncthreads();
   // only redone problems received counts here
   H.flush(a, 1, kBins1);
-  if (a.fuse_tail && last_cta(a, 0)) select_tail(a, 1, H.sh);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1381,14 +1357,6 @@ __global__ void __launch_bounds__(1024) select_kernel(Sel a, int level) {
   select_problem(a, blockIdx.x, level, h, sh);
 }
 
-// The fused tail of a kernel that ran with a.fuse_tail: every problem's select at this level (and
-// before level 1, the numbering of the work units), in the last CTA to finish.
-__device__ void select_tail(const Sel& a, int level, uint32_t* h) {
-  __shared__ int64_t sh[33];
-  if (level == 1) number_units(a, sh);
-  __syncthreads();
-  for (int64_t p = 0; p < (int64_t)a.T * a.C; ++p) select_problem(a, p, level, h, sh);
-}
 
 template <int C>
 __global__ void __launch_bounds__(kThreads) hist_kernel(Sel a, int level) {
@@ -1418,13 +1386,10 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(Sel a, int level) {
   }
   __syncthreads();
   H.flush(a, level, level == 2 ? kBins2 : kBins3);
-  if (a.fuse_tail && last_cta(a, level - 1)) select_tail(a, level, H.sh);
 }
 
 // ------------------------------------------------------------------------------------------
 // 8. count + scan
-
-__device__ void scan_problem(const Sel& a, int64_t p, int64_t* sh);
 
 template <int C>
 __global__ void __launch_bounds__(kThreads) count_kernel(Sel a) {
@@ -1460,13 +1425,6 @@ __global__ void __launch_bounds__(kThreads) count_kernel(Sel a) {
         a.pgt[u * C + c] = G;
         a.peq[u * C + c] = E;
       }
-    }
-  }
-  if (a.fuse_tail && last_cta(a, 3)) {
-    __shared__ int64_t sh[33];
-    for (int64_t p = 0; p < (int64_t)a.T * a.C; ++p) {
-      scan_problem(a, p, sh);
-      __syncthreads();
     }
   }
 }
@@ -1556,7 +1514,7 @@ __device__ __forceinline__ void emit_unit(const Sel& a, int64_t u, int32_t* out_
                                           int64_t limit, EmitStage& stg);
 
 template <int C>
-__global__ void __launch_bounds__(kThreads, 3) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
+__global__ void __launch_bounds__(kThreads, 4) emit_kernel(Sel a, int32_t* out_idx, float* out_val,
                                                         int64_t limit) {
   pdl_begin();
   __shared__ EmitStage stage[kWarps];
@@ -2244,17 +2202,14 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   int64_t uc = cdiv(a.units_bound, kWarps);
   if (uc > (int64_t)sm_count() * 8) uc = (int64_t)sm_count() * 8;
   const unsigned unit_ctas = piece_ctas ? (unsigned)uc : 0u;
-  // with few problems each select level (and the scan) runs as the tail of the kernel before it
-  const bool fuse = piece_ctas && (int64_t)T * C <= kFuseProblems;
-  a.fuse_tail = fuse ? 1 : 0;
   if (piece_ctas) launch(restore_kernel<C>, piece_ctas, kThreads, 0, st, a);
-  if (!fuse) launch(select_kernel, (unsigned)(T * C), 1024, 0, st, a, 1);
+  launch(select_kernel, (unsigned)(T * C), 1024, 0, st, a, 1);
   if (unit_ctas) launch(hist_kernel<C>, unit_ctas, kThreads, 0, st, a, 2);
-  if (!fuse) launch(select_kernel, (unsigned)(T * C), 1024, 0, st, a, 2);
+  launch(select_kernel, (unsigned)(T * C), 1024, 0, st, a, 2);
   if (unit_ctas) launch(hist_kernel<C>, unit_ctas, kThreads, 0, st, a, 3);
-  if (!fuse) launch(select_kernel, (unsigned)(T * C), 1024, 0, st, a, 3);
+  launch(select_kernel, (unsigned)(T * C), 1024, 0, st, a, 3);
   if (unit_ctas) launch(count_kernel<C>, unit_ctas, kThreads, 0, st, a);
-  if (!fuse) launch(scan_kernel, (unsigned)(T * C), 1024, 0, st, a);
+  launch(scan_kernel, (unsigned)(T * C), 1024, 0, st, a);
   if (unit_ctas)
     launch(emit_kernel<C>, unit_ctas, kThreads, 0, st, a, out_idx, out_val,
                                                     C == 1 ? out_capacity : 2 * L.kbound);
