@@ -161,7 +161,7 @@ def run_ours(args, rank, world, dist):
     keep = keep_of(args.drop)
     b = gs.golomb_b_star(1.0 - args.drop)
     cap = gs.k_for(n, keep)
-    chunk = 64
+    chunk = gs.golomb_chunk_hint(cap)
 
     # inputs: generated on the host (pinned, for the end-to-end leg), copied once to the device
     g_host = []
@@ -375,7 +375,7 @@ def run_exchange(args, rank, world, dist):
     keep = keep_of(args.drop)
     b = gs.golomb_b_star(1.0 - args.drop)
     cap = gs.k_for(n, keep)
-    chunk = 64
+    chunk = gs.golomb_chunk_hint(cap)
     nch = (cap + chunk - 1) // chunk
     nwords = gs.golomb_word_capacity(cap, b, n)
     g = torch.from_numpy(synth.laplace_outliers(rank, n)).to(dev)
@@ -564,7 +564,8 @@ def run_workload(args):
     mean = [torch.zeros(T, device=dev) for _ in range(W)]
     words = [torch.empty(gs.golomb_word_capacity(cap, b, n), dtype=torch.int32, device=dev) for _ in range(W)]
     nbits = [torch.zeros(1, dtype=torch.int64, device=dev) for _ in range(W)]
-    table = [torch.empty(((cap + 63) // 64, 2), dtype=torch.int64, device=dev) for _ in range(W)]
+    chunk = gs.golomb_chunk_hint(cap)
+    table = [torch.empty(((cap + chunk - 1) // chunk, 2), dtype=torch.int64, device=dev) for _ in range(W)]
     dec = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(W)]
     out = [torch.empty(n, device=dev) for _ in range(W)]
     dense = torch.empty(n, device=dev)
@@ -599,9 +600,9 @@ def run_workload(args):
                                      means=means[w], workspace=ws_q, d_status=st, capacity=cap)
             if name in ("flat2e20", "resnet50"):
                 end = off[w][T:T + 1]
-                gs.golomb_encode(idx[w], end, b, n, chunk=64, words=words[w], nbits=nbits[w], table=table[w],
+                gs.golomb_encode(idx[w], end, b, n, chunk=chunk, words=words[w], nbits=nbits[w], table=table[w],
                                  workspace=ws_g, d_status=st, capacity=cap)
-                gs.golomb_decode(words[w], nbits[w], end, cap, b, table=table[w], chunk=64, n_limit=n,
+                gs.golomb_decode(words[w], nbits[w], end, cap, b, table=table[w], chunk=chunk, n_limit=n,
                                  out_idx=dec[w], d_status=st)
         rec(1)
         src = dec if name in ("flat2e20", "resnet50") else idx

@@ -51,6 +51,7 @@ _SIGNATURES = {
     "gsparse_version": (ctypes.c_char_p, []),
     "gsparse_k_for": (_i64, [_i64, _i64, _i64]),
     "gsparse_golomb_b_star": (_i32, [_f64]),
+    "gsparse_golomb_chunk_hint": (_i32, [_i64]),
     "gsparse_warmup_keep_num": (_i64, [_i64, _i64, _f64, _f64, _i64]),
     "gsparse_residual_topk_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
     "gsparse_residual_topk_workspace_min": (_sz, [_i64, _i32]),
@@ -137,6 +138,11 @@ def k_for(n_s: int, keep: Tuple[int, int]) -> int:
 
 def golomb_b_star(p: float) -> int:
     return int(lib().gsparse_golomb_b_star(p))
+
+
+def golomb_chunk_hint(capacity: int) -> int:
+    """Side-table chunk recommended for lists of up to `capacity` codewords."""
+    return int(lib().gsparse_golomb_chunk_hint(capacity))
 
 
 def warmup_keep(t: int, T: int, start: float = 0.25, end: float = 0.001, den: int = 1_000_000) -> Tuple[int, int]:

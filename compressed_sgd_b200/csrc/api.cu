@@ -46,6 +46,12 @@ int32_t gsparse_golomb_b_star(double p) {
   return 1 + (int32_t)floor(log2(log(phi - 1.0) / log(1.0 - p)));
 }
 
+int32_t gsparse_golomb_chunk_hint(int64_t capacity) {
+  int32_t c = 64;
+  while (c > 4 && capacity / c < 16384) c >>= 1;
+  return c;
+}
+
 int64_t gsparse_warmup_keep_num(int64_t t, int64_t T, double start, double end, int64_t den) {
   if (den <= 0 || t < 0 || T < 0 || !(start > 0.0) || !(start <= 1.0) || !(end > 0.0) || !(end <= 1.0))
     return -1;

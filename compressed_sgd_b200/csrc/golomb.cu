@@ -16,9 +16,11 @@
 namespace gs {
 namespace {
 
-constexpr int kPer = 8;                      // codewords per thread
 constexpr int kCodeThreads = 256;
-constexpr int kBlockCodes = kPer * kCodeThreads;  // codewords per block
+// codewords per thread: 8 for long lists; 2 for short ones (below kShortList), which then spread
+// over four times as many blocks
+constexpr int kPerLong = 8, kPerShort = 2;
+constexpr int64_t kShortList = 1 << 20;
 constexpr int kPackWords = 4096;             // shared word buffer of a block (128 Kbit)
 constexpr long long kLookbackCycles = 1ll << 31;  // bound of one block's look-back (about a second)
 
@@ -51,26 +53,27 @@ __device__ __forceinline__ bool list_bounds(const int64_t* d_begin, const int64_
   return !(b < 0 || l < 0 || l > capacity);
 }
 
-// Gaps of this thread's kPer consecutive codewords (entries j0 .. j0+kPer-1 of the list); an
+// Gaps of this thread's KP consecutive codewords (entries j0 .. j0+KP-1 of the list); an
 // invalid (negative) gap is reported and coded as 0. Indices are non-negative int32, so a gap
-// fits 32 bits. The eight entries come in as two 16-byte loads when they are aligned.
+// fits 32 bits. The entries come in as 16-byte loads when they are aligned.
+template <int KP>
 __device__ __forceinline__ void thread_gaps(const int32_t* x, int64_t len, int64_t base, int64_t j0,
-                                            uint32_t (&d)[kPer], int32_t* d_status) {
-  static_assert(kPer == 8, "two int4 loads per thread");
-  int32_t v[kPer];
-  if (j0 + kPer <= len && (reinterpret_cast<uintptr_t>(x + j0) & 15u) == 0) {
-    const int4 a = *reinterpret_cast<const int4*>(x + j0);
-    const int4 c = *reinterpret_cast<const int4*>(x + j0 + 4);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+                                            uint32_t (&d)[KP], int32_t* d_status) {
+  int32_t v[KP];
+  if (KP % 4 == 0 && j0 + KP <= len && (reinterpret_cast<uintptr_t>(x + j0) & 15u) == 0) {
+#pragma unroll
+    for (int h = 0; h < KP / 4; ++h) {
+      const int4 a = *reinterpret_cast<const int4*>(x + j0 + 4 * h);
+      v[4 * h] = a.x; v[4 * h + 1] = a.y; v[4 * h + 2] = a.z; v[4 * h + 3] = a.w;
+    }
   } else {
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) v[e] = j0 + e < len ? x[j0 + e] : 0;
+    for (int e = 0; e < KP; ++e) v[e] = j0 + e < len ? x[j0 + e] : 0;
   }
   int64_t prev = j0 == 0 ? base - 1 : (j0 - 1 < len ? (int64_t)x[j0 - 1] : 0);
   bool bad = false;
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) {
+  for (int e = 0; e < KP; ++e) {
     d[e] = 0;
     if (j0 + e < len) {
       const int64_t g = (int64_t)v[e] - prev - 1;
@@ -146,6 +149,7 @@ __device__ bool lookback(const uint64_t* flags, uint32_t vb, int lane, uint64_t*
 // may hold bits of the neighbouring block: those two go to head[]/tail[] and the fix-up kernel
 // merges them. A block whose bits do not fit the shared buffer (very long unary runs) looks back
 // first, zeroes its interior words and ORs its codewords into them.
+template <int KP>
 __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
     const int32_t* idx, const int64_t* d_begin, const int64_t* d_end, int64_t capacity, int64_t base,
     int b, uint32_t* words, int64_t word_capacity, uint64_t* d_nbits, int64_t* table, int32_t chunk,
@@ -169,22 +173,22 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
     }
     return;
   }
-  const int64_t nact = cdiv(len, kBlockCodes);
+  const int64_t nact = cdiv(len, (KP * kCodeThreads));
   if (len == 0) {
     if (vb == 0 && threadIdx.x == 0) *d_nbits = 0;
     return;
   }
   if ((int64_t)vb >= nact) return;
   const int32_t* x = idx + lb;
-  const int64_t jb = (int64_t)vb * kBlockCodes;
-  const int64_t j0 = jb + (int64_t)threadIdx.x * kPer;
-  uint32_t d[kPer];
-  thread_gaps(x, len, base, j0, d, d_status);
+  const int64_t jb = (int64_t)vb * (KP * kCodeThreads);
+  const int64_t j0 = jb + (int64_t)threadIdx.x * KP;
+  uint32_t d[KP];
+  thread_gaps<KP>(x, len, base, j0, d, d_status);
   // codewords of this thread: entries j0 .. j0 + nv - 1 of the list
-  const int nv = len - j0 >= kPer ? kPer : (len > j0 ? (int)(len - j0) : 0);
+  const int nv = len - j0 >= KP ? KP : (len > j0 ? (int)(len - j0) : 0);
   uint64_t lu = 0;
 #pragma unroll
-  for (int e = 0; e < kPer; ++e)
+  for (int e = 0; e < KP; ++e)
     if (e < nv) lu += (uint64_t)(d[e] >> b) + 1u + (uint32_t)b;
   const int64_t l = (int64_t)lu;
   int64_t tot;
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
     __syncthreads();
     uint32_t p = (uint32_t)ex;   // relative bit position (< 2^17 here)
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) {
+    for (int e = 0; e < KP; ++e) {
       if (e >= nv) break;
       const uint32_t q = d[e] >> b;
       const uint32_t rem = d[e] & ((1u << b) - 1u);
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
       int64_t o = o0;
       uint32_t next = e0;
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) {
+      for (int e = 0; e < KP; ++e) {
         if (e >= nv) break;
         if ((uint32_t)e == next) {
           next += (uint32_t)chunk;
@@ -301,7 +305,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
   __syncthreads();
   int64_t o = o0;
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) {
+  for (int e = 0; e < KP; ++e) {
     if (e >= nv) break;
     Code c;
     c.o = (uint64_t)o;
@@ -329,12 +333,13 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
 // The words shared by two blocks: word (S_j >> 5) for every block j > 0 that starts inside a
 // word holds the end of block j - 1 (its tail) and the start of block j (its head).
 __global__ void g_fix_kernel(const int64_t* d_begin, const int64_t* d_end, int64_t capacity,
-                             const GState* state, const uint64_t* flags, const uint32_t* head,
-                             const uint32_t* tail, uint32_t* words, int64_t word_capacity) {
+                             int32_t block_codes, const GState* state, const uint64_t* flags,
+                             const uint32_t* head, const uint32_t* tail, uint32_t* words,
+                             int64_t word_capacity) {
   pdl_begin();
   int64_t lb, len;
   if (!list_bounds(d_begin, d_end, capacity, &lb, &len) || state->abort) return;
-  const int64_t nact = cdiv(len, kBlockCodes);
+  const int64_t nact = cdiv(len, block_codes);
   const int64_t j = 1 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= nact) return;
   const uint64_t S = flags[j - 1] & kValMask;   // inclusive total of the blocks before j
@@ -623,10 +628,12 @@ struct GLayout {
   size_t bytes;
 };
 
+int32_t codes_per_thread(int64_t capacity) { return capacity < kShortList ? kPerShort : kPerLong; }
+
 GLayout g_carve(int64_t capacity, void* ws) {
   GLayout L;
   Carver cv(ws);
-  L.nblk = cdiv(capacity > 0 ? capacity : 1, kBlockCodes);
+  L.nblk = cdiv(capacity > 0 ? capacity : 1, (int64_t)codes_per_thread(capacity) * kCodeThreads);
   L.state = cv.take<GState>(1);
   L.flags = cv.take<uint64_t>(L.nblk);
   L.zero_bytes = cv.off;
@@ -662,12 +669,18 @@ int gsparse_golomb_encode(const int32_t* idx, const int64_t* d_begin, const int6
   GLayout L = g_carve(capacity, workspace);
   if (workspace_bytes < L.bytes) return GSPARSE_ERR_WORKSPACE;
   if (cudaMemsetAsync(workspace, 0, L.zero_bytes, st) != cudaSuccess) return GSPARSE_ERR_CUDA;
-  launch(g_encode_kernel, (unsigned)L.nblk, kCodeThreads, 0, st, idx, d_begin, d_end, capacity, base, b, words,
-                                                             word_capacity, d_nbits, chunk_table, chunk,
-                                                             L.state, L.flags, L.head, L.tail, d_status);
+  const int32_t kp = codes_per_thread(capacity);
+  if (kp == kPerShort)
+    launch(g_encode_kernel<kPerShort>, (unsigned)L.nblk, kCodeThreads, 0, st, idx, d_begin, d_end, capacity,
+           base, b, words, word_capacity, d_nbits, chunk_table, chunk, L.state, L.flags, L.head, L.tail,
+           d_status);
+  else
+    launch(g_encode_kernel<kPerLong>, (unsigned)L.nblk, kCodeThreads, 0, st, idx, d_begin, d_end, capacity,
+           base, b, words, word_capacity, d_nbits, chunk_table, chunk, L.state, L.flags, L.head, L.tail,
+           d_status);
   if (L.nblk > 1)
-    launch(g_fix_kernel, (unsigned)cdiv(L.nblk - 1, 256), 256, 0, st, d_begin, d_end, capacity, L.state, L.flags,
-                                                                 L.head, L.tail, words, word_capacity);
+    launch(g_fix_kernel, (unsigned)cdiv(L.nblk - 1, 256), 256, 0, st, d_begin, d_end, capacity,
+           kp * kCodeThreads, L.state, L.flags, L.head, L.tail, words, word_capacity);
   return launch_status();
 }
 

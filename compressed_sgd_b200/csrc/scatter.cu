@@ -230,19 +230,17 @@ __global__ void __launch_bounds__(kTileThreads) sa_merge_kernel(Lists L, int32_t
 
 // Fused receive side. The tile-start table (the bounds kernel above) gives each worker's entries
 // of every tile. Persistent CTAs take tiles from a shared counter, so tiles crowded with entries
-// (dense embedding rows) do not hold up the others. For each tile a CTA first requests the
-// local-gradient tile with one bulk asynchronous copy into shared memory (mbarrier completion,
-// bounded wait; the copy reads this GPU's own memory, no multicast) and the first batch of every
-// one of the first kCombPre workers' entries of the tile into registers, then adds the workers'
-// entries of the tile worker by worker into a shared accumulator (so the sums keep the fixed
-// order), streams out fl(fl(alpha * G) + fl(beta * L)) and finally clears only the entries it
+// (dense embedding rows) do not hold up the others. For each tile a CTA requests the
+// local-gradient tile first, adds the workers' entries of the tile into a shared accumulator
+// (worker by worker, so the sums keep the fixed order; four independent list loads per thread in
+// flight), streams out fl(fl(alpha * G) + fl(beta * L)) and finally clears only the entries it
 // touched, so the accumulator is zeroed once per CTA rather than once per tile.
 constexpr int kCombThreads = 256;
 constexpr int kCombPer = 4;
-constexpr int kCombPre = 2;  // workers whose first batch of entries is requested with the tile
-constexpr size_t kCombDynSmem = 2 * kTile * sizeof(float);   // the local-gradient tile + accumulator
 
-__global__ void __launch_bounds__(kCombThreads, 3) sa_combine_kernel(Lists L, int32_t W, int64_t n,
+constexpr int kCombPre = 2;  // workers whose first batch of entries is requested together
+
+__global__ void __launch_bounds__(kCombThreads, 4) sa_combine_kernel(Lists L, int32_t W, int64_t n,
                                                                   const int64_t* start,
                                                                   uint32_t* next_tile,
                                                                   const float* Lg, float* out,
@@ -251,24 +249,16 @@ __global__ void __launch_bounds__(kCombThreads, 3) sa_combine_kernel(Lists L, in
                                                                   int32_t* d_status) {
   pdl_begin();
   constexpr int kVec = kTile / 4 / kCombThreads;  // float4s of a tile per thread
-  extern __shared__ __align__(128) unsigned char comb_dyn[];
-  float* lbuf = reinterpret_cast<float*>(comb_dyn);   // the local-gradient tile
-  float* acc = lbuf + kTile;                          // the worker-ordered sum of the tile
+  __shared__ __align__(16) float acc[kTile];
   __shared__ uint32_t touched[kTile / 32];
   __shared__ uint32_t tnext;
   __shared__ int64_t cnt[GSPARSE_MAX_WORKERS], rb[GSPARSE_MAX_WORKERS], re[GSPARSE_MAX_WORKERS];
-  __shared__ uint64_t bar;
   const int64_t ntiles = cdiv(n, kTile);
   for (int i = threadIdx.x; i < kTile; i += blockDim.x) acc[i] = 0.0f;
   for (int i = threadIdx.x; i < kTile / 32; i += blockDim.x) touched[i] = 0u;
-  if (threadIdx.x == 0) {
-    tnext = atomicAdd(next_tile, 1u);
-    mbar_init(&bar, 1);
-  }
-  fence_mbarrier_init();
+  if (threadIdx.x == 0) tnext = atomicAdd(next_tile, 1u);
   __syncthreads();
   int64_t t = tnext;
-  uint32_t phase = 0;
   // the entry ranges of the tile being worked on sit in rb/re; those of the next tile are loaded
   // (by thread w for worker w) while the current tile is finished
   for (int w = threadIdx.x; w < W; w += blockDim.x) {
@@ -276,32 +266,27 @@ __global__ void __launch_bounds__(kCombThreads, 3) sa_combine_kernel(Lists L, in
     if (t < ntiles) tile_range(start, t, W, w, cnt[w], &rb[w], &re[w]);
   }
   while (t < ntiles) {
-    __syncthreads();  // every thread has read tnext; rb/re hold tile t; lbuf is free
+    __syncthreads();  // every thread has read tnext; rb/re hold tile t
+    if (threadIdx.x == 0) tnext = atomicAdd(next_tile, 1u);  // claimed now, read after the tile
     const int64_t t0 = t * kTile;
     const int64_t m = (n - t0) < kTile ? (n - t0) : kTile;
-    const bool bulk = m == kTile;
-    if (threadIdx.x == 0) {
-      tnext = atomicAdd(next_tile, 1u);  // claimed now, read after the tile
-      if (bulk) {
-        mbar_arrive_expect_tx(&bar, (uint32_t)(kTile * sizeof(float)));
-        bulk_load(lbuf, Lg + t0, (uint32_t)(kTile * sizeof(float)), &bar);
-      }
+    float4 lv[kVec];
+    if (m == kTile) {
+#pragma unroll
+      for (int k = 0; k < kVec; ++k) lv[k] = ld_stream(Lg + t0 + 4 * (threadIdx.x + k * kCombThreads));
     }
-    // the first batch of the first kCombPre workers, requested together with the tile
-    int32_t pi[kCombPre][kCombPer];
-    float px[kCombPre][kCombPer];
+    // first batch of the first kCombPre workers, requested together
+    int32_t pi[kCombPre];
+    float px[kCombPre];
 #pragma unroll
     for (int w = 0; w < kCombPre; ++w) {
-#pragma unroll
-      for (int k = 0; k < kCombPer; ++k) {
-        pi[w][k] = 0;
-        px[w][k] = 0.0f;
-        if (w < W) {
-          const int64_t j = rb[w] + k * kCombThreads + threadIdx.x;
-          if (j < re[w]) {
-            pi[w][k] = L.idx[w][j];
-            px[w][k] = L.val[w] ? L.val[w][j] : (L.uni[w] ? *L.uni[w] : 0.0f);
-          }
+      pi[w] = 0;
+      px[w] = 0.0f;
+      if (w < W) {
+        const int64_t j = rb[w] + threadIdx.x;
+        if (j < re[w]) {
+          pi[w] = L.idx[w][j];
+          px[w] = L.val[w] ? L.val[w][j] : (L.uni[w] ? *L.uni[w] : 0.0f);
         }
       }
     }
@@ -313,16 +298,14 @@ __global__ void __launch_bounds__(kCombThreads, 3) sa_combine_kernel(Lists L, in
       for (int64_t jb = b; jb < e; jb += kCombThreads * kCombPer) {
         int32_t iv[kCombPer];
         float xv[kCombPer];
-        if (jb == b && w < kCombPre) {
 #pragma unroll
-          for (int k = 0; k < kCombPer; ++k) {
-            iv[k] = w == 0 ? pi[0][k] : pi[1][k];
-            xv[k] = w == 0 ? px[0][k] : px[1][k];
-          }
-        } else {
+        for (int k = 0; k < kCombPer; ++k) {
+          const int64_t j = jb + k * kCombThreads + threadIdx.x;
+          if (k == 0 && jb == b && w < kCombPre) {
 #pragma unroll
-          for (int k = 0; k < kCombPer; ++k) {
-            const int64_t j = jb + k * kCombThreads + threadIdx.x;
+            for (int ww = 0; ww < kCombPre; ++ww)
+              if (ww == w) { iv[0] = pi[ww]; xv[0] = px[ww]; }
+          } else {
             iv[k] = j < e ? ix[j] : 0;
             xv[k] = j < e ? (vv ? vv[j] : u) : 0.0f;
           }
@@ -363,30 +346,18 @@ __global__ void __launch_bounds__(kCombThreads, 3) sa_combine_kernel(Lists L, in
       }
       __syncthreads();
     }
-    if (bulk) {
-      // the local-gradient tile: every thread waits (bounded) for the copy
-      const bool ok = mbar_wait_bounded(&bar, phase);
-      phase ^= 1u;
-      if (__syncthreads_or(!ok)) {
-        if (threadIdx.x == 0) {
-          raise(d_status, GSPARSE_DERR_TIMEOUT);
-          mbar_wait_bounded(&bar, phase ^ 1u);   // let the copy land before the CTA leaves
-        }
-        return;
-      }
+    if (m == kTile) {
 #pragma unroll
       for (int k = 0; k < kVec; ++k) {
         const int v = threadIdx.x + k * kCombThreads;
         const float4 g = reinterpret_cast<const float4*>(acc)[v];
-        const float4 l = reinterpret_cast<const float4*>(lbuf)[v];
         float4 o;
-        o.x = __fadd_rn(__fmul_rn(alpha, g.x), __fmul_rn(beta, l.x));
-        o.y = __fadd_rn(__fmul_rn(alpha, g.y), __fmul_rn(beta, l.y));
-        o.z = __fadd_rn(__fmul_rn(alpha, g.z), __fmul_rn(beta, l.z));
-        o.w = __fadd_rn(__fmul_rn(alpha, g.w), __fmul_rn(beta, l.w));
+        o.x = __fadd_rn(__fmul_rn(alpha, g.x), __fmul_rn(beta, lv[k].x));
+        o.y = __fadd_rn(__fmul_rn(alpha, g.y), __fmul_rn(beta, lv[k].y));
+        o.z = __fadd_rn(__fmul_rn(alpha, g.z), __fmul_rn(beta, lv[k].z));
+        o.w = __fadd_rn(__fmul_rn(alpha, g.w), __fmul_rn(beta, lv[k].w));
         st_stream(out + t0 + 4 * v, o);
       }
-      fence_proxy_async_smem();   // these reads of lbuf come before the next copy into it
     } else {
       for (int i = threadIdx.x; i < m; i += blockDim.x)
         out[t0 + i] = __fadd_rn(__fmul_rn(alpha, acc[i]), __fmul_rn(beta, Lg[t0 + i]));
@@ -565,11 +536,8 @@ int gsparse_accumulate_combine(const gsparse_list* lists, int32_t W, int64_t n, 
   if (ntiles == 0) return launch_status();
   uint32_t* next_tile = reinterpret_cast<uint32_t*>(S.ctl + 1);
   launch_starts(Ls, W, n, ntiles, S.start, next_tile, d_status, st);
-  const int64_t ctas = (int64_t)sm_count() * 3 < ntiles ? (int64_t)sm_count() * 3 : ntiles;
-  if (cudaFuncSetAttribute(sa_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombDynSmem) !=
-      cudaSuccess)
-    return GSPARSE_ERR_CUDA;
-  launch(sa_combine_kernel, (unsigned)ctas, kCombThreads, kCombDynSmem, st, 
+  const int64_t ctas = (int64_t)sm_count() * 4 < ntiles ? (int64_t)sm_count() * 4 : ntiles;
+  launch(sa_combine_kernel, (unsigned)ctas, kCombThreads, 0, st, 
       Ls, W, n, S.start, next_tile, L, out, alpha, beta, mode == 1 ? own : -1, dense_out, d_status);
   return launch_status();
 }

@@ -569,12 +569,10 @@ __device__ __forceinline__ int cand_class(float x) {
 // Per-warp state of pass 1 over one piece.
 struct P1State {
   uint32_t count;   // candidates found so far
-  // sliding window of 128 pending writes: slot k of lane l holds list entry cp + 32 k + l. Writes
-  // of earlier chunks stay in it until the lower half is used up; then the upper half moves down
-  // and the next 64 writes are requested, about a chunk before they are needed.
-  uint32_t cp;      // list position of slot 0, lane 0
-  int32_t wi[4];
-  float wv[4];
+  uint32_t cp;      // next pending write of this piece
+  // pending window of 64 writes (entries cp + lane and cp + 32 + lane), loaded one chunk ahead
+  int32_t win_idx, win_idx2;
+  float win_val, win_val2;
   // the store: positions below `room` have slots; the newest region (primary store or pool
   // chunk) starts at position ch_lo, slot ch_base; the one before it at pv_lo, pv_base
   uint32_t room, nch, ch_lo, pv_lo;
@@ -602,43 +600,13 @@ __device__ __forceinline__ void p1_reserve(const Sel& a, int64_t q, uint32_t nee
   S.nch += 1;
 }
 
-// Slots k0 .. k1 - 1 of the window from list position cp (entries past the list read as +inf).
-__device__ __forceinline__ void load_slots(const Sel& a, uint32_t cend, int lane, P1State& S, int k0,
-                                           int k1) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    if (k < k0 || k >= k1) continue;
-    const uint32_t j = S.cp + 32u * k + lane;
-    S.wi[k] = j < cend ? a.pw_idx[j] : INT32_MAX;
-    S.wv[k] = j < cend ? a.pw_val[j] : 0.0f;
-  }
-}
-
-// Applies the pending writes in [base, lim) to the chunk staged in st (entry base + o at st[o])
-// and slides the window. The list ascends, so the window's entries below lim are a prefix of it:
-// once that prefix covers the lower half, the upper half moves down and the next 64 writes are
-// requested; a chunk holding more writes than the window reloads it whole and goes on.
-__device__ __forceinline__ void apply_pending(const Sel& a, uint32_t base, uint32_t lim, uint32_t cend,
-                                              int lane, P1State& S, float* st) {
-  for (;;) {
-    uint32_t below = 0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      if (S.wi[k] >= (int32_t)base && S.wi[k] < (int32_t)lim) st[S.wi[k] - (int32_t)base] = S.wv[k];
-      below += __popc(__ballot_sync(kFull, S.wi[k] < (int32_t)lim));
-    }
-    if (below < 64u) return;
-    __syncwarp();
-    if (below < 128u) {
-      S.wi[0] = S.wi[2]; S.wv[0] = S.wv[2];
-      S.wi[1] = S.wi[3]; S.wv[1] = S.wv[3];
-      S.cp += 64u;
-      load_slots(a, cend, lane, S, 2, 4);
-      return;
-    }
-    S.cp += 128u;   // every write of the window lies before lim: take the next 128
-    load_slots(a, cend, lane, S, 0, 4);
-  }
+__device__ __forceinline__ void load_window(const Sel& a, uint32_t cp, uint32_t cend, int lane,
+                                            P1State& S) {
+  const uint32_t j = cp + lane;
+  S.win_idx = j < cend ? a.pw_idx[j] : INT32_MAX;
+  S.win_val = j < cend ? a.pw_val[j] : 0.0f;
+  S.win_idx2 = j + 32 < cend ? a.pw_idx[j + 32] : INT32_MAX;
+  S.win_val2 = j + 32 < cend ? a.pw_val[j + 32] : 0.0f;
 }
 
 // One chunk of 512 entries [base, base + 512) of the piece [lo, hi): pending writes, acc, the
@@ -657,7 +625,22 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
   float* r = a.r;
   if (kRing) {
     // pending writes that fall in this chunk replace those residual entries in the slot
-    if (S.cp < cend) apply_pending(a, base, base + (uint32_t)kGranule, cend, lane, S, st);
+    if (S.cp < cend) {
+      const uint32_t lim = base + (uint32_t)kGranule;
+      for (;;) {
+        // the window's writes inside the chunk are a prefix of it (the list ascends)
+        const bool in = S.win_idx >= (int32_t)base && S.win_idx < (int32_t)lim;
+        const bool in2 = S.win_idx2 >= (int32_t)base && S.win_idx2 < (int32_t)lim;
+        const uint32_t mask = __ballot_sync(kFull, in), mask2 = __ballot_sync(kFull, in2);
+        if (!mask) break;
+        if (in) st[S.win_idx - (int32_t)base] = S.win_val;
+        if (in2) st[S.win_idx2 - (int32_t)base] = S.win_val2;
+        S.cp += __popc(mask) + __popc(mask2);
+        __syncwarp();
+        load_window(a, S.cp, cend, lane, S);
+        if (mask2 != kFull) break;
+      }
+    }
     const float4* g4 = reinterpret_cast<const float4*>(gs_);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -675,18 +658,29 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
     }
     __syncwarp();
   } else if (S.cp < cend) {
-    // pending residual writes that fall in this chunk replace those residual entries (the chunk
-    // goes through shared memory only when one does)
+    // pending residual writes that fall in this chunk replace those residual entries
     const uint32_t lim = base + (uint32_t)kGranule < hi ? base + (uint32_t)kGranule : hi;
-    bool any = false;
+    bool staged = false;
+    for (;;) {
+      // the window's writes inside the chunk are a prefix of it (the list ascends)
+      const bool in = S.win_idx >= (int32_t)base && S.win_idx < (int32_t)lim;
+      const bool in2 = S.win_idx2 >= (int32_t)base && S.win_idx2 < (int32_t)lim;
+      const uint32_t mask = __ballot_sync(kFull, in), mask2 = __ballot_sync(kFull, in2);
+      if (!mask) break;
+      if (!staged) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) any |= S.wi[k] >= (int32_t)base && S.wi[k] < (int32_t)lim;
-    if (__any_sync(kFull, any)) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = rv[u];
+        for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = rv[u];
+        __syncwarp();
+        staged = true;
+      }
+      if (in) st[S.win_idx - (int32_t)base] = S.win_val;
+      if (in2) st[S.win_idx2 - (int32_t)base] = S.win_val2;
+      S.cp += __popc(mask) + __popc(mask2);
       __syncwarp();
-      apply_pending(a, base, lim, cend, lane, S, st);
-      __syncwarp();
+      load_window(a, S.cp, cend, lane, S);   // the next window (for this chunk if it was full)
+      if (mask2 != kFull) break;
+    }
+    if (staged) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) rv[u] = st4[u * 32 + lane];
       __syncwarp();
@@ -824,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
     S.ch_lo = S.pv_lo = 0;
     S.ch_base = S.pv_base = q * a.cap;
     if (cend) S.cp = a.pstart[q];
-    load_slots(a, cend, lane, S, 0, 4);
+    load_window(a, S.cp, cend, lane, S);
     uint32_t base = lo & ~3u;
     float4 gv[4], rv[4];
     if (base < lo || base + (uint32_t)kGranule > hi) {
@@ -944,7 +938,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
     S.ch_lo = S.pv_lo = 0;
     S.ch_base = S.pv_base = q * a.cap;
     if (cend) S.cp = a.pstart[q];
-    load_slots(a, cend, lane, S, 0, 4);
+    load_window(a, S.cp, cend, lane, S);
     uint32_t base = lo & ~3u;
     float4 gv[4], rv[4];
     if (base < lo || base + (uint32_t)kGranule > hi) {

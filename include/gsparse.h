@@ -317,6 +317,12 @@ int gsparse_binarize(const float* g, float* residual, int64_t n, const int64_t* 
  *             decoding; not part of the stream.
  * b           0..30.
  */
+/* Recommended side-table chunk for a list of up to `capacity` codewords: the largest power of
+ * two in [4, 64] that still gives at least 16384 chunks (one decoding thread each), so short
+ * lists are decoded by enough threads and long ones keep a small table (16 bytes per chunk).
+ * Returns 4 for capacity <= 0. Any chunk >= 1 is valid; this only chooses speed. */
+int32_t gsparse_golomb_chunk_hint(int64_t capacity);
+
 size_t gsparse_golomb_encode_workspace_size(int64_t capacity);
 int gsparse_golomb_encode(const int32_t* idx, const int64_t* d_begin, const int64_t* d_end,
                           int64_t capacity, int64_t base, int32_t b, uint32_t* words,

@@ -67,3 +67,15 @@ def test_workspace_queries(gs):
     assert lib.gsparse_scatter_accumulate_workspace_size(4, 1 << 20) > 0
     for s in range(6):
         assert lib.gsparse_status_string(s)
+
+
+def test_golomb_chunk_hint(gs):
+    # the largest power of two in [4, 64] leaving at least 16384 chunks
+    assert gs.golomb_chunk_hint(0) == 4 and gs.golomb_chunk_hint(25_558) == 4
+    assert gs.golomb_chunk_hint(16384 * 64) == 64 and gs.golomb_chunk_hint(16384 * 64 - 1) == 32
+    assert gs.golomb_chunk_hint(16384 * 8) == 8 and gs.golomb_chunk_hint(10_737_419) == 64
+    for cap in [1, 1000, 10 ** 5, 10 ** 6, 10 ** 8]:
+        c = gs.golomb_chunk_hint(cap)
+        assert c in (4, 8, 16, 32, 64)
+        assert c == 4 or cap // c >= 16384
+        assert c == 64 or cap // (2 * c) < 16384

@@ -430,6 +430,28 @@ def test_golomb_parity(b, K):
     assert np.array_equal(host(out2)[:K], idx)
 
 
+@pytest.mark.parametrize("chunk", [4, 7, 64])
+@pytest.mark.parametrize("b, K", [(3, (1 << 20) + 7), (9, 25_558), (0, 4097)])
+def test_golomb_parity_chunks_and_list_lengths(b, K, chunk):
+    # short lists (2 codewords per encoding thread) and long ones (8), small and odd side-table
+    # chunks (the decoder's 16-byte output path and its scalar tail)
+    n = 1 << 27 if b else 1 << 14
+    gen = np.random.default_rng(b * 7 + K + chunk)
+    idx = np.unique(gen.integers(0, n, size=int(K * 1.2)))[:K].astype(np.int32)
+    K = idx.size
+    wwords, wbits, wtable = oracle.golomb_encode(idx, b, 0, chunk=chunk)
+    end = torch.tensor([K], dtype=torch.int64, device="cuda")
+    st = gs.status_tensor()
+    words, nbits, table = gs.golomb_encode(dev(idx), end, b, n, chunk=chunk, d_status=st, capacity=K)
+    nb = int(host(nbits)[0])
+    assert int(host(st)[0]) == 0 and nb == wbits
+    assert np.array_equal(host(words)[:(nb + 31) // 32].view(np.uint32), wwords)
+    assert np.array_equal(host(table)[: wtable.shape[0]], wtable)
+    out = gs.golomb_decode(words, nbits, end, K, b, table=table, chunk=chunk, n_limit=n, d_status=st)
+    assert int(host(st)[0]) == 0
+    assert np.array_equal(host(out)[:K], idx)
+
+
 def test_golomb_huge_gaps_and_base():
     idx = np.array([5, 6, 100000, 100001, 2_000_000_000], np.int32)
     for b in [0, 2, 20]:
