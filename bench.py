@@ -39,7 +39,7 @@ import numpy as np  # noqa: E402
 
 METRIC = "gradient GB/s compressed (top-1% residual select+compact)"
 UNIT = "GB/s"
-PROFILE = os.path.join(ROOT, "profiles", "pass1_kernel_flat_fp32.md")
+PROFILE = os.path.join(ROOT, "profiles", "pass1_ring_kernel_flat_fp32.md")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -69,13 +69,21 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def source_sha():
+    """First 16 hex digits of the sha256 of select.cu followed by common.cuh."""
+    h = hashlib.sha256()
+    for f in ("select.cu", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "compressed_sgd_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def profiled_traffic(n):
     """Per-launch DRAM bytes of the pass-1 kernel from the committed ncu summary, scaled to n
-    entries; None if the summary is missing or the kernel source changed since the capture."""
+    entries; None if the summary is missing or the kernel source (select.cu and the shared
+    common.cuh) changed since the capture."""
     try:
         text = open(PROFILE).read()
-        src = open(os.path.join(ROOT, "compressed_sgd_b200", "csrc", "select.cu"), "rb").read()
-        sha = hashlib.sha256(src).hexdigest()[:16]
+        sha = source_sha()
         m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
         m_b = re.search(r"dram_bytes_per_entry:\s*([0-9.]+)", text)
         if not m_sha or not m_b or m_sha.group(1) != sha:
@@ -332,7 +340,7 @@ def run_ours(args, rank, world, dist):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(n, W, args.drop, b, {"parallelism": f"replicas x{world}"}
                                   if mom is None else {"parallelism": f"replicas x{world}", "momentum": mom}),
-        "roofline": {"bound": "hbm", "kernel": ("pass1_kernel" if mom is None else "pass1_ring_kernel") + " (streaming pass of residual top-k)",
+        "roofline": {"bound": "hbm", "kernel": "pass1_ring_kernel<1, " + ("momentum" if mom is not None else "two streams") + "> (streaming pass of residual top-k)",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": profiled_traffic(n) if mom is None else None,
                      "algorithmic_bytes_per_launch": p1_bytes, "launch_ms": round(p1, 4)},

@@ -357,8 +357,10 @@ __device__ __forceinline__ uint32_t* shist_of(const Sel& a, int64_t p, int level
 // smallest s with 2^s >= v (v >= 1)
 __device__ __forceinline__ uint32_t ceil_log2(uint32_t v) { return v <= 1 ? 0u : 32u - __clz(v - 1u); }
 
+constexpr int kSampleThreads = 512;    // two sampled entries per thread, two CTAs per SM
+
 template <int C>
-__global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhaustive) {
+__global__ void __launch_bounds__(kSampleThreads) sample_kernel(Sel a, int level, int exhaustive) {
   pdl_begin();
   __shared__ uint32_t h[C * kBins1];
   __shared__ uint32_t cnt[C];
@@ -435,11 +437,13 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
     run_e[threadIdx.x] = e;
   }
   __syncthreads();
-  // the CTA's slice holds at most 1024 entries: every thread loads its (up to) four first
-  static_assert(kSample / kSampleCtas <= 4 * 256, "four sampled entries per thread");
-  float xs[4];
+  // the CTA's slice holds at most 1024 entries: every thread loads its (at most two) before any
+  // is histogrammed
+  static_assert(kSample / kSampleCtas <= 2 * kSampleThreads, "two sampled entries per thread");
+  constexpr int kIt = (kSample / kSampleCtas + kSampleThreads - 1) / kSampleThreads;
+  float xs[kIt];
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {
+  for (int it = 0; it < kIt; ++it) {
     const int64_t j = j0 + threadIdx.x + (int64_t)it * blockDim.x;
     xs[it] = 0.0f;
     if (j < j1) {
@@ -450,7 +454,7 @@ __global__ void __launch_bounds__(256) sample_kernel(Sel a, int level, int exhau
     }
   }
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {
+  for (int it = 0; it < kIt; ++it) {
     const int64_t j = j0 + threadIdx.x + (int64_t)it * blockDim.x;
     const float x = xs[it];
     const int c = j < j1 ? class_of<C>(x) : -1;
@@ -2121,8 +2125,8 @@ int run_select(const float* g, float* r, int64_t n, const int64_t* seg, int32_t 
   const unsigned piece_ctas = (unsigned)cdiv(L.Q, kWarps);
   const int exhaustive = (flags & GSPARSE_SELECT_EXHAUSTIVE) ? 1 : 0;
   const dim3 sgrid(kSampleCtas, (unsigned)T);
-  launch(sample_kernel<C>, sgrid, 256, 0, st, a, 1, exhaustive);
-  launch(sample_kernel<C>, sgrid, 256, 0, st, a, 2, exhaustive);
+  launch(sample_kernel<C>, sgrid, kSampleThreads, 0, st, a, 1, exhaustive);
+  launch(sample_kernel<C>, sgrid, kSampleThreads, 0, st, a, 2, exhaustive);
   const bool timed = events && events->before && events->after;
   if (timed) cudaEventRecord((cudaEvent_t)events->before, st);
   if (piece_ctas) {
