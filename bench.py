@@ -69,11 +69,20 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def code_text(src):
+    """CUDA source with its comments and blank lines removed: edits to comments alone leave the
+    compiled kernel, and so its counters, unchanged."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip())
+
+
 def source_sha():
-    """First 16 hex digits of the sha256 of select.cu followed by common.cuh."""
+    """First 16 hex digits of the sha256 of the code of select.cu followed by common.cuh."""
     h = hashlib.sha256()
     for f in ("select.cu", "common.cuh"):
-        h.update(open(os.path.join(ROOT, "compressed_sgd_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "compressed_sgd_b200", "csrc", f)).read()
+        h.update(code_text(src).encode())
     return h.hexdigest()[:16]
 
 

@@ -156,7 +156,6 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
     GState* state, uint64_t* flags, uint32_t* head, uint32_t* tail, int32_t* d_status) {
   pdl_begin();
   __shared__ uint32_t wbuf[kPackWords + 1];
-  __shared__ uint32_t cpos[KP * kCodeThreads], cpat[KP * kCodeThreads];   // the gather path's codewords
   __shared__ int64_t sh[33];
   __shared__ uint32_t s_vb;
   __shared__ uint64_t s_prefix;
@@ -215,47 +214,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
     }
     __syncthreads();
   };
-  bool longcw = false;
-#pragma unroll
-  for (int e = 0; e < KP; ++e) longcw |= e < nv && (d[e] >> b) + 1u + (uint32_t)b > 32u;
-  const bool gather = fits && !__syncthreads_or(longcw);
-  if (gather) {
-    // every codeword is at most 32 bits: its relative position and bit pattern go to shared
-    // memory, and each relative word is assembled by the one thread whose bits contain the
-    // word's first bit (plain stores, no atomics)
-    constexpr uint32_t kJ = KP * kCodeThreads;
-    uint32_t p = (uint32_t)ex;
-#pragma unroll
-    for (int e = 0; e < KP; ++e) {
-      const uint32_t j = threadIdx.x * KP + e;
-      if (e < nv) {
-        const uint32_t q = d[e] >> b;
-        const uint32_t rem = d[e] & ((1u << b) - 1u);
-        const uint32_t tl = b ? (__brev(rem) >> (32 - b)) << 1 : 0u;
-        cpos[j] = p;
-        cpat[j] = (q ? 0xffffffffu >> (32u - q) : 0u) | (tl << q);
-        p += q + 1u + (uint32_t)b;
-      } else {
-        cpos[j] = 0xffffffffu;   // past every word
-        cpat[j] = 0u;
-      }
-    }
-    if (threadIdx.x == 0) wbuf[nrel] = 0u;
-    __syncthreads();
-    const uint32_t p0 = (uint32_t)ex, p1 = (uint32_t)(ex + l);
-    uint32_t j = threadIdx.x * KP;
-    for (uint32_t w = (p0 + 31u) >> 5; 32u * w < p1; ++w) {
-      const uint32_t lo = 32u * w;
-      while (j + 1 < kJ && cpos[j + 1] <= lo) ++j;   // the codeword holding bit lo
-      uint32_t acc = 0;
-      for (uint32_t jj = j; jj < kJ && cpos[jj] < lo + 32u; ++jj) {
-        const uint32_t sp = cpos[jj], pt = cpat[jj];
-        acc |= sp >= lo ? pt << (sp - lo) : pt >> (lo - sp);
-      }
-      wbuf[w] = acc;
-    }
-    find_prefix();   // includes the barrier that completes the packing
-  } else if (fits) {
+  if (fits) {
     for (int64_t i = threadIdx.x; i <= nrel; i += blockDim.x) wbuf[i] = 0u;
     __syncthreads();
     uint32_t p = (uint32_t)ex;   // relative bit position (< 2^17 here)

@@ -95,3 +95,13 @@ def test_reference_arm_with_momentum():
     assert out.returncode == 0, out.stderr
     line = json.loads(out.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0
+
+
+def test_profile_hash_ignores_comments_only():
+    """The pass-1 profile stays valid across comment edits and is invalidated by a code edit."""
+    src = "// header\n__global__ void k(int* p) {  /* note */\n  p[0] = 1;  // store\n}\n"
+    same = "// another header\n\n__global__ void k(int* p) {\n  p[0] = 1;\n}\n"
+    other = "__global__ void k(int* p) {\n  p[0] = 2;\n}\n"
+    assert bench.code_text(src) == bench.code_text(same)
+    assert bench.code_text(src) != bench.code_text(other)
+    assert len(bench.source_sha()) == 16
