@@ -95,6 +95,11 @@ __device__ __forceinline__ void st_stream(float* p, float4 v) {
   __stcs(reinterpret_cast<float4*>(p), v);
 }
 
+// Brings the 128-byte line holding p into L2 (a hint: nothing waits for it).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(__cvta_generic_to_global(p)));
+}
+
 // Upper bound search: number of entries of a[0..len) that are <= x (a ascending).
 __device__ __forceinline__ int64_t upper_bound_i64(const int64_t* a, int64_t len, int64_t x) {
   int64_t lo = 0, hi = len;

@@ -859,17 +859,19 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_kernel(Sel a) {
 }
 
 // ------------------------------------------------------------------------------------------
-// 3b. pass 1 through a shared-memory ring (top-k with momentum)
+// 3b. pass 1 through a shared-memory ring (fp32 top-k, with or without momentum)
 //
-// The same pass for three input streams (g, u, r): the interior chunks of a piece reach shared
-// memory by bulk asynchronous copies (one lane issues 2 KB per stream and chunk, completion is
-// counted on a per-slot mbarrier), kStagesM - 1 chunks ahead of the one being processed, so a
-// warp keeps its loads outstanding without holding them in registers. (With two streams the
-// register pipeline above is as fast on flat gradients and faster when candidates cluster.) Every wait is
-// bounded (about a second of SM clock); a wait that gives up raises GSPARSE_DERR_TIMEOUT, stops
-// the call and lets the warp's remaining copies land before it exits.
+// The same pass, with the interior chunks of a piece brought into shared memory by bulk
+// asynchronous copies (one lane issues 2 KB per stream and chunk, completion is counted on a
+// per-slot mbarrier), kStages - 1 chunks ahead of the one being processed (two streams, g and r)
+// or kStagesM - 1 ahead (three streams, g, u and r), so a warp keeps its loads outstanding
+// without holding them in registers. The register pipeline above serves the sign-split
+// binarisation (two classes per problem). Every wait is bounded (about a second of SM
+// clock); a wait that gives up raises GSPARSE_DERR_TIMEOUT, stops the call and lets the warp's
+// remaining copies land before it exits.
 
 constexpr int kStages = 3;
+constexpr uint32_t kPendChunks = 3;    // chunks of pending writes kept requested ahead in L2
 constexpr uint32_t kChunkBytes = (uint32_t)kGranule * 4u;
 constexpr long long kTestWaitCycles = 1ll << 16;   // the test hook's wait (about 33 us)
 
@@ -943,6 +945,14 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
     S.ch_base = S.pv_base = q * a.cap;
     if (cend) S.cp = a.pstart[q];
     load_window(a, S.cp, cend, lane, S);
+    // pending writes up to entry pf have been requested into L2 (see the chunk loop), at most up
+    // to pf_end (the piece's last write) and about kPendChunks chunks' worth ahead of the window
+    uint32_t pf = S.cp, pf_end = S.cp, lead = 0;
+    if (cend) {
+      pf_end = a.pstart[q + 1];
+      const uint64_t per = (uint64_t)(pf_end - S.cp) * (kPendChunks * (uint64_t)kGranule) / (hi > lo ? hi - lo : 1u);
+      lead = (uint32_t)(per + 32u < 512u ? per + 32u : 512u);
+    }
     uint32_t base = lo & ~3u;
     float4 gv[4], rv[4];
     if (base < lo || base + (uint32_t)kGranule > hi) {
@@ -986,6 +996,19 @@ __global__ void __launch_bounds__(kThreads, 2) pass1_ring_kernel(Sel a) {
         break;
       }
       parity ^= 1u << k;
+      // Keep the pending writes of the next few chunks requested into L2: a window load that
+      // missed would queue behind the ring's copies in flight (several microseconds), while the
+      // line is needed one chunk later; a longer lead loses the lines to the stream before use.
+      // Lanes 0-15 take index lines, 16-31 value lines, one 32-entry line each, only lines not
+      // requested before.
+      if (pf < pf_end) {
+        const uint32_t want = S.cp + lead < pf_end ? S.cp + lead : pf_end;
+        if (pf < want) {
+          const uint32_t j = pf + 32u * (uint32_t)(lane & 15);
+          if (j < want) prefetch_l2(lane < 16 ? (const void*)(a.pw_idx + j) : (const void*)(a.pw_val + j));
+          pf = pf + 512u < want ? pf + 512u : want;
+        }
+      }
       const float* us_ = nullptr;
       if constexpr (kMom) us_ = ring[k].u;
       pass1_chunk<C, true>(a, q, base + c * (uint32_t)kGranule, lo, hi, true, 0xFFFFu, gv, rv, S, cend,
