@@ -14,6 +14,8 @@ namespace gs {
 namespace {
 
 constexpr int kTile = 8192;
+constexpr int kTileShift = 13;
+static_assert(kTile == 1 << kTileShift, "tiles are a power of two");
 constexpr int kTileThreads = 256;
 
 struct Lists {
@@ -67,9 +69,12 @@ __global__ void __launch_bounds__(256) sa_starts_kernel(Lists L, int32_t W, int6
     if (c > 0 && (ix[0] < 0 || (int64_t)ix[c - 1] >= n)) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
   }
   const int64_t j0 = kStartsPer * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
-  if (j0 > c) return;
+  // lanes past the list stay for the shuffle below (they mark nothing)
   int32_t v[kStartsPer];
-  if (j0 + kStartsPer <= c && (reinterpret_cast<uintptr_t>(ix) & 15u) == 0) {
+  if (j0 > c) {
+#pragma unroll
+    for (int e = 0; e < kStartsPer; ++e) v[e] = 0;
+  } else if (j0 + kStartsPer <= c && (reinterpret_cast<uintptr_t>(ix) & 15u) == 0) {
 #pragma unroll
     for (int h = 0; h < kStartsPer / 4; ++h) {
       const int4 q = *reinterpret_cast<const int4*>(ix + j0 + 4 * h);
@@ -79,21 +84,26 @@ __global__ void __launch_bounds__(256) sa_starts_kernel(Lists L, int32_t W, int6
 #pragma unroll
     for (int e = 0; e < kStartsPer; ++e) v[e] = j0 + e < c ? ix[j0 + e] : 0;
   }
-  // fast scan: the entries whose tile differs from their predecessor's (or that lie outside
-  // [0, n), or close the list) are marked; the rest start nothing
-  const int32_t p0 = j0 > 0 ? ix[j0 - 1] : -1;
-  const uint32_t un = (uint32_t)(n < INT32_MAX ? n : INT32_MAX);
-  uint32_t mark = 0;
-  int32_t pv = p0;
+  // fast scan, 32-bit: an entry is marked when its raw tile (index >> 13, as unsigned) differs
+  // from its predecessor's, which includes every change of the clamped tile and every negative
+  // index, and so is the end of the list; starts_at clamps, and a marked entry whose clamped tile
+  // equals its predecessor's starts nothing. The predecessor of a thread's first entry is the
+  // last entry of the lane before (one load per warp).
+  const int lane = threadIdx.x & 31;
+  int32_t p0 = __shfl_up_sync(kFull, v[kStartsPer - 1], 1);
+  if (j0 > c) return;
+  if (lane == 0) p0 = j0 > 0 ? ix[j0 - 1] : -1;
+  uint32_t change = 0;
+  uint32_t tp = (uint32_t)p0 >> kTileShift;
 #pragma unroll
   for (int e = 0; e < kStartsPer; ++e) {
-    const int64_t j = j0 + e;
-    const bool in = j < c;
-    const bool odd = !in || v[e] < 0 || (uint32_t)v[e] >= un || pv < 0 ||
-                     ((uint32_t)v[e] / (uint32_t)kTile) != ((uint32_t)pv / (uint32_t)kTile);
-    mark |= (uint32_t)(odd && j <= c) << e;
-    pv = v[e];
+    const uint32_t tv = (uint32_t)v[e] >> kTileShift;
+    change |= (uint32_t)(tv != tp) << e;
+    tp = tv;
   }
+  const int64_t left = c - j0;   // entries of the list from j0 on (>= 0 here)
+  uint32_t mark = left < kStartsPer ? (change & ((1u << (uint32_t)left) - 1u)) | (1u << (uint32_t)left)
+                                    : change;   // entries of the list, and the list's end
   // the marked entries, in order (rolled loop: the list values come again from L1)
   while (mark) {
     const int e = __ffs(mark) - 1;
