@@ -60,6 +60,26 @@ template <int KP>
 __device__ __forceinline__ void thread_gaps(const int32_t* x, int64_t len, int64_t base, int64_t j0,
                                             uint32_t (&d)[KP], int32_t* d_status) {
   int32_t v[KP];
+  if (KP % 4 == 0 && j0 > 0 && j0 + KP <= len && (reinterpret_cast<uintptr_t>(x + j0) & 15u) == 0) {
+    // a full run after the list's first entry: 32-bit differences (indices are int32, so
+    // idx - prev - 1 fits 32 unsigned bits whenever idx > prev)
+#pragma unroll
+    for (int h = 0; h < KP / 4; ++h) {
+      const int4 a = *reinterpret_cast<const int4*>(x + j0 + 4 * h);
+      v[4 * h] = a.x; v[4 * h + 1] = a.y; v[4 * h + 2] = a.z; v[4 * h + 3] = a.w;
+    }
+    int32_t prev = x[j0 - 1];
+    bool bad = false;
+#pragma unroll
+    for (int e = 0; e < KP; ++e) {
+      const bool up = v[e] > prev;
+      bad |= !up;
+      d[e] = up ? (uint32_t)v[e] - (uint32_t)prev - 1u : 0u;
+      prev = v[e];
+    }
+    if (bad) raise(d_status, GSPARSE_DERR_INDEX_RANGE);
+    return;
+  }
   if (KP % 4 == 0 && j0 + KP <= len && (reinterpret_cast<uintptr_t>(x + j0) & 15u) == 0) {
 #pragma unroll
     for (int h = 0; h < KP / 4; ++h) {
@@ -150,7 +170,7 @@ __device__ bool lookback(const uint64_t* flags, uint32_t vb, int lane, uint64_t*
 // merges them. A block whose bits do not fit the shared buffer (very long unary runs) looks back
 // first, zeroes its interior words and ORs its codewords into them.
 template <int KP>
-__global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
+__global__ void __launch_bounds__(kCodeThreads, 5) g_encode_kernel(
     const int32_t* idx, const int64_t* d_begin, const int64_t* d_end, int64_t capacity, int64_t base,
     int b, uint32_t* words, int64_t word_capacity, uint64_t* d_nbits, int64_t* table, int32_t chunk,
     GState* state, uint64_t* flags, uint32_t* head, uint32_t* tail, int32_t* d_status) {
@@ -186,10 +206,24 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
   thread_gaps<KP>(x, len, base, j0, d, d_status);
   // codewords of this thread: entries j0 .. j0 + nv - 1 of the list
   const int nv = len - j0 >= KP ? KP : (len > j0 ? (int)(len - j0) : 0);
-  uint64_t lu = 0;
+  // this thread's bits: 32-bit sums unless a unary part reaches 2^26
+  uint32_t l32 = 0;
+  bool wide = false;
 #pragma unroll
-  for (int e = 0; e < KP; ++e)
-    if (e < nv) lu += (uint64_t)(d[e] >> b) + 1u + (uint32_t)b;
+  for (int e = 0; e < KP; ++e) {
+    if (e < nv) {
+      const uint32_t q = d[e] >> b;
+      wide |= q >= (1u << 26);
+      l32 += q + 1u + (uint32_t)b;
+    }
+  }
+  uint64_t lu = l32;
+  if (wide) {
+    lu = 0;
+#pragma unroll
+    for (int e = 0; e < KP; ++e)
+      if (e < nv) lu += (uint64_t)(d[e] >> b) + 1u + (uint32_t)b;
+  }
   const int64_t l = (int64_t)lu;
   int64_t tot;
   const int64_t ex = block_exclusive_scan(l, sh, &tot);   // this thread's first bit in the block
@@ -260,7 +294,11 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
   // thread; indices < 2^31)
   if (table) {
     // the chunk starts among this thread's codewords: e = e0, e0 + chunk, ... below nv
-    const uint32_t e0 = (uint32_t)((chunk - (int64_t)((uint32_t)j0 % (uint32_t)chunk)) % chunk);
+    const bool p2 = (chunk & (chunk - 1)) == 0;   // power-of-two chunks: masks and shifts
+    const uint32_t cm = (uint32_t)chunk - 1u;
+    const int cs = __ffs(chunk) - 1;
+    const uint32_t e0 = p2 ? (((uint32_t)chunk - ((uint32_t)j0 & cm)) & cm)
+                           : (uint32_t)((chunk - (int64_t)((uint32_t)j0 % (uint32_t)chunk)) % chunk);
     if (e0 < (uint32_t)nv) {
       int64_t o = o0;
       uint32_t next = e0;
@@ -270,7 +308,7 @@ __global__ void __launch_bounds__(kCodeThreads) g_encode_kernel(
         if ((uint32_t)e == next) {
           next += (uint32_t)chunk;
           const int64_t j = j0 + e;
-          const int64_t c = (int64_t)((uint32_t)j / (uint32_t)chunk);
+          const int64_t c = (int64_t)(p2 ? (uint32_t)j >> cs : (uint32_t)j / (uint32_t)chunk);
           table[2 * c] = o;
           table[2 * c + 1] = j == 0 ? base - 1 : (int64_t)x[j - 1];
         }
