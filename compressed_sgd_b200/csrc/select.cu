@@ -1080,14 +1080,29 @@ __global__ void __launch_bounds__(256) pending_check_kernel(Sel a) {
     int64_t next_lo = q_prev + 1 < Qn ? piece_of(a, q_prev + 1).lo : INT64_MAX;
     // fast scan: validity, and a mark on every write at or beyond the next piece's start
     uint32_t mark = 0;
-    int64_t ip = ip0;
+    if (j0 + kCheckPer <= c) {
+      // a full run: 32-bit tests (indices are int32; n <= 2^31 - 1, so an unsigned compare with n
+      // also catches negative indices)
+      const uint32_t un = (uint32_t)a.n;
+      const uint32_t nl = next_lo <= (int64_t)UINT32_MAX ? (uint32_t)next_lo : UINT32_MAX;
+      int32_t ip = (int32_t)ip0;
 #pragma unroll
-    for (int e = 0; e < kCheckPer; ++e) {
-      const int64_t j = j0 + e;
-      const int64_t i = v[e];
-      if (j < c) bad |= i < 0 || i >= a.n || (j > 0 && ip >= i);
-      mark |= (uint32_t)(j <= c && (j == c || i >= next_lo)) << e;
-      ip = i;
+      for (int e = 0; e < kCheckPer; ++e) {
+        bad |= (uint32_t)v[e] >= un || ((j0 + e) > 0 && ip >= v[e]);
+        mark |= (uint32_t)((uint32_t)v[e] >= nl && (uint32_t)v[e] < un) << e;
+        ip = v[e];
+      }
+      // every write at or beyond the next start is marked; out-of-range ones raise anyway
+    } else {
+      int64_t ip = ip0;
+#pragma unroll
+      for (int e = 0; e < kCheckPer; ++e) {
+        const int64_t j = j0 + e;
+        const int64_t i = v[e];
+        if (j < c) bad |= i < 0 || i >= a.n || (j > 0 && ip >= i);
+        mark |= (uint32_t)(j <= c && (j == c || i >= next_lo)) << e;
+        ip = i;
+      }
     }
     // the marked writes, in order (rolled loop)
     while (mark && Qn > 0) {

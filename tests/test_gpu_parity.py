@@ -676,6 +676,32 @@ def test_pending_writes_must_be_ascending():
     assert bool((r == 0).all())                       # nothing written
 
 
+@pytest.mark.parametrize("defect", ["descent", "repeat", "past_n", "negative", "first_negative"])
+def test_pending_writes_invalid_inside_a_long_list(defect):
+    # the same check on a list long enough that the defect sits inside a full run of writes
+    n = 200_000
+    g = synth.gaussian(n, 3)
+    r = torch.zeros(n, device="cuda")
+    base = np.arange(1000, dtype=np.int64) * 150 + 7
+    if defect == "descent":
+        base[500] = base[499] - 3
+    elif defect == "repeat":
+        base[500] = base[499]
+    elif defect == "past_n":
+        base[500:] += n          # ascending, but out of range from entry 500 on
+    elif defect == "negative":
+        base[:501] -= base[500] + 1   # entries 0..500 negative, still ascending
+    else:
+        base[0] = -1
+    pidx = torch.tensor(base.astype(np.int32), device="cuda")
+    pval = torch.ones(1000, device="cuda")
+    st = gs.status_tensor()
+    gs.residual_topk(dev(g), r, (1, 10), d_status=st,
+                     pending=gs.make_pending(pidx, pval, torch.tensor([1000], device="cuda")))
+    assert int(host(st)[0]) & gs.DERR_INDEX_RANGE
+    assert bool((r == 0).all())                       # nothing written
+
+
 # ------------------------------------------------------------------- segmented quantisation
 
 @pytest.mark.parametrize("layout", [[1000], [37, 0, 5000, 256, 1, 70001], [0], [300, 0, 0]])
