@@ -37,7 +37,8 @@ constexpr uint32_t kNone = 0x80000000u;  // a threshold no 31-bit key reaches
 constexpr int kBins1 = 2048, kBins2 = 2048, kBins3 = 512;
 constexpr int kHist = kBins1 + kBins2 + kBins3;  // per problem
 constexpr int64_t kGranule = 512;                // entries per warp iteration (32 lanes x 16)
-constexpr int64_t kTargetPieces = 148 * 32;      // warps streaming at once on a B200
+constexpr int64_t kTargetPieces = 148 * 64;      // four pieces per pass-1 warp slot of a B200 (16 per
+                                                  // SM), so a crowded piece holds up less of the pass
 constexpr int kSample = 1 << 18;                 // sampled entries per segment
 constexpr int kSampleRuns = kSample / 32;        // ... as evenly spaced runs of 32 entries
 constexpr int kSampleCtas = 256;                 // CTAs sharing one segment's sample
