@@ -586,11 +586,15 @@ struct P1State {
 
 // Makes room for `need` more candidates (need <= 512 <= a chunk) by claiming one pool chunk.
 // Warp-uniform; once a candidate has been dropped nothing more is claimed (the piece is re-read).
-__device__ __forceinline__ void p1_reserve(const Sel& a, int64_t q, uint32_t need, P1State& S,
-                                           int lane) {
+// A piece whose candidates so far are more than a quarter of the `seen` entries it has streamed
+// claims none either: candidates that dense are cheaper to re-read from the residual in the later
+// steps (4 bytes per entry) than to store here (8 bytes per candidate and a scattered write
+// each), and refusing at the first spill leaves only the primary store to restore.
+__device__ __forceinline__ void p1_reserve(const Sel& a, int64_t q, uint32_t need, uint32_t seen,
+                                           P1State& S, int lane) {
   if (S.count + need <= S.room || S.count > S.room) return;
   uint32_t c = 0xFFFFFFFFu;
-  if (lane == 0 && S.nch < (uint32_t)a.max_chunks) {
+  if (lane == 0 && S.nch < (uint32_t)a.max_chunks && 4ull * (S.count + need) <= (uint64_t)seen) {
     c = atomicAdd(reinterpret_cast<uint32_t*>(a.ctl + 2), 1u);
     if (c >= (uint64_t)a.pool_chunks) c = 0xFFFFFFFFu;
     else a.pchunk[q * a.max_chunks + S.nch] = (int32_t)c;
@@ -707,13 +711,24 @@ __device__ __forceinline__ void pass1_chunk(const Sel& a, int64_t q, uint32_t ba
   const uint32_t incl = warp_inclusive_scan(packed);
   const uint32_t tot = __shfl_sync(kFull, incl, 31);
   bool from_stage = false;
-  if (tot) {
+  if (tot && S.count > S.room) {
+    // the piece is past its store and will be re-read: only the histogram
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float xs[4] = {av[u].x, av[u].y, av[u].z, av[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((m16 >> (4 * u + e)) & 1u)
+          atomicAdd(hsink + cand_class<C>(xs[e]) * hstride + (mag_key(xs[e]) >> 20), 1u);
+    }
+    S.count += (tot & 0xFFu) + ((tot >> 8) & 0xFFu) + ((tot >> 16) & 0xFFu) + (tot >> 24);
+  } else if (tot) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) st4[u * 32 + lane] = av[u];
     __syncwarp();
     const uint32_t excl = incl - packed;
     const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu;
-    p1_reserve(a, q, t0 + t1 + t2 + (tot >> 24), S, lane);
+    p1_reserve(a, q, t0 + t1 + t2 + (tot >> 24), base + (uint32_t)kGranule - lo, S, lane);
     uint32_t stored = 0;
     for (uint32_t m = m16; m; m &= m - 1) {
       const int b = __ffs(m) - 1;
