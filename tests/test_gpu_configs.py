@@ -256,15 +256,27 @@ def test_config5_2e30_two_workers_three_drops():
                 sb, mm = gs.quantize(idx, val.clone(), off[1:2], d_status=st)
                 assert np.array_equal(bits(host(mm)), bits(qm))
                 assert np.array_equal(host(sb)[:qb.size].view(np.uint32), qb)
-                ww, wnb, _ = oracle.golomb_encode(wi, b, chunk=64)
+                ww, wnb, wt = oracle.golomb_encode(wi, b, chunk=64)
+            elif w == 0:
+                # 90% and 99.9%: quantisation and Golomb words of the library's own list (pinned
+                # above by exact k, order, threshold, ties and the residual invariant), bitwise
+                # against the oracle on the same list
+                hi, hv = host(idx)[:K], host(val)[:K]
+                qb, qm, qv, _ = oracle.quantize(hi, hv, write_dequantized=True)
+                sb, mm = gs.quantize(idx, val.clone(), off[1:2], d_status=st)
+                assert np.array_equal(bits(host(mm)), bits(qm))
+                assert np.array_equal(host(sb)[:qb.size].view(np.uint32), qb)
+                ww, wnb, wt = oracle.golomb_encode(hi, b, chunk=64)
+                del hi, hv, qv
             end = off[1:2]
             words, nbits, table = gs.golomb_encode(idx, end, b, n, chunk=64, d_status=st)
             ids = idx[:K].long()
             gaps = torch.diff(ids, prepend=torch.tensor([-1], device="cuda")) - 1
             assert int(host(nbits)[0]) == K * (b + 1) + int((gaps >> b).sum())        # closed form
-            if w == 0 and drop_den == 100:
+            if w == 0:
                 assert int(host(nbits)[0]) == wnb
                 assert np.array_equal(host(words)[:ww.size].view(np.uint32), ww)
+                assert np.array_equal(host(table)[:wt.shape[0]], wt)                     # side table
             dec = gs.golomb_decode(words, nbits, end, idx.numel(), b, table=table, chunk=64, n_limit=n, d_status=st)
             assert torch.equal(dec[:K], idx[:K])
             lists.append(gs.make_list(dec, end, val=val))
