@@ -587,14 +587,16 @@ struct P1State {
 // Makes room for `need` more candidates (need <= 512 <= a chunk) by claiming one pool chunk.
 // Warp-uniform; once a candidate has been dropped nothing more is claimed (the piece is re-read).
 // A piece whose candidates so far are more than a quarter of the `seen` entries it has streamed
-// claims none either: candidates that dense are cheaper to re-read from the residual in the later
-// steps (4 bytes per entry) than to store here (8 bytes per candidate and a scattered write
-// each), and refusing at the first spill leaves only the primary store to restore.
+// (once it has streamed four chunks, so that one dense row at its start does not decide) claims
+// none either: candidates that dense are cheaper to re-read from the residual in the later steps
+// (4 bytes per entry) than to store here (8 bytes per candidate and a scattered write each), and
+// refusing early leaves little to restore.
 __device__ __forceinline__ void p1_reserve(const Sel& a, int64_t q, uint32_t need, uint32_t seen,
                                            P1State& S, int lane) {
   if (S.count + need <= S.room || S.count > S.room) return;
   uint32_t c = 0xFFFFFFFFu;
-  if (lane == 0 && S.nch < (uint32_t)a.max_chunks && 4ull * (S.count + need) <= (uint64_t)seen) {
+  if (lane == 0 && S.nch < (uint32_t)a.max_chunks &&
+      (seen < 4u * (uint32_t)kGranule || 4ull * (S.count + need) <= (uint64_t)seen)) {
     c = atomicAdd(reinterpret_cast<uint32_t*>(a.ctl + 2), 1u);
     if (c >= (uint64_t)a.pool_chunks) c = 0xFFFFFFFFu;
     else a.pchunk[q * a.max_chunks + S.nch] = (int32_t)c;
@@ -1245,10 +1247,22 @@ __global__ void __launch_bounds__(kThreads) restore_kernel(Sel a) {
     const uint32_t room = room_of(a, q);
     if (redo || cnt > room) {
       if (a.zero_mode) {
+        // the stored candidates get their acc back, eight per lane with their loads in flight
         const uint32_t stored = cnt < room ? cnt : room;
-        for (uint32_t j = lane; j < stored; j += 32) {
-          const int64_t sl = slot_of(a, q, j);
-          a.r[a.cidx[sl]] = a.cval[sl];
+        constexpr int kB = 8;
+        for (uint32_t j0 = lane; j0 < stored; j0 += 32 * kB) {
+          int32_t ix[kB];
+          float xv[kB];
+#pragma unroll
+          for (int k = 0; k < kB; ++k) {
+            const uint32_t j = j0 + 32u * k;
+            const int64_t sl = j < stored ? slot_of(a, q, j) : 0;
+            ix[k] = j < stored ? a.cidx[sl] : -1;
+            xv[k] = j < stored ? a.cval[sl] : 0.0f;
+          }
+#pragma unroll
+          for (int k = 0; k < kB; ++k)
+            if (ix[k] >= 0) a.r[ix[k]] = xv[k];
         }
       }
       __syncwarp();
