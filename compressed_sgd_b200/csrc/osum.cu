@@ -65,14 +65,15 @@ __global__ void __launch_bounds__(kLeafWarps * 32) osum_leaves_kernel(SumJob* jo
     }
     __syncwarp();
     const int m = cnt - base < kLeafRound ? cnt - base : kLeafRound;
+    // a value outside the job's sign class is added as +0, which leaves the sum's bits as they
+    // are (a positive-class sum starts at +0 and only grows; a negative-class one is +0 until its
+    // first member and negative after); no divergent branch when lanes hold different modes
     for (int j = 0; j < m; ++j) {
       const float x = tile[wid][lane][j];
-      switch (mode) {
-        case kSumPositive: if (x > 0.0f) { s = __dadd_rn(s, (double)x); ++members; } break;
-        case kSumNegative: if (x < 0.0f) { s = __dadd_rn(s, (double)x); ++members; } break;
-        case kSumNegated: s = __dadd_rn(s, -(double)x); ++members; break;
-        default: s = __dadd_rn(s, (double)x); ++members;
-      }
+      const bool take = mode == kSumPositive ? x > 0.0f : (mode == kSumNegative ? x < 0.0f : true);
+      const double v = mode == kSumNegated ? -(double)x : (double)x;
+      s = __dadd_rn(s, take ? v : 0.0);
+      members += take;
     }
     __syncwarp();
   }
@@ -146,10 +147,16 @@ __global__ void __launch_bounds__(kLeafWarps * 32) osum_pair_leaves_kernel(SumJo
     }
     __syncwarp();
     const int m = cnt - base < kLeafRound ? cnt - base : kLeafRound;
+    // both sums take every position, the other sign's values as +0: sp starts at +0 and only
+    // grows, sn is +0 until its first negative value and negative after, so adding +0 changes
+    // neither (the same bits as adding each value to its own sum only); no divergent branch
     for (int j = 0; j < m; ++j) {
       const float x = tile[wid][lane][j];
-      if (x > 0.0f) { sp = __dadd_rn(sp, (double)x); ++np; }
-      else if (x < 0.0f) { sn = __dadd_rn(sn, (double)x); ++nn; }
+      const bool pos = x > 0.0f, neg = x < 0.0f;
+      sp = __dadd_rn(sp, (double)(pos ? x : 0.0f));
+      sn = __dadd_rn(sn, (double)(neg ? x : 0.0f));
+      np += pos;
+      nn += neg;
     }
     __syncwarp();
   }
