@@ -22,7 +22,7 @@ def _free_port():
 
 
 N = 200003
-KEEPS = [(1, 100), (0, 1)]   # rank 1 sends nothing in the second round
+KEEPS = [(1, 100), (0, 1)]   # rank 1 sends nothing in the second exchange
 
 
 def _compress(rank, rnd):
@@ -117,7 +117,7 @@ CAP_KEEP = (1, 50)
 
 def _fixed_payload(rank, rnd):
     """Oracle payload laid out in fixed-capacity buffers: words, side table, values and an int64
-    header {bits, count}; rank 1 sends nothing in round 1."""
+    header {bits, count}; rank 1 sends nothing in exchange 1 (the second)."""
     g = synth.flat_mixture(N, seed=3000 * rnd + rank)
     keep = CAP_KEEP if not (rank == 1 and rnd == 1) else (0, 1)
     idx, val, _, _ = oracle.residual_topk(g, np.zeros(N, np.float32), keep)
@@ -173,7 +173,7 @@ def test_fixed_capacity_gather_two_ranks():
 def _lib_keep(rank, rnd):
     if rnd == 0:
         return (1, 10) if rank == 0 else (1, 100)
-    return (1, 100) if rank == 0 else (0, 1)      # rank 1 sends nothing in round 1
+    return (1, 100) if rank == 0 else (0, 1)      # rank 1 sends nothing in exchange 1
 
 
 def _lib_rank_main(rank, world, port, out):
